@@ -1,0 +1,401 @@
+"""Benchmark of the MoE layout -> dispatch -> combine step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 2]
+
+One step = the whole token-choice hot path on one batch: ep_get_layout,
+ep_dispatch (bf16, compact per-expert buffers) and ep_combine (gate-weighted,
+fp32 accumulate, bf16 out), the expert function between them being the
+identity.  Default workload: 4096 tokens x 7168 hidden, 256 experts in 8
+logical ranks, top-8 (sigmoid router with bias), seeded synthetic inputs.
+
+Timing: W untimed warm-up steps; then K steps, each preceded by a 256 MiB
+memset that flushes the 126 MB L2 outside the timed events; CUDA events on
+the launching stream around every step and every kernel; barrier + device
+synchronize on both sides; the max over ranks.  value = algorithmic HBM bytes
+of all steps on all ranks / max time (GB/s).  With N > 1 (torchrun) every rank
+runs its own token batch (its own seed): the units are independent, there is
+no collective on the data path, and the scaling is weak.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine HBM GB/s and tokens/s at 4096×7168 top-8; % of HBM peak"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=2, choices=[2, 5])
+    ap.add_argument("--e2e-steps", type=int, default=40)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def algorithmic_bytes(cfg, n_valid):
+    """HBM bytes the step must move, by kernel (each input read once, each
+    output written once)."""
+    T, H, K, R, E = cfg["T"], cfg["H"], cfg["K"], cfg["R"], cfg["E"]
+    layout = T * K * 8 + T * K * 4 + T * R + E * 4 * 2 + 4 + R * 4
+    dispatch = T * H * 2 + n_valid * H * 2 + T * K * 8 + T * K * 4 + E * 4
+    combine = n_valid * H * 2 + T * H * 2 + T * K * 8 + T * K * 4 + T * K * 4 + E * 4
+    return dict(layout=layout, dispatch=dispatch, combine=combine)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "combine_ep_get_10_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = source_digest()
+    for line in open(path):
+        fields = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+        if fields.get("kernel") == kernel and fields.get("source_sha") == want:
+            try:
+                return int(fields["dram_bytes_per_launch"])
+            except (KeyError, ValueError):
+                return None
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index, uuid=None):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid else pynvml.nvmlDeviceGetHandleByIndex(index)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = self._reasons_fn(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0,
+                    "source": "nvml unavailable" if self._nv is None else "nvml"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (n_gpus, world))
+    return world, rank, local
+
+
+def cpu_oracle_run(cfg_id, seed, n_tokens, reps_budget_s, min_reps=1):
+    """Time the CPU oracle (single thread) on the first n_tokens tokens of the
+    workload: layout + dispatch + combine, as a bounded sample."""
+    import oracle
+    from combine_ep_get_10_b200 import workloads as W
+
+    inp = W.make_inputs(cfg_id, seed=seed)
+    cfg = inp["cfg"]
+    x = np.ascontiguousarray(inp["x"][:n_tokens])
+    idx = np.ascontiguousarray(inp["topk_idx"][:n_tokens])
+    w = np.ascontiguousarray(inp["topk_weights"][:n_tokens])
+    sub = dict(cfg, T=n_tokens)
+    n_valid = int((idx >= 0).sum())
+    times = []
+    t_end = time.perf_counter() + reps_budget_s
+    while len(times) < min_reps or time.perf_counter() < t_end:
+        t0 = time.perf_counter()
+        L = oracle.tc_layout(idx, cfg["E"], cfg["R"])
+        D = oracle.tc_dispatch(x, idx, cfg["E"], L)
+        oracle.tc_combine(D["recv"], idx, cfg["E"], L, w, out_dtype=oracle.BF16)
+        times.append(time.perf_counter() - t0)
+    b = sum(algorithmic_bytes(sub, n_valid).values())
+    return times, b
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: every step is a bounded sample
+    (the first 256 tokens of the workload), single-threaded on the host."""
+    world, rank, _ = dist_setup(args.gpus)
+    if rank != 0:
+        return 0
+    import oracle
+
+    oracle.build()
+    from combine_ep_get_10_b200 import workloads as W
+
+    cfg = W.CONFIGS[args.workload]
+    n_tok = 256
+    inp = W.make_inputs(args.workload)
+    x = np.ascontiguousarray(inp["x"][:n_tok])
+    idx = np.ascontiguousarray(inp["topk_idx"][:n_tok])
+    w = np.ascontiguousarray(inp["topk_weights"][:n_tok])
+    n_valid = int((idx >= 0).sum())
+    bytes_step = sum(algorithmic_bytes(dict(cfg, T=n_tok), n_valid).values())
+
+    def step():
+        L = oracle.tc_layout(idx, cfg["E"], cfg["R"])
+        D = oracle.tc_dispatch(x, idx, cfg["E"], L)
+        oracle.tc_combine(D["recv"], idx, cfg["E"], L, w, out_dtype=oracle.BF16)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = bytes_step * args.steps / dt / 1e9
+    sample = "first %d of %d tokens of workload %s per step" % (n_tok, cfg["T"], cfg["name"])
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": cfg["name"], "sample_tokens": n_tok},
+            "tokens_per_s": n_tok * args.steps / dt,
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    from combine_ep_get_10_b200 import binding as B
+    from combine_ep_get_10_b200 import build as build_mod
+    from combine_ep_get_10_b200 import workloads as W
+
+    if not os.path.exists(build_mod.LIB) and rank == 0:
+        build_mod.build()
+    if world > 1:
+        dist.barrier()
+    B.lib()
+
+    seed = W.CONFIGS[args.workload]["seed"] + 1000 * rank
+    inp = W.make_inputs(args.workload, seed=seed)
+    cfg = inp["cfg"]
+    T, H, K, E, R = cfg["T"], cfg["H"], cfg["K"], cfg["E"], cfg["R"]
+    n_valid = int((inp["topk_idx"] >= 0).sum())
+    nbytes = algorithmic_bytes(cfg, n_valid)
+    step_bytes = sum(nbytes.values())
+
+    dev = torch.device("cuda", local)
+    x_h = torch.from_numpy(inp["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    idx_h = torch.from_numpy(inp["topk_idx"]).pin_memory()
+    w_h = torch.from_numpy(inp["topk_weights"]).pin_memory()
+    x = x_h.to(dev)
+    idx = idx_h.to(dev)
+    w = w_h.to(dev)
+    routing = B.Routing.topk(idx, E, R)
+    lay = B.Layout(routing, device=dev)
+    recv = torch.empty((T * K, H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        B.ep_get_layout(routing, lay, stream=stream)
+        B.ep_dispatch(x, routing, lay, recv, num_recv_rows=T * K, stream=stream)
+        B.ep_combine(recv, routing, lay, w, out, num_y_rows=T * K, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if B.ep_get_device_error(lay) != 0:
+        raise RuntimeError("device error flagged during warm-up")
+
+    K_steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    props = torch.cuda.get_device_properties(dev)
+    uuid = ("GPU-" + str(props.uuid)) if getattr(props, "uuid", None) is not None else None
+    with ClockSampler(local, uuid) as clocks:
+        for i in range(K_steps):
+            flush.zero_()
+            e0, e1, e2, e3 = ev[i]
+            e0.record(stream)
+            B.ep_get_layout(routing, lay, stream=stream)
+            e1.record(stream)
+            B.ep_dispatch(x, routing, lay, recv, num_recv_rows=T * K, stream=stream)
+            e2.record(stream)
+            B.ep_combine(recv, routing, lay, w, out, num_y_rows=T * K, stream=stream)
+            e3.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t_layout = [a[0].elapsed_time(a[1]) for a in ev]
+    t_disp = [a[1].elapsed_time(a[2]) for a in ev]
+    t_comb = [a[2].elapsed_time(a[3]) for a in ev]
+    t_step = [a[0].elapsed_time(a[3]) for a in ev]
+    total_ms = float(sum(t_step))
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    if B.ep_get_device_error(lay) != 0:
+        raise RuntimeError("device error flagged during the timed steps")
+
+    # end to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, the three calls, D2H of the combined output
+    out_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(1, min(args.e2e_steps, K_steps))
+    h2d = x_h.numel() * 2 + idx_h.numel() * 8 + w_h.numel() * 4
+    d2h = out_h.numel() * 2
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(e2e_steps):
+        flush.zero_()
+        ee[i][0].record(stream)
+        x.copy_(x_h, non_blocking=True)
+        idx.copy_(idx_h, non_blocking=True)
+        w.copy_(w_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        ee[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = float(sum(a.elapsed_time(b) for a, b in ee))
+    if world > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+        dist.barrier()
+
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        mean = lambda a: float(sum(a) / len(a))  # noqa: E731
+        k_ms = {"layout": mean(t_layout), "dispatch": mean(t_disp), "combine": mean(t_comb)}
+        dominant = max(("dispatch", "combine"), key=lambda k: k_ms[k])
+        achieved = nbytes[dominant] / (k_ms[dominant] * 1e-3) / 1e9
+        traffic = recorded_traffic(dominant)
+        value = step_bytes * K_steps * world / (total_ms * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K_steps,
+            "warmup": max(3, args.warmup), "ms_per_step": total_ms / K_steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded numpy PCG64 per rank; no dataset)",
+            "config": {"workload": cfg["name"], "num_tokens": T, "hidden": H, "num_topk": K, "num_experts": E,
+                       "logical_ranks": R, "valid_pairs": n_valid, "dispatch": "bf16 compact",
+                       "combine": "bf16 out, fp32 accumulate", "l2": "flushed: 256 MiB memset before every step",
+                       "parallelism": "replicas, one token batch per GPU" if world > 1 else "single GPU"},
+            "tokens_per_s": T * K_steps * world / (total_ms * 1e-3),
+            "kernels_us": {k: v * 1e3 for k, v in k_ms.items()},
+            "kernels_gbs": {k: nbytes[k] / (k_ms[k] * 1e-3) / 1e9 for k in k_ms},
+            "algorithmic_bytes_per_step": nbytes,
+            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": peak_kind, "traffic": traffic},
+            "gpu_launches": 3 * K_steps,
+            "e2e": {"value": step_bytes * e2e_steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "tokens_per_s": T * e2e_steps * world / (e2e_ms * 1e-3), "steps": e2e_steps,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            n_tok = 1024
+            times, b = cpu_oracle_run(args.workload, seed, n_tok, reps_budget_s=10.0)
+            med = statistics.median(times)
+            line["cpu_baseline"] = {"value": b / med / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                    "sample": "first %d of %d tokens, layout+dispatch+combine, median of %d reps"
+                                              % (n_tok, T, len(times)),
+                                    "tokens_per_s": n_tok / med}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,254 @@
+"""Thin ctypes binding of libep_b200.so (C ABI in include/ep.h).
+
+Argument marshalling only: torch tensors are turned into device pointers and
+sizes, the current CUDA stream is passed through, and a non-OK status raises
+EPError.  Every step of layout / dispatch / combine runs in the library's
+CUDA kernels; this module does no arithmetic on the data and has no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libep_b200.so")
+
+# enums of include/ep.h
+EP_OK = 0
+STATUS_NAMES = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_BAD_INDEX", 3: "EP_ERR_OVERFLOW",
+                4: "EP_ERR_WORKSPACE", 5: "EP_ERR_CUDA", 6: "EP_ERR_UNSUPPORTED", 7: "EP_ERR_TIMEOUT"}
+EP_BF16, EP_FP32, EP_FP8_E4M3 = 0, 1, 2
+EP_LAYOUT_COMPACT, EP_LAYOUT_PADDED = 0, 1
+EP_ROUTING_TOPK, EP_ROUTING_EXPERT_CHOICE = 0, 1
+EP_DEVERR_BAD_INDEX, EP_DEVERR_OVERFLOW, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
+
+EXPORTED = ("ep_workspace_bytes", "ep_workspace_init", "ep_get_layout", "ep_dispatch", "ep_combine",
+            "ep_dispatch_expert_choice", "ep_combine_expert_choice", "ep_get_device_error", "ep_status_string",
+            "ep_version")
+
+
+class EPError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s (%s)" % (what, STATUS_NAMES.get(status, status), _status_text(status)))
+
+
+class RoutingDesc(ctypes.Structure):
+    _fields_ = [("routing", ctypes.c_int), ("topk_idx", ctypes.c_void_p), ("token_indices", ctypes.c_void_p),
+                ("num_tokens", ctypes.c_int32), ("num_topk", ctypes.c_int32), ("capacity", ctypes.c_int32),
+                ("num_experts", ctypes.c_int32), ("num_ranks", ctypes.c_int32)]
+
+
+class LayoutDesc(ctypes.Structure):
+    _fields_ = [("num_tokens_per_expert", ctypes.c_void_p), ("expert_offsets", ctypes.c_void_p),
+                ("num_tokens_per_rank", ctypes.c_void_p), ("is_token_in_rank", ctypes.c_void_p),
+                ("slot", ctypes.c_void_p), ("token_offsets", ctypes.c_void_p), ("token_slots", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library; raises if it is missing (build it with
+    ``python -m combine_ep_get_10_b200.build``).  There is no fallback."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libep_b200.so is not built (%s); run python -m combine_ep_get_10_b200.build"
+                              % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, i64, st = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int
+        RP, LP = ctypes.POINTER(RoutingDesc), ctypes.POINTER(LayoutDesc)
+        L.ep_workspace_bytes.restype = ctypes.c_size_t
+        L.ep_workspace_bytes.argtypes = [RP]
+        L.ep_workspace_init.restype = st
+        L.ep_workspace_init.argtypes = [P, ctypes.c_size_t, P]
+        L.ep_get_layout.restype = st
+        L.ep_get_layout.argtypes = [RP, LP, P]
+        L.ep_dispatch.restype = st
+        L.ep_dispatch.argtypes = [P, i32, RP, LP, st, i32, i64, st, P, P, P, P, P, P]
+        L.ep_combine.restype = st
+        L.ep_combine.argtypes = [P, i32, i64, RP, LP, st, i32, P, P, st, P]
+        L.ep_dispatch_expert_choice.restype = st
+        L.ep_dispatch_expert_choice.argtypes = [P, i32, RP, LP, P, P]
+        L.ep_combine_expert_choice.restype = st
+        L.ep_combine_expert_choice.argtypes = [P, i32, RP, LP, P, P, st, P]
+        L.ep_get_device_error.restype = st
+        L.ep_get_device_error.argtypes = [LP, ctypes.POINTER(ctypes.c_uint32), st, P]
+        L.ep_status_string.restype = ctypes.c_char_p
+        L.ep_status_string.argtypes = [st]
+        L.ep_version.restype = ctypes.c_int
+        L.ep_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _status_text(status: int) -> str:
+    try:
+        return lib().ep_status_string(status).decode()
+    except Exception:
+        return "?"
+
+
+def _check(status: int, what: str) -> None:
+    if status != EP_OK:
+        raise EPError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return EP_BF16
+    if t.dtype == torch.float32:
+        return EP_FP32
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return EP_FP8_E4M3
+    raise TypeError("unsupported dtype %s" % t.dtype)
+
+
+class Routing:
+    """A routing decision on the device plus its C descriptor."""
+
+    def __init__(self, desc: RoutingDesc, keep):
+        self.desc = desc
+        self._keep = keep
+
+    @staticmethod
+    def topk(topk_idx: torch.Tensor, num_experts: int, num_ranks: int) -> "Routing":
+        if topk_idx.dtype != torch.int64 or topk_idx.dim() != 2 or not topk_idx.is_contiguous():
+            raise TypeError("topk_idx must be a contiguous int64 [T, K] tensor")
+        d = RoutingDesc(EP_ROUTING_TOPK, topk_idx.data_ptr(), None, topk_idx.shape[0], topk_idx.shape[1], 0,
+                        num_experts, num_ranks)
+        return Routing(d, topk_idx)
+
+    @staticmethod
+    def expert_choice(token_indices: torch.Tensor, num_tokens: int, num_ranks: int) -> "Routing":
+        if token_indices.dtype != torch.int32 or token_indices.dim() != 2 or not token_indices.is_contiguous():
+            raise TypeError("token_indices must be a contiguous int32 [E, C] tensor")
+        E, C = token_indices.shape
+        d = RoutingDesc(EP_ROUTING_EXPERT_CHOICE, None, token_indices.data_ptr(), num_tokens, 0, C, E, num_ranks)
+        return Routing(d, token_indices)
+
+    @property
+    def T(self):
+        return self.desc.num_tokens
+
+    @property
+    def E(self):
+        return self.desc.num_experts
+
+    @property
+    def R(self):
+        return self.desc.num_ranks
+
+
+def ep_workspace_bytes(routing: Routing) -> int:
+    n = lib().ep_workspace_bytes(ctypes.byref(routing.desc))
+    if n == 0:
+        raise EPError(1, "ep_workspace_bytes")
+    return int(n)
+
+
+def ep_workspace_init(workspace: torch.Tensor, stream=None) -> None:
+    _check(lib().ep_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+           "ep_workspace_init")
+
+
+class Layout:
+    """Device buffers of one layout (allocated by torch, i.e. by the caller
+    of the C ABI) plus the C descriptor pointing at them."""
+
+    def __init__(self, routing: Routing, device="cuda", workspace: torch.Tensor | None = None, stream=None):
+        T, E, R = routing.T, routing.E, routing.R
+        i32 = dict(dtype=torch.int32, device=device)
+        self.num_tokens_per_expert = torch.empty(E, **i32)
+        self.num_tokens_per_rank = torch.empty(R, **i32)
+        self.is_token_in_rank = torch.empty((T, R), dtype=torch.uint8, device=device)
+        self.expert_offsets = self.slot = self.token_offsets = self.token_slots = None
+        if routing.desc.routing == EP_ROUTING_TOPK:
+            self.expert_offsets = torch.empty(E + 1, **i32)
+            self.slot = torch.empty((T, routing.desc.num_topk), **i32)
+        else:
+            self.token_offsets = torch.empty(T + 1, **i32)
+            self.token_slots = torch.empty(E * routing.desc.capacity, **i32)
+        need = ep_workspace_bytes(routing)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=device)
+            ep_workspace_init(workspace, stream)
+        elif workspace.numel() * workspace.element_size() < need:
+            raise ValueError("workspace too small: %d < %d" % (workspace.numel(), need))
+        self.workspace = workspace
+        self.desc = LayoutDesc(*(None if t is None else t.data_ptr() for t in (
+            self.num_tokens_per_expert, self.expert_offsets, self.num_tokens_per_rank, self.is_token_in_rank,
+            self.slot, self.token_offsets, self.token_slots, self.workspace)),
+            self.workspace.numel() * self.workspace.element_size())
+
+
+def ep_get_layout(routing: Routing, layout: Layout, stream=None) -> Layout:
+    _check(lib().ep_get_layout(ctypes.byref(routing.desc), ctypes.byref(layout.desc), _stream(stream)),
+           "ep_get_layout")
+    return layout
+
+
+def ep_dispatch(x: torch.Tensor, routing: Routing, layout: Layout, recv_x: torch.Tensor, *, mode=EP_LAYOUT_COMPACT,
+                max_tokens_per_expert=0, num_recv_rows=None, topk_weights=None, recv_scales=None, recv_src=None,
+                recv_weights=None, stream=None) -> None:
+    """out dtype follows recv_x (bfloat16, or uint8 / float8_e4m3fn for FP8)."""
+    out_dtype = _dtype_code(recv_x)
+    rows = recv_x.shape[0] if num_recv_rows is None else int(num_recv_rows)
+    _check(lib().ep_dispatch(_ptr(x), x.shape[1], ctypes.byref(routing.desc), ctypes.byref(layout.desc), int(mode),
+                             int(max_tokens_per_expert), rows, out_dtype, _ptr(topk_weights), _ptr(recv_x),
+                             _ptr(recv_scales), _ptr(recv_src), _ptr(recv_weights), _stream(stream)), "ep_dispatch")
+
+
+def ep_combine(y: torch.Tensor, routing: Routing, layout: Layout, topk_weights: torch.Tensor, out: torch.Tensor, *,
+               mode=EP_LAYOUT_COMPACT, max_tokens_per_expert=0, num_y_rows=None, stream=None) -> None:
+    """out dtype follows `out` (bfloat16 or float32)."""
+    rows = y.shape[0] if num_y_rows is None else int(num_y_rows)
+    _check(lib().ep_combine(_ptr(y), y.shape[1], rows, ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                            int(mode), int(max_tokens_per_expert), _ptr(topk_weights), _ptr(out), _dtype_code(out),
+                            _stream(stream)), "ep_combine")
+
+
+def ep_dispatch_expert_choice(x: torch.Tensor, routing: Routing, layout: Layout, recv_x: torch.Tensor,
+                              stream=None) -> None:
+    _check(lib().ep_dispatch_expert_choice(_ptr(x), x.shape[1], ctypes.byref(routing.desc),
+                                           ctypes.byref(layout.desc), _ptr(recv_x), _stream(stream)),
+           "ep_dispatch_expert_choice")
+
+
+def ep_combine_expert_choice(y: torch.Tensor, routing: Routing, layout: Layout, expert_weights: torch.Tensor,
+                             out: torch.Tensor, stream=None) -> None:
+    _check(lib().ep_combine_expert_choice(_ptr(y), y.shape[1], ctypes.byref(routing.desc),
+                                          ctypes.byref(layout.desc), _ptr(expert_weights), _ptr(out),
+                                          _dtype_code(out), _stream(stream)), "ep_combine_expert_choice")
+
+
+def ep_get_device_error(layout: Layout, clear: bool = True, stream=None) -> int:
+    """Synchronises the stream; returns the EP_DEVERR_* bits (0 = none)."""
+    flags = ctypes.c_uint32(0)
+    st = lib().ep_get_device_error(ctypes.byref(layout.desc), ctypes.byref(flags), 1 if clear else 0,
+                                   _stream(stream))
+    if st not in (EP_OK, 2, 3, 7):
+        raise EPError(st, "ep_get_device_error")
+    return int(flags.value)
+
+
+def ep_status_string(status: int) -> str:
+    return lib().ep_status_string(status).decode()
+
+
+def ep_version() -> int:
+    return int(lib().ep_version())

@@ -1,0 +1,366 @@
+// ep_api.cu -- the C ABI declared in include/ep.h: argument checks on the
+// host, then one launcher per operation.  Nothing here allocates device
+// memory; only ep_get_device_error synchronises.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ep.h"
+#include "ep_internal.h"
+
+namespace {
+
+using ep::kWorkspaceHeaderBytes;
+
+bool aligned(const void* p, uintptr_t n)
+{
+    return (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0;
+}
+
+ep_status_t from_cuda(cudaError_t e)
+{
+    return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+ep_status_t check_routing(const ep_routing_desc_t* r)
+{
+    if (r == nullptr)
+        return EP_ERR_INVALID_ARG;
+    if (r->num_tokens < 0 || r->num_experts < 1 || r->num_ranks < 1 || r->num_ranks > 32 ||
+        r->num_experts % r->num_ranks != 0)
+        return EP_ERR_INVALID_ARG;
+    if (r->routing == EP_ROUTING_TOPK) {
+        if (r->num_topk < 1)
+            return EP_ERR_INVALID_ARG;
+        if (static_cast<int64_t>(r->num_tokens) * r->num_topk >= (int64_t{1} << 31))
+            return EP_ERR_INVALID_ARG;
+        if (r->num_tokens > 0 && (r->topk_idx == nullptr || !aligned(r->topk_idx, 8)))
+            return EP_ERR_INVALID_ARG;
+        return EP_OK;
+    }
+    if (r->routing == EP_ROUTING_EXPERT_CHOICE) {
+        if (r->capacity < 1)
+            return EP_ERR_INVALID_ARG;
+        if (static_cast<int64_t>(r->num_experts) * r->capacity >= (int64_t{1} << 31))
+            return EP_ERR_INVALID_ARG;
+        if (r->token_indices == nullptr || !aligned(r->token_indices, 4))
+            return EP_ERR_INVALID_ARG;
+        return EP_OK;
+    }
+    return EP_ERR_INVALID_ARG;
+}
+
+size_t workspace_need(const ep_routing_desc_t* r)
+{
+    if (r->routing == EP_ROUTING_EXPERT_CHOICE)
+        return ep::ec_layout_workspace_bytes(r->num_tokens, r->num_experts, r->capacity);
+    return kWorkspaceHeaderBytes;
+}
+
+ep_status_t check_workspace(const ep_routing_desc_t* r, const ep_layout_t* l)
+{
+    if (l == nullptr)
+        return EP_ERR_INVALID_ARG;
+    if (l->workspace == nullptr || !aligned(l->workspace, 256) || l->workspace_bytes < workspace_need(r))
+        return EP_ERR_WORKSPACE;
+    return EP_OK;
+}
+
+bool valid_mode(ep_buffer_mode_t m)
+{
+    return m == EP_LAYOUT_COMPACT || m == EP_LAYOUT_PADDED;
+}
+
+ep_status_t check_rows(const ep_routing_desc_t* r, const ep_layout_t* l, ep_buffer_mode_t mode, int32_t max_tokens,
+                       int64_t num_rows)
+{
+    if (!valid_mode(mode) || num_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    if (mode == EP_LAYOUT_PADDED && max_tokens < 1)
+        return EP_ERR_INVALID_ARG;
+    if (r->num_tokens > 0 && (l->slot == nullptr || !aligned(l->slot, 4)))
+        return EP_ERR_INVALID_ARG;
+    if (mode == EP_LAYOUT_COMPACT && (l->expert_offsets == nullptr || !aligned(l->expert_offsets, 4)))
+        return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+ep::TcRows tc_rows(const ep_routing_desc_t* r, const ep_layout_t* l, ep_buffer_mode_t mode, int32_t max_tokens,
+                   int64_t num_rows)
+{
+    ep::TcRows rows{};
+    rows.topk_idx = r->topk_idx;
+    rows.slot = l->slot;
+    rows.offsets = l->expert_offsets;
+    rows.K = r->num_topk;
+    rows.E = r->num_experts;
+    rows.mode = static_cast<int32_t>(mode);
+    rows.max_tokens = max_tokens;
+    rows.num_rows = num_rows;
+    return rows;
+}
+
+} // namespace
+
+extern "C" {
+
+size_t ep_workspace_bytes(const ep_routing_desc_t* routing)
+{
+    if (check_routing(routing) != EP_OK)
+        return 0;
+    return workspace_need(routing);
+}
+
+ep_status_t ep_workspace_init(void* workspace, size_t bytes, ep_stream_t stream)
+{
+    if (workspace == nullptr || !aligned(workspace, 256) || bytes < kWorkspaceHeaderBytes)
+        return EP_ERR_WORKSPACE;
+    return from_cuda(cudaMemsetAsync(workspace, 0, bytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream)
+{
+    ep_status_t st = check_routing(routing);
+    if (st != EP_OK)
+        return st;
+    st = check_workspace(routing, layout);
+    if (st != EP_OK)
+        return st;
+    const int32_t T = routing->num_tokens, E = routing->num_experts, R = routing->num_ranks;
+    if (layout->num_tokens_per_expert == nullptr || layout->num_tokens_per_rank == nullptr ||
+        !aligned(layout->num_tokens_per_expert, 4) || !aligned(layout->num_tokens_per_rank, 4))
+        return EP_ERR_INVALID_ARG;
+    if (T > 0 && layout->is_token_in_rank == nullptr)
+        return EP_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* err = ep::error_word(layout->workspace);
+    if (routing->routing == EP_ROUTING_TOPK) {
+        if (E > ep::kMaxTopkLayoutExperts)
+            return EP_ERR_UNSUPPORTED;
+        if (layout->expert_offsets == nullptr || !aligned(layout->expert_offsets, 4))
+            return EP_ERR_INVALID_ARG;
+        if (T > 0 && (layout->slot == nullptr || !aligned(layout->slot, 4)))
+            return EP_ERR_INVALID_ARG;
+        ep::TcLayoutLaunch a{routing->topk_idx,
+                             T,
+                             routing->num_topk,
+                             E,
+                             R,
+                             layout->num_tokens_per_expert,
+                             layout->expert_offsets,
+                             layout->num_tokens_per_rank,
+                             layout->is_token_in_rank,
+                             layout->slot,
+                             err};
+        return from_cuda(ep::launch_tc_layout(a, s));
+    }
+    if (layout->token_offsets == nullptr || layout->token_slots == nullptr || !aligned(layout->token_offsets, 4) ||
+        !aligned(layout->token_slots, 4))
+        return EP_ERR_INVALID_ARG;
+    ep::EcLayoutLaunch a{routing->token_indices,
+                         T,
+                         E,
+                         routing->capacity,
+                         R,
+                         layout->num_tokens_per_expert,
+                         layout->num_tokens_per_rank,
+                         layout->is_token_in_rank,
+                         layout->token_offsets,
+                         layout->token_slots,
+                         layout->workspace,
+                         err};
+    return from_cuda(ep::launch_ec_layout(a, s));
+}
+
+ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                        ep_buffer_mode_t mode, int32_t max_tokens_per_expert, int64_t num_recv_rows,
+                        ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, float* recv_scales,
+                        int32_t* recv_src, float* recv_weights, ep_stream_t stream)
+{
+    ep_status_t st = check_routing(routing);
+    if (st != EP_OK)
+        return st;
+    if (routing->routing != EP_ROUTING_TOPK)
+        return EP_ERR_INVALID_ARG;
+    st = check_workspace(routing, layout);
+    if (st != EP_OK)
+        return st;
+    st = check_rows(routing, layout, mode, max_tokens_per_expert, num_recv_rows);
+    if (st != EP_OK)
+        return st;
+    if (hidden < 1 || hidden % 8 != 0)
+        return EP_ERR_INVALID_ARG;
+    if (out_dtype != EP_BF16 && out_dtype != EP_FP8_E4M3)
+        return EP_ERR_INVALID_ARG;
+    if (out_dtype == EP_FP8_E4M3 && (hidden % 128 != 0 || (num_recv_rows > 0 && recv_scales == nullptr) ||
+                                     !aligned(recv_scales, 4)))
+        return EP_ERR_INVALID_ARG;
+    const int32_t T = routing->num_tokens;
+    if (T > 0 && (x == nullptr || !aligned(x, 16)))
+        return EP_ERR_INVALID_ARG;
+    if (num_recv_rows > 0 && (recv_x == nullptr || !aligned(recv_x, 16)))
+        return EP_ERR_INVALID_ARG;
+    if (recv_weights != nullptr && (topk_weights == nullptr || !aligned(topk_weights, 4) || !aligned(recv_weights, 4)))
+        return EP_ERR_INVALID_ARG;
+    if (recv_src != nullptr && !aligned(recv_src, 4))
+        return EP_ERR_INVALID_ARG;
+    ep::TcDispatchLaunch a{x,
+                           T,
+                           hidden,
+                           tc_rows(routing, layout, mode, max_tokens_per_expert, num_recv_rows),
+                           static_cast<int32_t>(out_dtype),
+                           topk_weights,
+                           recv_x,
+                           recv_scales,
+                           recv_src,
+                           recv_weights,
+                           ep::error_word(layout->workspace)};
+    return from_cuda(ep::launch_tc_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_combine(const void* y, int32_t hidden, int64_t num_y_rows, const ep_routing_desc_t* routing,
+                       const ep_layout_t* layout, ep_buffer_mode_t mode, int32_t max_tokens_per_expert,
+                       const float* topk_weights, void* out, ep_dtype_t out_dtype, ep_stream_t stream)
+{
+    ep_status_t st = check_routing(routing);
+    if (st != EP_OK)
+        return st;
+    if (routing->routing != EP_ROUTING_TOPK)
+        return EP_ERR_INVALID_ARG;
+    st = check_workspace(routing, layout);
+    if (st != EP_OK)
+        return st;
+    st = check_rows(routing, layout, mode, max_tokens_per_expert, num_y_rows);
+    if (st != EP_OK)
+        return st;
+    if (hidden < 1 || hidden % 8 != 0 || (out_dtype != EP_BF16 && out_dtype != EP_FP32))
+        return EP_ERR_INVALID_ARG;
+    const int32_t T = routing->num_tokens;
+    if (num_y_rows > 0 && (y == nullptr || !aligned(y, 16)))
+        return EP_ERR_INVALID_ARG;
+    if (T > 0 && (out == nullptr || !aligned(out, 16) || topk_weights == nullptr || !aligned(topk_weights, 4)))
+        return EP_ERR_INVALID_ARG;
+    ep::TcCombineLaunch a{y,
+                          T,
+                          hidden,
+                          tc_rows(routing, layout, mode, max_tokens_per_expert, num_y_rows),
+                          topk_weights,
+                          out,
+                          static_cast<int32_t>(out_dtype),
+                          ep::error_word(layout->workspace)};
+    return from_cuda(ep::launch_tc_combine(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_dispatch_expert_choice(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                      const ep_layout_t* layout, void* recv_x, ep_stream_t stream)
+{
+    ep_status_t st = check_routing(routing);
+    if (st != EP_OK)
+        return st;
+    if (routing->routing != EP_ROUTING_EXPERT_CHOICE)
+        return EP_ERR_INVALID_ARG;
+    if (layout == nullptr || layout->workspace == nullptr || !aligned(layout->workspace, 256) ||
+        layout->workspace_bytes < kWorkspaceHeaderBytes)
+        return EP_ERR_WORKSPACE;
+    if (hidden < 1 || hidden % 8 != 0)
+        return EP_ERR_INVALID_ARG;
+    if ((routing->num_tokens > 0 && (x == nullptr || !aligned(x, 16))) || recv_x == nullptr || !aligned(recv_x, 16))
+        return EP_ERR_INVALID_ARG;
+    ep::EcDispatchLaunch a{x,
+                           routing->num_tokens,
+                           hidden,
+                           routing->num_experts,
+                           routing->capacity,
+                           routing->token_indices,
+                           recv_x,
+                           ep::error_word(layout->workspace)};
+    return from_cuda(ep::launch_ec_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_combine_expert_choice(const void* y, int32_t hidden, const ep_routing_desc_t* routing,
+                                     const ep_layout_t* layout, const float* expert_weights, void* out,
+                                     ep_dtype_t out_dtype, ep_stream_t stream)
+{
+    ep_status_t st = check_routing(routing);
+    if (st != EP_OK)
+        return st;
+    if (routing->routing != EP_ROUTING_EXPERT_CHOICE)
+        return EP_ERR_INVALID_ARG;
+    if (layout == nullptr || layout->workspace == nullptr || !aligned(layout->workspace, 256) ||
+        layout->workspace_bytes < kWorkspaceHeaderBytes)
+        return EP_ERR_WORKSPACE;
+    if (hidden < 1 || hidden % 8 != 0 || (out_dtype != EP_BF16 && out_dtype != EP_FP32))
+        return EP_ERR_INVALID_ARG;
+    if (y == nullptr || !aligned(y, 16) || expert_weights == nullptr || !aligned(expert_weights, 4))
+        return EP_ERR_INVALID_ARG;
+    if (layout->token_offsets == nullptr || layout->token_slots == nullptr || !aligned(layout->token_offsets, 4) ||
+        !aligned(layout->token_slots, 4))
+        return EP_ERR_INVALID_ARG;
+    if (routing->num_tokens > 0 && (out == nullptr || !aligned(out, 16)))
+        return EP_ERR_INVALID_ARG;
+    ep::EcCombineLaunch a{y,
+                          routing->num_tokens,
+                          hidden,
+                          static_cast<int64_t>(routing->num_experts) * routing->capacity,
+                          layout->token_offsets,
+                          layout->token_slots,
+                          expert_weights,
+                          out,
+                          static_cast<int32_t>(out_dtype),
+                          ep::error_word(layout->workspace)};
+    return from_cuda(ep::launch_ec_combine(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_get_device_error(const ep_layout_t* layout, uint32_t* flags, int clear, ep_stream_t stream)
+{
+    if (layout == nullptr || layout->workspace == nullptr || !aligned(layout->workspace, 256) ||
+        layout->workspace_bytes < kWorkspaceHeaderBytes)
+        return EP_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, layout->workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess && clear)
+        e = cudaMemsetAsync(layout->workspace, 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess)
+        return EP_ERR_CUDA;
+    if (flags != nullptr)
+        *flags = word;
+    if (word & EP_DEVERR_BAD_INDEX)
+        return EP_ERR_BAD_INDEX;
+    if (word & EP_DEVERR_OVERFLOW)
+        return EP_ERR_OVERFLOW;
+    if (word & EP_DEVERR_TIMEOUT)
+        return EP_ERR_TIMEOUT;
+    return EP_OK;
+}
+
+const char* ep_status_string(ep_status_t status)
+{
+    switch (status) {
+    case EP_OK:
+        return "ok";
+    case EP_ERR_INVALID_ARG:
+        return "invalid argument";
+    case EP_ERR_BAD_INDEX:
+        return "routing index out of range";
+    case EP_ERR_OVERFLOW:
+        return "destination row beyond the buffer";
+    case EP_ERR_WORKSPACE:
+        return "workspace missing, misaligned or too small";
+    case EP_ERR_CUDA:
+        return "CUDA runtime error";
+    case EP_ERR_UNSUPPORTED:
+        return "unsupported configuration";
+    case EP_ERR_TIMEOUT:
+        return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+int ep_version(void)
+{
+    return EP_ABI_VERSION;
+}
+
+} // extern "C"

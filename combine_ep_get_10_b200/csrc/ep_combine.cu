@@ -1,0 +1,250 @@
+// ep_combine.cu -- combine (gather-reduce) kernels.
+//
+// Token choice: DeepEP-Ascend README, API Overview, combine and
+// low_latency_combine (the reduce weighted by topk_weights).  Expert choice:
+// DeepEP issue #595, Solution 1 (the reduce over the slots that picked the
+// token, no [T, K] padding, no cap on their number).  Both skip -1 entries
+// (issue #595, Solution 2).
+//
+// One warp per (token, hidden segment).  A segment is kVecPerLane 16-byte
+// vectors per lane (8 bf16 each); the warp fetches the token's entries (row,
+// weight) once, 32 at a time, broadcasts them by shuffles and, for groups of
+// kGroup entries, issues every 16-byte load of the group before any FMA so
+// that kGroup * kVecPerLane loads per lane are in flight.  Each accumulator
+// sees its entries in ascending order: acc = fmaf(w, y, acc) from 0 in fp32.
+#include "ep_device.cuh"
+#include "ep_internal.h"
+
+namespace ep {
+
+namespace {
+
+constexpr int kCombineThreads = 256;
+constexpr int kWarpsPerCta = kCombineThreads / 32;
+constexpr int kVecPerLane = 2;
+constexpr int kGroup = 8;
+constexpr int kSegVec = 32 * kVecPerLane;
+
+struct CombineArgs {
+    const uint8_t* y;
+    int32_t T, H, nvec, nseg;
+    int64_t num_y_rows;
+    // token choice
+    const int64_t* topk_idx;
+    const int32_t* slot;
+    const int32_t* offsets;
+    int32_t K, E, mode, max_tokens;
+    const float* topk_weights;
+    // expert choice
+    const int32_t* token_offsets;
+    const int32_t* token_slots;
+    const float* expert_weights;
+    void* out;
+    uint32_t* err;
+    int64_t warp_base; // first (token, segment) item of this launch
+};
+
+template <bool kExpertChoice>
+__device__ __forceinline__ void entry(const CombineArgs& a, int64_t t, int64_t beg, int j, int64_t& row, float& w,
+                                      uint32_t& errbits)
+{
+    row = -1;
+    w = 0.0f;
+    if (kExpertChoice) {
+        const int64_t s = __ldg(a.token_slots + beg + j);
+        if (s < 0 || s >= a.num_y_rows) {
+            errbits |= EP_DEVERR_OVERFLOW;
+            return;
+        }
+        row = s;
+        w = __ldg(a.expert_weights + s);
+    } else {
+        const int64_t e = __ldg(a.topk_idx + t * a.K + j);
+        const int32_t s = __ldg(a.slot + t * a.K + j);
+        if (e < 0 || e >= a.E || s < 0) {
+            if (e < -1 || e >= a.E)
+                errbits |= EP_DEVERR_BAD_INDEX;
+            return;
+        }
+        int64_t r;
+        if (a.mode == EP_LAYOUT_PADDED) {
+            if (s >= a.max_tokens) {
+                errbits |= EP_DEVERR_OVERFLOW;
+                return;
+            }
+            r = e * a.max_tokens + s;
+        } else {
+            r = static_cast<int64_t>(__ldg(a.offsets + e)) + s;
+        }
+        if (r >= a.num_y_rows) {
+            errbits |= EP_DEVERR_OVERFLOW;
+            return;
+        }
+        row = r;
+        w = __ldg(a.topk_weights + t * a.K + j);
+    }
+}
+
+template <bool kExpertChoice, bool kOutF32>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = a.warp_base + static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
+    const int64_t t = gw / a.nseg;
+    const int seg = static_cast<int>(gw - t * a.nseg);
+    if (t >= a.T)
+        return;
+
+    int64_t beg = 0;
+    int n;
+    if (kExpertChoice) {
+        beg = __ldg(a.token_offsets + t);
+        n = __ldg(a.token_offsets + t + 1) - static_cast<int>(beg);
+    } else {
+        n = a.K;
+    }
+
+    int v[kVecPerLane];
+    bool vin[kVecPerLane];
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j) {
+        v[j] = seg * kSegVec + j * 32 + lane;
+        vin[j] = v[j] < a.nvec;
+    }
+    float acc[kVecPerLane][8];
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            acc[j][i] = 0.0f;
+
+    uint32_t errbits = 0;
+    const int64_t row_bytes = static_cast<int64_t>(a.H) * 2;
+    for (int k0 = 0; k0 < n; k0 += 32) {
+        int64_t my_row = -1;
+        float my_w = 0.0f;
+        if (k0 + lane < n)
+            entry<kExpertChoice>(a, t, beg, k0 + lane, my_row, my_w, errbits);
+        const int m = min(32, n - k0);
+        for (int g0 = 0; g0 < m; g0 += kGroup) {
+            int64_t rows[kGroup];
+            float ws[kGroup];
+#pragma unroll
+            for (int g = 0; g < kGroup; ++g) {
+                const int src = (g0 + g) & 31;
+                rows[g] = __shfl_sync(kFullMask, my_row, src);
+                ws[g] = __shfl_sync(kFullMask, my_w, src);
+                if (g0 + g >= m)
+                    rows[g] = -1;
+            }
+            uint4 d[kGroup][kVecPerLane];
+#pragma unroll
+            for (int g = 0; g < kGroup; ++g)
+#pragma unroll
+                for (int j = 0; j < kVecPerLane; ++j)
+                    d[g][j] = (rows[g] >= 0 && vin[j]) ? ld_nc_v4(a.y + rows[g] * row_bytes + static_cast<int64_t>(v[j]) * 16)
+                                                        : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int g = 0; g < kGroup; ++g) {
+                if (rows[g] < 0)
+                    continue;
+#pragma unroll
+                for (int j = 0; j < kVecPerLane; ++j) {
+                    acc[j][0] = fmaf(ws[g], bf16_lo(d[g][j].x), acc[j][0]);
+                    acc[j][1] = fmaf(ws[g], bf16_hi(d[g][j].x), acc[j][1]);
+                    acc[j][2] = fmaf(ws[g], bf16_lo(d[g][j].y), acc[j][2]);
+                    acc[j][3] = fmaf(ws[g], bf16_hi(d[g][j].y), acc[j][3]);
+                    acc[j][4] = fmaf(ws[g], bf16_lo(d[g][j].z), acc[j][4]);
+                    acc[j][5] = fmaf(ws[g], bf16_hi(d[g][j].z), acc[j][5]);
+                    acc[j][6] = fmaf(ws[g], bf16_lo(d[g][j].w), acc[j][6]);
+                    acc[j][7] = fmaf(ws[g], bf16_hi(d[g][j].w), acc[j][7]);
+                }
+            }
+        }
+    }
+
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j) {
+        if (!vin[j])
+            continue;
+        if (kOutF32) {
+            float* o = static_cast<float*>(a.out) + t * a.H + static_cast<int64_t>(v[j]) * 8;
+            st_cs_v4(o, make_uint4(__float_as_uint(acc[j][0]), __float_as_uint(acc[j][1]), __float_as_uint(acc[j][2]),
+                                   __float_as_uint(acc[j][3])));
+            st_cs_v4(o + 4, make_uint4(__float_as_uint(acc[j][4]), __float_as_uint(acc[j][5]),
+                                       __float_as_uint(acc[j][6]), __float_as_uint(acc[j][7])));
+        } else {
+            uint8_t* o = static_cast<uint8_t*>(a.out) + t * row_bytes + static_cast<int64_t>(v[j]) * 16;
+            st_cs_v4(o, make_uint4(pack_bf16x2(acc[j][0], acc[j][1]), pack_bf16x2(acc[j][2], acc[j][3]),
+                                   pack_bf16x2(acc[j][4], acc[j][5]), pack_bf16x2(acc[j][6], acc[j][7])));
+        }
+    }
+    if (seg == 0) {
+        const uint32_t any = __reduce_or_sync(kFullMask, errbits);
+        if (lane == 0)
+            flag_error(a.err, any);
+    }
+}
+
+template <bool kExpertChoice>
+cudaError_t launch_combine(CombineArgs k, bool out_f32, cudaStream_t stream)
+{
+    constexpr int64_t kMaxBlocks = int64_t{1} << 30;
+    const int64_t warps = static_cast<int64_t>(k.T) * k.nseg;
+    const int64_t blocks = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
+    for (int64_t b0 = 0; b0 < blocks; b0 += kMaxBlocks) {
+        k.warp_base = b0 * kWarpsPerCta;
+        const unsigned n = static_cast<unsigned>(blocks - b0 < kMaxBlocks ? blocks - b0 : kMaxBlocks);
+        if (out_f32)
+            combine_kernel<kExpertChoice, true><<<n, kCombineThreads, 0, stream>>>(k);
+        else
+            combine_kernel<kExpertChoice, false><<<n, kCombineThreads, 0, stream>>>(k);
+        cudaError_t st = cudaGetLastError();
+        if (st != cudaSuccess)
+            return st;
+    }
+    return cudaSuccess;
+}
+
+} // namespace
+
+cudaError_t launch_tc_combine(const TcCombineLaunch& a, cudaStream_t stream)
+{
+    CombineArgs k{};
+    k.y = static_cast<const uint8_t*>(a.y);
+    k.T = a.T;
+    k.H = a.H;
+    k.nvec = a.H / 8;
+    k.nseg = (k.nvec + kSegVec - 1) / kSegVec;
+    k.num_y_rows = a.rows.num_rows;
+    k.topk_idx = a.rows.topk_idx;
+    k.slot = a.rows.slot;
+    k.offsets = a.rows.offsets;
+    k.K = a.rows.K;
+    k.E = a.rows.E;
+    k.mode = a.rows.mode;
+    k.max_tokens = a.rows.max_tokens;
+    k.topk_weights = a.topk_weights;
+    k.out = a.out;
+    k.err = a.err;
+    return launch_combine<false>(k, a.out_dtype == EP_FP32, stream);
+}
+
+cudaError_t launch_ec_combine(const EcCombineLaunch& a, cudaStream_t stream)
+{
+    CombineArgs k{};
+    k.y = static_cast<const uint8_t*>(a.y);
+    k.T = a.T;
+    k.H = a.H;
+    k.nvec = a.H / 8;
+    k.nseg = (k.nvec + kSegVec - 1) / kSegVec;
+    k.num_y_rows = a.num_y_rows;
+    k.token_offsets = a.token_offsets;
+    k.token_slots = a.token_slots;
+    k.expert_weights = a.expert_weights;
+    k.out = a.out;
+    k.err = a.err;
+    return launch_combine<true>(k, a.out_dtype == EP_FP32, stream);
+}
+
+} // namespace ep

@@ -1,0 +1,310 @@
+// ep_dispatch.cu -- dispatch kernels.
+//
+// bf16 dispatch (token choice: DeepEP-Ascend README, API Overview,
+// dispatch / low_latency_dispatch; expert choice: DeepEP issue #595,
+// Solution 1) is a pure row copy: each source row chunk is read from HBM
+// exactly once by the TMA engine (cp.async.bulk global->shared, completion on
+// an mbarrier) and written to every destination row by bulk stores
+// (cp.async.bulk shared->global), one per destination, issued by different
+// lanes.  A CTA is one warp and moves one (row, chunk) item; up to 32 CTAs
+// per SM keep ~200 KB of copies in flight per SM and the block scheduler
+// balances the tail.
+//
+// FP8 dispatch (README, "Quantization Modes in Normal Dispatch"; one fp32
+// scale per 128 channels): one CTA per token quantises the row once in
+// registers -- a half-warp owns a 128-channel group, amax by shuffles,
+// scale = amax/448, codes = cvt.rn.satfinite.e4m3x2(x * 448/amax) -- and
+// stores the 8-byte code runs and the scale to each destination row.
+#include <algorithm>
+
+#include "ep_device.cuh"
+#include "ep_internal.h"
+
+namespace ep {
+
+namespace {
+
+constexpr int64_t kChunkTarget = 8192; // bytes per bulk-copy item
+
+struct RowMap {
+    const int64_t* topk_idx;
+    const int32_t* slot;
+    const int32_t* offsets;
+    int32_t K, E, mode, max_tokens;
+    int64_t num_rows;
+
+    // Destination row of pair (t,k), or -1 (not routed / no room).
+    __device__ __forceinline__ int64_t row(int64_t t, int k, uint32_t& errbits) const
+    {
+        const int64_t e = __ldg(topk_idx + t * K + k);
+        const int32_t s = __ldg(slot + t * K + k);
+        if (e < 0 || e >= E || s < 0) {
+            if (e < -1 || e >= E)
+                errbits |= EP_DEVERR_BAD_INDEX;
+            return -1;
+        }
+        int64_t r;
+        if (mode == EP_LAYOUT_PADDED) {
+            if (s >= max_tokens) {
+                errbits |= EP_DEVERR_OVERFLOW;
+                return -1;
+            }
+            r = e * max_tokens + s;
+        } else {
+            r = static_cast<int64_t>(__ldg(offsets + e)) + s;
+        }
+        if (r >= num_rows) {
+            errbits |= EP_DEVERR_OVERFLOW;
+            return -1;
+        }
+        return r;
+    }
+};
+
+struct BulkArgs {
+    const uint8_t* src;
+    uint8_t* dst;
+    int64_t row_bytes;
+    int64_t chunk_bytes;
+    int32_t nchunks;
+    RowMap map;                 // token choice
+    const float* topk_weights;  // token choice, optional outputs
+    int32_t* recv_src;
+    float* recv_weights;
+    const int32_t* token_indices; // expert choice
+    int32_t T;
+    uint32_t* err;
+    int64_t item_base; // first item of this launch
+};
+
+// One warp per (row, chunk) item.  kExpertChoice: item row = slot s, source
+// token = token_indices[s], one destination (row s).  Otherwise item row =
+// token t, destinations = its K routed pairs.
+template <bool kExpertChoice>
+__global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
+{
+    __shared__ __align__(8) uint64_t bar;
+    extern __shared__ __align__(128) uint8_t buf[];
+    const int lane = threadIdx.x;
+    const int64_t item = a.item_base + blockIdx.x;
+    const int64_t r = item / a.nchunks;
+    const int c = static_cast<int>(item - r * a.nchunks);
+    const int64_t off = static_cast<int64_t>(c) * a.chunk_bytes;
+    const uint32_t bytes = static_cast<uint32_t>(min(a.chunk_bytes, a.row_bytes - off));
+    uint32_t errbits = 0;
+
+    int64_t src_row;
+    if (kExpertChoice) {
+        const int t = __ldg(a.token_indices + r);
+        if (t < 0 || t >= a.T) {
+            if (lane == 0 && c == 0 && t != -1)
+                flag_error(a.err, EP_DEVERR_BAD_INDEX);
+            return;
+        }
+        src_row = t;
+    } else {
+        src_row = r;
+    }
+
+    if (lane == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&bar, bytes);
+        bulk_load_g2s(buf, a.src + src_row * a.row_bytes + off, bytes, &bar);
+    }
+    // destination rows of the first 32 pairs while the load is in flight
+    int64_t dst_row = -1;
+    if (kExpertChoice) {
+        dst_row = lane == 0 ? r : -1;
+    } else if (lane < a.map.K) {
+        dst_row = a.map.row(r, lane, errbits);
+    }
+    __syncwarp();
+    const bool ok = mbar_wait_bounded(&bar, 0, a.err);
+    if (ok) {
+        if (dst_row >= 0)
+            bulk_store_s2g(a.dst + dst_row * a.row_bytes + off, buf, bytes);
+        if (!kExpertChoice) {
+            for (int k = lane + 32; k < a.map.K; k += 32) {
+                const int64_t rk = a.map.row(r, k, errbits);
+                if (rk >= 0)
+                    bulk_store_s2g(a.dst + rk * a.row_bytes + off, buf, bytes);
+            }
+        }
+        bulk_commit();
+        bulk_wait_read_all();
+    }
+    if (!kExpertChoice && c == 0 && (a.recv_src != nullptr || a.recv_weights != nullptr)) {
+        uint32_t ignored = 0;
+        for (int k = lane; k < a.map.K; k += 32) {
+            const int64_t rk = k < 32 ? dst_row : a.map.row(r, k, ignored);
+            if (rk < 0)
+                continue;
+            if (a.recv_src != nullptr)
+                a.recv_src[rk] = static_cast<int32_t>(r);
+            if (a.recv_weights != nullptr)
+                a.recv_weights[rk] = __ldg(a.topk_weights + r * a.map.K + k);
+        }
+    }
+    if (c == 0) {
+        const uint32_t any = __reduce_or_sync(kFullMask, errbits);
+        if (lane == 0)
+            flag_error(a.err, any);
+    }
+}
+
+struct Fp8Args {
+    const uint16_t* x;
+    int32_t H;
+    RowMap map;
+    uint8_t* recv;
+    float* scales;
+    const float* topk_weights;
+    int32_t* recv_src;
+    float* recv_weights;
+    uint32_t* err;
+};
+
+constexpr int kFp8Threads = 256;
+
+__global__ void __launch_bounds__(kFp8Threads) fp8_dispatch_kernel(Fp8Args a)
+{
+    extern __shared__ __align__(16) int64_t rows[]; // [K]
+    const int64_t t = blockIdx.x;
+    const int tid = threadIdx.x;
+    uint32_t errbits = 0;
+    for (int k = tid; k < a.map.K; k += kFp8Threads) {
+        const int64_t rk = a.map.row(t, k, errbits);
+        rows[k] = rk;
+        if (rk >= 0) {
+            if (a.recv_src != nullptr)
+                a.recv_src[rk] = static_cast<int32_t>(t);
+            if (a.recv_weights != nullptr)
+                a.recv_weights[rk] = __ldg(a.topk_weights + t * a.map.K + k);
+        }
+    }
+    if (errbits)
+        flag_error(a.err, errbits);
+    __syncthreads();
+
+    const int nvec = a.H / 8;   // 16-byte vectors of 8 bf16
+    const int groups = a.H / 128;
+    const uint8_t* xrow = reinterpret_cast<const uint8_t*>(a.x) + t * static_cast<int64_t>(a.H) * 2;
+    for (int base = 0; base < nvec; base += kFp8Threads) {
+        const int v = base + tid;
+        const bool active = v < nvec; // a 16-lane group is all-in or all-out (nvec % 16 == 0)
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (active)
+            raw = ld_nc_v4(xrow + static_cast<int64_t>(v) * 16);
+        float f[8];
+        f[0] = bf16_lo(raw.x);
+        f[1] = bf16_hi(raw.x);
+        f[2] = bf16_lo(raw.y);
+        f[3] = bf16_hi(raw.y);
+        f[4] = bf16_lo(raw.z);
+        f[5] = bf16_hi(raw.z);
+        f[6] = bf16_lo(raw.w);
+        f[7] = bf16_hi(raw.w);
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+        for (int d = 8; d >= 1; d >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
+        float scale = 0.0f;
+        uint2 q = make_uint2(0, 0);
+        if (amax > 0.0f) {
+            scale = __fdiv_rn(amax, 448.0f);
+            float inv = __fdiv_rn(448.0f, amax);
+            inv = fminf(inv, 3.40282347e38f);
+            float p[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                p[i] = __fmul_rn(f[i], inv);
+            q.x = pack_e4m3x2(p[0], p[1]) | (pack_e4m3x2(p[2], p[3]) << 16);
+            q.y = pack_e4m3x2(p[4], p[5]) | (pack_e4m3x2(p[6], p[7]) << 16);
+        }
+        if (active) {
+            const int g = v >> 4;
+            for (int k = 0; k < a.map.K; ++k) {
+                const int64_t rk = rows[k];
+                if (rk < 0)
+                    continue;
+                st_v2(a.recv + rk * a.H + static_cast<int64_t>(v) * 8, q);
+                if ((tid & 15) == 0)
+                    a.scales[rk * groups + g] = scale;
+            }
+        }
+    }
+}
+
+constexpr int64_t kMaxGrid = int64_t{1} << 30;
+
+template <bool kExpertChoice>
+cudaError_t launch_bulk(BulkArgs k, int64_t items, cudaStream_t stream)
+{
+    for (int64_t base = 0; base < items; base += kMaxGrid) {
+        k.item_base = base;
+        const unsigned n = static_cast<unsigned>(std::min(kMaxGrid, items - base));
+        bulk_dispatch_kernel<kExpertChoice><<<n, 32, static_cast<size_t>(k.chunk_bytes), stream>>>(k);
+        cudaError_t st = cudaGetLastError();
+        if (st != cudaSuccess)
+            return st;
+    }
+    return cudaSuccess;
+}
+
+} // namespace
+
+cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream)
+{
+    if (a.T == 0)
+        return cudaSuccess;
+    RowMap m{a.rows.topk_idx, a.rows.slot, a.rows.offsets, a.rows.K, a.rows.E, a.rows.mode, a.rows.max_tokens,
+             a.rows.num_rows};
+    if (a.out_dtype == EP_FP8_E4M3) {
+        Fp8Args k{static_cast<const uint16_t*>(a.x), a.H, m, static_cast<uint8_t*>(a.recv_x), a.recv_scales,
+                  a.topk_weights, a.recv_src, a.recv_weights, a.err};
+        const size_t smem = sizeof(int64_t) * static_cast<size_t>(a.rows.K);
+        if (smem > 48 * 1024) {
+            cudaError_t st = cudaFuncSetAttribute(fp8_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(smem));
+            if (st != cudaSuccess)
+                return st;
+        }
+        fp8_dispatch_kernel<<<a.T, kFp8Threads, smem, stream>>>(k);
+        return cudaGetLastError();
+    }
+    BulkArgs k{};
+    k.src = static_cast<const uint8_t*>(a.x);
+    k.dst = static_cast<uint8_t*>(a.recv_x);
+    k.row_bytes = static_cast<int64_t>(a.H) * 2;
+    k.nchunks = static_cast<int32_t>((k.row_bytes + kChunkTarget - 1) / kChunkTarget);
+    k.chunk_bytes = ((k.row_bytes / k.nchunks + 15) / 16) * 16;
+    k.nchunks = static_cast<int32_t>((k.row_bytes + k.chunk_bytes - 1) / k.chunk_bytes);
+    k.map = m;
+    k.topk_weights = a.topk_weights;
+    k.recv_src = a.recv_src;
+    k.recv_weights = a.recv_weights;
+    k.err = a.err;
+    return launch_bulk<false>(k, static_cast<int64_t>(a.T) * k.nchunks, stream);
+}
+
+cudaError_t launch_ec_dispatch(const EcDispatchLaunch& a, cudaStream_t stream)
+{
+    const int64_t S = static_cast<int64_t>(a.E) * a.C;
+    BulkArgs k{};
+    k.src = static_cast<const uint8_t*>(a.x);
+    k.dst = static_cast<uint8_t*>(a.recv_x);
+    k.row_bytes = static_cast<int64_t>(a.H) * 2;
+    k.nchunks = static_cast<int32_t>((k.row_bytes + kChunkTarget - 1) / kChunkTarget);
+    k.chunk_bytes = ((k.row_bytes / k.nchunks + 15) / 16) * 16;
+    k.nchunks = static_cast<int32_t>((k.row_bytes + k.chunk_bytes - 1) / k.chunk_bytes);
+    k.token_indices = a.token_indices;
+    k.T = a.T;
+    k.err = a.err;
+    return launch_bulk<true>(k, S * k.nchunks, stream);
+}
+
+} // namespace ep

@@ -1,0 +1,107 @@
+// ep_internal.h -- host-side launch interfaces between the C-ABI layer
+// (ep_api.cu) and the kernel files.  Arguments reaching these launchers have
+// been validated by ep_api.cu.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ep.h"
+
+namespace ep {
+
+constexpr size_t kWorkspaceHeaderBytes = 256; // error word + reserved
+constexpr int kMaxTopkLayoutExperts = 1024;   // token-choice layout keeps E counters per warp
+
+inline uint32_t* error_word(void* workspace)
+{
+    return static_cast<uint32_t*>(workspace);
+}
+
+// ------------------------------------------------------------------ layout
+struct TcLayoutLaunch {
+    const int64_t* topk_idx;
+    int32_t T, K, E, R;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* rank_counts;
+    uint8_t* in_rank;
+    int32_t* slot;
+    uint32_t* err;
+};
+cudaError_t launch_tc_layout(const TcLayoutLaunch& a, cudaStream_t stream);
+
+struct EcLayoutLaunch {
+    const int32_t* token_indices;
+    int32_t T, E, C, R;
+    int32_t* counts;
+    int32_t* rank_counts;
+    uint8_t* in_rank;
+    int32_t* token_offsets;
+    int32_t* token_slots;
+    void* workspace; // header, then tmask[T], fill[T], scratch[E*C]
+    uint32_t* err;
+};
+size_t ec_layout_workspace_bytes(int64_t T, int64_t E, int64_t C);
+cudaError_t launch_ec_layout(const EcLayoutLaunch& a, cudaStream_t stream);
+
+// --------------------------------------------------------------- dispatch
+// Token-choice destination rows (shared by dispatch and combine).
+struct TcRows {
+    const int64_t* topk_idx;
+    const int32_t* slot;
+    const int32_t* offsets;
+    int32_t K, E, mode, max_tokens;
+    int64_t num_rows;
+};
+
+struct TcDispatchLaunch {
+    const void* x;
+    int32_t T, H;
+    TcRows rows;
+    int32_t out_dtype;
+    const float* topk_weights;
+    void* recv_x;
+    float* recv_scales;
+    int32_t* recv_src;
+    float* recv_weights;
+    uint32_t* err;
+};
+cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream);
+
+struct EcDispatchLaunch {
+    const void* x;
+    int32_t T, H, E, C;
+    const int32_t* token_indices;
+    void* recv_x;
+    uint32_t* err;
+};
+cudaError_t launch_ec_dispatch(const EcDispatchLaunch& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- combine
+struct TcCombineLaunch {
+    const void* y;
+    int32_t T, H;
+    TcRows rows;
+    const float* topk_weights;
+    void* out;
+    int32_t out_dtype;
+    uint32_t* err;
+};
+cudaError_t launch_tc_combine(const TcCombineLaunch& a, cudaStream_t stream);
+
+struct EcCombineLaunch {
+    const void* y;
+    int32_t T, H;
+    int64_t num_y_rows;
+    const int32_t* token_offsets;
+    const int32_t* token_slots;
+    const float* expert_weights;
+    void* out;
+    int32_t out_dtype;
+    uint32_t* err;
+};
+cudaError_t launch_ec_combine(const EcCombineLaunch& a, cudaStream_t stream);
+
+} // namespace ep

@@ -1,0 +1,208 @@
+/*
+ * ep.h -- MoE token layout, dispatch and combine on one B200 (sm_100a).
+ *
+ * C ABI of libep_b200.so.  All tensors are plain device pointers, row-major
+ * and densely packed; all memory belongs to the caller.  No entry point
+ * allocates or frees device memory, and none synchronises the host except
+ * ep_get_device_error().  Every call is asynchronous on `stream`
+ * (a cudaStream_t; NULL = the legacy default stream).
+ *
+ * The operations follow these pages (title, section):
+ *   [README] "DeepEP-Ascend" README (sgl-kernel-npu python/deep_ep),
+ *            "API Overview" table: get_dispatch_layout, dispatch, combine,
+ *            low_latency_dispatch, low_latency_combine; "Quantization Modes
+ *            in Normal Dispatch"; "Environment Variables":
+ *            MOE_EXPERT_TOKEN_NUMS_TYPE (count vs prefix-sum form),
+ *            MOE_ENABLE_TOPK_NEG_ONE (-1 = not dispatched).
+ *   [EC]     DeepEP issue #595, "Support Expert-Choice Routing via Native
+ *            Expert-Centric API ([num_experts, capacity])": "Proposed
+ *            Solutions", Solution 1 (token_indices [num_experts, capacity]
+ *            and its dispatch/combine pair) and Solution 2 (skip -1 padding).
+ *
+ * Notation: T tokens, H hidden, K top-k width, E experts, R logical ranks
+ * (rank r owns experts [r*E/R, (r+1)*E/R)), C expert capacity.
+ *
+ * Status and errors
+ *   Argument problems found on the host return EP_ERR_INVALID_ARG (or
+ *   EP_ERR_UNSUPPORTED / EP_ERR_WORKSPACE) before anything is launched.
+ *   A failed launch returns EP_ERR_CUDA.  Problems only the device can see
+ *   (an index out of range, a padded buffer that is full, a bounded wait
+ *   that ran out) never fault: the offending element is skipped and a bit
+ *   is OR-ed into the error word at the start of the layout workspace,
+ *   read back by ep_get_device_error().
+ */
+#ifndef EP_B200_H_
+#define EP_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EP_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define EP_API __attribute__((visibility("default")))
+#else
+#define EP_API
+#endif
+
+typedef struct CUstream_st* ep_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    EP_OK = 0,
+    EP_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer, bad enum */
+    EP_ERR_BAD_INDEX = 2,   /* device: routing id outside [-1, E) or [-1, T) */
+    EP_ERR_OVERFLOW = 3,    /* device: destination row beyond the buffer */
+    EP_ERR_WORKSPACE = 4,   /* workspace missing, misaligned or too small */
+    EP_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+    EP_ERR_UNSUPPORTED = 6, /* valid request this build does not handle */
+    EP_ERR_TIMEOUT = 7      /* device: a bounded wait gave up */
+} ep_status_t;
+
+typedef enum { EP_BF16 = 0, EP_FP32 = 1, EP_FP8_E4M3 = 2 } ep_dtype_t;
+
+/* COMPACT: expert e's rows are [expert_offsets[e], expert_offsets[e+1]) of
+ *   one buffer (normal-mode dispatch); rank r's rows are the contiguous
+ *   range [expert_offsets[r*E/R], expert_offsets[(r+1)*E/R]).
+ * PADDED: expert e owns rows [e*max_tokens, (e+1)*max_tokens), as the
+ *   low-latency per-expert receive buffers of num_max_dispatch_tokens rows;
+ *   rows past num_tokens_per_expert[e] are never written. */
+typedef enum { EP_LAYOUT_COMPACT = 0, EP_LAYOUT_PADDED = 1 } ep_buffer_mode_t;
+
+typedef enum { EP_ROUTING_TOPK = 0, EP_ROUTING_EXPERT_CHOICE = 1 } ep_routing_t;
+
+/* bits of the device error word */
+#define EP_DEVERR_BAD_INDEX 0x1u
+#define EP_DEVERR_OVERFLOW 0x2u
+#define EP_DEVERR_TIMEOUT 0x4u
+
+/* The routing decision, read-only.
+ *   TOPK:          topk_idx  int64 [T, K]; entry -1 = slot not dispatched.
+ *   EXPERT_CHOICE: token_indices int32 [E, C]; entry -1 = empty slot.
+ * Ids outside [-1, E) (resp. [-1, T)) are treated as -1 and flagged
+ * EP_DEVERR_BAD_INDEX.  Limits: T >= 0; K, E, C >= 1; 1 <= R <= 32;
+ * E % R == 0; T*K and E*C below 2^31; token-choice layout needs E <= 1024. */
+typedef struct {
+    ep_routing_t routing;
+    const int64_t* topk_idx;
+    const int32_t* token_indices;
+    int32_t num_tokens;
+    int32_t num_topk;
+    int32_t capacity;
+    int32_t num_experts;
+    int32_t num_ranks;
+} ep_routing_desc_t;
+
+/* Layout outputs (written by ep_get_layout) and the handle that dispatch
+ * and combine read back.  Pointers not used by a routing kind may be NULL.
+ *   num_tokens_per_expert int32 [E]    pairs (TOPK) or filled slots (EC) per expert
+ *   expert_offsets        int32 [E+1]  TOPK: exclusive scan of the counts
+ *   num_tokens_per_rank   int32 [R]    tokens with >= 1 expert in rank r
+ *   is_token_in_rank      uint8 [T, R] 0/1
+ *   slot                  int32 [T, K] TOPK: rank of pair (t,k) among the
+ *                                      pairs of its expert in ascending
+ *                                      (t, k) order; -1 if not routed
+ *   token_offsets         int32 [T+1]  EC: exclusive scan of picks per token
+ *   token_slots           int32 [E*C]  EC: slot ids s = e*C + c picking each
+ *                                      token, ascending; [0, token_offsets[T])
+ *                                      is written
+ *   workspace             device scratch of ep_workspace_bytes() bytes,
+ *                         256-byte aligned.  Zero it once (ep_workspace_init)
+ *                         before first use; calls leave it reusable.  One
+ *                         workspace per stream: calls that share one must not
+ *                         overlap on the GPU. */
+typedef struct {
+    int32_t* num_tokens_per_expert;
+    int32_t* expert_offsets;
+    int32_t* num_tokens_per_rank;
+    uint8_t* is_token_in_rank;
+    int32_t* slot;
+    int32_t* token_offsets;
+    int32_t* token_slots;
+    void* workspace;
+    size_t workspace_bytes;
+} ep_layout_t;
+
+/* Bytes of workspace the layout of this routing needs (>= 256; the first
+ * 256 bytes hold the device error word).  Pure host function. */
+EP_API size_t ep_workspace_bytes(const ep_routing_desc_t* routing);
+
+/* Zero `bytes` of workspace on `stream` (a cudaMemsetAsync). */
+EP_API ep_status_t ep_workspace_init(void* workspace, size_t bytes, ep_stream_t stream);
+
+/* get_dispatch_layout ([README] API Overview; count and prefix-sum forms per
+ * MOE_EXPERT_TOKEN_NUMS_TYPE; -1 per MOE_ENABLE_TOPK_NEG_ONE).
+ * TOPK writes num_tokens_per_expert, expert_offsets, num_tokens_per_rank,
+ * is_token_in_rank and slot.  EXPERT_CHOICE ([EC] Solution 1) writes
+ * num_tokens_per_expert, num_tokens_per_rank, is_token_in_rank,
+ * token_offsets and token_slots.  Deterministic: the same routing gives the
+ * same bytes on every call. */
+EP_API ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream);
+
+/* Token-choice dispatch ([README] API Overview: dispatch; low_latency_dispatch
+ * for PADDED).  For every routed pair (t,k) of expert e with slot s:
+ *   row = expert_offsets[e] + s          (COMPACT)
+ *   row = e * max_tokens_per_expert + s  (PADDED; s >= max_tokens -> skipped,
+ *                                         EP_DEVERR_OVERFLOW)
+ * and row >= num_recv_rows is skipped with EP_DEVERR_OVERFLOW.
+ *   x            bf16 [T, H], 16-byte aligned, H % 8 == 0
+ *   out_dtype    EP_BF16: recv_x bf16 [rows, H] receives x[t] bit for bit.
+ *                EP_FP8_E4M3 (H % 128 == 0): recv_x uint8 [rows, H] receives
+ *                e4m3 codes and recv_scales fp32 [rows, H/128] one scale per
+ *                128 channels: scale = amax/448, code = RNE-satfinite of
+ *                x * (448/amax) (448/amax clamped to FLT_MAX; amax == 0 gives
+ *                scale 0 and code 0x00) -- [README] "Quantization Modes".
+ *   topk_weights fp32 [T, K], needed only when recv_weights != NULL
+ *   recv_src     optional int32 [rows]: source token of each written row
+ *   recv_weights optional fp32 [rows]: gate weight of each written row
+ * Rows not named by any pair are left untouched. */
+EP_API ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                        ep_buffer_mode_t mode, int32_t max_tokens_per_expert, int64_t num_recv_rows,
+                        ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, float* recv_scales,
+                        int32_t* recv_src, float* recv_weights, ep_stream_t stream);
+
+/* Token-choice combine ([README] API Overview: combine / low_latency_combine,
+ * the weighted reduce; [EC] Solution 2: -1 slots are skipped).
+ *   out[t] = sum over k = 0..K-1 of topk_weights[t,k] * y[row(t,k)], over the
+ *   routed pairs only, accumulated in fp32 as acc = fmaf(w, y, acc) from 0
+ *   in ascending k; written as fp32 or rounded once (RNE) to bf16.  A token
+ *   with no routed pair gets +0.  row(t,k) is the dispatch row above; rows
+ *   >= num_y_rows are skipped with EP_DEVERR_OVERFLOW.
+ *   y   bf16 [num_y_rows, H], 16-byte aligned;  out [T, H] (out_dtype BF16 or FP32). */
+EP_API ep_status_t ep_combine(const void* y, int32_t hidden, int64_t num_y_rows, const ep_routing_desc_t* routing,
+                       const ep_layout_t* layout, ep_buffer_mode_t mode, int32_t max_tokens_per_expert,
+                       const float* topk_weights, void* out, ep_dtype_t out_dtype, ep_stream_t stream);
+
+/* Expert-choice dispatch ([EC] Solution 1, dispatch_expert_choice):
+ *   recv_x[e*C + c] = x[token_indices[e, c]] for every filled slot; rows of
+ *   empty slots are untouched.  x bf16 [T, H]; recv_x bf16 [E*C, H]; both
+ *   16-byte aligned, H % 8 == 0.  Needs only routing and layout->workspace. */
+EP_API ep_status_t ep_dispatch_expert_choice(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                      const ep_layout_t* layout, void* recv_x, ep_stream_t stream);
+
+/* Expert-choice combine ([EC] Solution 1, the combine of the new API pair):
+ *   out[t] = sum over the token's slots s in token_slots[token_offsets[t] ..
+ *   token_offsets[t+1]) (ascending s) of expert_weights[s] * y[s], as an fmaf
+ *   chain in fp32 from 0; unpicked tokens get +0.  y bf16 [E*C, H];
+ *   expert_weights fp32 [E, C]; out [T, H] (BF16 or FP32).  Uses the CSR
+ *   written by ep_get_layout for the same routing. */
+EP_API ep_status_t ep_combine_expert_choice(const void* y, int32_t hidden, const ep_routing_desc_t* routing,
+                                     const ep_layout_t* layout, const float* expert_weights, void* out,
+                                     ep_dtype_t out_dtype, ep_stream_t stream);
+
+/* Synchronise `stream`, read the device error word of layout->workspace into
+ * *flags (EP_DEVERR_* bits), clear it if `clear`, and return EP_OK when it is
+ * zero, else the status of the lowest set bit (BAD_INDEX, OVERFLOW, TIMEOUT).
+ * After EP_ERR_TIMEOUT re-run ep_workspace_init on the workspace. */
+EP_API ep_status_t ep_get_device_error(const ep_layout_t* layout, uint32_t* flags, int clear, ep_stream_t stream);
+
+EP_API const char* ep_status_string(ep_status_t status);
+EP_API int ep_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EP_B200_H_ */

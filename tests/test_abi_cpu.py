@@ -1,0 +1,126 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point include/ep.h declares, and rejects bad arguments on the host before it
+touches CUDA (no compute call runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from combine_ep_get_10_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from combine_ep_get_10_b200 import build
+
+    build.build()
+    return B.lib()
+
+
+def declared_entry_points():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"^EP_API\s+[\w\s\*]+?\b(ep_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = declared_entry_points()
+    for required in ("ep_get_layout", "ep_dispatch", "ep_combine", "ep_dispatch_expert_choice",
+                     "ep_combine_expert_choice"):
+        assert required in names
+    assert set(B.EXPORTED) <= set(names)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_entry_points():
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings(L):
+    assert B.ep_version() == 1
+    for s in range(8):
+        assert B.ep_status_string(s)
+    assert B.ep_status_string(99) == "unknown status"
+
+
+def _topk_desc(T=16, K=2, E=8, R=2, ptr=0x1000):
+    return B.RoutingDesc(B.EP_ROUTING_TOPK, ptr, None, T, K, 0, E, R)
+
+
+def _ec_desc(T=16, E=8, C=4, R=2, ptr=0x1000):
+    return B.RoutingDesc(B.EP_ROUTING_EXPERT_CHOICE, None, ptr, T, 0, C, E, R)
+
+
+def test_workspace_bytes(L):
+    assert L.ep_workspace_bytes(ctypes.byref(_topk_desc())) == 256
+    n = L.ep_workspace_bytes(ctypes.byref(_ec_desc(T=1000, E=128, C=128)))
+    assert n >= 256 + 4 * (2 * 1000 + 128 * 128) and n % 256 == 0
+    assert L.ep_workspace_bytes(ctypes.byref(_topk_desc(E=9, R=2))) == 0  # E % R != 0
+    assert L.ep_workspace_bytes(None) == 0
+
+
+@pytest.mark.parametrize("desc", [
+    _topk_desc(E=9, R=2), _topk_desc(R=0), _topk_desc(R=33, E=66), _topk_desc(K=0), _topk_desc(T=-1),
+    _topk_desc(ptr=0), _topk_desc(ptr=0x1004), _topk_desc(T=1 << 28, K=8), _ec_desc(C=0), _ec_desc(ptr=0),
+    _ec_desc(E=1 << 16, C=1 << 16, R=1), B.RoutingDesc(7, 0x1000, 0x1000, 4, 2, 2, 4, 1)])
+def test_layout_rejects_bad_routing(L, desc):
+    lay = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x100000, 1 << 20)
+    assert L.ep_get_layout(ctypes.byref(desc), ctypes.byref(lay), None) == 1
+
+
+def test_layout_rejects_bad_workspace(L):
+    d = _topk_desc()
+    for ws, n in [(0, 1 << 20), (0x100010, 1 << 20), (0x100000, 255)]:
+        lay = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, ws, n)
+        assert L.ep_get_layout(ctypes.byref(d), ctypes.byref(lay), None) == 4
+    ec = _ec_desc(T=100, E=8, C=4)
+    lay = B.LayoutDesc(0x1000, None, 0x1000, 0x1000, None, 0x1000, 0x1000, 0x100000, 512)
+    assert L.ep_get_layout(ctypes.byref(ec), ctypes.byref(lay), None) == 4
+
+
+def test_layout_unsupported_expert_count(L):
+    d = _topk_desc(E=2048, R=1)
+    lay = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x100000, 1 << 20)
+    assert L.ep_get_layout(ctypes.byref(d), ctypes.byref(lay), None) == 6
+
+
+def test_dispatch_and_combine_reject_bad_args(L):
+    d = _topk_desc()
+    lay = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x100000, 256)
+    ok = dict(x=0x2000, hidden=256, mode=0, mt=0, rows=32, dt=B.EP_BF16, w=0x3000, recv=0x4000, sc=None)
+
+    def disp(**kw):
+        a = dict(ok, **kw)
+        return L.ep_dispatch(a["x"], a["hidden"], ctypes.byref(d), ctypes.byref(lay), a["mode"], a["mt"], a["rows"],
+                             a["dt"], a["w"], a["recv"], a["sc"], None, None, None)
+
+    assert disp(hidden=12) == 1  # not a multiple of 8
+    assert disp(x=0x2008) == 1  # x not 16-byte aligned
+    assert disp(recv=0x4004) == 1
+    assert disp(mode=5) == 1
+    assert disp(mode=1, mt=0) == 1  # padded needs max_tokens >= 1
+    assert disp(dt=B.EP_FP32) == 1  # dispatch writes bf16 or fp8
+    assert disp(dt=B.EP_FP8_E4M3, hidden=136) == 1  # fp8 needs H % 128 == 0
+    assert disp(dt=B.EP_FP8_E4M3, sc=None) == 1  # fp8 needs scales
+    assert disp(rows=-1) == 1
+    assert L.ep_combine(0x2000, 256, 32, ctypes.byref(d), ctypes.byref(lay), 0, 0, None, 0x5000, B.EP_BF16,
+                        None) == 1  # weights missing
+    assert L.ep_combine(0x2000, 256, 32, ctypes.byref(d), ctypes.byref(lay), 0, 0, 0x3000, 0x5000, B.EP_FP8_E4M3,
+                        None) == 1  # combine writes bf16 or fp32
+    ec = _ec_desc()
+    assert L.ep_dispatch(0x2000, 256, ctypes.byref(ec), ctypes.byref(lay), 0, 0, 32, 0, None, 0x4000, None, None,
+                         None, None) == 1  # token-choice call with expert-choice routing
+    assert L.ep_dispatch_expert_choice(0x2000, 256, ctypes.byref(d), ctypes.byref(lay), 0x4000, None) == 1
+    assert L.ep_combine_expert_choice(0x2000, 256, ctypes.byref(ec), ctypes.byref(lay), None, 0x5000, 0, None) == 1
+
+
+def test_device_error_rejects_missing_workspace(L):
+    lay = B.LayoutDesc(None, None, None, None, None, None, None, None, 0)
+    flags = ctypes.c_uint32(0)
+    assert L.ep_get_device_error(ctypes.byref(lay), ctypes.byref(flags), 1, None) == 4
