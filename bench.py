@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--workload", type=int, default=2, choices=[2, 5])
     ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--print-digests", action="store_true", help="print kernel source digests and exit")
     return ap.parse_args()
 
 
@@ -69,12 +70,19 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_digest():
+KERNEL_SOURCES = {"layout": "ep_layout.cu", "dispatch": "ep_dispatch.cu", "combine": "ep_combine.cu"}
+
+
+def source_digest(kernel):
+    """Digest of the sources a kernel is compiled from (its .cu file and the
+    shared headers): a recorded ncu traffic figure is valid only for it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "combine_ep_get_10_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted([KERNEL_SOURCES[kernel], "ep_device.cuh", "ep_internal.h"]):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
+    with open(os.path.join(ROOT, "include", "ep.h"), "rb") as f:
+        h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -84,7 +92,7 @@ def recorded_traffic(kernel):
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
-    want = source_digest()
+    want = source_digest(kernel)
     for line in open(path):
         fields = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
         if fields.get("kernel") == kernel and fields.get("source_sha") == want:
@@ -160,6 +168,26 @@ def dist_setup(n_gpus):
     if world != n_gpus:
         raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (n_gpus, world))
     return world, rank, local
+
+
+def rank_seed(workload, rank):
+    """Seed of rank `rank`'s token batch: the workload seed for rank 0, then
+    one independent stream per rank (replicas on disjoint data)."""
+    from combine_ep_get_10_b200 import workloads as W
+
+    return W.CONFIGS[workload]["seed"] + 1000 * rank
+
+
+def max_over_ranks(value, world, device=None):
+    """Max of a float over all ranks (all ranks must call it)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def cpu_oracle_run(cfg_id, seed, n_tokens, reps_budget_s, min_reps=1):
@@ -252,7 +280,7 @@ def run_ours(args):
         dist.barrier()
     B.lib()
 
-    seed = W.CONFIGS[args.workload]["seed"] + 1000 * rank
+    seed = rank_seed(args.workload, rank)
     inp = W.make_inputs(args.workload, seed=seed)
     cfg = inp["cfg"]
     T, H, K, E, R = cfg["T"], cfg["H"], cfg["K"], cfg["E"], cfg["R"]
@@ -311,11 +339,7 @@ def run_ours(args):
     t_disp = [a[1].elapsed_time(a[2]) for a in ev]
     t_comb = [a[2].elapsed_time(a[3]) for a in ev]
     t_step = [a[0].elapsed_time(a[3]) for a in ev]
-    total_ms = float(sum(t_step))
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(float(sum(t_step)), world, dev)
     if B.ep_get_device_error(lay) != 0:
         raise RuntimeError("device error flagged during the timed steps")
 
@@ -339,11 +363,8 @@ def run_ours(args):
         out_h.copy_(out, non_blocking=True)
         ee[i][1].record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = float(sum(a.elapsed_time(b) for a, b in ee))
+    e2e_ms = max_over_ranks(float(sum(a.elapsed_time(b) for a, b in ee)), world, dev)
     if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
         dist.barrier()
 
     if rank == 0:
@@ -392,6 +413,9 @@ def run_ours(args):
 
 def main():
     args = parse()
+    if args.print_digests:
+        print(json.dumps({k: source_digest(k) for k in KERNEL_SOURCES}))
+        return 0
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

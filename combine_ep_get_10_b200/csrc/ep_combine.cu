@@ -19,10 +19,20 @@ namespace ep {
 
 namespace {
 
-constexpr int kCombineThreads = 256;
+#ifndef EP_COMBINE_VEC
+#define EP_COMBINE_VEC 2
+#endif
+#ifndef EP_COMBINE_GROUP
+#define EP_COMBINE_GROUP 8
+#endif
+#ifndef EP_COMBINE_THREADS
+#define EP_COMBINE_THREADS 256
+#endif
+
+constexpr int kCombineThreads = EP_COMBINE_THREADS;
 constexpr int kWarpsPerCta = kCombineThreads / 32;
-constexpr int kVecPerLane = 2;
-constexpr int kGroup = 8;
+constexpr int kVecPerLane = EP_COMBINE_VEC; // 16-byte vectors per lane per segment
+constexpr int kGroup = EP_COMBINE_GROUP;    // entries whose loads are issued together
 constexpr int kSegVec = 32 * kVecPerLane;
 
 struct CombineArgs {

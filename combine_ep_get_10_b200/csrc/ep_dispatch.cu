@@ -24,7 +24,11 @@ namespace ep {
 
 namespace {
 
-constexpr int64_t kChunkTarget = 8192; // bytes per bulk-copy item
+#ifndef EP_DISPATCH_CHUNK
+#define EP_DISPATCH_CHUNK 8192
+#endif
+
+constexpr int64_t kChunkTarget = EP_DISPATCH_CHUNK; // bytes per bulk-copy item
 
 struct RowMap {
     const int64_t* topk_idx;

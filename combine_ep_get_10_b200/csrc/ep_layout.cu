@@ -17,6 +17,8 @@
 // global atomics (order-free integer sums), one-CTA scan, an unordered fill,
 // then each token's slot list is put in ascending order by a warp that ranks
 // every entry against the others (slot ids are distinct).
+#include <algorithm>
+
 #include <cooperative_groups.h>
 
 #include "ep_device.cuh"
@@ -32,6 +34,7 @@ constexpr int kLayoutThreads = 1024;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
 constexpr int kPrefetch = 8; // 32-pair steps a warp loads before ranking them
 constexpr int64_t kPairsPerCta = 2048;
+constexpr int kMaxCluster = 16;
 
 struct TcArgs {
     const int64_t* topk_idx;
@@ -106,50 +109,68 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(Tc
     const uint32_t lanes_below = (1u << lane) - 1u;
     bool bad = false;
 
-    // phase 1: per-warp stable ranks (stored in slot[] for now) and counters
+    // phase 1: per-warp stable ranks and counters.  When the warp's run fits
+    // one prefetch batch (<= 256 pairs) the ids and ranks stay in registers;
+    // longer runs park the rank in slot[] and re-read it in phase 3.
+    const bool in_regs = (we - wb) <= 32 * kPrefetch;
+    int ev[kPrefetch]; // expert id, or -1 for a pair that is not routed
+    int loc[kPrefetch];
     for (int64_t base = wb; base < we; base += 32 * kPrefetch) {
-        int64_t ev[kPrefetch];
+        int64_t raw[kPrefetch];
 #pragma unroll
         for (int j = 0; j < kPrefetch; ++j) {
             const int64_t p = base + j * 32 + lane;
-            ev[j] = p < we ? __ldg(a.topk_idx + p) : -1;
+            raw[j] = p < we ? __ldg(a.topk_idx + p) : -1;
         }
 #pragma unroll
         for (int j = 0; j < kPrefetch; ++j) {
+            const bool ok = raw[j] >= 0 && raw[j] < a.E;
+            bad |= !ok && raw[j] != -1;
+            ev[j] = ok ? static_cast<int>(raw[j]) : -1;
+        }
+#pragma unroll
+        for (int j = 0; j < kPrefetch; ++j) {
+            loc[j] = -1;
             const int64_t step = base + j * 32;
             if (step >= we)
                 break; // warp-uniform
             const int64_t p = step + lane;
             const bool in = p < we;
-            const int64_t e = ev[j];
-            const bool good = in && e >= 0 && e < a.E;
-            bad |= in && !good && e != -1;
-            const uint32_t peers = __match_any_sync(kFullMask, good ? static_cast<int>(e) : -1);
+            const int e = ev[j];
+            const bool good = e >= 0;
+            const uint32_t peers = __match_any_sync(kFullMask, e);
             int prior = 0;
             if (good)
                 prior = mine[e];
             __syncwarp();
             if (good) {
                 const int r = __popc(peers & lanes_below);
-                a.slot[p] = prior + r;
+                loc[j] = prior + r;
                 if (r == 0)
                     mine[e] = prior + __popc(peers);
-            } else if (in) {
-                a.slot[p] = -1;
             }
+            if (!in_regs && in)
+                a.slot[p] = loc[j];
             __syncwarp();
         }
     }
 
-    // phase 1b: rank membership of this CTA's tokens
+    // phase 1b: rank membership of this CTA's tokens (ids re-read from L1/L2,
+    // all of a token's loads issued before any is used)
+    constexpr int kMaskBatch = 8;
     for (int64_t tb = t0 + static_cast<int64_t>(warp) * 32; tb < t1; tb += kLayoutThreads) {
         const int64_t t = tb + lane;
         uint32_t mask = 0;
         if (t < t1) {
-            for (int k = 0; k < a.K; ++k) {
-                const int64_t e = __ldg(a.topk_idx + t * a.K + k);
-                if (e >= 0 && e < a.E)
-                    mask |= 1u << static_cast<uint32_t>(e / a.per_rank);
+            for (int k0 = 0; k0 < a.K; k0 += kMaskBatch) {
+                int64_t ids[kMaskBatch];
+#pragma unroll
+                for (int k = 0; k < kMaskBatch; ++k)
+                    ids[k] = k0 + k < a.K ? __ldg(a.topk_idx + t * a.K + k0 + k) : -1;
+#pragma unroll
+                for (int k = 0; k < kMaskBatch; ++k)
+                    if (ids[k] >= 0 && ids[k] < a.E)
+                        mask |= 1u << static_cast<uint32_t>(ids[k] / a.per_rank);
             }
             uint8_t* row = a.in_rank + t * a.R;
             if (a.in_rank_words) {
@@ -186,18 +207,28 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(Tc
     }
     cluster.sync();
 
+    // totals of every CTA of the cluster, all loads in flight together
     int base = 0, all = 0;
     if (e < a.E) {
-        for (int j = 0; j < cs; ++j) {
-            const int v = cluster.map_shared_rank(tot, j)[e];
-            base += j < b ? v : 0;
-            all += v;
+        int v[kMaxCluster];
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j)
+            v[j] = j < cs ? cluster.map_shared_rank(tot, j)[e] : 0;
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j) {
+            base += j < b ? v[j] : 0;
+            all += v[j];
         }
     }
     int rank_total = 0;
     if (b == 0 && tid < a.R) {
-        for (int j = 0; j < cs; ++j)
-            rank_total += cluster.map_shared_rank(srank, j)[tid];
+        int v[kMaxCluster];
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j)
+            v[j] = j < cs ? cluster.map_shared_rank(srank, j)[tid] : 0;
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j)
+            rank_total += v[j];
     }
     cluster.sync(); // no CTA leaves or reuses its shared memory while others read it
 
@@ -219,14 +250,23 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(Tc
     }
     __syncthreads();
 
-    // phase 3: add the base of (earlier CTAs + earlier warps); same lane
-    // owns the same pair as in phase 1
-    for (int64_t step = wb; step < we; step += 32) {
-        const int64_t p = step + lane;
-        if (p < we) {
-            const int64_t ex = __ldg(a.topk_idx + p);
-            if (ex >= 0 && ex < a.E)
-                a.slot[p] += mine[ex];
+    // phase 3: slot = rank inside the warp's run + (earlier warps + earlier
+    // CTAs); the same lane owns the same pair as in phase 1
+    if (in_regs) {
+#pragma unroll
+        for (int j = 0; j < kPrefetch; ++j) {
+            const int64_t p = wb + j * 32 + lane;
+            if (p < we)
+                a.slot[p] = loc[j] >= 0 ? loc[j] + mine[ev[j]] : -1;
+        }
+    } else {
+        for (int64_t step = wb; step < we; step += 32) {
+            const int64_t p = step + lane;
+            if (p < we) {
+                const int32_t l = a.slot[p];
+                if (l >= 0)
+                    a.slot[p] = l + mine[__ldg(a.topk_idx + p)];
+            }
         }
     }
 }
@@ -369,6 +409,30 @@ __global__ void __launch_bounds__(kEcThreads) ec_sort_kernel(EcArgs a)
 }
 
 int cluster_limit_cache[64];
+size_t smem_attr_cache[64];
+
+// Kernel attributes (dynamic shared memory limit, 16-CTA clusters) are set
+// once per device and shared-memory size; later calls skip the driver calls.
+cudaError_t prepare_layout_kernel(size_t smem)
+{
+    int dev = 0;
+    cudaError_t st = cudaGetDevice(&dev);
+    if (st != cudaSuccess)
+        return st;
+    if (dev >= 0 && dev < 64 && smem_attr_cache[dev] >= smem)
+        return cudaSuccess;
+    const size_t want = std::max<size_t>(smem, sizeof(int32_t) * (kLayoutWarps * 256 + 256 + 64));
+    st = cudaFuncSetAttribute(tc_layout_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(want));
+    if (st != cudaSuccess)
+        return st;
+    st = cudaFuncSetAttribute(tc_layout_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (st != cudaSuccess)
+        return st;
+    if (dev >= 0 && dev < 64)
+        smem_attr_cache[dev] = want;
+    return cudaSuccess;
+}
 
 int max_layout_cluster(size_t smem_bytes)
 {
@@ -418,11 +482,7 @@ cudaError_t launch_tc_layout(const TcLayoutLaunch& a, cudaStream_t stream)
     k.in_rank_words = (a.R % 4 == 0 && (reinterpret_cast<uintptr_t>(a.in_rank) & 3u) == 0) ? 1 : 0;
 
     const size_t smem = sizeof(int32_t) * (static_cast<size_t>(kLayoutWarps) * a.E + a.E + 64);
-    cudaError_t st = cudaFuncSetAttribute(tc_layout_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(smem));
-    if (st != cudaSuccess)
-        return st;
-    st = cudaFuncSetAttribute(tc_layout_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaError_t st = prepare_layout_kernel(smem);
     if (st != cudaSuccess)
         return st;
     const int64_t pairs = static_cast<int64_t>(a.T) * a.K;
