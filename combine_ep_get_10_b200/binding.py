@@ -26,7 +26,7 @@ EP_DEVERR_BAD_INDEX, EP_DEVERR_OVERFLOW, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 EXPORTED = ("ep_workspace_bytes", "ep_workspace_init", "ep_get_layout", "ep_dispatch", "ep_combine",
             "ep_dispatch_expert_choice", "ep_combine_expert_choice", "ep_get_device_error", "ep_status_string",
-            "ep_version")
+            "ep_version", "ep_get_layout_no_alloc")
 
 
 class EPError(RuntimeError):
@@ -82,6 +82,8 @@ def lib():
         L.ep_status_string.argtypes = [st]
         L.ep_version.restype = ctypes.c_int
         L.ep_version.argtypes = []
+        L.ep_get_layout_no_alloc.restype = st
+        L.ep_get_layout_no_alloc.argtypes = [RP, LP, P, P]
         _lib = L
     return _lib
 
@@ -248,6 +250,17 @@ def ep_get_device_error(layout: Layout, clear: bool = True, stream=None) -> int:
 
 def ep_status_string(status: int) -> str:
     return lib().ep_status_string(status).decode()
+
+
+def ep_get_layout_no_alloc(routing: Routing, layout: Layout, device_error_flags: torch.Tensor | None = None,
+                           stream=None) -> Layout:
+    """The layout without a caller workspace (for callers that cannot
+    allocate): layout.workspace is ignored; the library's fixed scratch
+    array is used.  device_error_flags: optional one-element int32/uint32
+    device tensor that receives the EP_DEVERR_* bits of this call."""
+    _check(lib().ep_get_layout_no_alloc(ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                                        _ptr(device_error_flags), _stream(stream)), "ep_get_layout_no_alloc")
+    return layout
 
 
 def ep_version() -> int:

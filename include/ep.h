@@ -193,6 +193,35 @@ EP_API ep_status_t ep_combine_expert_choice(const void* y, int32_t hidden, const
                                      const ep_layout_t* layout, const float* expert_weights, void* out,
                                      ep_dtype_t out_dtype, ep_stream_t stream);
 
+/* ep_get_layout for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this is a deployment variant of the layout call.
+ *
+ * Who needs it: code that must not call cudaMalloc (or any allocator) when
+ * it builds a layout -- a host capturing the MoE step into a CUDA graph
+ * (allocation is not allowed during stream capture), a plugin inside an
+ * inference server or framework that is handed only its input and output
+ * tensors, or a decode loop where an allocation could synchronise the device.
+ *
+ * It computes exactly what ep_get_layout computes, writing the same outputs
+ * in `layout`, but ignores layout->workspace / workspace_bytes: its scratch is
+ * a fixed array of EP_STATIC_WORKSPACE_BYTES inside the library, held by
+ * every GPU that loads the library until the process exits.  A routing whose
+ * ep_workspace_bytes() exceeds that size is rejected with EP_ERR_WORKSPACE
+ * before anything is launched (token choice needs 256 bytes and always fits;
+ * expert choice needs 256 + 4*(2*T + E*C) bytes rounded up to 256).  Nothing
+ * is allocated or freed.
+ *   device_error_flags  optional device pointer to one uint32: zeroed at the
+ *                       start of the call, then receives the EP_DEVERR_* bits
+ *                       the layout kernels raise (NULL: not reported).
+ * The first call on a device looks up the array's device address (with that
+ * device current), so make one call per device before any stream capture.
+ * All calls share the array and it keeps the last call's contents: calls that
+ * overlap on the GPU (other streams, other host threads) race on it and must
+ * be serialised by the caller. */
+#define EP_STATIC_WORKSPACE_BYTES ((size_t)4 << 20)
+EP_API ep_status_t ep_get_layout_no_alloc(const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                                          uint32_t* device_error_flags, ep_stream_t stream);
+
 /* Synchronise `stream`, read the device error word of layout->workspace into
  * *flags (EP_DEVERR_* bits), clear it if `clear`, and return EP_OK when it is
  * zero, else the status of the lowest set bit (BAD_INDEX, OVERFLOW, TIMEOUT).
