@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-digests", action="store_true", help="print kernel source digests and exit")
+    ap.add_argument("--workloads", action="store_true",
+                    help="time every op on all five workloads (one JSON line each) instead of the step")
+    ap.add_argument("--only", type=int, default=0, choices=[0, 1, 2, 3, 4, 5],
+                    help="with --workloads: just this workload")
     return ap.parse_args()
 
 
@@ -411,8 +415,106 @@ def run_ours(args):
     return 0
 
 
+def run_workload_table(args):
+    """Per-op timings on every workload (layout, dispatch, combine; expert
+    choice for workload 4): one JSON line per (workload, op), L2 flushed
+    before every repetition, median of --steps repetitions."""
+    import torch
+
+    from combine_ep_get_10_b200 import binding as B
+    from combine_ep_get_10_b200 import workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    peak, peak_kind = measured_peak()
+    reps = max(10, min(args.steps, 200))
+
+    def timeit(fn):
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b) * 1e3)
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    def emit(cfg, op, us, nbytes, tokens):
+        print(json.dumps({"workload": cfg["name"], "op": op, "us": round(us, 2), "bytes": int(nbytes),
+                          "gbs": round(nbytes / us / 1e3, 1), "frac_of_peak": round(nbytes / us / 1e3 / peak, 3),
+                          "peak_gbs": peak, "peak_source": peak_kind, "tokens_per_s": round(tokens / us * 1e6),
+                          "reps": reps, "l2": "flushed"}), flush=True)
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    for wl in ([args.only] if args.only else (1, 2, 3, 4, 5)):
+        inp = W.make_inputs(wl)
+        cfg = inp["cfg"]
+        T, H, E, R = cfg["T"], cfg["H"], cfg["E"], cfg["R"]
+        x = bf(inp["x"])
+        if cfg["routing"] == "topk":
+            K = cfg["K"]
+            idx_np = inp["topk_idx"]
+            n_valid = int((idx_np >= 0).sum())
+            idx = torch.from_numpy(idx_np).to(dev)
+            w = torch.from_numpy(inp["topk_weights"]).to(dev)
+            rt = B.Routing.topk(idx, E, R)
+            lay = B.Layout(rt, device=dev)
+            emit(cfg, "layout", timeit(lambda: B.ep_get_layout(rt, lay)),
+                 T * K * 12 + T * R + E * 8 + R * 4, T)
+            mode, mt = cfg["mode"], cfg["max_tokens"]
+            rows = E * mt if mode == W.PADDED else T * K
+            meta = T * K * 12 + E * 4
+            if cfg["dispatch_dtype"] == W.FP8_E4M3:
+                recv = torch.empty((rows, H), dtype=torch.uint8, device=dev)
+                sc = torch.empty((rows, H // 128), dtype=torch.float32, device=dev)
+                emit(cfg, "dispatch_fp8", timeit(lambda: B.ep_dispatch(x, rt, lay, recv, mode=mode,
+                                                                       max_tokens_per_expert=mt, recv_scales=sc)),
+                     T * H * 2 + n_valid * (H + H // 128 * 4) + meta, T)
+                y = torch.zeros((rows, H), dtype=torch.bfloat16, device=dev)
+            else:
+                recv = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)
+                emit(cfg, "dispatch", timeit(lambda: B.ep_dispatch(x, rt, lay, recv, mode=mode,
+                                                                   max_tokens_per_expert=mt)),
+                     T * H * 2 + n_valid * H * 2 + meta, T)
+                y = recv
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+            emit(cfg, "combine", timeit(lambda: B.ep_combine(y, rt, lay, w, out, mode=mode,
+                                                             max_tokens_per_expert=mt)),
+                 n_valid * H * 2 + T * H * 2 + T * K * 16 + E * 4, T)
+        else:
+            C = cfg["C"]
+            ti_np = inp["token_indices"]
+            S = E * C
+            uniq = len(np.unique(ti_np[ti_np >= 0]))
+            ti = torch.from_numpy(ti_np).to(dev)
+            ew = torch.from_numpy(inp["expert_weights"]).to(dev)
+            rt = B.Routing.expert_choice(ti, T, R)
+            lay = B.Layout(rt, device=dev)
+            emit(cfg, "ec_layout", timeit(lambda: B.ep_get_layout(rt, lay)),
+                 S * 4 + (T + 1) * 4 + S * 4 + T * R + E * 4 + R * 4, T)
+            recv = torch.empty((S, H), dtype=torch.bfloat16, device=dev)
+            emit(cfg, "ec_dispatch", timeit(lambda: B.ep_dispatch_expert_choice(x, rt, lay, recv)),
+                 uniq * H * 2 + S * H * 2 + S * 4, T)
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+            emit(cfg, "ec_combine", timeit(lambda: B.ep_combine_expert_choice(recv, rt, lay, ew, out)),
+                 S * H * 2 + T * H * 2 + S * 8 + (T + 1) * 4, T)
+        if B.ep_get_device_error(lay) != 0:
+            raise RuntimeError("device error flagged on workload %d" % wl)
+    return 0
+
+
 def main():
     args = parse()
+    if args.workloads:
+        return run_workload_table(args)
     if args.print_digests:
         print(json.dumps({k: source_digest(k) for k in KERNEL_SOURCES}))
         return 0

@@ -7,11 +7,16 @@
 // (issue #595, Solution 2).
 //
 // One warp per (token, hidden segment).  A segment is kVecPerLane 16-byte
-// vectors per lane (8 bf16 each); the warp fetches the token's entries (row,
-// weight) once, 32 at a time, broadcasts them by shuffles and, for groups of
-// kGroup entries, issues every 16-byte load of the group before any FMA so
-// that kGroup * kVecPerLane loads per lane are in flight.  Each accumulator
-// sees its entries in ascending order: acc = fmaf(w, y, acc) from 0 in fp32.
+// vectors per lane (8 bf16 each; 4 vectors = 2 KB of a row per warp); the
+// warp fetches the token's entries (row, weight) once, 32 at a time,
+// broadcasts them by shuffles and, for groups of kGroup entries, issues every
+// 16-byte load of the group before any FMA so that kGroup * kVecPerLane loads
+// per lane are in flight.  Each accumulator sees its entries in ascending
+// order: acc = fmaf(w, y, acc) from 0 in fp32.  (A TMA-pipelined variant --
+// a producer warp streaming row chunks into a shared-memory ring -- measured
+// no faster at 4096 tokens and slower under expert-choice skew.)
+#include <algorithm>
+
 #include "ep_device.cuh"
 #include "ep_internal.h"
 
@@ -20,10 +25,10 @@ namespace ep {
 namespace {
 
 #ifndef EP_COMBINE_VEC
-#define EP_COMBINE_VEC 2
+#define EP_COMBINE_VEC 4
 #endif
 #ifndef EP_COMBINE_GROUP
-#define EP_COMBINE_GROUP 8
+#define EP_COMBINE_GROUP 4
 #endif
 #ifndef EP_COMBINE_THREADS
 #define EP_COMBINE_THREADS 256
@@ -31,9 +36,27 @@ namespace {
 
 constexpr int kCombineThreads = EP_COMBINE_THREADS;
 constexpr int kWarpsPerCta = kCombineThreads / 32;
-constexpr int kVecPerLane = EP_COMBINE_VEC; // 16-byte vectors per lane per segment
-constexpr int kGroup = EP_COMBINE_GROUP;    // entries whose loads are issued together
-constexpr int kSegVec = 32 * kVecPerLane;
+// token choice: kTcVec 16-byte vectors per lane per segment, kTcGroup
+// entries whose loads are issued together (K is small and uniform)
+constexpr int kTcVec = EP_COMBINE_VEC;
+constexpr int kTcGroup = EP_COMBINE_GROUP;
+// expert choice: most tokens have few or no picks and a few have long lists
+#ifndef EP_COMBINE_EC_VEC
+#define EP_COMBINE_EC_VEC 2
+#endif
+#ifndef EP_COMBINE_EC_GROUP
+#define EP_COMBINE_EC_GROUP 8
+#endif
+// token choice: uniform items, so one resident wave of persistent warps;
+// expert choice: item cost varies by 100x, so blocks are scheduled dynamically
+#ifndef EP_COMBINE_PERSIST_TC
+#define EP_COMBINE_PERSIST_TC 1
+#endif
+#ifndef EP_COMBINE_PERSIST_EC
+#define EP_COMBINE_PERSIST_EC 0
+#endif
+constexpr int kEcVec = EP_COMBINE_EC_VEC;
+constexpr int kEcGroup = EP_COMBINE_EC_GROUP;
 
 struct CombineArgs {
     const uint8_t* y;
@@ -95,120 +118,167 @@ __device__ __forceinline__ void entry(const CombineArgs& a, int64_t t, int64_t b
     }
 }
 
-template <bool kExpertChoice, bool kOutF32>
+template <bool kExpertChoice, bool kOutF32, int kVecPerLane, int kGroup>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 {
+    constexpr int kSegVec = 32 * kVecPerLane;
+    // token choice lists are short (K); expert-choice lists reach E entries
+    constexpr int kLookup = kExpertChoice ? 4 : 1;
     const int lane = threadIdx.x & 31;
-    const int64_t gw = a.warp_base + static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
-    const int64_t t = gw / a.nseg;
-    const int seg = static_cast<int>(gw - t * a.nseg);
-    if (t >= a.T)
-        return;
-
-    int64_t beg = 0;
-    int n;
-    if (kExpertChoice) {
-        beg = __ldg(a.token_offsets + t);
-        n = __ldg(a.token_offsets + t + 1) - static_cast<int>(beg);
-    } else {
-        n = a.K;
-    }
-
-    int v[kVecPerLane];
-    bool vin[kVecPerLane];
-#pragma unroll
-    for (int j = 0; j < kVecPerLane; ++j) {
-        v[j] = seg * kSegVec + j * 32 + lane;
-        vin[j] = v[j] < a.nvec;
-    }
-    float acc[kVecPerLane][8];
-#pragma unroll
-    for (int j = 0; j < kVecPerLane; ++j)
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            acc[j][i] = 0.0f;
-
+    const int64_t items = static_cast<int64_t>(a.T) * a.nseg;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarpsPerCta;
     uint32_t errbits = 0;
-    const int64_t row_bytes = static_cast<int64_t>(a.H) * 2;
-    for (int k0 = 0; k0 < n; k0 += 32) {
-        int64_t my_row = -1;
-        float my_w = 0.0f;
-        if (k0 + lane < n)
-            entry<kExpertChoice>(a, t, beg, k0 + lane, my_row, my_w, errbits);
-        const int m = min(32, n - k0);
-        for (int g0 = 0; g0 < m; g0 += kGroup) {
-            int64_t rows[kGroup];
-            float ws[kGroup];
+    for (int64_t gw = a.warp_base + static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
+         gw < items; gw += stride) {
+        const int64_t t = gw / a.nseg;
+        const int seg = static_cast<int>(gw - t * a.nseg);
+
+        int64_t beg = 0;
+        int n;
+        if (kExpertChoice) {
+            beg = __ldg(a.token_offsets + t);
+            n = __ldg(a.token_offsets + t + 1) - static_cast<int>(beg);
+        } else {
+            n = a.K;
+        }
+
+        int v[kVecPerLane];
+        bool vin[kVecPerLane];
 #pragma unroll
-            for (int g = 0; g < kGroup; ++g) {
-                const int src = (g0 + g) & 31;
-                rows[g] = __shfl_sync(kFullMask, my_row, src);
-                ws[g] = __shfl_sync(kFullMask, my_w, src);
-                if (g0 + g >= m)
-                    rows[g] = -1;
+        for (int j = 0; j < kVecPerLane; ++j) {
+            v[j] = seg * kSegVec + j * 32 + lane;
+            vin[j] = v[j] < a.nvec;
+        }
+        float acc[kVecPerLane][8];
+#pragma unroll
+        for (int j = 0; j < kVecPerLane; ++j)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                acc[j][i] = 0.0f;
+
+        const int64_t row_bytes = static_cast<int64_t>(a.H) * 2;
+        // entries are looked up kLookup at a time (all of their loads in flight),
+        // then folded kGroup at a time in ascending order
+        for (int k0 = 0; k0 < n; k0 += 32 * kLookup) {
+            int64_t my_row[kLookup];
+            float my_w[kLookup];
+#pragma unroll
+            for (int i = 0; i < kLookup; ++i) {
+                my_row[i] = -1;
+                my_w[i] = 0.0f;
+                const int j = k0 + 32 * i + lane;
+                if (j < n)
+                    entry<kExpertChoice>(a, t, beg, j, my_row[i], my_w[i], errbits);
             }
-            uint4 d[kGroup][kVecPerLane];
 #pragma unroll
-            for (int g = 0; g < kGroup; ++g)
+            for (int i = 0; i < kLookup; ++i) {
+                const int kb = k0 + 32 * i;
+                if (kb >= n)
+                    break; // warp-uniform
+                const int m = min(32, n - kb);
+                for (int g0 = 0; g0 < m; g0 += kGroup) {
+                    int64_t rows[kGroup];
+                    float ws[kGroup];
 #pragma unroll
-                for (int j = 0; j < kVecPerLane; ++j)
-                    d[g][j] = (rows[g] >= 0 && vin[j]) ? ld_nc_v4(a.y + rows[g] * row_bytes + static_cast<int64_t>(v[j]) * 16)
-                                                        : make_uint4(0, 0, 0, 0);
+                    for (int g = 0; g < kGroup; ++g) {
+                        const int src = (g0 + g) & 31;
+                        rows[g] = __shfl_sync(kFullMask, my_row[i], src);
+                        ws[g] = __shfl_sync(kFullMask, my_w[i], src);
+                        if (g0 + g >= m)
+                            rows[g] = -1;
+                    }
+                    uint4 d[kGroup][kVecPerLane];
 #pragma unroll
-            for (int g = 0; g < kGroup; ++g) {
-                if (rows[g] < 0)
-                    continue;
+                    for (int g = 0; g < kGroup; ++g)
 #pragma unroll
-                for (int j = 0; j < kVecPerLane; ++j) {
-                    acc[j][0] = fmaf(ws[g], bf16_lo(d[g][j].x), acc[j][0]);
-                    acc[j][1] = fmaf(ws[g], bf16_hi(d[g][j].x), acc[j][1]);
-                    acc[j][2] = fmaf(ws[g], bf16_lo(d[g][j].y), acc[j][2]);
-                    acc[j][3] = fmaf(ws[g], bf16_hi(d[g][j].y), acc[j][3]);
-                    acc[j][4] = fmaf(ws[g], bf16_lo(d[g][j].z), acc[j][4]);
-                    acc[j][5] = fmaf(ws[g], bf16_hi(d[g][j].z), acc[j][5]);
-                    acc[j][6] = fmaf(ws[g], bf16_lo(d[g][j].w), acc[j][6]);
-                    acc[j][7] = fmaf(ws[g], bf16_hi(d[g][j].w), acc[j][7]);
+                        for (int j = 0; j < kVecPerLane; ++j)
+                            d[g][j] = (rows[g] >= 0 && vin[j])
+                                          ? ld_nc_v4(a.y + rows[g] * row_bytes + static_cast<int64_t>(v[j]) * 16)
+                                          : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int g = 0; g < kGroup; ++g) {
+                        if (rows[g] < 0)
+                            continue;
+#pragma unroll
+                        for (int j = 0; j < kVecPerLane; ++j) {
+                            acc[j][0] = fmaf(ws[g], bf16_lo(d[g][j].x), acc[j][0]);
+                            acc[j][1] = fmaf(ws[g], bf16_hi(d[g][j].x), acc[j][1]);
+                            acc[j][2] = fmaf(ws[g], bf16_lo(d[g][j].y), acc[j][2]);
+                            acc[j][3] = fmaf(ws[g], bf16_hi(d[g][j].y), acc[j][3]);
+                            acc[j][4] = fmaf(ws[g], bf16_lo(d[g][j].z), acc[j][4]);
+                            acc[j][5] = fmaf(ws[g], bf16_hi(d[g][j].z), acc[j][5]);
+                            acc[j][6] = fmaf(ws[g], bf16_lo(d[g][j].w), acc[j][6]);
+                            acc[j][7] = fmaf(ws[g], bf16_hi(d[g][j].w), acc[j][7]);
+                        }
+                    }
                 }
             }
         }
-    }
 
 #pragma unroll
-    for (int j = 0; j < kVecPerLane; ++j) {
-        if (!vin[j])
-            continue;
-        if (kOutF32) {
-            float* o = static_cast<float*>(a.out) + t * a.H + static_cast<int64_t>(v[j]) * 8;
-            st_cs_v4(o, make_uint4(__float_as_uint(acc[j][0]), __float_as_uint(acc[j][1]), __float_as_uint(acc[j][2]),
-                                   __float_as_uint(acc[j][3])));
-            st_cs_v4(o + 4, make_uint4(__float_as_uint(acc[j][4]), __float_as_uint(acc[j][5]),
-                                       __float_as_uint(acc[j][6]), __float_as_uint(acc[j][7])));
-        } else {
-            uint8_t* o = static_cast<uint8_t*>(a.out) + t * row_bytes + static_cast<int64_t>(v[j]) * 16;
-            st_cs_v4(o, make_uint4(pack_bf16x2(acc[j][0], acc[j][1]), pack_bf16x2(acc[j][2], acc[j][3]),
-                                   pack_bf16x2(acc[j][4], acc[j][5]), pack_bf16x2(acc[j][6], acc[j][7])));
+        for (int j = 0; j < kVecPerLane; ++j) {
+            if (!vin[j])
+                continue;
+            if (kOutF32) {
+                float* o = static_cast<float*>(a.out) + t * a.H + static_cast<int64_t>(v[j]) * 8;
+                st_cs_v4(o, make_uint4(__float_as_uint(acc[j][0]), __float_as_uint(acc[j][1]), __float_as_uint(acc[j][2]),
+                                       __float_as_uint(acc[j][3])));
+                st_cs_v4(o + 4, make_uint4(__float_as_uint(acc[j][4]), __float_as_uint(acc[j][5]),
+                                           __float_as_uint(acc[j][6]), __float_as_uint(acc[j][7])));
+            } else {
+                uint8_t* o = static_cast<uint8_t*>(a.out) + t * row_bytes + static_cast<int64_t>(v[j]) * 16;
+                st_cs_v4(o, make_uint4(pack_bf16x2(acc[j][0], acc[j][1]), pack_bf16x2(acc[j][2], acc[j][3]),
+                                       pack_bf16x2(acc[j][4], acc[j][5]), pack_bf16x2(acc[j][6], acc[j][7])));
+            }
         }
     }
-    if (seg == 0) {
-        const uint32_t any = __reduce_or_sync(kFullMask, errbits);
-        if (lane == 0)
-            flag_error(a.err, any);
-    }
+    const uint32_t any = __reduce_or_sync(kFullMask, errbits);
+    if (lane == 0)
+        flag_error(a.err, any);
 }
 
-template <bool kExpertChoice>
-cudaError_t launch_combine(CombineArgs k, bool out_f32, cudaStream_t stream)
+// Blocks of 256 threads of `kernel` resident on the whole device (SMs x
+// blocks per SM), cached per device in `cache`.
+template <typename Kernel>
+int64_t resident_blocks(Kernel kernel, int* cache)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 0;
+    if (cache[dev] == 0) {
+        int sms = 0, per_sm = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kCombineThreads, 0) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        cache[dev] = sms * std::max(per_sm, 1);
+    }
+    return cache[dev];
+}
+
+// persistent: one resident wave of warps loops over the (token, segment)
+// items instead of one short-lived block per 8 items
+template <bool kExpertChoice, int kVec, int kGrp>
+cudaError_t launch_combine(CombineArgs k, bool out_f32, bool persistent, cudaStream_t stream)
 {
     constexpr int64_t kMaxBlocks = int64_t{1} << 30;
+    k.nseg = (k.nvec + 32 * kVec - 1) / (32 * kVec);
     const int64_t warps = static_cast<int64_t>(k.T) * k.nseg;
-    const int64_t blocks = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
+    int64_t blocks = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
+    if (persistent) {
+        static int cache[64];
+        const int64_t res = resident_blocks(combine_kernel<kExpertChoice, false, kVec, kGrp>, cache);
+        if (res > 0)
+            blocks = std::min(blocks, res);
+    }
     for (int64_t b0 = 0; b0 < blocks; b0 += kMaxBlocks) {
         k.warp_base = b0 * kWarpsPerCta;
         const unsigned n = static_cast<unsigned>(blocks - b0 < kMaxBlocks ? blocks - b0 : kMaxBlocks);
         if (out_f32)
-            combine_kernel<kExpertChoice, true><<<n, kCombineThreads, 0, stream>>>(k);
+            combine_kernel<kExpertChoice, true, kVec, kGrp><<<n, kCombineThreads, 0, stream>>>(k);
         else
-            combine_kernel<kExpertChoice, false><<<n, kCombineThreads, 0, stream>>>(k);
+            combine_kernel<kExpertChoice, false, kVec, kGrp><<<n, kCombineThreads, 0, stream>>>(k);
         cudaError_t st = cudaGetLastError();
         if (st != cudaSuccess)
             return st;
@@ -225,7 +295,6 @@ cudaError_t launch_tc_combine(const TcCombineLaunch& a, cudaStream_t stream)
     k.T = a.T;
     k.H = a.H;
     k.nvec = a.H / 8;
-    k.nseg = (k.nvec + kSegVec - 1) / kSegVec;
     k.num_y_rows = a.rows.num_rows;
     k.topk_idx = a.rows.topk_idx;
     k.slot = a.rows.slot;
@@ -237,7 +306,7 @@ cudaError_t launch_tc_combine(const TcCombineLaunch& a, cudaStream_t stream)
     k.topk_weights = a.topk_weights;
     k.out = a.out;
     k.err = a.err;
-    return launch_combine<false>(k, a.out_dtype == EP_FP32, stream);
+    return launch_combine<false, kTcVec, kTcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0, stream);
 }
 
 cudaError_t launch_ec_combine(const EcCombineLaunch& a, cudaStream_t stream)
@@ -247,14 +316,13 @@ cudaError_t launch_ec_combine(const EcCombineLaunch& a, cudaStream_t stream)
     k.T = a.T;
     k.H = a.H;
     k.nvec = a.H / 8;
-    k.nseg = (k.nvec + kSegVec - 1) / kSegVec;
     k.num_y_rows = a.num_y_rows;
     k.token_offsets = a.token_offsets;
     k.token_slots = a.token_slots;
     k.expert_weights = a.expert_weights;
     k.out = a.out;
     k.err = a.err;
-    return launch_combine<true>(k, a.out_dtype == EP_FP32, stream);
+    return launch_combine<true, kEcVec, kEcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_EC != 0, stream);
 }
 
 } // namespace ep

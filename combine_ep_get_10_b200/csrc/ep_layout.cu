@@ -30,11 +30,24 @@ namespace ep {
 
 namespace {
 
-constexpr int kLayoutThreads = 1024;
+#ifndef EP_LAYOUT_THREADS
+#define EP_LAYOUT_THREADS 512
+#endif
+#ifndef EP_LAYOUT_PAIRS_PER_CTA
+#define EP_LAYOUT_PAIRS_PER_CTA 2048
+#endif
+#ifndef EP_LAYOUT_MAX_CLUSTER
+#define EP_LAYOUT_MAX_CLUSTER 16
+#endif
+constexpr int kLayoutThreads = EP_LAYOUT_THREADS;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
-constexpr int kPrefetch = 8; // 32-pair steps a warp loads before ranking them
-constexpr int64_t kPairsPerCta = 2048;
+// 32-pair steps a warp keeps in registers: a full 16-CTA cluster holds 8192
+// pairs per CTA (131072 pairs) on the register path
+constexpr int kPrefetch = 8192 / kLayoutThreads;
+constexpr int kLoadBatch = 8;                       // ids loaded together
+constexpr int64_t kPairsPerCta = EP_LAYOUT_PAIRS_PER_CTA;
 constexpr int kMaxCluster = 16;
+constexpr int64_t kSmemIds = 8192; // pairs per CTA whose ids are staged in shared memory
 
 struct TcArgs {
     const int64_t* topk_idx;
@@ -47,6 +60,31 @@ struct TcArgs {
     uint32_t* err;
     int32_t in_rank_words; // 1: write is_token_in_rank as 32-bit words
 };
+
+__device__ __forceinline__ void write_rank_row(const TcArgs& a, int64_t t, uint32_t mask)
+{
+    uint8_t* row = a.in_rank + t * a.R;
+    if (a.in_rank_words) {
+        for (int r = 0; r < a.R; r += 4) {
+            const uint32_t w = ((mask >> r) & 1u) | (((mask >> (r + 1)) & 1u) << 8) |
+                               (((mask >> (r + 2)) & 1u) << 16) | (((mask >> (r + 3)) & 1u) << 24);
+            *reinterpret_cast<uint32_t*>(row + r) = w;
+        }
+    } else {
+        for (int r = 0; r < a.R; ++r)
+            row[r] = static_cast<uint8_t>((mask >> r) & 1u);
+    }
+}
+
+__device__ __forceinline__ void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
 
 // Exclusive scan of one int per thread over the block; returns the block total.
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& total)
@@ -86,10 +124,14 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(Tc
     const int cs = static_cast<int>(cluster.num_blocks());
     const int b = static_cast<int>(cluster.block_rank());
     extern __shared__ __align__(16) int32_t smem[];
-    int32_t* wtab = smem;                      // [32][E] per-warp counters, later prefixes
+    int32_t* wtab = smem;                      // [warps][E] per-warp counters, later prefixes
     int32_t* tot = wtab + kLayoutWarps * a.E;  // [E] this CTA's pairs per expert
-    int32_t* srank = tot + a.E;                // [32] this CTA's tokens per rank
+    int32_t* base = tot + a.E;                 // [E] pairs of each expert in earlier CTAs
+    int32_t* all = base + a.E;                 // [E] pairs of each expert in the cluster
+    int32_t* srank = all + a.E;                // [32] this CTA's tokens per rank
     int32_t* sscan = srank + 32;               // [32] scan scratch
+    int* sid = sscan + 32;                     // [<= kSmemIds] expert id of each pair (or -1)
+    uint32_t* smask = reinterpret_cast<uint32_t*>(sid + kSmemIds); // [<= kSmemIds] rank bits per token
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     for (int i = tid; i < kLayoutWarps * a.E; i += kLayoutThreads)
@@ -110,79 +152,87 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(Tc
     bool bad = false;
 
     // phase 1: per-warp stable ranks and counters.  When the warp's run fits
-    // one prefetch batch (<= 256 pairs) the ids and ranks stay in registers;
-    // longer runs park the rank in slot[] and re-read it in phase 3.
+    // kPrefetch steps the ids and ranks stay in registers; longer runs park
+    // the rank in slot[] and re-read it in phase 3.
     const bool in_regs = (we - wb) <= 32 * kPrefetch;
+    // with the whole CTA on the register path its ids are also staged in
+    // shared memory for the rank-membership pass
+    const bool ids_in_smem = (p1 - p0) <= kSmemIds;
     int ev[kPrefetch]; // expert id, or -1 for a pair that is not routed
     int loc[kPrefetch];
-    for (int64_t base = wb; base < we; base += 32 * kPrefetch) {
-        int64_t raw[kPrefetch];
+    for (int64_t start = wb; start < we; start += 32 * kPrefetch) {
 #pragma unroll
-        for (int j = 0; j < kPrefetch; ++j) {
-            const int64_t p = base + j * 32 + lane;
-            raw[j] = p < we ? __ldg(a.topk_idx + p) : -1;
-        }
+        for (int j0 = 0; j0 < kPrefetch; j0 += kLoadBatch) {
+            int64_t raw[kLoadBatch];
 #pragma unroll
-        for (int j = 0; j < kPrefetch; ++j) {
-            const bool ok = raw[j] >= 0 && raw[j] < a.E;
-            bad |= !ok && raw[j] != -1;
-            ev[j] = ok ? static_cast<int>(raw[j]) : -1;
+            for (int j = 0; j < kLoadBatch; ++j) {
+                const int64_t p = start + (j0 + j) * 32 + lane;
+                raw[j] = p < we ? __ldg(a.topk_idx + p) : -1;
+            }
+#pragma unroll
+            for (int j = 0; j < kLoadBatch; ++j) {
+                const bool ok = raw[j] >= 0 && raw[j] < a.E;
+                bad |= !ok && raw[j] != -1;
+                ev[j0 + j] = ok ? static_cast<int>(raw[j]) : -1;
+                const int64_t p = start + (j0 + j) * 32 + lane;
+                if (ids_in_smem && p < we)
+                    sid[p - p0] = ev[j0 + j];
+            }
         }
+        // the steps' equal-id lane sets are independent: issue them together,
+        // then run the dependent counter updates step after step
+        uint32_t peers[kPrefetch];
+#pragma unroll
+        for (int j = 0; j < kPrefetch; ++j)
+            peers[j] = start + j * 32 < we ? __match_any_sync(kFullMask, ev[j]) : 0u;
 #pragma unroll
         for (int j = 0; j < kPrefetch; ++j) {
             loc[j] = -1;
-            const int64_t step = base + j * 32;
+            const int64_t step = start + j * 32;
             if (step >= we)
                 break; // warp-uniform
             const int64_t p = step + lane;
-            const bool in = p < we;
             const int e = ev[j];
-            const bool good = e >= 0;
-            const uint32_t peers = __match_any_sync(kFullMask, e);
             int prior = 0;
-            if (good)
+            if (e >= 0)
                 prior = mine[e];
             __syncwarp();
-            if (good) {
-                const int r = __popc(peers & lanes_below);
+            if (e >= 0) {
+                const int r = __popc(peers[j] & lanes_below);
                 loc[j] = prior + r;
                 if (r == 0)
-                    mine[e] = prior + __popc(peers);
+                    mine[e] = prior + __popc(peers[j]);
             }
-            if (!in_regs && in)
+            if (!in_regs && p < we)
                 a.slot[p] = loc[j];
             __syncwarp();
         }
     }
 
-    // phase 1b: rank membership of this CTA's tokens (ids re-read from L1/L2,
-    // all of a token's loads issued before any is used)
-    constexpr int kMaskBatch = 8;
+    // phase 1b: rank membership of this CTA's tokens, from the staged ids in
+    // shared memory, else re-read from L1/L2 (a token's loads issued together)
+    __syncthreads();
     for (int64_t tb = t0 + static_cast<int64_t>(warp) * 32; tb < t1; tb += kLayoutThreads) {
         const int64_t t = tb + lane;
         uint32_t mask = 0;
-        if (t < t1) {
-            for (int k0 = 0; k0 < a.K; k0 += kMaskBatch) {
-                int64_t ids[kMaskBatch];
+        if (t < t1 && ids_in_smem) {
+            const int* ids = sid + (t - t0) * a.K;
+            for (int k = 0; k < a.K; ++k)
+                if (ids[k] >= 0)
+                    mask |= 1u << static_cast<uint32_t>(ids[k] / a.per_rank);
+            smask[t - t0] = mask; // written out after the cluster barriers
+        } else if (t < t1) {
+            for (int k0 = 0; k0 < a.K; k0 += kLoadBatch) {
+                int64_t ids[kLoadBatch];
 #pragma unroll
-                for (int k = 0; k < kMaskBatch; ++k)
+                for (int k = 0; k < kLoadBatch; ++k)
                     ids[k] = k0 + k < a.K ? __ldg(a.topk_idx + t * a.K + k0 + k) : -1;
 #pragma unroll
-                for (int k = 0; k < kMaskBatch; ++k)
+                for (int k = 0; k < kLoadBatch; ++k)
                     if (ids[k] >= 0 && ids[k] < a.E)
                         mask |= 1u << static_cast<uint32_t>(ids[k] / a.per_rank);
             }
-            uint8_t* row = a.in_rank + t * a.R;
-            if (a.in_rank_words) {
-                for (int r = 0; r < a.R; r += 4) {
-                    uint32_t w = ((mask >> r) & 1u) | (((mask >> (r + 1)) & 1u) << 8) |
-                                 (((mask >> (r + 2)) & 1u) << 16) | (((mask >> (r + 3)) & 1u) << 24);
-                    *reinterpret_cast<uint32_t*>(row + r) = w;
-                }
-            } else {
-                for (int r = 0; r < a.R; ++r)
-                    row[r] = static_cast<uint8_t>((mask >> r) & 1u);
-            }
+            write_rank_row(a, t, mask);
         }
         for (int r = 0; r < a.R; ++r) {
             const int c = __popc(__ballot_sync(kFullMask, (mask >> r) & 1u));
@@ -195,9 +245,9 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(Tc
     __syncthreads();
 
     // phase 2: counters -> exclusive prefix down the warps; CTA totals
-    const int e = tid; // E <= kLayoutThreads
-    if (e < a.E) {
+    for (int e = tid; e < a.E; e += kLayoutThreads) {
         int run = 0;
+#pragma unroll
         for (int w = 0; w < kLayoutWarps; ++w) {
             const int c = wtab[w * a.E + e];
             wtab[w * a.E + e] = run;
@@ -208,17 +258,19 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(Tc
     cluster.sync();
 
     // totals of every CTA of the cluster, all loads in flight together
-    int base = 0, all = 0;
-    if (e < a.E) {
+    for (int e = tid; e < a.E; e += kLayoutThreads) {
         int v[kMaxCluster];
 #pragma unroll
         for (int j = 0; j < kMaxCluster; ++j)
             v[j] = j < cs ? cluster.map_shared_rank(tot, j)[e] : 0;
+        int bs = 0, al = 0;
 #pragma unroll
         for (int j = 0; j < kMaxCluster; ++j) {
-            base += j < b ? v[j] : 0;
-            all += v[j];
+            bs += j < b ? v[j] : 0;
+            al += v[j];
         }
+        base[e] = bs;
+        all[e] = al;
     }
     int rank_total = 0;
     if (b == 0 && tid < a.R) {
@@ -230,23 +282,36 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(Tc
         for (int j = 0; j < kMaxCluster; ++j)
             rank_total += v[j];
     }
-    cluster.sync(); // no CTA leaves or reuses its shared memory while others read it
+    // every remote read above has completed (its value is in registers or
+    // shared memory); the matching wait sits at the end of the kernel so that
+    // no CTA exits while another may still read its shared memory
+    cluster_arrive_relaxed();
 
     if (b == 0) {
-        int total = 0;
-        const int excl = block_exclusive_scan(e < a.E ? all : 0, sscan, total);
-        if (e < a.E) {
-            a.counts[e] = all;
-            a.offsets[e] = excl;
+        // expert offsets: exclusive scan of the cluster totals, one block-wide
+        // pass per kLayoutThreads experts
+        int carry = 0;
+        for (int e0 = 0; e0 < a.E; e0 += kLayoutThreads) {
+            const int e = e0 + tid;
+            const int v = e < a.E ? all[e] : 0;
+            int total = 0;
+            const int excl = block_exclusive_scan(v, sscan, total);
+            if (e < a.E) {
+                a.counts[e] = v;
+                a.offsets[e] = carry + excl;
+            }
+            carry += total;
         }
         if (tid == 0)
-            a.offsets[a.E] = total;
+            a.offsets[a.E] = carry;
         if (tid < a.R)
             a.rank_counts[tid] = rank_total;
     }
-    if (e < a.E) {
+    for (int e = tid; e < a.E; e += kLayoutThreads) {
+        const int bs = base[e];
+#pragma unroll
         for (int w = 0; w < kLayoutWarps; ++w)
-            wtab[w * a.E + e] += base;
+            wtab[w * a.E + e] += bs;
     }
     __syncthreads();
 
@@ -269,6 +334,11 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(Tc
             }
         }
     }
+    if (ids_in_smem) {
+        for (int64_t t = t0 + tid; t < t1; t += kLayoutThreads)
+            write_rank_row(a, t, smask[t - t0]);
+    }
+    cluster_wait();
 }
 
 // ---------------------------------------------------------------- expert choice
@@ -408,6 +478,271 @@ __global__ void __launch_bounds__(kEcThreads) ec_sort_kernel(EcArgs a)
     }
 }
 
+// Expert choice in one launch: a cluster of up to 16 CTAs, CTA j holding a
+// contiguous range of slots and owning a contiguous range of tokens.
+//   1. one warp walks the CTA's slots in order (32 at a time, equal token ids
+//      ranked by __match_any_sync) keeping a per-token counter in shared
+//      memory: the rank of a slot among the CTA's slots of its token;
+//      the other warps OR rank bits per token and count each expert's row;
+//   2. cluster barrier; each owner reads every CTA's counters of its tokens
+//      over DSMEM: degree, rank mask, and the CTA's total; the degrees are
+//      scanned over the owner's range;
+//   3. cluster barrier; owners add the totals of earlier owners, write
+//      token_offsets, and store into every CTA i's shared memory the start of
+//      CTA i's run inside each owned token's list (offset + counts of CTAs
+//      before i);
+//   4. cluster barrier; every slot is written at start + its rank.
+// Slot lists come out in ascending slot order with integer arithmetic only.
+constexpr int kEcClusterThreads = 256;
+constexpr int64_t kEcClusterMaxT = 16384;
+constexpr int64_t kEcClusterSlotsPerCta = 2048;
+constexpr int kEcClusterPrefetch = 16; // ranking steps whose lane sets are formed together
+constexpr int64_t kEcClusterOwnMax = 4 * kEcClusterThreads; // tokens owned per CTA, 4 per thread
+constexpr int64_t kEcClusterMaxE = 2048;
+
+struct EcClusterArgs {
+    const int32_t* ti;
+    int32_t T, E, C, R, per_rank;
+    int32_t* counts;
+    int32_t* rank_counts;
+    uint8_t* in_rank;
+    int32_t* token_offsets;
+    int32_t* token_slots;
+    uint32_t* err;
+};
+
+// per-token arrays are padded to a multiple of 4 tokens for 16-byte DSMEM access
+__host__ __device__ inline int64_t ec_padded_tokens(int64_t T)
+{
+    return (T + 3) / 4 * 4;
+}
+
+size_t ec_cluster_smem_bytes(int64_t T, int64_t spc, int64_t E)
+{
+    return sizeof(int32_t) * static_cast<size_t>(3 * ec_padded_tokens(T) + 2 * spc + E + 32 + 32 + 8);
+}
+
+__global__ void __launch_bounds__(kEcClusterThreads, 1) ec_layout_cluster_kernel(EcClusterArgs a, int32_t spc)
+{
+    cg::cluster_group cluster = cg::this_cluster();
+    const int cs = static_cast<int>(cluster.num_blocks());
+    const int b = static_cast<int>(cluster.block_rank());
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t S = static_cast<int64_t>(a.E) * a.C;
+    const int64_t Tp = ec_padded_tokens(a.T);
+    // owned token ranges are multiples of 4 tokens
+    const int64_t own = ((Tp / 4 + cs - 1) / cs) * 4;
+    extern __shared__ __align__(16) int32_t smem[];
+    int32_t* hist = smem;                                      // [Tp] this CTA's slots per token
+    uint32_t* tmask = reinterpret_cast<uint32_t*>(hist + Tp);  // [Tp] rank bits of this CTA's slots
+    int32_t* start = reinterpret_cast<int32_t*>(tmask + Tp);   // [Tp] where this CTA's run of a token starts
+    int32_t* sid = start + Tp;                                 // [spc] token of each slot (-1: none)
+    int32_t* lrank = sid + spc;                                // [spc] rank of each slot in its token's run
+    int32_t* pcount = lrank + spc;                             // [E] this CTA's filled slots per expert
+    int32_t* srank = pcount + a.E;                             // [32] owner: tokens per rank
+    int32_t* sscan = srank + 32;                               // [32] scan scratch
+    int32_t* rtot = sscan + 32;                                // [1] owner: total picks of its tokens
+
+    for (int64_t i = tid; i < Tp; i += kEcClusterThreads) {
+        hist[i] = 0;
+        tmask[i] = 0u;
+    }
+    for (int e = tid; e < a.E; e += kEcClusterThreads)
+        pcount[e] = 0;
+    if (tid < 32)
+        srank[tid] = 0;
+    __syncthreads();
+
+    // 1. the CTA's slots: ids into shared memory (all warps, one pass),
+    // rank bits per token and filled slots per expert
+    const int64_t s0 = min(S, static_cast<int64_t>(b) * spc);
+    const int64_t s1 = min(S, s0 + spc);
+    bool bad = false;
+    for (int64_t sb = s0 + (tid & ~31); sb < s1; sb += kEcClusterThreads) {
+        const int64_t s = sb + lane;
+        const bool in = s < s1;
+        const int t = in ? __ldg(a.ti + s) : -1;
+        const bool good = in && t >= 0 && t < a.T;
+        bad |= in && !good && t != -1;
+        const int e = in ? static_cast<int>(s / a.C) : -1;
+        if (in)
+            sid[s - s0] = good ? t : -1;
+        if (good)
+            atomicOr(&tmask[t], 1u << static_cast<uint32_t>(e / a.per_rank));
+        // lanes of one expert add their filled slots once
+        const uint32_t peers = __match_any_sync(kFullMask, e);
+        const int n = __popc(__ballot_sync(kFullMask, good) & peers);
+        if (in && (__ffs(peers) - 1) == lane && n)
+            atomicAdd(&pcount[e], n);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // ranking walk over the staged ids, 32 slots per step
+        const uint32_t lanes_below = (1u << lane) - 1u;
+        for (int64_t base = s0; base < s1; base += 32 * kEcClusterPrefetch) {
+            // equal-token lane sets of kEcClusterPrefetch steps issued together,
+            // then the dependent counter updates step after step
+            int key[kEcClusterPrefetch];
+            uint32_t peers[kEcClusterPrefetch];
+#pragma unroll
+            for (int j = 0; j < kEcClusterPrefetch; ++j) {
+                const int64_t s = base + j * 32 + lane;
+                key[j] = s < s1 ? sid[s - s0] : -1;
+            }
+#pragma unroll
+            for (int j = 0; j < kEcClusterPrefetch; ++j)
+                peers[j] = base + j * 32 < s1 ? __match_any_sync(kFullMask, key[j]) : 0u;
+#pragma unroll
+            for (int j = 0; j < kEcClusterPrefetch; ++j) {
+                if (base + j * 32 >= s1)
+                    break; // warp-uniform
+                const int64_t s = base + j * 32 + lane;
+                int prior = 0;
+                if (key[j] >= 0)
+                    prior = hist[key[j]];
+                __syncwarp();
+                if (key[j] >= 0) {
+                    const int r = __popc(peers[j] & lanes_below);
+                    lrank[s - s0] = prior + r;
+                    if (r == 0)
+                        hist[key[j]] = prior + __popc(peers[j]);
+                }
+                __syncwarp();
+            }
+        }
+    }
+    if (__any_sync(kFullMask, bad) && lane == 0)
+        flag_error(a.err, EP_DEVERR_BAD_INDEX);
+    __syncthreads();
+    cluster.sync();
+
+    // 2. owner of tokens [u0, u1), four per thread: every CTA's counters of
+    // the four tokens in one 16-byte DSMEM load each, kept in registers
+    const int64_t u0 = min(Tp, static_cast<int64_t>(b) * own);
+    const int64_t u1 = min(static_cast<int64_t>(a.T), u0 + own);
+    const int64_t t4 = u0 + 4 * static_cast<int64_t>(tid);
+    const bool owns = t4 < u1;
+    int4 h[kMaxCluster];
+    int deg[4] = {0, 0, 0, 0};
+    uint32_t mask[4] = {0u, 0u, 0u, 0u};
+    if (owns) {
+        uint4 m[kMaxCluster];
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j) {
+            h[j] = j < cs ? *reinterpret_cast<const int4*>(cluster.map_shared_rank(hist, j) + t4) : make_int4(0, 0, 0, 0);
+            m[j] = j < cs ? *reinterpret_cast<const uint4*>(cluster.map_shared_rank(tmask, j) + t4)
+                          : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j) {
+            deg[0] += h[j].x;
+            deg[1] += h[j].y;
+            deg[2] += h[j].z;
+            deg[3] += h[j].w;
+            mask[0] |= m[j].x;
+            mask[1] |= m[j].y;
+            mask[2] |= m[j].z;
+            mask[3] |= m[j].w;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        for (int r = 0; r < a.R; ++r) {
+            const int c = __popc(__ballot_sync(kFullMask, (mask[i] >> r) & 1u));
+            if (lane == 0 && c)
+                atomicAdd(&srank[r], c);
+        }
+    }
+    // CTA 0: filled slots per expert, summed over the cluster
+    int ecount = 0;
+    const int e_own = tid;
+    if (b == 0) {
+        for (int e = tid; e < a.E; e += kEcClusterThreads) {
+            int n = 0;
+            for (int j = 0; j < cs; ++j)
+                n += cluster.map_shared_rank(pcount, j)[e];
+            if (e == e_own)
+                ecount = n;
+            else
+                a.counts[e] = n; // E > threads: rare, written directly
+        }
+    }
+    int range_total = 0;
+    const int excl = block_exclusive_scan(deg[0] + deg[1] + deg[2] + deg[3], sscan, range_total);
+    if (tid == 0)
+        rtot[0] = range_total;
+    __syncthreads();
+    cluster.sync();
+
+    // 3. owners: global offsets, and the start of every CTA's run in each token
+    int carry = 0;
+    {
+        int v[kMaxCluster];
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j)
+            v[j] = j < b ? cluster.map_shared_rank(rtot, j)[0] : 0;
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j)
+            carry += v[j];
+    }
+    int off[4];
+    off[0] = carry + excl;
+    off[1] = off[0] + deg[0];
+    off[2] = off[1] + deg[1];
+    off[3] = off[2] + deg[2];
+    if (owns) {
+        int4 pre = make_int4(off[0], off[1], off[2], off[3]);
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j) {
+            if (j < cs) {
+                *reinterpret_cast<int4*>(cluster.map_shared_rank(start, j) + t4) = pre;
+                pre.x += h[j].x;
+                pre.y += h[j].y;
+                pre.z += h[j].z;
+                pre.w += h[j].w;
+            }
+        }
+    }
+    int rank_total = 0;
+    if (b == 0 && tid < a.R) {
+        int v[kMaxCluster];
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j)
+            v[j] = j < cs ? cluster.map_shared_rank(srank, j)[tid] : 0;
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j)
+            rank_total += v[j];
+    }
+    cluster.sync();
+
+    // 4. global outputs, after the last cluster barrier (so no barrier waits
+    // for them): every filled slot at its run's start + its rank, then the
+    // owners' offsets and rank rows, CTA 0's counts
+    for (int64_t s = s0 + tid; s < s1; s += kEcClusterThreads) {
+        const int t = sid[s - s0];
+        if (t >= 0)
+            a.token_slots[start[t] + lrank[s - s0]] = static_cast<int32_t>(s);
+    }
+    if (owns) {
+        for (int i = 0; i < 4; ++i) {
+            if (t4 + i >= u1)
+                break;
+            a.token_offsets[t4 + i] = off[i];
+            uint8_t* row = a.in_rank + (t4 + i) * a.R;
+            for (int r = 0; r < a.R; ++r)
+                row[r] = static_cast<uint8_t>((mask[i] >> r) & 1u);
+        }
+    }
+    if (b == cs - 1 && tid == 0)
+        a.token_offsets[a.T] = carry + rtot[0];
+    if (b == 0) {
+        if (e_own < a.E)
+            a.counts[e_own] = ecount;
+        if (tid < a.R)
+            a.rank_counts[tid] = rank_total;
+    }
+}
+
 int cluster_limit_cache[64];
 size_t smem_attr_cache[64];
 
@@ -421,7 +756,7 @@ cudaError_t prepare_layout_kernel(size_t smem)
         return st;
     if (dev >= 0 && dev < 64 && smem_attr_cache[dev] >= smem)
         return cudaSuccess;
-    const size_t want = std::max<size_t>(smem, sizeof(int32_t) * (kLayoutWarps * 256 + 256 + 64));
+    const size_t want = std::max<size_t>(smem, sizeof(int32_t) * (kLayoutWarps * 256 + 3 * 256 + 64 + 2 * kSmemIds));
     st = cudaFuncSetAttribute(tc_layout_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(want));
     if (st != cudaSuccess)
@@ -462,6 +797,42 @@ int max_layout_cluster(size_t smem_bytes)
     return best;
 }
 
+int ec_cluster_limit_cache[64];
+
+// 16-CTA clusters of the expert-choice kernel fit on this device (else 8).
+int max_ec_cluster()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 8;
+    if (ec_cluster_limit_cache[dev] > 0)
+        return ec_cluster_limit_cache[dev];
+    int best = 8;
+    const size_t smem = ec_cluster_smem_bytes(kEcClusterMaxT, kEcClusterSlotsPerCta, kEcClusterMaxE);
+    if (cudaFuncSetAttribute(ec_layout_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) == cudaSuccess &&
+        cudaFuncSetAttribute(ec_layout_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        cfg.gridDim = dim3(16);
+        cfg.blockDim = dim3(kEcClusterThreads);
+        cfg.dynamicSmemBytes = smem;
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 16;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, ec_layout_cluster_kernel, &cfg) == cudaSuccess && n >= 1)
+            best = 16;
+    }
+    cudaGetLastError();
+    ec_cluster_limit_cache[dev] = best;
+    return best;
+}
+
 } // namespace
 
 cudaError_t launch_tc_layout(const TcLayoutLaunch& a, cudaStream_t stream)
@@ -481,12 +852,14 @@ cudaError_t launch_tc_layout(const TcLayoutLaunch& a, cudaStream_t stream)
     k.err = a.err;
     k.in_rank_words = (a.R % 4 == 0 && (reinterpret_cast<uintptr_t>(a.in_rank) & 3u) == 0) ? 1 : 0;
 
-    const size_t smem = sizeof(int32_t) * (static_cast<size_t>(kLayoutWarps) * a.E + a.E + 64);
+    const size_t smem =
+        sizeof(int32_t) * (static_cast<size_t>(kLayoutWarps) * a.E + 3 * static_cast<size_t>(a.E) + 64 + 2 * kSmemIds);
     cudaError_t st = prepare_layout_kernel(smem);
     if (st != cudaSuccess)
         return st;
     const int64_t pairs = static_cast<int64_t>(a.T) * a.K;
-    int cs = static_cast<int>(std::min<int64_t>(16, std::max<int64_t>(1, (pairs + kPairsPerCta - 1) / kPairsPerCta)));
+    int cs = static_cast<int>(
+        std::min<int64_t>(EP_LAYOUT_MAX_CLUSTER, std::max<int64_t>(1, (pairs + kPairsPerCta - 1) / kPairsPerCta)));
     if (cs > 8)
         cs = std::min(cs, max_layout_cluster(smem));
 
@@ -511,8 +884,63 @@ size_t ec_layout_workspace_bytes(int64_t T, int64_t E, int64_t C)
     return kWorkspaceHeaderBytes + ((arrays + 255) / 256) * 256;
 }
 
+int ec_smem_attr_dev[64];
+
+cudaError_t launch_ec_layout_cluster(const EcLayoutLaunch& a, cudaStream_t stream, bool& launched)
+{
+    launched = false;
+    const int64_t S = static_cast<int64_t>(a.E) * a.C;
+    if (a.T > kEcClusterMaxT || S > kMaxCluster * kEcClusterSlotsPerCta)
+        return cudaSuccess;
+    // enough CTAs for <= 1024 slots and <= kEcClusterOwnMax owned tokens each, if possible
+    const int64_t Tp = ec_padded_tokens(a.T);
+    int cs = static_cast<int>(std::min<int64_t>(
+        kMaxCluster, std::max<int64_t>({int64_t{1}, (S + 1023) / 1024, (Tp + kEcClusterOwnMax - 1) / kEcClusterOwnMax})));
+    if (cs > 8 && max_ec_cluster() < 16)
+        cs = 8;
+    const int64_t spc = (S + cs - 1) / cs;
+    const int64_t own = ((Tp / 4 + cs - 1) / cs) * 4;
+    if (spc > kEcClusterSlotsPerCta || own > kEcClusterOwnMax || a.E > kEcClusterMaxE)
+        return cudaSuccess; // too large for one cluster: the multi-kernel path below
+    const size_t smem = ec_cluster_smem_bytes(a.T, spc, a.E);
+    int dev = 0;
+    cudaError_t st = cudaGetDevice(&dev);
+    if (st != cudaSuccess)
+        return st;
+    if (dev < 0 || dev >= 64 || ec_smem_attr_dev[dev] == 0) {
+        st = cudaFuncSetAttribute(ec_layout_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(ec_cluster_smem_bytes(kEcClusterMaxT, kEcClusterSlotsPerCta, kEcClusterMaxE)));
+        if (st == cudaSuccess)
+            st = cudaFuncSetAttribute(ec_layout_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (st != cudaSuccess)
+            return st;
+        if (dev >= 0 && dev < 64)
+            ec_smem_attr_dev[dev] = 1;
+    }
+    EcClusterArgs k{a.token_indices, a.T, a.E, a.C, a.R, a.E / a.R, a.counts, a.rank_counts, a.in_rank,
+                    a.token_offsets, a.token_slots, a.err};
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(cs);
+    cfg.blockDim = dim3(kEcClusterThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    launched = true;
+    return cudaLaunchKernelEx(&cfg, ec_layout_cluster_kernel, k, static_cast<int32_t>(spc));
+}
+
 cudaError_t launch_ec_layout(const EcLayoutLaunch& a, cudaStream_t stream)
 {
+    bool launched = false;
+    cudaError_t cst = launch_ec_layout_cluster(a, stream, launched);
+    if (cst != cudaSuccess || launched)
+        return cst;
     EcArgs k{};
     k.ti = a.token_indices;
     k.T = a.T;
