@@ -143,6 +143,18 @@ class Routing:
         d = RoutingDesc(EP_ROUTING_EXPERT_CHOICE, None, token_indices.data_ptr(), num_tokens, 0, C, E, num_ranks)
         return Routing(d, token_indices)
 
+    def tokens(self, t0: int, t1: int) -> "Routing":
+        """Token-choice routing of tokens [t0, t1) only (a view: the topk_idx
+        pointer is offset).  With Layout.tokens() it lets dispatch and combine
+        run on a chunk of tokens, e.g. to overlap host transfers of the next
+        chunk, or to bound per-call working sets on long sequences."""
+        if self.desc.routing != EP_ROUTING_TOPK or not (0 <= t0 <= t1 <= self.desc.num_tokens):
+            raise ValueError("token range [%d, %d) of a token-choice routing of %d tokens"
+                             % (t0, t1, self.desc.num_tokens))
+        d = RoutingDesc(EP_ROUTING_TOPK, self.desc.topk_idx + t0 * self.desc.num_topk * 8, None, t1 - t0,
+                        self.desc.num_topk, 0, self.desc.num_experts, self.desc.num_ranks)
+        return Routing(d, self)
+
     @property
     def T(self):
         return self.desc.num_tokens
@@ -196,6 +208,25 @@ class Layout:
             self.num_tokens_per_expert, self.expert_offsets, self.num_tokens_per_rank, self.is_token_in_rank,
             self.slot, self.token_offsets, self.token_slots, self.workspace)),
             self.workspace.numel() * self.workspace.element_size())
+
+
+class LayoutView:
+    """A token-choice layout restricted to tokens [t0, t1) of its routing:
+    the slot pointer is offset; counts, offsets and workspace are shared."""
+
+    def __init__(self, parent: Layout, t0: int, k: int):
+        self.parent = parent
+        self.desc = LayoutDesc.from_buffer_copy(parent.desc)
+        if parent.slot is not None:
+            self.desc.slot = parent.desc.slot + t0 * k * 4
+        self.desc.is_token_in_rank = parent.desc.is_token_in_rank + t0 * parent.num_tokens_per_rank.numel()
+
+
+def layout_tokens(layout: Layout, routing: Routing, t0: int, t1: int) -> LayoutView:
+    """View of `layout` for tokens [t0, t1) of `routing` (see Routing.tokens)."""
+    if not (0 <= t0 <= t1 <= routing.T):
+        raise ValueError("bad token range")
+    return LayoutView(layout, t0, routing.desc.num_topk)
 
 
 def ep_get_layout(routing: Routing, layout: Layout, stream=None) -> Layout:

@@ -287,6 +287,34 @@ def test_tc_pipeline_prefill_gpu_end_to_end():
     assert_combine_close(host(out), ref, True, "pipeline")
 
 
+def test_tc_dispatch_combine_in_token_chunks():
+    """Dispatch and combine called on token sub-ranges (offset views of the
+    routing, layout, x, weights and out) give the same bytes as one call."""
+    inp = inputs(2)
+    c = inp["cfg"]
+    x, idx, w = inp["x"], inp["topk_idx"], inp["topk_weights"]
+    ref_l = oracle.tc_layout(idx, c["E"], c["R"])
+    ref_y = oracle.tc_dispatch(x, idx, c["E"], ref_l)["recv"]
+    ref = oracle.tc_combine(ref_y, idx, c["E"], ref_l, w, out_dtype=W.BF16)
+    routing, lay, _ = gpu_tc_layout(idx, c["E"], c["R"])
+    n = c["T"] * c["K"]
+    xd, wd = to_dev(x, bf16=True), to_dev(w)
+    recv = torch.empty((n, c["H"]), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((c["T"], c["H"]), dtype=torch.bfloat16, device="cuda")
+    bounds = [0, 1, 1000, 1000, 2555, 4096]  # includes an empty and a one-token chunk
+    for t0, t1 in zip(bounds[:-1], bounds[1:]):
+        r = routing.tokens(t0, t1)
+        v = B.layout_tokens(lay, routing, t0, t1)
+        B.ep_dispatch(xd[t0:t1], r, v, recv, num_recv_rows=n)
+    for t0, t1 in zip(bounds[:-1], bounds[1:]):
+        r = routing.tokens(t0, t1)
+        v = B.layout_tokens(lay, routing, t0, t1)
+        B.ep_combine(recv, r, v, wd[t0:t1], out[t0:t1], num_y_rows=n)
+    assert B.ep_get_device_error(lay) == 0
+    assert np.array_equal(host(recv), ref_y)
+    assert np.array_equal(host(out), ref)
+
+
 def test_tc_combine_decode_padded():
     inp = inputs(3)
     c = inp["cfg"]
