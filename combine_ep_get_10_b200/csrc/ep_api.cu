@@ -53,14 +53,17 @@ size_t workspace_need(const ep_routing_desc_t* r)
 {
     if (r->routing == EP_ROUTING_EXPERT_CHOICE)
         return ep::ec_layout_workspace_bytes(r->num_tokens, r->num_experts, r->capacity);
-    return kWorkspaceHeaderBytes;
+    return ep::tc_layout_workspace_bytes(r->num_experts);
 }
 
-ep_status_t check_workspace(const ep_routing_desc_t* r, const ep_layout_t* l)
+// The layout needs its full workspace; dispatch and combine only the header
+// (the device error word).
+ep_status_t check_workspace(const ep_routing_desc_t* r, const ep_layout_t* l, bool full)
 {
     if (l == nullptr)
         return EP_ERR_INVALID_ARG;
-    if (l->workspace == nullptr || !aligned(l->workspace, 256) || l->workspace_bytes < workspace_need(r))
+    const size_t need = full ? workspace_need(r) : kWorkspaceHeaderBytes;
+    if (l->workspace == nullptr || !aligned(l->workspace, 256) || l->workspace_bytes < need)
         return EP_ERR_WORKSPACE;
     return EP_OK;
 }
@@ -122,7 +125,7 @@ ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* l
     ep_status_t st = check_routing(routing);
     if (st != EP_OK)
         return st;
-    st = check_workspace(routing, layout);
+    st = check_workspace(routing, layout, true);
     if (st != EP_OK)
         return st;
     const int32_t T = routing->num_tokens, E = routing->num_experts, R = routing->num_ranks;
@@ -150,7 +153,8 @@ ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* l
                              layout->num_tokens_per_rank,
                              layout->is_token_in_rank,
                              layout->slot,
-                             err};
+                             err,
+                             layout->workspace};
         return from_cuda(ep::launch_tc_layout(a, s));
     }
     if (layout->token_offsets == nullptr || layout->token_slots == nullptr || !aligned(layout->token_offsets, 4) ||
@@ -181,7 +185,7 @@ ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* 
         return st;
     if (routing->routing != EP_ROUTING_TOPK)
         return EP_ERR_INVALID_ARG;
-    st = check_workspace(routing, layout);
+    st = check_workspace(routing, layout, false);
     if (st != EP_OK)
         return st;
     st = check_rows(routing, layout, mode, max_tokens_per_expert, num_recv_rows);
@@ -226,7 +230,7 @@ ep_status_t ep_combine(const void* y, int32_t hidden, int64_t num_y_rows, const 
         return st;
     if (routing->routing != EP_ROUTING_TOPK)
         return EP_ERR_INVALID_ARG;
-    st = check_workspace(routing, layout);
+    st = check_workspace(routing, layout, false);
     if (st != EP_OK)
         return st;
     st = check_rows(routing, layout, mode, max_tokens_per_expert, num_y_rows);

@@ -29,7 +29,9 @@ struct TcLayoutLaunch {
     uint8_t* in_rank;
     int32_t* slot;
     uint32_t* err;
+    void* workspace; // header + per-CTA totals of the grid-wide kernel
 };
+size_t tc_layout_workspace_bytes(int64_t E);
 cudaError_t launch_tc_layout(const TcLayoutLaunch& a, cudaStream_t stream);
 
 struct EcLayoutLaunch {

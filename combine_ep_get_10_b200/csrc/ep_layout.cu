@@ -39,6 +39,10 @@ namespace {
 #ifndef EP_LAYOUT_MAX_CLUSTER
 #define EP_LAYOUT_MAX_CLUSTER 16
 #endif
+// from this many (token, k) pairs on, the grid-wide kernel is used
+#ifndef EP_LAYOUT_GRID_MIN_PAIRS
+#define EP_LAYOUT_GRID_MIN_PAIRS 8192
+#endif
 constexpr int kLayoutThreads = EP_LAYOUT_THREADS;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
 // 32-pair steps a warp keeps in registers: a full 16-CTA cluster holds 8192
@@ -339,6 +343,252 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(Tc
             write_rank_row(a, t, smask[t - t0]);
     }
     cluster_wait();
+}
+
+// ---------------------------------------------------------------------------
+// Token choice over the whole device: one CTA per SM (cooperative launch),
+// each with a contiguous token range.  Phase 1 is the cluster kernel's
+// (per-warp runs ranked with match.any, per-warp counters in shared memory);
+// each CTA then publishes its per-expert totals and per-rank token counts in
+// the workspace, all CTAs meet at a grid barrier (bounded wait), and every
+// CTA sums the totals of the CTAs before it to get its base per expert.  The
+// bookkeeping is spread over every SM instead of 16.
+constexpr int kGridThreads = 256;
+constexpr int kGridWarps = kGridThreads / 32;
+constexpr int kGridPrefetch = 8;                          // 32-pair steps per warp in registers
+constexpr int64_t kGridIds = kGridWarps * kGridPrefetch * 32; // pairs per CTA staged in shared memory
+constexpr int kGridMaxBlocks = 64;                      // workspace holds this many CTAs' totals
+constexpr int64_t kGridPairsPerCta = 1024;
+
+struct GridBar {
+    uint32_t* arrive;
+    uint32_t* generation;
+};
+
+// All CTAs of a cooperative launch meet here; false if the wait ran out.
+__device__ __forceinline__ bool grid_sync(GridBar bar, uint32_t nblocks, uint32_t* err, int* ok_smem)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        volatile uint32_t* gen = bar.generation;
+        const uint32_t g = *gen;
+        __threadfence();
+        bool ok = true;
+        if (atomicAdd(bar.arrive, 1u) == nblocks - 1) {
+            atomicExch(bar.arrive, 0u);
+            __threadfence();
+            atomicAdd(bar.generation, 1u);
+        } else {
+            const uint64_t t0 = global_timer_ns();
+            for (uint32_t i = 1; *gen == g; ++i) {
+                if ((i & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+                    flag_error(err, EP_DEVERR_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        __threadfence();
+        *ok_smem = ok ? 1 : 0;
+    }
+    __syncthreads();
+    return *ok_smem != 0;
+}
+
+__global__ void __launch_bounds__(kGridThreads) tc_layout_grid_kernel(TcArgs a, int32_t* tile_counts,
+                                                                      int32_t* tile_ranks, GridBar bar)
+{
+    const int G = static_cast<int>(gridDim.x);
+    const int b = static_cast<int>(blockIdx.x);
+    extern __shared__ __align__(16) int32_t smem[];
+    int32_t* wtab = smem;                      // [warps][E] per-warp counters, later prefixes
+    int32_t* srank = wtab + kGridWarps * a.E;  // [32] this CTA's tokens per rank
+    int32_t* sscan = srank + 32;               // [32] scan scratch
+    int* sid = sscan + 32;                     // [kGridIds] expert id of each pair (or -1)
+    uint32_t* smask = reinterpret_cast<uint32_t*>(sid + kGridIds); // [kGridIds] rank bits per token
+    int* ok_smem = reinterpret_cast<int*>(smask + kGridIds);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    for (int i = tid; i < kGridWarps * a.E; i += kGridThreads)
+        wtab[i] = 0;
+    if (tid < 32)
+        srank[tid] = 0;
+    __syncthreads();
+
+    const int64_t tpc = (static_cast<int64_t>(a.T) + G - 1) / G;
+    const int64_t t0 = min(static_cast<int64_t>(a.T), static_cast<int64_t>(b) * tpc);
+    const int64_t t1 = min(static_cast<int64_t>(a.T), t0 + tpc);
+    const int64_t p0 = t0 * a.K, p1 = t1 * a.K;
+    const int64_t ppw = ((p1 - p0 + kGridWarps - 1) / kGridWarps + 31) / 32 * 32;
+    const int64_t wb = min(p1, p0 + warp * ppw);
+    const int64_t we = min(p1, wb + ppw);
+    int32_t* mine = wtab + warp * a.E;
+    const uint32_t lanes_below = (1u << lane) - 1u;
+    bool bad = false;
+    const bool in_regs = (we - wb) <= 32 * kGridPrefetch;
+    const bool ids_in_smem = (p1 - p0) <= kGridIds;
+
+    // phase 1: per-warp stable ranks and counters (as in the cluster kernel)
+    int ev[kGridPrefetch];
+    int loc[kGridPrefetch];
+    for (int64_t start = wb; start < we; start += 32 * kGridPrefetch) {
+        int64_t raw[kGridPrefetch];
+#pragma unroll
+        for (int j = 0; j < kGridPrefetch; ++j) {
+            const int64_t p = start + j * 32 + lane;
+            raw[j] = p < we ? __ldg(a.topk_idx + p) : -1;
+        }
+#pragma unroll
+        for (int j = 0; j < kGridPrefetch; ++j) {
+            const bool ok = raw[j] >= 0 && raw[j] < a.E;
+            bad |= !ok && raw[j] != -1;
+            ev[j] = ok ? static_cast<int>(raw[j]) : -1;
+            const int64_t p = start + j * 32 + lane;
+            if (ids_in_smem && p < we)
+                sid[p - p0] = ev[j];
+        }
+        uint32_t peers[kGridPrefetch];
+#pragma unroll
+        for (int j = 0; j < kGridPrefetch; ++j)
+            peers[j] = start + j * 32 < we ? __match_any_sync(kFullMask, ev[j]) : 0u;
+#pragma unroll
+        for (int j = 0; j < kGridPrefetch; ++j) {
+            loc[j] = -1;
+            const int64_t step = start + j * 32;
+            if (step >= we)
+                break; // warp-uniform
+            const int64_t p = step + lane;
+            const int e = ev[j];
+            int prior = 0;
+            if (e >= 0)
+                prior = mine[e];
+            __syncwarp();
+            if (e >= 0) {
+                const int r = __popc(peers[j] & lanes_below);
+                loc[j] = prior + r;
+                if (r == 0)
+                    mine[e] = prior + __popc(peers[j]);
+            }
+            if (!in_regs && p < we)
+                a.slot[p] = loc[j];
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+
+    // phase 1b: rank membership of this CTA's tokens
+    for (int64_t tb = t0 + static_cast<int64_t>(warp) * 32; tb < t1; tb += kGridThreads) {
+        const int64_t t = tb + lane;
+        uint32_t mask = 0;
+        if (t < t1) {
+            if (ids_in_smem) {
+                const int* ids = sid + (t - t0) * a.K;
+                for (int k = 0; k < a.K; ++k)
+                    if (ids[k] >= 0)
+                        mask |= 1u << static_cast<uint32_t>(ids[k] / a.per_rank);
+                smask[t - t0] = mask;
+            } else {
+                for (int k = 0; k < a.K; ++k) {
+                    const int64_t e = __ldg(a.topk_idx + t * a.K + k);
+                    if (e >= 0 && e < a.E)
+                        mask |= 1u << static_cast<uint32_t>(e / a.per_rank);
+                }
+                write_rank_row(a, t, mask);
+            }
+        }
+        for (int r = 0; r < a.R; ++r) {
+            const int c = __popc(__ballot_sync(kFullMask, (mask >> r) & 1u));
+            if (lane == 0 && c)
+                atomicAdd(&srank[r], c);
+        }
+    }
+    if (__any_sync(kFullMask, bad) && lane == 0)
+        flag_error(a.err, EP_DEVERR_BAD_INDEX);
+    __syncthreads();
+
+    // phase 2: exclusive prefix down the warps; publish this CTA's totals
+    for (int e = tid; e < a.E; e += kGridThreads) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < kGridWarps; ++w) {
+            const int c = wtab[w * a.E + e];
+            wtab[w * a.E + e] = run;
+            run += c;
+        }
+        tile_counts[static_cast<int64_t>(b) * a.E + e] = run;
+    }
+    if (tid < a.R)
+        tile_ranks[b * 32 + tid] = srank[tid];
+    if (!grid_sync(bar, static_cast<uint32_t>(G), a.err, ok_smem))
+        return;
+
+    // phase 3: base per expert = totals of the CTAs before this one; CTA 0
+    // also forms the counts, offsets and rank totals
+    constexpr int kUnroll = 16;
+    int carry = 0;
+    for (int e0 = 0; e0 < a.E; e0 += kGridThreads) {
+        const int e = e0 + tid;
+        int bs = 0, all = 0;
+        if (e < a.E) {
+            for (int j0 = 0; j0 < G; j0 += kUnroll) {
+                int v[kUnroll];
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u)
+                    v[u] = j0 + u < G ? __ldcg(tile_counts + static_cast<int64_t>(j0 + u) * a.E + e) : 0;
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    bs += j0 + u < b ? v[u] : 0;
+                    all += v[u];
+                }
+            }
+#pragma unroll
+            for (int w = 0; w < kGridWarps; ++w)
+                wtab[w * a.E + e] += bs;
+        }
+        if (b == 0) {
+            int total = 0;
+            const int excl = block_exclusive_scan(e < a.E ? all : 0, sscan, total);
+            if (e < a.E) {
+                a.counts[e] = all;
+                a.offsets[e] = carry + excl;
+            }
+            carry += total;
+        }
+    }
+    if (b == 0) {
+        if (tid == 0)
+            a.offsets[a.E] = carry;
+        if (tid < a.R) {
+            int n = 0;
+            for (int j = 0; j < G; ++j)
+                n += __ldcg(tile_ranks + j * 32 + tid);
+            a.rank_counts[tid] = n;
+        }
+    }
+    __syncthreads();
+
+    // phase 4: slots and rank rows
+    if (in_regs) {
+#pragma unroll
+        for (int j = 0; j < kGridPrefetch; ++j) {
+            const int64_t p = wb + j * 32 + lane;
+            if (p < we)
+                a.slot[p] = loc[j] >= 0 ? loc[j] + mine[ev[j]] : -1;
+        }
+    } else {
+        for (int64_t step = wb; step < we; step += 32) {
+            const int64_t p = step + lane;
+            if (p < we) {
+                const int32_t l = a.slot[p];
+                if (l >= 0)
+                    a.slot[p] = l + mine[__ldg(a.topk_idx + p)];
+            }
+        }
+    }
+    if (ids_in_smem) {
+        for (int64_t t = t0 + tid; t < t1; t += kGridThreads)
+            write_rank_row(a, t, smask[t - t0]);
+    }
 }
 
 // ---------------------------------------------------------------- expert choice
@@ -835,6 +1085,59 @@ int max_ec_cluster()
 
 } // namespace
 
+size_t tc_layout_workspace_bytes(int64_t E)
+{
+    return kWorkspaceHeaderBytes + sizeof(int32_t) * static_cast<size_t>(kGridMaxBlocks) * (E + 32);
+}
+
+int grid_blocks_cache[64];
+
+cudaError_t launch_tc_layout_grid(const TcArgs& k, void* workspace, cudaStream_t stream)
+{
+    int dev = 0;
+    cudaError_t st = cudaGetDevice(&dev);
+    if (st != cudaSuccess)
+        return st;
+    const size_t smem = sizeof(int32_t) * (static_cast<size_t>(kGridWarps) * k.E + 64 + 2 * kGridIds + 4);
+    int resident = dev >= 0 && dev < 64 ? grid_blocks_cache[dev] : 0;
+    if (resident == 0) {
+        const size_t max_smem = sizeof(int32_t) * (static_cast<size_t>(kGridWarps) * kMaxTopkLayoutExperts + 64 +
+                                                   2 * kGridIds + 4);
+        st = cudaFuncSetAttribute(tc_layout_grid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(max_smem));
+        if (st != cudaSuccess)
+            return st;
+        int sms = 0, per_sm = 0;
+        st = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (st == cudaSuccess)
+            st = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc_layout_grid_kernel, kGridThreads, max_smem);
+        if (st != cudaSuccess)
+            return st;
+        resident = std::max(1, sms * per_sm);
+        if (dev >= 0 && dev < 64)
+            grid_blocks_cache[dev] = resident;
+    }
+    const int64_t pairs = static_cast<int64_t>(k.T) * k.K;
+    const int G = static_cast<int>(std::min<int64_t>(
+        {static_cast<int64_t>(kGridMaxBlocks), static_cast<int64_t>(resident),
+         std::max<int64_t>(1, (pairs + kGridPairsPerCta - 1) / kGridPairsPerCta)}));
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* tile_counts = reinterpret_cast<int32_t*>(ws + kWorkspaceHeaderBytes);
+    int32_t* tile_ranks = tile_counts + static_cast<int64_t>(kGridMaxBlocks) * k.E;
+    GridBar bar{reinterpret_cast<uint32_t*>(ws + 64), reinterpret_cast<uint32_t*>(ws + 128)};
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kGridThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tc_layout_grid_kernel, k, tile_counts, tile_ranks, bar);
+}
+
 cudaError_t launch_tc_layout(const TcLayoutLaunch& a, cudaStream_t stream)
 {
     TcArgs k{};
@@ -851,6 +1154,9 @@ cudaError_t launch_tc_layout(const TcLayoutLaunch& a, cudaStream_t stream)
     k.slot = a.slot;
     k.err = a.err;
     k.in_rank_words = (a.R % 4 == 0 && (reinterpret_cast<uintptr_t>(a.in_rank) & 3u) == 0) ? 1 : 0;
+
+    if (static_cast<int64_t>(a.T) * a.K >= EP_LAYOUT_GRID_MIN_PAIRS && a.workspace != nullptr)
+        return launch_tc_layout_grid(k, a.workspace, stream);
 
     const size_t smem =
         sizeof(int32_t) * (static_cast<size_t>(kLayoutWarps) * a.E + 3 * static_cast<size_t>(a.E) + 64 + 2 * kSmemIds);

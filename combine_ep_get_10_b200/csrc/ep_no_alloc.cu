@@ -119,7 +119,8 @@ ep_status_t ep_get_layout_no_alloc(const ep_routing_desc_t* routing, const ep_la
                              layout->num_tokens_per_rank,
                              layout->is_token_in_rank,
                              layout->slot,
-                             err};
+                             err,
+                             ws};
         return ep::launch_tc_layout(a, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
     }
     ep::EcLayoutLaunch a{routing->token_indices,

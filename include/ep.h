@@ -110,10 +110,13 @@ typedef struct {
  *                                      token, ascending; [0, token_offsets[T])
  *                                      is written
  *   workspace             device scratch of ep_workspace_bytes() bytes,
- *                         256-byte aligned.  Zero it once (ep_workspace_init)
- *                         before first use; calls leave it reusable.  One
- *                         workspace per stream: calls that share one must not
- *                         overlap on the GPU. */
+ *                         256-byte aligned: the device error word, the
+ *                         grid-barrier words of the token-choice layout and
+ *                         its per-CTA expert totals, or the expert-choice
+ *                         layout's per-token arrays.  Zero it once
+ *                         (ep_workspace_init) before first use; calls leave
+ *                         it reusable.  One workspace per stream: calls that
+ *                         share one must not overlap on the GPU. */
 typedef struct {
     int32_t* num_tokens_per_expert;
     int32_t* expert_offsets;
@@ -207,9 +210,9 @@ EP_API ep_status_t ep_combine_expert_choice(const void* y, int32_t hidden, const
  * a fixed array of EP_STATIC_WORKSPACE_BYTES inside the library, held by
  * every GPU that loads the library until the process exits.  A routing whose
  * ep_workspace_bytes() exceeds that size is rejected with EP_ERR_WORKSPACE
- * before anything is launched (token choice needs 256 bytes and always fits;
- * expert choice needs 256 + 4*(2*T + E*C) bytes rounded up to 256).  Nothing
- * is allocated or freed.
+ * before anything is launched (token choice needs 256 + 256*(E + 32) bytes,
+ * at most 270 KB, and always fits; expert choice needs 256 + 4*(2*T + E*C)
+ * bytes rounded up to 256).  Nothing is allocated or freed.
  *   device_error_flags  optional device pointer to one uint32: zeroed at the
  *                       start of the call, then receives the EP_DEVERR_* bits
  *                       the layout kernels raise (NULL: not reported).

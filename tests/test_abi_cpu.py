@@ -58,7 +58,8 @@ def _ec_desc(T=16, E=8, C=4, R=2, ptr=0x1000):
 
 
 def test_workspace_bytes(L):
-    assert L.ep_workspace_bytes(ctypes.byref(_topk_desc())) == 256
+    n_tc = L.ep_workspace_bytes(ctypes.byref(_topk_desc(E=8)))
+    assert n_tc >= 256 + 4 * 64 * (8 + 32) and n_tc % 256 == 0
     n = L.ep_workspace_bytes(ctypes.byref(_ec_desc(T=1000, E=128, C=128)))
     assert n >= 256 + 4 * (2 * 1000 + 128 * 128) and n % 256 == 0
     assert L.ep_workspace_bytes(ctypes.byref(_topk_desc(E=9, R=2))) == 0  # E % R != 0
