@@ -6,9 +6,10 @@
 // exactly once by the TMA engine (cp.async.bulk global->shared, completion on
 // an mbarrier) and written to every destination row by bulk stores
 // (cp.async.bulk shared->global), one per destination, issued by different
-// lanes.  A CTA is one warp and moves one (row, chunk) item; up to 32 CTAs
+// lanes.  A CTA is one warp and moves one (row, chunk) item; up to 28 CTAs
 // per SM keep ~200 KB of copies in flight per SM and the block scheduler
-// balances the tail.
+// balances the tail.  (A persistent variant streaming each CTA's items
+// through a 3-4 stage ring measured 10-15% slower.)
 //
 // FP8 dispatch (README, "Quantization Modes in Normal Dispatch"; one fp32
 // scale per 128 channels): one CTA per token quantises the row once in
