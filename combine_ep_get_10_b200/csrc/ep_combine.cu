@@ -55,6 +55,9 @@ constexpr int kTcGroup = EP_COMBINE_GROUP;
 #ifndef EP_COMBINE_PERSIST_EC
 #define EP_COMBINE_PERSIST_EC 0
 #endif
+#ifndef EP_COMBINE_HEAVY_FIRST
+#define EP_COMBINE_HEAVY_FIRST 1
+#endif
 constexpr int kEcVec = EP_COMBINE_EC_VEC;
 constexpr int kEcGroup = EP_COMBINE_EC_GROUP;
 
@@ -75,7 +78,13 @@ struct CombineArgs {
     void* out;
     uint32_t* err;
     int64_t warp_base; // first (token, segment) item of this launch
+    int32_t heavy_first; // expert choice: list heavy tokens first (persistent launch)
 };
+
+// expert choice, heavy first (see combine_kernel)
+constexpr int kHeavyDeg = 16;
+constexpr int kMaxHeavy = 2048;
+constexpr int kHeavyFirstMaxT = 65536;
 
 template <bool kExpertChoice>
 __device__ __forceinline__ void entry(const CombineArgs& a, int64_t t, int64_t beg, int j, int64_t& row, float& w,
@@ -118,29 +127,94 @@ __device__ __forceinline__ void entry(const CombineArgs& a, int64_t t, int64_t b
     }
 }
 
+// Expert choice: virtual item g -> (token, segment); the first heavy_items
+// items are the listed heavy tokens' segments, then every token in order.
+__device__ __forceinline__ void item_token(int64_t g, int64_t heavy_items, int nseg, const int* heavy, int64_t& t,
+                                           int& seg)
+{
+    if (g < heavy_items) {
+        t = heavy[g / nseg];
+        seg = static_cast<int>(g % nseg);
+    } else {
+        t = (g - heavy_items) / nseg;
+        seg = static_cast<int>((g - heavy_items) - t * nseg);
+    }
+}
+
 template <bool kExpertChoice, bool kOutF32, int kVecPerLane, int kGroup>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 {
     constexpr int kSegVec = 32 * kVecPerLane;
     // token choice lists are short (K); expert-choice lists reach E entries
-    constexpr int kLookup = kExpertChoice ? 4 : 1;
+    constexpr int kLookup = kExpertChoice ? 2 : 1;
     const int lane = threadIdx.x & 31;
-    const int64_t items = static_cast<int64_t>(a.T) * a.nseg;
+    const int warp = threadIdx.x >> 5;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarpsPerCta;
     uint32_t errbits = 0;
-    for (int64_t gw = a.warp_base + static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
-         gw < items; gw += stride) {
-        const int64_t t = gw / a.nseg;
-        const int seg = static_cast<int>(gw - t * a.nseg);
 
+    // Expert choice, heavy first: every CTA lists, in token order, the tokens
+    // with at least kHeavyDeg picks (the same list in every CTA); warps take
+    // their items before all others, so the long lists start in the first
+    // wave and overlap the light work instead of trailing it.
+    __shared__ int s_heavy[kMaxHeavy];
+    __shared__ uint32_t s_flags[kHeavyFirstMaxT / 32];
+    __shared__ int s_wbase[kWarpsPerCta + 1];
+    int n_heavy = 0;
+    if (kExpertChoice && a.heavy_first) {
+        const int64_t per_warp = ((static_cast<int64_t>(a.T) + kWarpsPerCta * 32 - 1) / (kWarpsPerCta * 32)) * 32;
+        const int64_t w0 = min(static_cast<int64_t>(a.T), warp * per_warp);
+        const int64_t w1 = min(static_cast<int64_t>(a.T), w0 + per_warp);
+        int cnt = 0;
+        for (int64_t base = w0; base < w1; base += 32) {
+            const int64_t t = base + lane;
+            const bool heavy = t < w1 && __ldg(a.token_offsets + t + 1) - __ldg(a.token_offsets + t) >= kHeavyDeg;
+            const uint32_t bits = __ballot_sync(kFullMask, heavy);
+            if (lane == 0)
+                s_flags[base / 32] = bits;
+            cnt += __popc(bits);
+        }
+        if (lane == 0)
+            s_wbase[warp + 1] = cnt;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            s_wbase[0] = 0;
+            for (int w = 0; w < kWarpsPerCta; ++w)
+                s_wbase[w + 1] += s_wbase[w];
+        }
+        __syncthreads();
+        n_heavy = s_wbase[kWarpsPerCta];
+        if (n_heavy <= kMaxHeavy) {
+            int pos = s_wbase[warp];
+            for (int64_t base = w0; base < w1; base += 32) {
+                const uint32_t bits = s_flags[base / 32];
+                if ((bits >> lane) & 1u)
+                    s_heavy[pos + __popc(bits & ((1u << lane) - 1u))] = static_cast<int>(base + lane);
+                pos += __popc(bits);
+            }
+        } else {
+            n_heavy = 0; // too many to list: plain token order
+        }
+        __syncthreads();
+    }
+    const int64_t heavy_items = static_cast<int64_t>(n_heavy) * a.nseg;
+    const int64_t items = heavy_items + static_cast<int64_t>(a.T) * a.nseg;
+    for (int64_t gw = a.warp_base + static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + warp; gw < items;
+         gw += stride) {
+        int64_t t;
+        int seg;
         int64_t beg = 0;
         int n;
-        if (kExpertChoice) {
+        if constexpr (kExpertChoice) {
+            item_token(gw, heavy_items, a.nseg, s_heavy, t, seg);
             beg = __ldg(a.token_offsets + t);
             n = __ldg(a.token_offsets + t + 1) - static_cast<int>(beg);
         } else {
+            t = gw / a.nseg;
+            seg = static_cast<int>(gw - t * a.nseg);
             n = a.K;
         }
+        if (kExpertChoice && n_heavy > 0 && gw >= heavy_items && n >= kHeavyDeg)
+            continue; // done in the heavy phase
 
         int v[kVecPerLane];
         bool vin[kVecPerLane];
@@ -267,8 +341,9 @@ cudaError_t launch_combine(CombineArgs k, bool out_f32, bool persistent, cudaStr
     const int64_t warps = static_cast<int64_t>(k.T) * k.nseg;
     int64_t blocks = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
     if (persistent) {
-        static int cache[64];
-        const int64_t res = resident_blocks(combine_kernel<kExpertChoice, false, kVec, kGrp>, cache);
+        static int cache_bf16[64], cache_f32[64];
+        const int64_t res = out_f32 ? resident_blocks(combine_kernel<kExpertChoice, true, kVec, kGrp>, cache_f32)
+                                    : resident_blocks(combine_kernel<kExpertChoice, false, kVec, kGrp>, cache_bf16);
         if (res > 0)
             blocks = std::min(blocks, res);
     }
@@ -322,7 +397,9 @@ cudaError_t launch_ec_combine(const EcCombineLaunch& a, cudaStream_t stream)
     k.expert_weights = a.expert_weights;
     k.out = a.out;
     k.err = a.err;
-    return launch_combine<true, kEcVec, kEcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_EC != 0, stream);
+    k.heavy_first = EP_COMBINE_HEAVY_FIRST && a.T <= kHeavyFirstMaxT ? 1 : 0;
+    return launch_combine<true, kEcVec, kEcGroup>(k, a.out_dtype == EP_FP32,
+                                                  k.heavy_first != 0 || EP_COMBINE_PERSIST_EC != 0, stream);
 }
 
 } // namespace ep
