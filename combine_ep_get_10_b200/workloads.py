@@ -36,6 +36,7 @@ from __future__ import annotations
 import numpy as np
 
 BF16, FP32, FP8_E4M3 = 0, 1, 2
+INT8_PER_TOKEN, FP8_E4M3_PER_TOKEN, MXFP8_E4M3, MXFP8_E5M2, MXFP4_E2M1 = 3, 4, 5, 6, 7
 COMPACT, PADDED = 0, 1
 
 CONFIGS = {

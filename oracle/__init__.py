@@ -23,6 +23,8 @@ _LIB = os.path.join(_HERE, "libep_oracle.so")
 
 # numeric codes shared with the public interface (dtype / buffer layout)
 BF16, FP32, FP8_E4M3 = 0, 1, 2
+INT8_PER_TOKEN, FP8_E4M3_PER_TOKEN, MXFP8_E4M3, MXFP8_E5M2, MXFP4_E2M1 = 3, 4, 5, 6, 7
+QUANT_DTYPES = (FP8_E4M3, INT8_PER_TOKEN, FP8_E4M3_PER_TOKEN, MXFP8_E4M3, MXFP8_E5M2, MXFP4_E2M1)
 COMPACT, PADDED = 0, 1
 
 _lib = None
@@ -53,12 +55,26 @@ def load(path: str):
     L.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
     L.oracle_e4m3_to_f32.restype = ctypes.c_float
     L.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
-    for name in ("oracle_f32_to_bf16_array", "oracle_f32_to_e4m3_array", "oracle_e4m3_to_f32_array"):
+    for name in ("oracle_f32_to_bf16_array", "oracle_f32_to_e4m3_array", "oracle_e4m3_to_f32_array",
+                 "oracle_f32_to_e5m2_array", "oracle_e5m2_to_f32_array", "oracle_f32_to_e2m1_array",
+                 "oracle_e2m1_to_f32_array", "oracle_f32_to_int8_array"):
         fn = getattr(L, name)
         fn.restype = None
         fn.argtypes = [P, P, i64]
-    L.oracle_fp8_quant_row.restype = None
-    L.oracle_fp8_quant_row.argtypes = [P, i32, P, P]
+    for name in ("oracle_fp8_quant_row", "oracle_int8_quant_row", "oracle_fp8_pertoken_quant_row"):
+        fn = getattr(L, name)
+        fn.restype = None
+        fn.argtypes = [P, i32, P, P]
+    L.oracle_mx_quant_row.restype = None
+    L.oracle_mx_quant_row.argtypes = [i32, P, i32, P, P]
+    L.oracle_quant_row.restype = None
+    L.oracle_quant_row.argtypes = [i32, P, i32, P, P]
+    L.oracle_mx_shared_exp.restype = i32
+    L.oracle_mx_shared_exp.argtypes = [ctypes.c_float, i32]
+    L.oracle_row_code_bytes.restype = i64
+    L.oracle_row_code_bytes.argtypes = [i32, i32]
+    L.oracle_row_scale_bytes.restype = i64
+    L.oracle_row_scale_bytes.argtypes = [i32, i32]
     L.oracle_tc_layout.restype = i64
     L.oracle_tc_layout.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P]
     L.oracle_tc_dispatch.restype = i64
@@ -134,6 +150,68 @@ def fp8_quant_row(xrow_bits):
     return q, s
 
 
+def _array_fn(name, in_dtype, out_dtype):
+    def fn(a):
+        a = _c(a, in_dtype)
+        out = np.empty(a.shape, out_dtype)
+        getattr(lib(), name)(_p(a), _p(out), a.size)
+        return out
+
+    fn.__name__ = name.replace("oracle_", "").replace("_array", "")
+    return fn
+
+
+f32_to_e5m2 = _array_fn("oracle_f32_to_e5m2_array", np.float32, np.uint8)
+e5m2_to_f32 = _array_fn("oracle_e5m2_to_f32_array", np.uint8, np.float32)
+f32_to_e2m1 = _array_fn("oracle_f32_to_e2m1_array", np.float32, np.uint8)  # 4-bit codes, one per byte
+e2m1_to_f32 = _array_fn("oracle_e2m1_to_f32_array", np.uint8, np.float32)
+f32_to_int8 = _array_fn("oracle_f32_to_int8_array", np.float32, np.int8)
+
+
+def row_code_bytes(dtype, hidden):
+    return int(lib().oracle_row_code_bytes(int(dtype), int(hidden)))
+
+
+def row_scale_bytes(dtype, hidden):
+    return int(lib().oracle_row_scale_bytes(int(dtype), int(hidden)))
+
+
+def scale_array(dtype, rows, hidden):
+    """Zeroed scale buffer of the layout the output format uses."""
+    if dtype == FP8_E4M3:
+        return np.zeros((rows, hidden // 128), np.float32)
+    if dtype in (INT8_PER_TOKEN, FP8_E4M3_PER_TOKEN):
+        return np.zeros(rows, np.float32)
+    if dtype in (MXFP8_E4M3, MXFP8_E5M2, MXFP4_E2M1):
+        return np.zeros((rows, hidden // 32), np.uint8)
+    return None
+
+
+def code_array(dtype, rows, hidden):
+    """Zeroed code buffer of the layout the output format uses."""
+    if dtype == BF16:
+        return np.zeros((rows, hidden), np.uint16)
+    if dtype == INT8_PER_TOKEN:
+        return np.zeros((rows, hidden), np.int8)
+    return np.zeros((rows, row_code_bytes(dtype, hidden)), np.uint8)
+
+
+def quant_row(dtype, xrow_bits):
+    """One bf16 row -> (codes, scales) in output format `dtype` (any of
+    QUANT_DTYPES); shapes as one row of code_array / scale_array."""
+    x = _c(xrow_bits, np.uint16)
+    H = x.size
+    q = code_array(dtype, 1, H)[0]
+    s = scale_array(dtype, 1, H)
+    s = s[0] if s.ndim == 2 else s
+    lib().oracle_quant_row(int(dtype), _p(x), H, _p(q), _p(s))
+    return q, s
+
+
+def mx_shared_exp(amax, emax_elem):
+    return int(lib().oracle_mx_shared_exp(float(amax), int(emax_elem)))
+
+
 # ---------------------------------------------------------- token choice
 def tc_layout(topk_idx, num_experts, num_ranks):
     idx = _c(topk_idx, np.int64)
@@ -166,12 +244,8 @@ def tc_dispatch(x_bits, topk_idx, num_experts, layout, mode=COMPACT, max_tokens=
     if num_recv_rows is None:
         num_recv_rows = E * max_tokens if mode == PADDED else int(offs[E])
     rows = int(num_recv_rows)
-    if out_dtype == FP8_E4M3:
-        recv = np.zeros((rows, H), np.uint8)
-        scales = np.zeros((rows, H // 128), np.float32)
-    else:
-        recv = np.zeros((rows, H), np.uint16)
-        scales = None
+    recv = code_array(out_dtype, rows, H)
+    scales = scale_array(out_dtype, rows, H)
     src = np.full(rows, -1, np.int32) if want_src else None
     wts = np.zeros(rows, np.float32) if want_weights else None
     w = _c(topk_weights, np.float32) if topk_weights is not None else None

@@ -27,13 +27,17 @@
  * in the design notes): order inside an expert is ascending token, then
  * ascending k; logical rank r owns experts [r*E/R, (r+1)*E/R); one copy
  * per (token, expert) pair; FP8 scale = amax/448 per 128 channels and
- * q = e4m3_rne_satfinite(x * (448/amax)); combine is an fmaf chain from
+ * q = e4m3_rne_satfinite(x * (448/amax)); the other quantisation modes of
+ * the README table are read in the same way (dynamic symmetric scale from
+ * the amax of the row for the per-token modes; the OCP Microscaling shared
+ * exponent for the MX modes, see below); combine is an fmaf chain from
  * 0.0f in ascending k; an expert-choice token's slots are taken in
  * ascending slot id s = e*C + c.
  *
  * Parity pins: every function here is checked by the CPU test-suite
  * against brute-force enumeration, closed forms, invariants and library
- * conversions (torch's bf16 / float8_e4m3fn casts); none is unpinned.
+ * conversions (torch's bf16 / float8_e4m3fn / float8_e5m2 casts); none is
+ * unpinned.
  */
 #include <math.h>
 #include <stdint.h>
@@ -46,6 +50,11 @@
 #define OR_BF16 0
 #define OR_FP32 1
 #define OR_FP8_E4M3 2
+#define OR_INT8_PER_TOKEN 3
+#define OR_FP8_E4M3_PER_TOKEN 4
+#define OR_MXFP8_E4M3 5
+#define OR_MXFP8_E5M2 6
+#define OR_MXFP4_E2M1 7
 #define OR_COMPACT 0
 #define OR_PADDED 1
 
@@ -129,6 +138,150 @@ uint8_t oracle_f32_to_e4m3(float f)
     return (uint8_t)(sign | (uint8_t)code);
 }
 
+/* ---------------------------------------------------------------------
+ * More element formats of the README's quantization table
+ * ("Quantization Modes in Normal Dispatch": int8, float8_e5m2,
+ * float4_e2m1fn_x2, float8_e8m0fnu scales).  The bit layouts are those of
+ * the OCP 8-bit floating point and Microscaling (MX) v1.0 specifications.
+ *
+ * float8 e5m2: 1 sign, 5 exponent (bias 15), 2 mantissa bits; exponent
+ * field 31 holds infinities and NaNs; largest finite 1.75 * 2^15 = 57344;
+ * exponent field 0 encodes subnormals m/4 * 2^-14.
+ * float4 e2m1: 1 sign, 2 exponent (bias 1), 1 mantissa bit; no infinities
+ * or NaN; the magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+ * int8: two's complement; the symmetric range [-127, 127] is used.
+ * ------------------------------------------------------------------- */
+
+float oracle_e5m2_to_f32(uint8_t c)
+{
+    int s = (c >> 7) & 1;
+    int e = (c >> 2) & 0x1F;
+    int m = c & 3;
+    float v;
+    if (e == 0x1F)
+        v = (m == 0) ? INFINITY : NAN;
+    else if (e == 0)
+        v = ldexpf((float)m / 4.0f, -14);
+    else
+        v = ldexpf(1.0f + (float)m / 4.0f, e - 15);
+    return s ? -v : v;
+}
+
+/* Round to nearest e5m2 value, ties to even mantissa; magnitudes above
+ * 57344 saturate to 57344 (satfinite). */
+uint8_t oracle_f32_to_e5m2(float f)
+{
+    uint8_t sign = signbit(f) ? 0x80 : 0x00;
+    float a = fabsf(f);
+    if (isnan(f))
+        return (uint8_t)(sign | 0x7F);
+    if (a == 0.0f)
+        return sign;
+    if (a > 57344.0f)
+        return (uint8_t)(sign | 0x7B);
+    if (a < ldexpf(1.0f, -14)) {
+        /* subnormal range: value = m * 2^-16, m in [0, 4]; m == 4 is the
+         * smallest normal (code 0x04) */
+        int m = (int)nearbyintf(ldexpf(a, 16));
+        return (uint8_t)(sign | (uint8_t)m);
+    }
+    int ex;
+    float fr = frexpf(a, &ex); /* a = fr * 2^ex, fr in [0.5, 1) */
+    int unb = ex - 1;
+    int m = (int)nearbyintf(fr * 8.0f); /* significand in units of 1/4: [4, 8] */
+    if (m == 8) {
+        m = 4;
+        unb += 1;
+    }
+    int code = ((unb + 15) << 2) | (m - 4);
+    if (code > 0x7B)
+        code = 0x7B;
+    return (uint8_t)(sign | (uint8_t)code);
+}
+
+/* 4-bit code (low nibble) -> value. */
+float oracle_e2m1_to_f32(uint8_t c)
+{
+    int s = (c >> 3) & 1;
+    int e = (c >> 1) & 3;
+    int m = c & 1;
+    float v = (e == 0) ? 0.5f * (float)m : ldexpf(1.0f + 0.5f * (float)m, e - 1);
+    return s ? -v : v;
+}
+
+/* Round to nearest e2m1 value, ties to even mantissa; magnitudes above 6
+ * saturate to 6.  Returns the 4-bit code in the low nibble. */
+uint8_t oracle_f32_to_e2m1(float f)
+{
+    uint8_t sign = signbit(f) ? 0x8 : 0x0;
+    float a = fabsf(f);
+    if (isnan(f) || a > 6.0f)
+        return (uint8_t)(sign | 0x7);
+    if (a == 0.0f)
+        return sign;
+    if (a < 1.0f) {
+        /* subnormal range: value = m * 0.5, m in [0, 2]; m == 2 is 1.0 (code 2) */
+        int m = (int)nearbyintf(ldexpf(a, 1));
+        return (uint8_t)(sign | (uint8_t)m);
+    }
+    int ex;
+    float fr = frexpf(a, &ex);
+    int unb = ex - 1;
+    int m = (int)nearbyintf(fr * 4.0f); /* significand in units of 1/2: [2, 4] */
+    if (m == 4) {
+        m = 2;
+        unb += 1;
+    }
+    int code = ((unb + 1) << 1) | (m - 2);
+    if (code > 7)
+        code = 7;
+    return (uint8_t)(sign | (uint8_t)code);
+}
+
+/* Round to nearest integer, ties to even (the default rounding mode of
+ * nearbyintf), clamped to [-127, 127]. */
+int8_t oracle_f32_to_int8(float f)
+{
+    if (isnan(f))
+        return 0;
+    float r = nearbyintf(f);
+    if (r > 127.0f)
+        r = 127.0f;
+    if (r < -127.0f)
+        r = -127.0f;
+    return (int8_t)r;
+}
+
+void oracle_f32_to_e5m2_array(const float* in, uint8_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f32_to_e5m2(in[i]);
+}
+
+void oracle_e5m2_to_f32_array(const uint8_t* in, float* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_e5m2_to_f32(in[i]);
+}
+
+void oracle_f32_to_e2m1_array(const float* in, uint8_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f32_to_e2m1(in[i]);
+}
+
+void oracle_e2m1_to_f32_array(const uint8_t* in, float* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_e2m1_to_f32(in[i]);
+}
+
+void oracle_f32_to_int8_array(const float* in, int8_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f32_to_int8(in[i]);
+}
+
 void oracle_f32_to_bf16_array(const float* in, uint16_t* out, int64_t n)
 {
     for (int64_t i = 0; i < n; ++i)
@@ -183,6 +336,160 @@ void oracle_fp8_quant_row(const uint16_t* xrow, int32_t hidden, uint8_t* q, floa
             float prod = xv * inv;
             q[g * 128 + i] = oracle_f32_to_e4m3(prod);
         }
+    }
+}
+
+/* ---------------------------------------------------------------------
+ * Per-token modes of the README table: "int8" (INT8 dynamic, per-token
+ * float32 scale) and "pertoken_fp8_e4m3" (scalar FP8, per-token float32
+ * scale).  One scale for the whole row, from the amax of the row, in the
+ * same way as the 128-channel FP8 mode: scale = amax / qmax, inv = qmax /
+ * amax (clamped to FLT_MAX), q = encode(x * inv), with qmax = 127 (int8,
+ * round to nearest even, clamped to [-127, 127]) or 448 (e4m3
+ * satfinite).  amax == 0 gives scale 0 and all-zero codes.
+ * ------------------------------------------------------------------- */
+static float row_amax(const uint16_t* xrow, int32_t n)
+{
+    float amax = 0.0f;
+    for (int32_t i = 0; i < n; ++i) {
+        float v = fabsf(oracle_bf16_to_f32(xrow[i]));
+        if (v > amax)
+            amax = v;
+    }
+    return amax;
+}
+
+void oracle_int8_quant_row(const uint16_t* xrow, int32_t hidden, int8_t* q, float* scale)
+{
+    float amax = row_amax(xrow, hidden);
+    if (amax == 0.0f) {
+        *scale = 0.0f;
+        for (int32_t i = 0; i < hidden; ++i)
+            q[i] = 0;
+        return;
+    }
+    float inv = 127.0f / amax;
+    if (inv > FLT_MAX)
+        inv = FLT_MAX;
+    *scale = amax / 127.0f;
+    for (int32_t i = 0; i < hidden; ++i)
+        q[i] = oracle_f32_to_int8(oracle_bf16_to_f32(xrow[i]) * inv);
+}
+
+void oracle_fp8_pertoken_quant_row(const uint16_t* xrow, int32_t hidden, uint8_t* q, float* scale)
+{
+    float amax = row_amax(xrow, hidden);
+    if (amax == 0.0f) {
+        *scale = 0.0f;
+        for (int32_t i = 0; i < hidden; ++i)
+            q[i] = 0x00;
+        return;
+    }
+    float inv = 448.0f / amax;
+    if (inv > FLT_MAX)
+        inv = FLT_MAX;
+    *scale = amax / 448.0f;
+    for (int32_t i = 0; i < hidden; ++i)
+        q[i] = oracle_f32_to_e4m3(oracle_bf16_to_f32(xrow[i]) * inv);
+}
+
+/* ---------------------------------------------------------------------
+ * MX modes of the README table ("mx_fp8_e4m3", "mx_fp8_e5m2",
+ * "mx_fp4_e2m1": per 32 elements, float8_e8m0fnu scale).  The README gives
+ * the formats and the block size but not the scale rule; the rule here is
+ * the OCP Microscaling v1.0 conversion: for each block of 32 elements,
+ *   X = floor(log2(amax)) - emax,  emax = exponent of the element format's
+ *       largest normal (e4m3: 8, e5m2: 15, e2m1: 2),
+ * clamped to the E8M0 range [-127, 127] (amax == 0 gives -127); the scale
+ * byte is X + 127 (the block's scale is 2^X) and every element becomes
+ * encode(x * 2^-X), rounding to nearest even and saturating at the element
+ * format's largest finite value.  e2m1 codes are packed two per byte,
+ * element 2i in the low nibble and 2i+1 in the high nibble.
+ * ------------------------------------------------------------------- */
+int32_t oracle_mx_shared_exp(float amax, int32_t emax_elem)
+{
+    if (amax == 0.0f)
+        return -127;
+    int ex;
+    frexpf(amax, &ex); /* amax = fr * 2^ex, fr in [0.5, 1): floor(log2 amax) = ex - 1 */
+    int32_t X = (ex - 1) - emax_elem;
+    if (X < -127)
+        X = -127;
+    if (X > 127)
+        X = 127;
+    return X;
+}
+
+void oracle_mx_quant_row(int32_t dtype, const uint16_t* xrow, int32_t hidden, uint8_t* q, uint8_t* scales)
+{
+    int32_t emax = dtype == OR_MXFP8_E4M3 ? 8 : (dtype == OR_MXFP8_E5M2 ? 15 : 2);
+    for (int32_t g = 0; g < hidden / 32; ++g) {
+        float amax = row_amax(xrow + g * 32, 32);
+        int32_t X = oracle_mx_shared_exp(amax, emax);
+        scales[g] = (uint8_t)(X + 127);
+        for (int32_t i = 0; i < 32; ++i) {
+            int32_t h = g * 32 + i;
+            float v = ldexpf(oracle_bf16_to_f32(xrow[h]), -X); /* exact: a power-of-two scaling */
+            if (dtype == OR_MXFP8_E4M3) {
+                q[h] = oracle_f32_to_e4m3(v);
+            } else if (dtype == OR_MXFP8_E5M2) {
+                q[h] = oracle_f32_to_e5m2(v);
+            } else {
+                uint8_t c = oracle_f32_to_e2m1(v);
+                if (h % 2 == 0)
+                    q[h / 2] = c;
+                else
+                    q[h / 2] = (uint8_t)(q[h / 2] | (c << 4));
+            }
+        }
+    }
+}
+
+/* Bytes of codes and of scales that one quantised row of `hidden`
+ * channels takes in each output format (0 scale bytes for bf16). */
+int64_t oracle_row_code_bytes(int32_t dtype, int32_t hidden)
+{
+    if (dtype == OR_BF16)
+        return 2 * (int64_t)hidden;
+    if (dtype == OR_MXFP4_E2M1)
+        return hidden / 2;
+    return hidden;
+}
+
+int64_t oracle_row_scale_bytes(int32_t dtype, int32_t hidden)
+{
+    switch (dtype) {
+    case OR_FP8_E4M3:
+        return 4 * (int64_t)(hidden / 128);
+    case OR_INT8_PER_TOKEN:
+    case OR_FP8_E4M3_PER_TOKEN:
+        return 4;
+    case OR_MXFP8_E4M3:
+    case OR_MXFP8_E5M2:
+    case OR_MXFP4_E2M1:
+        return hidden / 32;
+    default:
+        return 0;
+    }
+}
+
+/* One bf16 row in output format `dtype`: codes into q, scales into
+ * `scales` (layouts as above). */
+void oracle_quant_row(int32_t dtype, const uint16_t* xrow, int32_t hidden, uint8_t* q, void* scales)
+{
+    switch (dtype) {
+    case OR_FP8_E4M3:
+        oracle_fp8_quant_row(xrow, hidden, q, (float*)scales);
+        break;
+    case OR_INT8_PER_TOKEN:
+        oracle_int8_quant_row(xrow, hidden, (int8_t*)q, (float*)scales);
+        break;
+    case OR_FP8_E4M3_PER_TOKEN:
+        oracle_fp8_pertoken_quant_row(xrow, hidden, q, (float*)scales);
+        break;
+    default:
+        oracle_mx_quant_row(dtype, xrow, hidden, q, (uint8_t*)scales);
+        break;
     }
 }
 
@@ -257,26 +564,28 @@ static int64_t pair_row(int64_t e, int32_t s, int32_t E, const int32_t* offsets,
 /* ---------------------------------------------------------------------
  * Token-choice dispatch.  [README] "API Overview", dispatch (normal) and
  * low_latency_dispatch (per-expert buffers of num_max_dispatch_tokens_per
- * _rank rows); "Quantization Modes in Normal Dispatch" (bf16 or FP8
- * payload with float32 scales).  For every routed pair (t,k), row
- * pair_row(...) of recv receives x[t] (bf16 copy) or its FP8 encoding
- * with scales; recv_src[row] = t and recv_weights[row] = w[t,k] when those
+ * _rank rows); "Quantization Modes in Normal Dispatch" (bf16 payload, or
+ * one of the quantised formats above with its scales).  For every routed
+ * pair (t,k), row pair_row(...) of recv receives x[t] (bf16 copy) or its
+ * encoding by oracle_quant_row, and the same row of recv_scales its
+ * scales; recv_src[row] = t and recv_weights[row] = w[t,k] when those
  * outputs are requested.  Returns the number of pairs that had no room
  * (padded slot >= max_tokens, or row beyond num_recv_rows).
  * ------------------------------------------------------------------- */
 int64_t oracle_tc_dispatch(const uint16_t* x, int32_t T, int32_t H, const int64_t* topk_idx, int32_t K,
                            int32_t E, const int32_t* slot, const int32_t* offsets, int32_t mode,
                            int32_t max_tokens, int64_t num_recv_rows, int32_t out_dtype,
-                           const float* topk_weights, void* recv, float* recv_scales,
+                           const float* topk_weights, void* recv, void* recv_scales,
                            int32_t* recv_src, float* recv_weights)
 {
     int64_t overflow = 0;
-    int32_t groups = H / 128;
+    int64_t code_bytes = oracle_row_code_bytes(out_dtype, H);
+    int64_t scale_bytes = oracle_row_scale_bytes(out_dtype, H);
     uint8_t* qrow = NULL;
-    float* srow = NULL;
-    if (out_dtype == OR_FP8_E4M3) {
-        qrow = (uint8_t*)malloc((size_t)H);
-        srow = (float*)malloc(sizeof(float) * (size_t)(groups > 0 ? groups : 1));
+    uint8_t* srow = NULL;
+    if (out_dtype != OR_BF16) {
+        qrow = (uint8_t*)malloc((size_t)code_bytes + 1);
+        srow = (uint8_t*)malloc((size_t)scale_bytes + 4);
     }
     for (int32_t t = 0; t < T; ++t) {
         for (int32_t k = 0; k < K; ++k) {
@@ -289,10 +598,10 @@ int64_t oracle_tc_dispatch(const uint16_t* x, int32_t T, int32_t H, const int64_
             }
             if (row < 0)
                 continue;
-            if (out_dtype == OR_FP8_E4M3) {
-                oracle_fp8_quant_row(x + (int64_t)t * H, H, qrow, srow);
-                memcpy((uint8_t*)recv + row * H, qrow, (size_t)H);
-                memcpy(recv_scales + row * groups, srow, sizeof(float) * (size_t)groups);
+            if (out_dtype != OR_BF16) {
+                oracle_quant_row(out_dtype, x + (int64_t)t * H, H, qrow, srow);
+                memcpy((uint8_t*)recv + row * code_bytes, qrow, (size_t)code_bytes);
+                memcpy((uint8_t*)recv_scales + row * scale_bytes, srow, (size_t)scale_bytes);
             } else {
                 memcpy((uint16_t*)recv + row * H, x + (int64_t)t * H, sizeof(uint16_t) * (size_t)H);
             }

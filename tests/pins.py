@@ -183,6 +183,303 @@ def pin_fp8_quant_error_bound(o):
             assert q[g * 128 + top] & 0x7F == 0x7E  # the amax element lands on 448
 
 
+# ------------------------------------------------ per-token and MX formats
+E2M1_MAGNITUDES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])  # OCP MX v1.0, FP4 E2M1 value table
+MX_EMAX = {W.MXFP8_E4M3: 8, W.MXFP8_E5M2: 15, W.MXFP4_E2M1: 2}
+MX_MAXFINITE = {W.MXFP8_E4M3: 448.0, W.MXFP8_E5M2: 57344.0, W.MXFP4_E2M1: 6.0}
+
+
+def _torch_e5m2_values():
+    return torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e5m2).to(torch.float32).numpy()
+
+
+def _e2m1_value(code):
+    v = E2M1_MAGNITUDES[code & 7]
+    return -v if code & 8 else v
+
+
+def _mx_element_values(dtype, codes):
+    """Element codes of one MX format -> float64 values, decoded without the
+    oracle (torch's float8 tables, the E2M1 value table)."""
+    if dtype == W.MXFP8_E4M3:
+        return _torch_e4m3_values()[codes].astype(np.float64)
+    if dtype == W.MXFP8_E5M2:
+        return _torch_e5m2_values()[codes].astype(np.float64)
+    nib = np.empty(codes.size * 2, np.uint8)
+    nib[0::2] = codes & 0xF
+    nib[1::2] = codes >> 4
+    return np.array([_e2m1_value(int(c)) for c in nib])
+
+
+def pin_e5m2_decode_vs_torch(o):
+    codes = np.arange(256, dtype=np.uint8)
+    got = o.e5m2_to_f32(codes)
+    ref = _torch_e5m2_values()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+    assert ref[0x7B] == 57344.0 and np.isinf(ref[0x7C])
+
+
+def pin_e5m2_encode_vs_torch(o):
+    """torch rounds to nearest-even and overflows to inf from 61440 up; this
+    pin covers |v| < 61440 (saturation has its own pin)."""
+    rng = _rng(51)
+    vals = _torch_e5m2_values()
+    fin = np.sort(np.unique(np.abs(vals[np.isfinite(vals)])))
+    mids = ((fin[1:].astype(np.float64) + fin[:-1]) / 2).astype(np.float32)
+    nudged = np.concatenate([np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(1e6))])
+    rnd = np.concatenate([rng.uniform(-61439, 61439, 100000), rng.standard_normal(100000) * 2.0 ** -12,
+                          rng.standard_normal(100000) * 2.0 ** -17,
+                          np.exp(rng.uniform(-30, 11, 100000)) * rng.choice([-1, 1], 100000)]).astype(np.float32)
+    a = np.concatenate([fin, -fin, mids, -mids, nudged, -nudged, rnd, np.array([61439.996, -61439.996], np.float32)])
+    got = o.f32_to_e5m2(a)
+    ref = torch.from_numpy(a).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    assert np.array_equal(got, ref), "e5m2 encoder differs from torch's cast"
+
+
+def pin_e5m2_saturation(o):
+    a = np.array([57344.0, 57345.0, 61439.0, 61440.0, 65536.0, 1e9, 3.4e38, np.inf], np.float32)
+    assert (o.f32_to_e5m2(a) == 0x7B).all()
+    assert (o.f32_to_e5m2(-a) == 0xFB).all()
+
+
+def pin_e2m1_decode_table(o):
+    got = o.e2m1_to_f32(np.arange(16, dtype=np.uint8)).astype(np.float64)
+    want = np.concatenate([E2M1_MAGNITUDES, -E2M1_MAGNITUDES])
+    assert np.array_equal(got, want)
+    assert np.signbit(got[8])
+
+
+def pin_e2m1_encode_bruteforce(o):
+    """Nearest of the eight magnitudes by search, ties to the even code, above
+    6 saturating to 6; the sign goes to bit 3 (negative zero included)."""
+    rng = _rng(52)
+    a = np.concatenate([rng.uniform(0, 7.5, 4000), rng.uniform(0, 1.2, 2000),
+                        np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 6.5, 7.0, 1e30, 0.0, 1e-40])])
+    a = np.concatenate([a, -a]).astype(np.float32)
+    got = o.f32_to_e2m1(a)
+    for v, g in zip(a.astype(np.float64), got):
+        m = abs(v)
+        if m > 6.0:
+            want = 7
+        else:
+            d = np.abs(E2M1_MAGNITUDES - m)
+            best = np.nonzero(d == d.min())[0]
+            want = int(best[0]) if len(best) == 1 else int([c for c in best if c % 2 == 0][0])
+        sign = 8 if math.copysign(1.0, v) < 0 else 0
+        assert int(g) == (want | sign), (v, int(g), want | sign)
+
+
+def pin_int8_encode_vs_torch(o):
+    """torch.round is round-half-to-even; codes are clamped to [-127, 127]."""
+    rng = _rng(53)
+    a = np.concatenate([rng.uniform(-140, 140, 100000), np.arange(-130, 131) + 0.5,
+                        np.array([-1e9, 1e9, -127.5, 127.5, -0.5, 0.5, -0.0])]).astype(np.float32)
+    ref = torch.from_numpy(a).round().clamp(-127, 127).to(torch.int8).numpy()
+    assert np.array_equal(o.f32_to_int8(a), ref)
+
+
+def pin_int8_quant_closed_form(o):
+    """Rows of integers in [-126, 126] times 2^m with one element +-127*2^m:
+    amax = 127*2^m, scale = 2^m and 127/amax = 2^-m exactly, so every code
+    comes back unchanged."""
+    rng = _rng(54)
+    for H, m, pos in [(7168, 0, 0), (256, 7, 255), (136, -20, 70), (8, 60, 3), (1024, -100, 511)]:
+        c = rng.integers(-126, 127, size=H)
+        c[pos] = 127 if m % 2 == 0 else -127
+        xf = c.astype(np.float64) * 2.0 ** m
+        xb = _torch_bf16_bits(xf.astype(np.float32))
+        assert np.array_equal(_bf16_f64(xb), xf)
+        q, s = o.quant_row(W.INT8_PER_TOKEN, xb)
+        assert np.array_equal(q.astype(np.int64), c), (H, m)
+        assert s[0] == np.float32(2.0 ** m)
+
+
+def pin_int8_quant_ties_and_bound(o):
+    # amax 127 gives 127/amax = 1 exactly: x = k + 1/2 must round to even
+    x = np.array([127.0, 2.5, 3.5, -2.5, -3.5, 0.5, -0.5, 126.5, 1.5] + [0.0] * 7, np.float32)
+    q, s = o.quant_row(W.INT8_PER_TOKEN, _torch_bf16_bits(x))
+    assert q.tolist() == [127, 2, 4, -2, -4, 0, 0, 126, 2] + [0] * 7 and s[0] == 1.0
+    # zero row, and amax = 2^-126, where 127/amax overflows fp32 and is
+    # clamped to FLT_MAX = (2 - 2^-23) 2^127: the code is rint(-(4 - 2^-22)) = -4
+    q, s = o.quant_row(W.INT8_PER_TOKEN, np.zeros(64, np.uint16))
+    assert (q == 0).all() and s[0] == 0.0
+    x = np.zeros(64, np.float32)
+    x[9] = -2.0 ** -126
+    q, s = o.quant_row(W.INT8_PER_TOKEN, _torch_bf16_bits(x))
+    assert q[9] == -4 and (np.delete(q, 9) == 0).all()
+    assert s[0] == np.float32(Fraction(2) ** -126 / 127)
+    rng = _rng(55)
+    for trial in range(4):
+        H = 7168
+        xb = _torch_bf16_bits((rng.standard_normal(H) * 10.0 ** rng.uniform(-3, 3)).astype(np.float32))
+        xf = _bf16_f64(xb)
+        q, s = o.quant_row(W.INT8_PER_TOKEN, xb)
+        amax = np.abs(xf).max()
+        sc = float(s[0])
+        assert abs(sc - amax / 127) <= U32 * amax / 127  # correctly rounded quotient
+        assert abs(int(q[np.argmax(np.abs(xf))])) == 127
+        assert (np.abs(q.astype(np.float64) * sc - xf) <= sc * (0.5 + 1e-5)).all()
+
+
+def pin_fp8_pertoken_reduces_to_group(o):
+    """With H = 128 the per-token FP8 row is the 128-channel FP8 row; for a
+    long row built from e4m3 values times 2^m with one element +-448*2^m the
+    codes come back unchanged and the scale is 2^m."""
+    rng = _rng(56)
+    for trial in range(20):
+        xb = _torch_bf16_bits((rng.standard_normal(128) * 10.0 ** rng.uniform(-20, 20)).astype(np.float32))
+        q, s = o.quant_row(W.FP8_E4M3_PER_TOKEN, xb)
+        q1, s1 = o.fp8_quant_row(xb)
+        assert np.array_equal(q, q1) and s[0] == s1[0]
+    vals = _torch_e4m3_values()
+    finite = np.array([c for c in range(256) if np.isfinite(vals[c]) and c not in (0x00, 0x80)], np.uint8)
+    for H, m, pos in [(7168, 0, 7167), (512, -30, 0), (136, 25, 77)]:
+        codes = rng.choice(finite, size=H) & 0xF7
+        codes[pos] = 0x7E if m % 2 == 0 else 0xFE
+        xf = vals[codes].astype(np.float64) * 2.0 ** m
+        xb = _torch_bf16_bits(xf.astype(np.float32))
+        assert np.array_equal(_bf16_f64(xb), xf)
+        q, s = o.quant_row(W.FP8_E4M3_PER_TOKEN, xb)
+        assert np.array_equal(q, codes) and s[0] == np.float32(2.0 ** m)
+    q, s = o.quant_row(W.FP8_E4M3_PER_TOKEN, np.zeros(256, np.uint16))
+    assert (q == 0).all() and s[0] == 0.0
+
+
+def _floor_log2_exact(v):
+    """floor(log2 v) for v > 0, exactly, from the rational value."""
+    f = Fraction(float(v))
+    n = f.numerator.bit_length() - f.denominator.bit_length()
+    while Fraction(2) ** n > f:
+        n -= 1
+    while Fraction(2) ** (n + 1) <= f:
+        n += 1
+    return n
+
+
+def pin_mx_shared_exp_exact(o):
+    rng = _rng(57)
+    vals = np.concatenate([np.exp2(rng.uniform(-149, 127.9, 3000)), np.array([1.0, 448.0, 447.9, 512.0, 6.0, 4.0,
+                           57344.0, 2.0 ** -126, 2.0 ** -149, 2.0 ** -130, 3.4e38])]).astype(np.float32)
+    for emax in (8, 15, 2):
+        assert o.mx_shared_exp(0.0, emax) == -127
+        for v in vals:
+            want = max(-127, min(127, _floor_log2_exact(v) - emax))
+            assert o.mx_shared_exp(float(v), emax) == want, (float(v), emax)
+
+
+def pin_mx_closed_form_roundtrip(o):
+    """Blocks of exact element values times 2^X whose largest element has the
+    format's top exponent: the shared exponent must be X (scale byte X+127)
+    and every code must come back unchanged."""
+    rng = _rng(58)
+    for dtype in (W.MXFP8_E4M3, W.MXFP8_E5M2, W.MXFP4_E2M1):
+        emax = MX_EMAX[dtype]
+        if dtype == W.MXFP4_E2M1:
+            allcodes = np.arange(16, dtype=np.uint8)
+            vals = np.array([_e2m1_value(int(c)) for c in allcodes])
+        else:
+            table = _torch_e4m3_values() if dtype == W.MXFP8_E4M3 else _torch_e5m2_values()
+            allcodes = np.array([c for c in range(256) if np.isfinite(table[c])], np.uint8)
+            vals = table.astype(np.float64)[allcodes]
+        top = allcodes[(np.abs(vals) >= 2.0 ** emax)]
+        rest = allcodes[(np.abs(vals) < 2.0 ** emax)]
+        nb = 6
+        H = 32 * nb
+        el = rng.choice(rest, size=H).astype(np.uint8)
+        Xs = [0, 5, -9, -100, 90, -120 + emax]
+        for g in range(nb):
+            el[g * 32 + rng.integers(0, 32)] = rng.choice(top)
+        value_of = {int(c): float(v) for c, v in zip(allcodes, vals)}
+        xf = np.array([value_of[int(c)] for c in el])
+        for g, X in enumerate(Xs):
+            xf[g * 32:(g + 1) * 32] *= 2.0 ** X
+        xb = _torch_bf16_bits(xf.astype(np.float32))
+        assert np.array_equal(_bf16_f64(xb), xf), "construction must be exact in bf16"
+        q, s = o.quant_row(dtype, xb)
+        assert np.array_equal(s.astype(np.int64), np.array(Xs) + 127), dtype
+        if dtype == W.MXFP4_E2M1:
+            want = (el[0::2] | (el[1::2] << 4)).astype(np.uint8)
+            assert np.array_equal(q, want)
+        else:
+            assert np.array_equal(q, el)
+
+
+def pin_mx_error_bound(o):
+    """Decoded codes times 2^X are within half an element-format spacing of
+    x, or saturated at the format's largest value when |x| / 2^X exceeds it;
+    the block's amax element decodes to at least 2^emax."""
+    rng = _rng(59)
+    for dtype in (W.MXFP8_E4M3, W.MXFP8_E5M2, W.MXFP4_E2M1):
+        emax, top = MX_EMAX[dtype], MX_MAXFINITE[dtype]
+        mbits = {W.MXFP8_E4M3: 3, W.MXFP8_E5M2: 2, W.MXFP4_E2M1: 1}[dtype]
+        emin = {W.MXFP8_E4M3: -6, W.MXFP8_E5M2: -14, W.MXFP4_E2M1: 0}[dtype]
+        for trial in range(6):
+            H = 32 * 64
+            xb = _torch_bf16_bits((rng.standard_normal(H) * np.exp2(rng.uniform(-40, 40, H // 32)).repeat(32))
+                                  .astype(np.float32))
+            xf = _bf16_f64(xb)
+            q, s = o.quant_row(dtype, xb)
+            deq_el = _mx_element_values(dtype, q)
+            for g in range(H // 32):
+                X = int(s[g]) - 127
+                seg = xf[g * 32:(g + 1) * 32] / 2.0 ** X
+                d = deq_el[g * 32:(g + 1) * 32]
+                e = np.floor(np.log2(np.maximum(np.abs(seg), 2.0 ** emin)))
+                half = 2.0 ** (e - mbits - 1)
+                sat = np.abs(seg) > top
+                assert (np.abs(d[~sat] - seg[~sat]) <= half[~sat] * (1 + 1e-9)).all(), (dtype, g)
+                assert (np.abs(d[sat]) == top).all() and (np.sign(d[sat]) == np.sign(seg[sat])).all()
+                assert np.abs(d).max() >= 2.0 ** emax
+
+
+def pin_mx_zero_tiny_and_packing(o):
+    for dtype in (W.MXFP8_E4M3, W.MXFP8_E5M2, W.MXFP4_E2M1):
+        q, s = o.quant_row(dtype, np.zeros(64, np.uint16))
+        assert (q == 0).all() and (s == 0).all()  # amax 0: X = -127
+        x = np.zeros(64, np.float32)
+        x[33] = 2.0 ** -133  # bf16 subnormal amax: X clamps to -127
+        x[40] = -2.0 ** -131
+        xb = _torch_bf16_bits(x)
+        xb[0] = 0x8000  # -0.0
+        q, s = o.quant_row(dtype, xb)
+        assert s.tolist() == [0, 0]
+        d = _mx_element_values(dtype, q)
+        assert np.isfinite(d).all() and np.signbit(d[0])
+        assert d[33] == x[33] * 2.0 ** 127 or dtype == W.MXFP4_E2M1
+    # packing: element 2i in the low nibble
+    x = np.array([1.0, 6.0, -0.5, 3.0] + [0.0] * 28, np.float32)
+    q, s = o.quant_row(W.MXFP4_E2M1, _torch_bf16_bits(x))
+    assert s[0] == 127 and q[0] == 0x72 and q[1] == 0x59 and (q[2:] == 0).all()
+
+
+def pin_quant_dispatch_rows(o):
+    """Each quantised dispatch row is the quantisation of its source row, in
+    the scale layout of its format, at the row routing gives it."""
+    rng = _rng(60)
+    for dt in (W.INT8_PER_TOKEN, W.FP8_E4M3_PER_TOKEN, W.MXFP8_E4M3, W.MXFP8_E5M2, W.MXFP4_E2M1):
+        for mode, max_tokens in ((W.COMPACT, 0), (W.PADDED, 5)):
+            T, E, R, K, H = 21, 8, 2, 3, 96
+            idx = W.random_topk(rng, T, E, K, p_neg=0.2, allow_dup=True)
+            x = _torch_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+            L = o.tc_layout(idx, E, R)
+            D = o.tc_dispatch(x, idx, E, L, mode=mode, max_tokens=max_tokens, out_dtype=dt, want_src=True)
+            seen = 0
+            for e in range(E):
+                pairs = [(t, k) for t in range(T) for k in range(K) if idx[t, k] == e]
+                for j, (t, k) in enumerate(pairs):
+                    if mode == W.PADDED and j >= max_tokens:
+                        continue
+                    row = _expected_row(e, j, L["expert_offsets"], mode, max_tokens)
+                    qq, ss = o.quant_row(dt, x[t])
+                    assert np.array_equal(D["recv"][row], qq), (dt, mode)
+                    assert np.array_equal(np.atleast_1d(D["recv_scales"][row]), ss), (dt, mode)
+                    assert D["recv_src"][row] == t
+                    seen += 1
+            assert seen == (D["recv_src"] >= 0).sum()
+
+
 # ----------------------------------------------------------- token choice
 def _brute_tc_layout(idx, E, R):
     T, K = idx.shape

@@ -43,6 +43,24 @@ PLANTS = [
     ("ec_combine_unfused", "acc[h] = fmaf(w, oracle_bf16_to_f32(y[s * H + h]), acc[h]);",
      "acc[h] = acc[h] + w * oracle_bf16_to_f32(y[s * H + h]);", "pin_ec"),
     ("ec_dispatch_wrong_row", "memcpy(recv + s * H, x + (int64_t)t * H", "memcpy(recv + s * H, x + (int64_t)((t + 1) % T) * H", "pin_ec_dispatch"),
+    ("e5m2_ties_away", "int m = (int)nearbyintf(fr * 8.0f);", "int m = (int)roundf(fr * 8.0f);", "pin_e5m2"),
+    ("e5m2_bias_16", "int code = ((unb + 15) << 2) | (m - 4);", "int code = ((unb + 16) << 2) | (m - 4);", "pin_e5m2"),
+    ("e5m2_subnormal_truncates", "int m = (int)nearbyintf(ldexpf(a, 16));", "int m = (int)ldexpf(a, 16);", "pin_e5m2"),
+    ("e2m1_ties_away", "int m = (int)nearbyintf(fr * 4.0f);", "int m = (int)roundf(fr * 4.0f);", "pin_e2m1"),
+    ("e2m1_subnormal_truncates", "int m = (int)nearbyintf(ldexpf(a, 1));", "int m = (int)ldexpf(a, 1);", "pin_e2m1"),
+    ("int8_truncates", "float r = nearbyintf(f);", "float r = truncf(f);", "pin_int8"),
+    ("int8_clamp_low_128", "if (r < -127.0f)\n        r = -127.0f;", "if (r < -128.0f)\n        r = -128.0f;", "pin_int8"),
+    ("int8_scale_128", "*scale = amax / 127.0f;", "*scale = amax / 128.0f;", "pin_int8"),
+    ("fp8_pertoken_first_group_amax", "float amax = row_amax(xrow, hidden);\n    if (amax == 0.0f) {\n        *scale = 0.0f;\n        for (int32_t i = 0; i < hidden; ++i)\n            q[i] = 0x00;",
+     "float amax = row_amax(xrow, hidden < 128 ? hidden : 128);\n    if (amax == 0.0f) {\n        *scale = 0.0f;\n        for (int32_t i = 0; i < hidden; ++i)\n            q[i] = 0x00;", "pin_fp8_pertoken"),
+    ("mx_exp_off_by_one", "int32_t X = (ex - 1) - emax_elem;", "int32_t X = ex - emax_elem;", "pin_mx"),
+    ("mx_no_low_clamp", "if (X < -127)\n        X = -127;", "if (X < -1000)\n        X = -127;", "pin_mx"),
+    ("mx_e5m2_emax_16", "dtype == OR_MXFP8_E5M2 ? 15 : 2", "dtype == OR_MXFP8_E5M2 ? 16 : 2", "pin_mx"),
+    ("mx_block_amax_of_16", "float amax = row_amax(xrow + g * 32, 32);", "float amax = row_amax(xrow + g * 32, 16);", "pin_mx"),
+    ("fp4_nibbles_swapped", "if (h % 2 == 0)\n                    q[h / 2] = c;\n                else\n                    q[h / 2] = (uint8_t)(q[h / 2] | (c << 4));",
+     "if (h % 2 == 0)\n                    q[h / 2] = (uint8_t)(c << 4);\n                else\n                    q[h / 2] = (uint8_t)(q[h / 2] | c);", "pin_mx"),
+    ("quant_dispatch_scale_row_shift", "memcpy((uint8_t*)recv_scales + row * scale_bytes, srow",
+     "memcpy((uint8_t*)recv_scales + (row / 2 * 2) * scale_bytes, srow", "pin_quant_dispatch"),
 ]
 
 
