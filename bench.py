@@ -53,6 +53,8 @@ def parse():
                     help="time every op on all five workloads (one JSON line each) instead of the step")
     ap.add_argument("--only", type=int, default=0, choices=[0, 1, 2, 3, 4, 5],
                     help="with --workloads: just this workload")
+    ap.add_argument("--quant", action="store_true",
+                    help="with --workloads: also time every quantised dispatch format on the token-choice workloads")
     return ap.parse_args()
 
 
@@ -454,6 +456,17 @@ def run_ours(args):
     return 0
 
 
+# quantised dispatch formats: (name, dtype code, code bytes per row, scale bytes per row)
+QUANT_FORMATS = [
+    ("fp8_g128", 2, lambda H: H, lambda H: H // 128 * 4),
+    ("int8_per_token", 3, lambda H: H, lambda H: 4),
+    ("fp8_per_token", 4, lambda H: H, lambda H: 4),
+    ("mxfp8_e4m3", 5, lambda H: H, lambda H: H // 32),
+    ("mxfp8_e5m2", 6, lambda H: H, lambda H: H // 32),
+    ("mxfp4_e2m1", 7, lambda H: H // 2, lambda H: H // 32),
+]
+
+
 def run_workload_table(args):
     """Per-op timings on every workload (layout, dispatch, combine; expert
     choice for workload 4): one JSON line per (workload, op), L2 flushed
@@ -528,6 +541,17 @@ def run_workload_table(args):
             emit(cfg, "combine", timeit(lambda: B.ep_combine(y, rt, lay, w, out, mode=mode,
                                                              max_tokens_per_expert=mt)),
                  n_valid * H * 2 + T * H * 2 + T * K * 16 + E * 4, T)
+            if args.quant:
+                del recv
+                for name, dt, code_b, scale_b in QUANT_FORMATS:
+                    cb, sb = code_b(H), scale_b(H)
+                    qrecv = torch.empty((rows, cb), dtype=torch.uint8, device=dev)
+                    qsc = torch.empty((rows, sb), dtype=torch.uint8, device=dev)
+                    emit(cfg, "dispatch_" + name,
+                         timeit(lambda: B.ep_dispatch(x, rt, lay, qrecv, mode=mode, max_tokens_per_expert=mt,
+                                                      recv_scales=qsc, out_dtype=dt)),
+                         T * H * 2 + n_valid * (cb + sb) + meta, T)
+                    del qrecv, qsc
         else:
             C = cfg["C"]
             ti_np = inp["token_indices"]

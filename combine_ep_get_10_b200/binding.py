@@ -20,6 +20,7 @@ EP_OK = 0
 STATUS_NAMES = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_BAD_INDEX", 3: "EP_ERR_OVERFLOW",
                 4: "EP_ERR_WORKSPACE", 5: "EP_ERR_CUDA", 6: "EP_ERR_UNSUPPORTED", 7: "EP_ERR_TIMEOUT"}
 EP_BF16, EP_FP32, EP_FP8_E4M3 = 0, 1, 2
+EP_INT8_PER_TOKEN, EP_FP8_E4M3_PER_TOKEN, EP_MXFP8_E4M3, EP_MXFP8_E5M2, EP_MXFP4_E2M1 = 3, 4, 5, 6, 7
 EP_LAYOUT_COMPACT, EP_LAYOUT_PADDED = 0, 1
 EP_ROUTING_TOPK, EP_ROUTING_EXPERT_CHOICE = 0, 1
 EP_DEVERR_BAD_INDEX, EP_DEVERR_OVERFLOW, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
@@ -237,9 +238,10 @@ def ep_get_layout(routing: Routing, layout: Layout, stream=None) -> Layout:
 
 def ep_dispatch(x: torch.Tensor, routing: Routing, layout: Layout, recv_x: torch.Tensor, *, mode=EP_LAYOUT_COMPACT,
                 max_tokens_per_expert=0, num_recv_rows=None, topk_weights=None, recv_scales=None, recv_src=None,
-                recv_weights=None, stream=None) -> None:
-    """out dtype follows recv_x (bfloat16, or uint8 / float8_e4m3fn for FP8)."""
-    out_dtype = _dtype_code(recv_x)
+                recv_weights=None, out_dtype=None, stream=None) -> None:
+    """out_dtype: one of the EP_* element formats; by default it follows
+    recv_x (bfloat16, or uint8 / float8_e4m3fn for 128-channel FP8)."""
+    out_dtype = _dtype_code(recv_x) if out_dtype is None else int(out_dtype)
     rows = recv_x.shape[0] if num_recv_rows is None else int(num_recv_rows)
     _check(lib().ep_dispatch(_ptr(x), x.shape[1], ctypes.byref(routing.desc), ctypes.byref(layout.desc), int(mode),
                              int(max_tokens_per_expert), rows, out_dtype, _ptr(topk_weights), _ptr(recv_x),

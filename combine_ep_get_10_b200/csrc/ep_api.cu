@@ -177,7 +177,7 @@ ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* l
 
 ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing, const ep_layout_t* layout,
                         ep_buffer_mode_t mode, int32_t max_tokens_per_expert, int64_t num_recv_rows,
-                        ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, float* recv_scales,
+                        ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, void* recv_scales,
                         int32_t* recv_src, float* recv_weights, ep_stream_t stream)
 {
     ep_status_t st = check_routing(routing);
@@ -193,11 +193,16 @@ ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* 
         return st;
     if (hidden < 1 || hidden % 8 != 0)
         return EP_ERR_INVALID_ARG;
-    if (out_dtype != EP_BF16 && out_dtype != EP_FP8_E4M3)
+    if (out_dtype == EP_FP32 || out_dtype < EP_BF16 || out_dtype > EP_MXFP4_E2M1)
         return EP_ERR_INVALID_ARG;
-    if (out_dtype == EP_FP8_E4M3 && (hidden % 128 != 0 || (num_recv_rows > 0 && recv_scales == nullptr) ||
-                                     !aligned(recv_scales, 4)))
-        return EP_ERR_INVALID_ARG;
+    if (out_dtype != EP_BF16) {
+        const bool mx = out_dtype == EP_MXFP8_E4M3 || out_dtype == EP_MXFP8_E5M2 || out_dtype == EP_MXFP4_E2M1;
+        const int group = out_dtype == EP_FP8_E4M3 ? 128 : (mx ? 32 : 8);
+        if (hidden % group != 0 || (num_recv_rows > 0 && recv_scales == nullptr) || !aligned(recv_scales, mx ? 1 : 4))
+            return EP_ERR_INVALID_ARG;
+        if (hidden > ep::kMaxQuantHidden)
+            return EP_ERR_UNSUPPORTED;
+    }
     const int32_t T = routing->num_tokens;
     if (T > 0 && (x == nullptr || !aligned(x, 16)))
         return EP_ERR_INVALID_ARG;

@@ -161,4 +161,29 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi)
     return static_cast<uint32_t>(r);
 }
 
+// Two floats to e5m2 codes (nearest, ties to even, saturating to +-57344);
+// `lo` lands in the low byte.
+__device__ __forceinline__ uint32_t pack_e5m2x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return static_cast<uint32_t>(r);
+}
+
+// Two floats to e2m1 codes (nearest, ties to even, saturating to +-6) in one
+// byte; `lo` lands in the low nibble.
+__device__ __forceinline__ uint32_t pack_e2m1x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\tcvt.u32.u8 %0, q;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ void st_u32(void* p, uint32_t v)
+{
+    asm volatile("st.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 } // namespace ep

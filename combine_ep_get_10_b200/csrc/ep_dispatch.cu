@@ -11,11 +11,13 @@
 // balances the tail.  (A persistent variant streaming each CTA's items
 // through a 3-4 stage ring measured 10-15% slower.)
 //
-// FP8 dispatch (README, "Quantization Modes in Normal Dispatch"; one fp32
-// scale per 128 channels): one CTA per token quantises the row once in
-// registers -- a half-warp owns a 128-channel group, amax by shuffles,
-// scale = amax/448, codes = cvt.rn.satfinite.e4m3x2(x * 448/amax) -- and
-// stores the 8-byte code runs and the scale to each destination row.
+// Quantised dispatch (README, "Quantization Modes in Normal Dispatch": FP8
+// with one fp32 scale per 128 channels, per-token INT8 and FP8, MX FP8/FP4
+// with an e8m0 scale per 32): one CTA per token holds the row in registers
+// (all loads issued at once), reduces the amax over each scale group by
+// shuffles (or over the CTA for per-token scales), encodes every element once
+// with the cvt.rn.satfinite packing instructions, and stores the code runs
+// and scales to each destination row of the token.
 #include <algorithm>
 
 #include "ep_device.cuh"
@@ -158,27 +160,109 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
     }
 }
 
-struct Fp8Args {
+// Quantised payload formats (values of ep_dtype_t handled by the kernel).
+enum QuantFmt : int {
+    kQFp8G128 = EP_FP8_E4M3,        // e4m3, fp32 scale per 128 channels
+    kQInt8Tok = EP_INT8_PER_TOKEN,  // int8, fp32 scale per row
+    kQFp8Tok = EP_FP8_E4M3_PER_TOKEN, // e4m3, fp32 scale per row
+    kQMxE4m3 = EP_MXFP8_E4M3,       // e4m3, e8m0 scale per 32
+    kQMxE5m2 = EP_MXFP8_E5M2,       // e5m2, e8m0 scale per 32
+    kQMxE2m1 = EP_MXFP4_E2M1        // e2m1 x2, e8m0 scale per 32
+};
+
+struct QuantArgs {
     const uint16_t* x;
     int32_t H;
+    int32_t nper; // 16-byte vectors per thread (<= kQuantMaxVec)
     RowMap map;
     uint8_t* recv;
-    float* scales;
+    void* scales;
     const float* topk_weights;
     int32_t* recv_src;
     float* recv_weights;
     uint32_t* err;
 };
 
-constexpr int kFp8Threads = 256;
+constexpr int kQuantMaxVec = 8;     // a row is held in registers: <= 8 vectors of 8 bf16 per thread
+constexpr int kQuantVecTarget = 4;  // vectors per thread the launch aims for
 
-__global__ void __launch_bounds__(kFp8Threads) fp8_dispatch_kernel(Fp8Args a)
+__device__ __forceinline__ float amax8(uint4 r)
 {
-    extern __shared__ __align__(16) int64_t rows[]; // [K]
+    // |x| of a bf16 is its bit pattern without the sign; max over floats
+    const float a0 = fmaxf(fabsf(bf16_lo(r.x)), fabsf(bf16_hi(r.x)));
+    const float a1 = fmaxf(fabsf(bf16_lo(r.y)), fabsf(bf16_hi(r.y)));
+    const float a2 = fmaxf(fabsf(bf16_lo(r.z)), fabsf(bf16_hi(r.z)));
+    const float a3 = fmaxf(fabsf(bf16_lo(r.w)), fabsf(bf16_hi(r.w)));
+    return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+}
+
+// Eight bf16 values times `mul` (one IEEE multiply each) encoded in format
+// kFmt: 8 bytes (int8 / fp8) in .x/.y, or 4 bytes (fp4) in .x.
+template <int kFmt>
+__device__ __forceinline__ uint2 encode8(uint4 r, float mul)
+{
+    float p[8];
+    p[0] = __fmul_rn(bf16_lo(r.x), mul);
+    p[1] = __fmul_rn(bf16_hi(r.x), mul);
+    p[2] = __fmul_rn(bf16_lo(r.y), mul);
+    p[3] = __fmul_rn(bf16_hi(r.y), mul);
+    p[4] = __fmul_rn(bf16_lo(r.z), mul);
+    p[5] = __fmul_rn(bf16_hi(r.z), mul);
+    p[6] = __fmul_rn(bf16_lo(r.w), mul);
+    p[7] = __fmul_rn(bf16_hi(r.w), mul);
+    uint2 q;
+    if constexpr (kFmt == kQInt8Tok) {
+        uint32_t b[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            b[i] = static_cast<uint32_t>(max(-127, min(127, __float2int_rn(p[i])))) & 0xFFu;
+        q.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+        q.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+    } else if constexpr (kFmt == kQMxE5m2) {
+        q.x = pack_e5m2x2(p[0], p[1]) | (pack_e5m2x2(p[2], p[3]) << 16);
+        q.y = pack_e5m2x2(p[4], p[5]) | (pack_e5m2x2(p[6], p[7]) << 16);
+    } else if constexpr (kFmt == kQMxE2m1) {
+        q.x = pack_e2m1x2(p[0], p[1]) | (pack_e2m1x2(p[2], p[3]) << 8) | (pack_e2m1x2(p[4], p[5]) << 16) |
+              (pack_e2m1x2(p[6], p[7]) << 24);
+        q.y = 0;
+    } else {
+        q.x = pack_e4m3x2(p[0], p[1]) | (pack_e4m3x2(p[2], p[3]) << 16);
+        q.y = pack_e4m3x2(p[4], p[5]) | (pack_e4m3x2(p[6], p[7]) << 16);
+    }
+    return q;
+}
+
+// One CTA per token.  Thread i holds vectors i, i + nthr, ... of the row
+// (all loads issued up front); the amax is reduced over the scale group --
+// 16 lanes (128 channels), 4 lanes (32, MX) or the whole CTA (per token) --
+// then every thread encodes its vectors once and stores them, with the
+// group's scale, to each destination row of the token.
+template <int kFmt>
+__global__ void __launch_bounds__(512, 1) quant_dispatch_kernel(QuantArgs a)
+{
+    constexpr bool kMx = kFmt == kQMxE4m3 || kFmt == kQMxE5m2 || kFmt == kQMxE2m1;
+    constexpr bool kPerToken = kFmt == kQInt8Tok || kFmt == kQFp8Tok;
+    constexpr int kGroupLanes = kFmt == kQFp8G128 ? 16 : 4; // group modes only
+    constexpr int kCodeBytes = kFmt == kQMxE2m1 ? 4 : 8;  // bytes per 8 channels
+    extern __shared__ __align__(16) int64_t rows[];         // [K]
+    __shared__ float warp_amax[32];
     const int64_t t = blockIdx.x;
     const int tid = threadIdx.x;
+    const int nthr = blockDim.x;
+    const int nvec = a.H / 8;
+
+    const uint8_t* xrow = reinterpret_cast<const uint8_t*>(a.x) + t * static_cast<int64_t>(a.H) * 2;
+    uint4 raw[kQuantMaxVec];
+#pragma unroll
+    for (int j = 0; j < kQuantMaxVec; ++j) {
+        const int v = j * nthr + tid;
+        raw[j] = make_uint4(0, 0, 0, 0);
+        if (j < a.nper && v < nvec)
+            raw[j] = ld_nc_v4(xrow + static_cast<int64_t>(v) * 16);
+    }
+
     uint32_t errbits = 0;
-    for (int k = tid; k < a.map.K; k += kFp8Threads) {
+    for (int k = tid; k < a.map.K; k += nthr) {
         const int64_t rk = a.map.row(t, k, errbits);
         rows[k] = rk;
         if (rk >= 0) {
@@ -190,58 +274,115 @@ __global__ void __launch_bounds__(kFp8Threads) fp8_dispatch_kernel(Fp8Args a)
     }
     if (errbits)
         flag_error(a.err, errbits);
-    __syncthreads();
 
-    const int nvec = a.H / 8;   // 16-byte vectors of 8 bf16
-    const int groups = a.H / 128;
-    const uint8_t* xrow = reinterpret_cast<const uint8_t*>(a.x) + t * static_cast<int64_t>(a.H) * 2;
-    for (int base = 0; base < nvec; base += kFp8Threads) {
-        const int v = base + tid;
-        const bool active = v < nvec; // a 16-lane group is all-in or all-out (nvec % 16 == 0)
-        uint4 raw = make_uint4(0, 0, 0, 0);
-        if (active)
-            raw = ld_nc_v4(xrow + static_cast<int64_t>(v) * 16);
-        float f[8];
-        f[0] = bf16_lo(raw.x);
-        f[1] = bf16_hi(raw.x);
-        f[2] = bf16_lo(raw.y);
-        f[3] = bf16_hi(raw.y);
-        f[4] = bf16_lo(raw.z);
-        f[5] = bf16_hi(raw.z);
-        f[6] = bf16_lo(raw.w);
-        f[7] = bf16_hi(raw.w);
-        float amax = 0.0f;
+    float tok_amax = 0.0f;
+    if constexpr (kPerToken) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            amax = fmaxf(amax, fabsf(f[i]));
+        for (int j = 0; j < kQuantMaxVec; ++j)
+            tok_amax = fmaxf(tok_amax, amax8(raw[j]));
 #pragma unroll
-        for (int d = 8; d >= 1; d >>= 1)
-            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
-        float scale = 0.0f;
-        uint2 q = make_uint2(0, 0);
-        if (amax > 0.0f) {
-            scale = __fdiv_rn(amax, 448.0f);
-            float inv = __fdiv_rn(448.0f, amax);
-            inv = fminf(inv, 3.40282347e38f);
-            float p[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                p[i] = __fmul_rn(f[i], inv);
-            q.x = pack_e4m3x2(p[0], p[1]) | (pack_e4m3x2(p[2], p[3]) << 16);
-            q.y = pack_e4m3x2(p[4], p[5]) | (pack_e4m3x2(p[6], p[7]) << 16);
-        }
-        if (active) {
-            const int g = v >> 4;
-            for (int k = 0; k < a.map.K; ++k) {
-                const int64_t rk = rows[k];
-                if (rk < 0)
-                    continue;
-                st_v2(a.recv + rk * a.H + static_cast<int64_t>(v) * 8, q);
-                if ((tid & 15) == 0)
-                    a.scales[rk * groups + g] = scale;
-            }
+        for (int d = 16; d >= 1; d >>= 1)
+            tok_amax = fmaxf(tok_amax, __shfl_xor_sync(kFullMask, tok_amax, d));
+        if ((tid & 31) == 0)
+            warp_amax[tid >> 5] = tok_amax;
+    }
+    __syncthreads();
+    if constexpr (kPerToken) {
+        tok_amax = 0.0f;
+        for (int w = 0; w < (nthr >> 5); ++w)
+            tok_amax = fmaxf(tok_amax, warp_amax[w]);
+    }
+
+    // codes and scale of each held vector
+    uint2 code[kQuantMaxVec];
+    float fscale[kQuantMaxVec];   // fp32 scale of the vector's group (128-channel mode)
+    uint32_t xbyte[kQuantMaxVec]; // e8m0 byte of the vector's block (MX)
+    float tok_scale = 0.0f, tok_mul = 0.0f;
+    if constexpr (kPerToken) {
+        constexpr float qmax = kFmt == kQInt8Tok ? 127.0f : 448.0f;
+        if (tok_amax > 0.0f) {
+            tok_scale = __fdiv_rn(tok_amax, qmax);
+            tok_mul = fminf(__fdiv_rn(qmax, tok_amax), 3.40282347e38f);
         }
     }
+#pragma unroll
+    for (int j = 0; j < kQuantMaxVec; ++j) {
+        float mul = tok_mul;
+        fscale[j] = 0.0f;
+        xbyte[j] = 0;
+        if constexpr (!kPerToken) {
+            float amax = amax8(raw[j]);
+#pragma unroll
+            for (int d = kGroupLanes / 2; d >= 1; d >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
+            if constexpr (kMx) {
+                constexpr int kEmax = kFmt == kQMxE4m3 ? 8 : (kFmt == kQMxE5m2 ? 15 : 2);
+                // floor(log2 amax) is the unbiased exponent of a normal amax; a
+                // zero or subnormal amax clamps to -127 either way
+                const int ef = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
+                const int X = max(ef - 127 - kEmax, -127);
+                xbyte[j] = static_cast<uint32_t>(X + 127);
+                mul = __uint_as_float(static_cast<uint32_t>(127 - X) << 23); // 2^-X, a normal float
+            } else {
+                mul = 0.0f;
+                if (amax > 0.0f) {
+                    fscale[j] = __fdiv_rn(amax, 448.0f);
+                    mul = fminf(__fdiv_rn(448.0f, amax), 3.40282347e38f);
+                }
+            }
+        }
+        // dynamic scales: a zero amax gives zero codes (no -0 codes either)
+        code[j] = (kMx || mul != 0.0f) ? encode8<kFmt>(raw[j], mul) : make_uint2(0, 0);
+    }
+
+    const int64_t code_row = static_cast<int64_t>(nvec) * kCodeBytes;
+    for (int k = 0; k < a.map.K; ++k) {
+        const int64_t rk = rows[k];
+        if (rk < 0)
+            continue;
+        uint8_t* dst = a.recv + rk * code_row;
+#pragma unroll
+        for (int j = 0; j < kQuantMaxVec; ++j) {
+            const int v = j * nthr + tid;
+            if (j >= a.nper || v >= nvec)
+                continue;
+            if constexpr (kCodeBytes == 8)
+                st_v2(dst + static_cast<int64_t>(v) * 8, code[j]);
+            else
+                st_u32(dst + static_cast<int64_t>(v) * 4, code[j].x);
+            if constexpr (kMx) {
+                if ((tid & 3) == 0)
+                    static_cast<uint8_t*>(a.scales)[rk * (nvec / 4) + v / 4] = static_cast<uint8_t>(xbyte[j]);
+            } else if constexpr (kFmt == kQFp8G128) {
+                if ((tid & 15) == 0)
+                    static_cast<float*>(a.scales)[rk * (nvec / 16) + v / 16] = fscale[j];
+            }
+        }
+        if constexpr (kPerToken) {
+            if (tid == 0)
+                static_cast<float*>(a.scales)[rk] = tok_scale;
+        }
+    }
+}
+
+template <int kFmt>
+cudaError_t launch_quant(const QuantArgs& k, int32_t T, int32_t K, cudaStream_t stream)
+{
+    const int nvec = k.H / 8;
+    int nthr = (nvec + kQuantVecTarget - 1) / kQuantVecTarget;
+    nthr = ((nthr + 31) / 32) * 32;
+    nthr = std::min(std::max(nthr, 32), 512);
+    QuantArgs a = k;
+    a.nper = (nvec + nthr - 1) / nthr;
+    const size_t smem = sizeof(int64_t) * static_cast<size_t>(K);
+    if (smem > 40 * 1024) {
+        cudaError_t st = cudaFuncSetAttribute(quant_dispatch_kernel<kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              static_cast<int>(smem));
+        if (st != cudaSuccess)
+            return st;
+    }
+    quant_dispatch_kernel<kFmt><<<T, nthr, smem, stream>>>(a);
+    return cudaGetLastError();
 }
 
 constexpr int64_t kMaxGrid = int64_t{1} << 30;
@@ -268,18 +409,25 @@ cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream)
         return cudaSuccess;
     RowMap m{a.rows.topk_idx, a.rows.slot, a.rows.offsets, a.rows.K, a.rows.E, a.rows.mode, a.rows.max_tokens,
              a.rows.num_rows};
-    if (a.out_dtype == EP_FP8_E4M3) {
-        Fp8Args k{static_cast<const uint16_t*>(a.x), a.H, m, static_cast<uint8_t*>(a.recv_x), a.recv_scales,
-                  a.topk_weights, a.recv_src, a.recv_weights, a.err};
-        const size_t smem = sizeof(int64_t) * static_cast<size_t>(a.rows.K);
-        if (smem > 48 * 1024) {
-            cudaError_t st = cudaFuncSetAttribute(fp8_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  static_cast<int>(smem));
-            if (st != cudaSuccess)
-                return st;
+    if (a.out_dtype != EP_BF16) {
+        QuantArgs k{static_cast<const uint16_t*>(a.x), a.H, 0, m, static_cast<uint8_t*>(a.recv_x), a.recv_scales,
+                    a.topk_weights, a.recv_src, a.recv_weights, a.err};
+        switch (a.out_dtype) {
+        case EP_FP8_E4M3:
+            return launch_quant<kQFp8G128>(k, a.T, a.rows.K, stream);
+        case EP_INT8_PER_TOKEN:
+            return launch_quant<kQInt8Tok>(k, a.T, a.rows.K, stream);
+        case EP_FP8_E4M3_PER_TOKEN:
+            return launch_quant<kQFp8Tok>(k, a.T, a.rows.K, stream);
+        case EP_MXFP8_E4M3:
+            return launch_quant<kQMxE4m3>(k, a.T, a.rows.K, stream);
+        case EP_MXFP8_E5M2:
+            return launch_quant<kQMxE5m2>(k, a.T, a.rows.K, stream);
+        case EP_MXFP4_E2M1:
+            return launch_quant<kQMxE2m1>(k, a.T, a.rows.K, stream);
+        default:
+            return cudaErrorInvalidValue;
         }
-        fp8_dispatch_kernel<<<a.T, kFp8Threads, smem, stream>>>(k);
-        return cudaGetLastError();
     }
     BulkArgs k{};
     k.src = static_cast<const uint8_t*>(a.x);

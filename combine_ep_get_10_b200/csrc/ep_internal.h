@@ -13,6 +13,7 @@ namespace ep {
 
 constexpr size_t kWorkspaceHeaderBytes = 256; // error word + reserved
 constexpr int kMaxTopkLayoutExperts = 1024;   // token-choice layout keeps E counters per warp
+constexpr int kMaxQuantHidden = 32768;        // quantising dispatch holds a row in registers (512 threads x 64)
 
 inline uint32_t* error_word(void* workspace)
 {
@@ -65,7 +66,7 @@ struct TcDispatchLaunch {
     int32_t out_dtype;
     const float* topk_weights;
     void* recv_x;
-    float* recv_scales;
+    void* recv_scales;
     int32_t* recv_src;
     float* recv_weights;
     uint32_t* err;

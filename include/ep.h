@@ -62,7 +62,37 @@ typedef enum {
     EP_ERR_TIMEOUT = 7      /* device: a bounded wait gave up */
 } ep_status_t;
 
-typedef enum { EP_BF16 = 0, EP_FP32 = 1, EP_FP8_E4M3 = 2 } ep_dtype_t;
+/* Element formats.  EP_BF16 / EP_FP32 are plain arrays.  The others are the
+ * quantised dispatch payloads of the [README] "Quantization Modes" table
+ * ("int8", "pertoken_fp8_e4m3", "mx_fp8_e4m3", "mx_fp8_e5m2",
+ * "mx_fp4_e2m1"; EP_FP8_E4M3 is the 128-channel FP8 of low_latency_dispatch):
+ *   value               codes per row            scales per row
+ *   EP_FP8_E4M3         H bytes, e4m3            H/128 fp32 (amax/448)
+ *   EP_INT8_PER_TOKEN   H bytes, int8            1 fp32 (amax/127)
+ *   EP_FP8_E4M3_PER_TOKEN H bytes, e4m3          1 fp32 (amax/448)
+ *   EP_MXFP8_E4M3       H bytes, e4m3            H/32 e8m0 bytes
+ *   EP_MXFP8_E5M2       H bytes, e5m2            H/32 e8m0 bytes
+ *   EP_MXFP4_E2M1       H/2 bytes, two e2m1      H/32 e8m0 bytes
+ *                       codes per byte, element
+ *                       2i in the low nibble
+ * Dynamic scales (fp32): scale = amax/qmax and code = encode(x * (qmax/amax))
+ * with qmax/amax clamped to FLT_MAX, qmax = 448 (e4m3, nearest-even,
+ * saturating) or 127 (int8, nearest-even, clamped to [-127, 127]); amax == 0
+ * gives scale 0 and zero codes.  MX scales (OCP Microscaling v1.0): per block
+ * of 32, X = floor(log2 amax) - emax (e4m3 8, e5m2 15, e2m1 2) clamped to
+ * [-127, 127] (amax == 0 gives -127), scale byte X + 127, code =
+ * encode(x * 2^-X), nearest-even and saturating to the format's largest
+ * finite value (448, 57344, 6). */
+typedef enum {
+    EP_BF16 = 0,
+    EP_FP32 = 1,
+    EP_FP8_E4M3 = 2,
+    EP_INT8_PER_TOKEN = 3,
+    EP_FP8_E4M3_PER_TOKEN = 4,
+    EP_MXFP8_E4M3 = 5,
+    EP_MXFP8_E5M2 = 6,
+    EP_MXFP4_E2M1 = 7
+} ep_dtype_t;
 
 /* COMPACT: expert e's rows are [expert_offsets[e], expert_offsets[e+1]) of
  *   one buffer (normal-mode dispatch); rank r's rows are the contiguous
@@ -153,18 +183,19 @@ EP_API ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layo
  * and row >= num_recv_rows is skipped with EP_DEVERR_OVERFLOW.
  *   x            bf16 [T, H], 16-byte aligned, H % 8 == 0
  *   out_dtype    EP_BF16: recv_x bf16 [rows, H] receives x[t] bit for bit.
- *                EP_FP8_E4M3 (H % 128 == 0): recv_x uint8 [rows, H] receives
- *                e4m3 codes and recv_scales fp32 [rows, H/128] one scale per
- *                128 channels: scale = amax/448, code = RNE-satfinite of
- *                x * (448/amax) (448/amax clamped to FLT_MAX; amax == 0 gives
- *                scale 0 and code 0x00) -- [README] "Quantization Modes".
+ *                A quantised format (see ep_dtype_t): recv_x receives the
+ *                codes of x[t] and recv_scales (fp32, or e8m0 bytes for MX)
+ *                its scales, both row-major with the row sizes listed at
+ *                ep_dtype_t.  Needs H % 128 == 0 (EP_FP8_E4M3), H % 32 == 0
+ *                (MX), H <= 32768, and recv_scales aligned to its element
+ *                ([README] "Quantization Modes in Normal Dispatch").
  *   topk_weights fp32 [T, K], needed only when recv_weights != NULL
  *   recv_src     optional int32 [rows]: source token of each written row
  *   recv_weights optional fp32 [rows]: gate weight of each written row
  * Rows not named by any pair are left untouched. */
 EP_API ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing, const ep_layout_t* layout,
                         ep_buffer_mode_t mode, int32_t max_tokens_per_expert, int64_t num_recv_rows,
-                        ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, float* recv_scales,
+                        ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, void* recv_scales,
                         int32_t* recv_src, float* recv_weights, ep_stream_t stream);
 
 /* Token-choice combine ([README] API Overview: combine / low_latency_combine,

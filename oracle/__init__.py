@@ -246,6 +246,8 @@ def tc_dispatch(x_bits, topk_idx, num_experts, layout, mode=COMPACT, max_tokens=
     rows = int(num_recv_rows)
     recv = code_array(out_dtype, rows, H)
     scales = scale_array(out_dtype, rows, H)
+    if want_weights and topk_weights is None:
+        raise ValueError("recv_weights needs topk_weights")
     src = np.full(rows, -1, np.int32) if want_src else None
     wts = np.zeros(rows, np.float32) if want_weights else None
     w = _c(topk_weights, np.float32) if topk_weights is not None else None

@@ -110,6 +110,12 @@ def test_dispatch_and_combine_reject_bad_args(L):
     assert disp(dt=B.EP_FP8_E4M3, hidden=136) == 1  # fp8 needs H % 128 == 0
     assert disp(dt=B.EP_FP8_E4M3, sc=None) == 1  # fp8 needs scales
     assert disp(rows=-1) == 1
+    assert disp(dt=8) == 1  # no such format
+    assert disp(dt=B.EP_MXFP8_E4M3, hidden=264, sc=0x6000) == 1  # MX needs H % 32 == 0
+    assert disp(dt=B.EP_MXFP4_E2M1, hidden=256, sc=None) == 1  # scales required
+    assert disp(dt=B.EP_INT8_PER_TOKEN, hidden=256, sc=0x6002) == 1  # fp32 scales misaligned
+    assert disp(dt=B.EP_FP8_E4M3_PER_TOKEN, hidden=32776, sc=0x6000) == 6  # row wider than 32768
+    assert disp(dt=B.EP_MXFP8_E5M2, hidden=32800, sc=0x6001) == 6
     assert L.ep_combine(0x2000, 256, 32, ctypes.byref(d), ctypes.byref(lay), 0, 0, None, 0x5000, B.EP_BF16,
                         None) == 1  # weights missing
     assert L.ep_combine(0x2000, 256, 32, ctypes.byref(d), ctypes.byref(lay), 0, 0, 0x3000, 0x5000, B.EP_FP8_E4M3,
