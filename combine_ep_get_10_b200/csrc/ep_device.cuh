@@ -100,6 +100,13 @@ __device__ __forceinline__ void bulk_store_s2g(void* dst, const void* src_smem, 
                  : "memory");
 }
 
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy (bulk copy) reads of them.
+__device__ __forceinline__ void fence_proxy_async_shared()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_commit()
 {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
@@ -179,6 +186,11 @@ __device__ __forceinline__ uint32_t pack_e2m1x2(float lo, float hi)
         : "=r"(r)
         : "f"(hi), "f"(lo));
     return r;
+}
+
+__device__ __forceinline__ void sts_v2(void* p, uint2 v)
+{
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(smem_addr(p)), "r"(v.x), "r"(v.y) : "memory");
 }
 
 __device__ __forceinline__ void st_u32(void* p, uint32_t v)

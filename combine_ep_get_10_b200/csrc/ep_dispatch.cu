@@ -173,7 +173,6 @@ enum QuantFmt : int {
 struct QuantArgs {
     const uint16_t* x;
     int32_t H;
-    int32_t nper; // 16-byte vectors per thread (<= kQuantMaxVec)
     RowMap map;
     uint8_t* recv;
     void* scales;
@@ -183,8 +182,7 @@ struct QuantArgs {
     uint32_t* err;
 };
 
-constexpr int kQuantMaxVec = 8;     // a row is held in registers: <= 8 vectors of 8 bf16 per thread
-constexpr int kQuantVecTarget = 4;  // vectors per thread the launch aims for
+constexpr int kQuantThreads = 128; // threads per token CTA
 
 __device__ __forceinline__ float amax8(uint4 r)
 {
@@ -232,37 +230,48 @@ __device__ __forceinline__ uint2 encode8(uint4 r, float mul)
     return q;
 }
 
-// One CTA per token.  Thread i holds vectors i, i + nthr, ... of the row
-// (all loads issued up front); the amax is reduced over the scale group --
-// 16 lanes (128 channels), 4 lanes (32, MX) or the whole CTA (per token) --
-// then every thread encodes its vectors once and stores them, with the
-// group's scale, to each destination row of the token.
+// One CTA per token, its row staged in shared memory: a TMA bulk load brings
+// the bf16 row in (completion on an mbarrier, bounded wait) while the
+// threads look up the token's destination rows.  Threads then walk the
+// 16-byte vectors of the row (vector v = j*nthr + tid) and reduce the amax
+// over each scale group by shuffles -- 16 lanes (128 channels), 4 lanes (32,
+// MX) -- or over the CTA for a per-token scale (an extra pass over shared
+// memory), encode every element once into a shared code row and scale row,
+// and hand those to the TMA engine: one bulk store per destination row,
+// issued by different threads.  Rows whose byte size is not a multiple of 16
+// are written with 8-byte stores instead.  Registers stay low, so many CTAs
+// (and their row loads) are resident per SM.
+//   shared memory: x row [2H] | codes [code_row] | scales [scale_row -> 16] | rows [K]
 template <int kFmt>
-__global__ void __launch_bounds__(512, 1) quant_dispatch_kernel(QuantArgs a)
+__global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs a)
 {
     constexpr bool kMx = kFmt == kQMxE4m3 || kFmt == kQMxE5m2 || kFmt == kQMxE2m1;
     constexpr bool kPerToken = kFmt == kQInt8Tok || kFmt == kQFp8Tok;
     constexpr int kGroupLanes = kFmt == kQFp8G128 ? 16 : 4; // group modes only
     constexpr int kCodeBytes = kFmt == kQMxE2m1 ? 4 : 8;  // bytes per 8 channels
-    extern __shared__ __align__(16) int64_t rows[];         // [K]
-    __shared__ float warp_amax[32];
+    extern __shared__ __align__(128) uint8_t qsmem[];
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ float warp_amax[kQuantThreads / 32];
     const int64_t t = blockIdx.x;
     const int tid = threadIdx.x;
-    const int nthr = blockDim.x;
     const int nvec = a.H / 8;
+    const int row_bytes = a.H * 2;
+    const int code_row = nvec * kCodeBytes;
+    const int scale_row = kMx ? nvec / 4 : (kPerToken ? 4 : nvec / 16 * 4);
+    uint8_t* s_x = qsmem;
+    uint8_t* s_codes = qsmem + row_bytes;
+    uint8_t* s_scales = s_codes + code_row;
+    int64_t* rows = reinterpret_cast<int64_t*>(s_scales + ((scale_row + 15) & ~15));
 
-    const uint8_t* xrow = reinterpret_cast<const uint8_t*>(a.x) + t * static_cast<int64_t>(a.H) * 2;
-    uint4 raw[kQuantMaxVec];
-#pragma unroll
-    for (int j = 0; j < kQuantMaxVec; ++j) {
-        const int v = j * nthr + tid;
-        raw[j] = make_uint4(0, 0, 0, 0);
-        if (j < a.nper && v < nvec)
-            raw[j] = ld_nc_v4(xrow + static_cast<int64_t>(v) * 16);
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(row_bytes));
+        bulk_load_g2s(s_x, reinterpret_cast<const uint8_t*>(a.x) + t * static_cast<int64_t>(row_bytes),
+                      static_cast<uint32_t>(row_bytes), &bar);
     }
-
     uint32_t errbits = 0;
-    for (int k = tid; k < a.map.K; k += nthr) {
+    for (int k = tid; k < a.map.K; k += kQuantThreads) {
         const int64_t rk = a.map.row(t, k, errbits);
         rows[k] = rk;
         if (rk >= 0) {
@@ -274,44 +283,43 @@ __global__ void __launch_bounds__(512, 1) quant_dispatch_kernel(QuantArgs a)
     }
     if (errbits)
         flag_error(a.err, errbits);
+    __syncthreads(); // barrier initialised before anyone waits on it
+    if (!mbar_wait_bounded(&bar, 0, a.err))
+        return;
 
-    float tok_amax = 0.0f;
+    float tok_mul = 0.0f;
     if constexpr (kPerToken) {
-#pragma unroll
-        for (int j = 0; j < kQuantMaxVec; ++j)
-            tok_amax = fmaxf(tok_amax, amax8(raw[j]));
+        float amax = 0.0f;
+        for (int v = tid; v < nvec; v += kQuantThreads)
+            amax = fmaxf(amax, amax8(*reinterpret_cast<const uint4*>(s_x + v * 16)));
 #pragma unroll
         for (int d = 16; d >= 1; d >>= 1)
-            tok_amax = fmaxf(tok_amax, __shfl_xor_sync(kFullMask, tok_amax, d));
+            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
         if ((tid & 31) == 0)
-            warp_amax[tid >> 5] = tok_amax;
-    }
-    __syncthreads();
-    if constexpr (kPerToken) {
-        tok_amax = 0.0f;
-        for (int w = 0; w < (nthr >> 5); ++w)
-            tok_amax = fmaxf(tok_amax, warp_amax[w]);
+            warp_amax[tid >> 5] = amax;
+        __syncthreads();
+        amax = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kQuantThreads / 32; ++w)
+            amax = fmaxf(amax, warp_amax[w]);
+        constexpr float qmax = kFmt == kQInt8Tok ? 127.0f : 448.0f;
+        float scale = 0.0f;
+        if (amax > 0.0f) {
+            scale = __fdiv_rn(amax, qmax);
+            tok_mul = fminf(__fdiv_rn(qmax, amax), 3.40282347e38f);
+        }
+        if (tid == 0)
+            *reinterpret_cast<float*>(s_scales) = scale;
     }
 
-    // codes and scale of each held vector
-    uint2 code[kQuantMaxVec];
-    float fscale[kQuantMaxVec];   // fp32 scale of the vector's group (128-channel mode)
-    uint32_t xbyte[kQuantMaxVec]; // e8m0 byte of the vector's block (MX)
-    float tok_scale = 0.0f, tok_mul = 0.0f;
-    if constexpr (kPerToken) {
-        constexpr float qmax = kFmt == kQInt8Tok ? 127.0f : 448.0f;
-        if (tok_amax > 0.0f) {
-            tok_scale = __fdiv_rn(tok_amax, qmax);
-            tok_mul = fminf(__fdiv_rn(qmax, tok_amax), 3.40282347e38f);
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < kQuantMaxVec; ++j) {
+    // uniform trip count: every lane takes part in the group shuffles
+    for (int base = 0; base < nvec; base += kQuantThreads) {
+        const int v = base + tid;
+        const bool active = v < nvec; // a scale group is all-in or all-out
+        const uint4 raw = active ? *reinterpret_cast<const uint4*>(s_x + v * 16) : make_uint4(0, 0, 0, 0);
         float mul = tok_mul;
-        fscale[j] = 0.0f;
-        xbyte[j] = 0;
         if constexpr (!kPerToken) {
-            float amax = amax8(raw[j]);
+            float amax = amax8(raw);
 #pragma unroll
             for (int d = kGroupLanes / 2; d >= 1; d >>= 1)
                 amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
@@ -321,66 +329,93 @@ __global__ void __launch_bounds__(512, 1) quant_dispatch_kernel(QuantArgs a)
                 // zero or subnormal amax clamps to -127 either way
                 const int ef = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
                 const int X = max(ef - 127 - kEmax, -127);
-                xbyte[j] = static_cast<uint32_t>(X + 127);
                 mul = __uint_as_float(static_cast<uint32_t>(127 - X) << 23); // 2^-X, a normal float
+                if (active && (tid & 3) == 0)
+                    s_scales[v / 4] = static_cast<uint8_t>(X + 127);
             } else {
+                float scale = 0.0f;
                 mul = 0.0f;
                 if (amax > 0.0f) {
-                    fscale[j] = __fdiv_rn(amax, 448.0f);
+                    scale = __fdiv_rn(amax, 448.0f);
                     mul = fminf(__fdiv_rn(448.0f, amax), 3.40282347e38f);
                 }
+                if (active && (tid & 15) == 0)
+                    reinterpret_cast<float*>(s_scales)[v / 16] = scale;
             }
         }
-        // dynamic scales: a zero amax gives zero codes (no -0 codes either)
-        code[j] = (kMx || mul != 0.0f) ? encode8<kFmt>(raw[j], mul) : make_uint2(0, 0);
-    }
-
-    const int64_t code_row = static_cast<int64_t>(nvec) * kCodeBytes;
-    for (int k = 0; k < a.map.K; ++k) {
-        const int64_t rk = rows[k];
-        if (rk < 0)
-            continue;
-        uint8_t* dst = a.recv + rk * code_row;
-#pragma unroll
-        for (int j = 0; j < kQuantMaxVec; ++j) {
-            const int v = j * nthr + tid;
-            if (j >= a.nper || v >= nvec)
-                continue;
+        if (active) {
+            // dynamic scales: a zero amax gives zero codes (no -0 codes either)
+            const uint2 q = (kMx || mul != 0.0f) ? encode8<kFmt>(raw, mul) : make_uint2(0, 0);
             if constexpr (kCodeBytes == 8)
-                st_v2(dst + static_cast<int64_t>(v) * 8, code[j]);
+                sts_v2(s_codes + v * 8, q);
             else
-                st_u32(dst + static_cast<int64_t>(v) * 4, code[j].x);
-            if constexpr (kMx) {
-                if ((tid & 3) == 0)
-                    static_cast<uint8_t*>(a.scales)[rk * (nvec / 4) + v / 4] = static_cast<uint8_t>(xbyte[j]);
-            } else if constexpr (kFmt == kQFp8G128) {
-                if ((tid & 15) == 0)
-                    static_cast<float*>(a.scales)[rk * (nvec / 16) + v / 16] = fscale[j];
-            }
-        }
-        if constexpr (kPerToken) {
-            if (tid == 0)
-                static_cast<float*>(a.scales)[rk] = tok_scale;
+                reinterpret_cast<uint32_t*>(s_codes)[v] = q.x;
         }
     }
+    fence_proxy_async_shared();
+    __syncthreads();
+
+    const bool bulk_codes = (code_row & 15) == 0;
+    const bool bulk_scales = (scale_row & 15) == 0 && (reinterpret_cast<uintptr_t>(a.scales) & 15) == 0;
+    if (bulk_codes) {
+        bool issued = false;
+        for (int k = tid; k < a.map.K; k += kQuantThreads) {
+            const int64_t rk = rows[k];
+            if (rk < 0)
+                continue;
+            bulk_store_s2g(a.recv + rk * code_row, s_codes, static_cast<uint32_t>(code_row));
+            if (bulk_scales)
+                bulk_store_s2g(static_cast<uint8_t*>(a.scales) + rk * scale_row, s_scales,
+                               static_cast<uint32_t>(scale_row));
+            issued = true;
+        }
+        if (issued)
+            bulk_commit();
+    } else {
+        for (int k = 0; k < a.map.K; ++k) {
+            const int64_t rk = rows[k];
+            if (rk < 0)
+                continue;
+            uint8_t* dst = a.recv + rk * code_row;
+            for (int i = tid; i < code_row / 8; i += kQuantThreads)
+                st_v2(dst + i * 8, *reinterpret_cast<const uint2*>(s_codes + i * 8));
+        }
+    }
+    if (!(bulk_codes && bulk_scales)) {
+        // scales by plain stores (per-token: 4 bytes; rows not 16-byte multiples)
+        for (int k = 0; k < a.map.K; ++k) {
+            const int64_t rk = rows[k];
+            if (rk < 0)
+                continue;
+            uint8_t* dst = static_cast<uint8_t*>(a.scales) + rk * scale_row;
+            if constexpr (kMx) {
+                for (int i = tid; i < scale_row; i += kQuantThreads)
+                    dst[i] = s_scales[i];
+            } else {
+                for (int i = tid; i < scale_row / 4; i += kQuantThreads)
+                    reinterpret_cast<float*>(dst)[i] = reinterpret_cast<const float*>(s_scales)[i];
+            }
+        }
+    }
+    if (bulk_codes)
+        bulk_wait_read_all(); // shared memory must outlive the copies' reads
 }
 
 template <int kFmt>
-cudaError_t launch_quant(const QuantArgs& k, int32_t T, int32_t K, cudaStream_t stream)
+cudaError_t launch_quant(const QuantArgs& a, int32_t T, int32_t K, cudaStream_t stream)
 {
-    const int nvec = k.H / 8;
-    int nthr = (nvec + kQuantVecTarget - 1) / kQuantVecTarget;
-    nthr = ((nthr + 31) / 32) * 32;
-    nthr = std::min(std::max(nthr, 32), 512);
-    QuantArgs a = k;
-    a.nper = (nvec + nthr - 1) / nthr;
-    const size_t smem = sizeof(int64_t) * static_cast<size_t>(K);
-    if (smem > 40 * 1024) {
+    const size_t nvec = static_cast<size_t>(a.H) / 8;
+    const bool mx = kFmt == kQMxE4m3 || kFmt == kQMxE5m2 || kFmt == kQMxE2m1;
+    const size_t code_row = nvec * (kFmt == kQMxE2m1 ? 4 : 8);
+    const size_t scale_row = mx ? nvec / 4 : ((kFmt == kQInt8Tok || kFmt == kQFp8Tok) ? 4 : nvec / 16 * 4);
+    const size_t smem = nvec * 16 + code_row + ((scale_row + 15) & ~static_cast<size_t>(15)) + sizeof(int64_t) * K;
+    if (smem > 48 * 1024) {
         cudaError_t st = cudaFuncSetAttribute(quant_dispatch_kernel<kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               static_cast<int>(smem));
         if (st != cudaSuccess)
             return st;
     }
+    const int nthr = kQuantThreads;
     quant_dispatch_kernel<kFmt><<<T, nthr, smem, stream>>>(a);
     return cudaGetLastError();
 }
@@ -410,7 +445,7 @@ cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream)
     RowMap m{a.rows.topk_idx, a.rows.slot, a.rows.offsets, a.rows.K, a.rows.E, a.rows.mode, a.rows.max_tokens,
              a.rows.num_rows};
     if (a.out_dtype != EP_BF16) {
-        QuantArgs k{static_cast<const uint16_t*>(a.x), a.H, 0, m, static_cast<uint8_t*>(a.recv_x), a.recv_scales,
+        QuantArgs k{static_cast<const uint16_t*>(a.x), a.H, m, static_cast<uint8_t*>(a.recv_x), a.recv_scales,
                     a.topk_weights, a.recv_src, a.recv_weights, a.err};
         switch (a.out_dtype) {
         case EP_FP8_E4M3:

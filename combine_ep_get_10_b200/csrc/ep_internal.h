@@ -13,7 +13,7 @@ namespace ep {
 
 constexpr size_t kWorkspaceHeaderBytes = 256; // error word + reserved
 constexpr int kMaxTopkLayoutExperts = 1024;   // token-choice layout keeps E counters per warp
-constexpr int kMaxQuantHidden = 32768;        // quantising dispatch holds a row in registers (512 threads x 64)
+constexpr int kMaxQuantHidden = 32768;        // quantising dispatch stages a row (2H + H bytes) in shared memory
 
 inline uint32_t* error_word(void* workspace)
 {
