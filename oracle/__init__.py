@@ -81,6 +81,12 @@ def load(path: str):
     L.oracle_tc_dispatch.argtypes = [P, i32, i32, P, i32, i32, P, P, i32, i32, i64, i32, P, P, P, P, P]
     L.oracle_tc_combine.restype = None
     L.oracle_tc_combine.argtypes = [P, i64, i32, i32, P, i32, i32, P, P, i32, i32, P, P, i32, i32, P]
+    L.oracle_rank_layout.restype = None
+    L.oracle_rank_layout.argtypes = [P, i32, i32, P, P]
+    L.oracle_rank_dispatch.restype = None
+    L.oracle_rank_dispatch.argtypes = [P, i32, i32, P, i32, i32, i32, P, P, P, P, P, P]
+    L.oracle_rank_combine.restype = None
+    L.oracle_rank_combine.argtypes = [P, i32, i32, i32, P, P, i32, i32, P]
     L.oracle_ec_layout.restype = i64
     L.oracle_ec_layout.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P]
     L.oracle_ec_dispatch.restype = None
@@ -270,6 +276,46 @@ def tc_combine(y_bits, topk_idx, num_experts, layout, topk_weights, mode=COMPACT
     out = np.empty((n, H), np.float32 if out_dtype == FP32 else np.uint16)
     lib().oracle_tc_combine(_p(y), y.shape[0], H, T, _p(idx), K, int(num_experts), _p(slot), _p(offs),
                             int(mode), int(max_tokens), _p(w), _p(tok), n, int(out_dtype), _p(out))
+    return out
+
+
+# ------------------------------------------- per-rank (deduplicated) path
+def rank_layout(is_token_in_rank):
+    """is_token_in_rank [T, R] -> dict(rank_offsets [R+1], rank_row [T, R])."""
+    m = _c(is_token_in_rank, np.uint8)
+    T, R = m.shape
+    out = dict(rank_offsets=np.empty(R + 1, np.int32), rank_row=np.empty((T, R), np.int32))
+    lib().oracle_rank_layout(_p(m), T, R, _p(out["rank_offsets"]), _p(out["rank_row"]))
+    return out
+
+
+def rank_dispatch(x_bits, topk_idx, num_experts, num_ranks, rlayout, topk_weights=None, want_src=False):
+    """Returns dict(recv [rows, H] bf16 bits, recv_topk_idx [rows, K], recv_topk_weights [rows, K], recv_src)."""
+    x = _c(x_bits, np.uint16)
+    idx = _c(topk_idx, np.int64)
+    T, H = x.shape
+    K = idx.shape[1]
+    rr = _c(rlayout["rank_row"], np.int32)
+    rows = int(rlayout["rank_offsets"][-1])
+    w = _c(topk_weights, np.float32) if topk_weights is not None else np.zeros((T, K), np.float32)
+    recv = np.zeros((rows, H), np.uint16)
+    ridx = np.full((rows, K), -2, np.int64)
+    rw = np.full((rows, K), np.nan, np.float32)
+    src = np.full(rows, -1, np.int32) if want_src else None
+    lib().oracle_rank_dispatch(_p(x), T, H, _p(idx), K, int(num_experts), int(num_ranks), _p(rr), _p(w), _p(recv),
+                               _p(ridx), _p(rw), _p(src))
+    return dict(recv=recv, recv_topk_idx=ridx, recv_topk_weights=rw, recv_src=src)
+
+
+def rank_combine(y_bits, rlayout, out_dtype=FP32, tokens=None):
+    y = _c(y_bits, np.uint16)
+    H = y.shape[1]
+    rr = _c(rlayout["rank_row"], np.int32)
+    T, R = rr.shape
+    tok = None if tokens is None else _c(tokens, np.int32)
+    n = T if tok is None else tok.size
+    out = np.empty((n, H), np.float32 if out_dtype == FP32 else np.uint16)
+    lib().oracle_rank_combine(_p(y), H, T, R, _p(rr), _p(tok), n, int(out_dtype), _p(out))
     return out
 
 

@@ -657,6 +657,99 @@ void oracle_tc_combine(const uint16_t* y, int64_t num_y_rows, int32_t H, int32_t
 }
 
 /* ---------------------------------------------------------------------
+ * Per-rank (deduplicated) dispatch and rank-level combine.  [README] "API
+ * Overview": normal-mode dispatch sends tokens to expert *ranks* and returns
+ * the received tokens with their top-k information; combine reduces the
+ * tokens coming back from the ranks, using the dispatch handle; the layout
+ * gives is_token_in_rank.  Reading: a token travels once to every rank
+ * that holds at least one of its experts (is_token_in_rank[t, r] = 1).
+ * Rank r's received rows are its tokens in ascending token order, and the
+ * ranks' row ranges are laid end to end: rank_offsets[R+1] is the exclusive
+ * scan of the per-rank token counts and rank_row[t, r] is token t's row
+ * (rank_offsets[r] + number of earlier tokens of rank r), -1 where t does
+ * not go to r.  Each received row carries the token's K entries as seen by
+ * the rank: the local expert id e - r*E/R for an expert of rank r and its
+ * gate weight, else -1 and 0.  The rank-level combine adds, for each token,
+ * the rows its ranks send back, in ascending rank order, in fp32 from 0
+ * (the gate weights were applied on the ranks), written as fp32 or rounded
+ * once to bf16.
+ * ------------------------------------------------------------------- */
+void oracle_rank_layout(const uint8_t* is_token_in_rank, int32_t T, int32_t R, int32_t* rank_offsets,
+                        int32_t* rank_row)
+{
+    int32_t* count = (int32_t*)calloc((size_t)R + 1, sizeof(int32_t));
+    for (int32_t t = 0; t < T; ++t) {
+        for (int32_t r = 0; r < R; ++r) {
+            if (is_token_in_rank[(int64_t)t * R + r]) {
+                rank_row[(int64_t)t * R + r] = count[r];
+                count[r] += 1;
+            } else {
+                rank_row[(int64_t)t * R + r] = -1;
+            }
+        }
+    }
+    rank_offsets[0] = 0;
+    for (int32_t r = 0; r < R; ++r)
+        rank_offsets[r + 1] = rank_offsets[r] + count[r];
+    for (int32_t t = 0; t < T; ++t)
+        for (int32_t r = 0; r < R; ++r)
+            if (rank_row[(int64_t)t * R + r] >= 0)
+                rank_row[(int64_t)t * R + r] += rank_offsets[r];
+    free(count);
+}
+
+void oracle_rank_dispatch(const uint16_t* x, int32_t T, int32_t H, const int64_t* topk_idx, int32_t K,
+                          int32_t E, int32_t R, const int32_t* rank_row, const float* topk_weights,
+                          uint16_t* recv, int64_t* recv_topk_idx, float* recv_topk_weights, int32_t* recv_src)
+{
+    int32_t per_rank = E / R;
+    for (int32_t t = 0; t < T; ++t) {
+        for (int32_t r = 0; r < R; ++r) {
+            int64_t row = rank_row[(int64_t)t * R + r];
+            if (row < 0)
+                continue;
+            memcpy(recv + row * H, x + (int64_t)t * H, sizeof(uint16_t) * (size_t)H);
+            if (recv_src)
+                recv_src[row] = t;
+            for (int32_t k = 0; k < K; ++k) {
+                int64_t e = topk_idx[(int64_t)t * K + k];
+                int local = e >= 0 && e < E && e / per_rank == r;
+                if (recv_topk_idx)
+                    recv_topk_idx[row * K + k] = local ? e - (int64_t)r * per_rank : -1;
+                if (recv_topk_weights)
+                    recv_topk_weights[row * K + k] = local ? topk_weights[(int64_t)t * K + k] : 0.0f;
+            }
+        }
+    }
+}
+
+void oracle_rank_combine(const uint16_t* y, int32_t H, int32_t T, int32_t R, const int32_t* rank_row,
+                         const int32_t* tokens, int32_t n_tokens, int32_t out_dtype, void* out)
+{
+    float* acc = (float*)malloc(sizeof(float) * (size_t)H);
+    int32_t n = tokens ? n_tokens : T;
+    for (int32_t i = 0; i < n; ++i) {
+        int32_t t = tokens ? tokens[i] : i;
+        for (int32_t h = 0; h < H; ++h)
+            acc[h] = 0.0f;
+        for (int32_t r = 0; r < R; ++r) {
+            int64_t row = rank_row[(int64_t)t * R + r];
+            if (row < 0)
+                continue;
+            for (int32_t h = 0; h < H; ++h)
+                acc[h] = acc[h] + oracle_bf16_to_f32(y[row * H + h]);
+        }
+        for (int32_t h = 0; h < H; ++h) {
+            if (out_dtype == OR_FP32)
+                ((float*)out)[(int64_t)i * H + h] = acc[h];
+            else
+                ((uint16_t*)out)[(int64_t)i * H + h] = oracle_f32_to_bf16(acc[h]);
+        }
+    }
+    free(acc);
+}
+
+/* ---------------------------------------------------------------------
  * Expert-choice layout.  [EC] "Proposed Solutions", Solution 1: the
  * routing is token_indices[E, C] (expert e picked token token_indices[e,c]
  * in slot c); no [T, K] inverse table with padding is built.  What the

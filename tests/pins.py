@@ -695,6 +695,128 @@ def pin_tc_cfg1_closed_form(o):
     assert (np.abs(out - exact) <= bound).all()
 
 
+# --------------------------------------------------- per-rank (dedup) path
+def _brute_rank(idx, E, R):
+    """Rank r's tokens by enumeration from topk_idx itself: the tokens with
+    at least one valid expert in r's block, ascending; rows laid end to end."""
+    T, K = idx.shape
+    per = E // R
+    lists = [[t for t in range(T) if any(0 <= idx[t, k] < E and idx[t, k] // per == r for k in range(K))]
+             for r in range(R)]
+    offsets = np.concatenate([[0], np.cumsum([len(l) for l in lists])])
+    row = np.full((T, R), -1, np.int64)
+    for r in range(R):
+        for j, t in enumerate(lists[r]):
+            row[t, r] = offsets[r] + j
+    return offsets, row
+
+
+def pin_rank_layout_bruteforce(o):
+    for T, E, R, K, p_neg, dup, p_bad, seed in TC_CASES:
+        idx = W.random_topk(_rng(seed), T, E, K, p_neg=p_neg, allow_dup=dup, p_bad=p_bad).reshape(T, K)
+        L = o.tc_layout(idx, E, R)
+        got = o.rank_layout(L["is_token_in_rank"])
+        offsets, row = _brute_rank(idx, E, R)
+        assert np.array_equal(got["rank_offsets"], offsets), (T, E, R, K)
+        assert np.array_equal(got["rank_row"], row)
+        assert got["rank_offsets"][-1] == L["num_tokens_per_rank"].sum()
+
+
+def pin_rank_dispatch_bruteforce(o):
+    """Each (token, rank) row holds x[t] once; its K entries are the local
+    ids and weights of the token's experts in that rank (-1 / 0 elsewhere);
+    every valid (t, k) pair appears in exactly one received row."""
+    rng = _rng(61)
+    for T, E, R, K, H in [(37, 16, 4, 5, 64), (20, 8, 8, 3, 128), (9, 64, 32, 40, 32)]:
+        idx = W.random_topk(rng, T, E, K, p_neg=0.2, allow_dup=True, p_bad=0.05)
+        x = _torch_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+        w = rng.random((T, K)).astype(np.float32)
+        L = o.tc_layout(idx, E, R)
+        RL = o.rank_layout(L["is_token_in_rank"])
+        D = o.rank_dispatch(x, idx, E, R, RL, w, want_src=True)
+        offsets, row = _brute_rank(idx, E, R)
+        per = E // R
+        seen = 0
+        for t in range(T):
+            for r in range(R):
+                rw = row[t, r]
+                if rw < 0:
+                    continue
+                assert np.array_equal(D["recv"][rw], x[t]) and D["recv_src"][rw] == t
+                for k in range(K):
+                    e = int(idx[t, k])
+                    if 0 <= e < E and e // per == r:
+                        assert D["recv_topk_idx"][rw, k] == e - r * per and D["recv_topk_weights"][rw, k] == w[t, k]
+                        seen += 1
+                    else:
+                        assert D["recv_topk_idx"][rw, k] == -1 and D["recv_topk_weights"][rw, k] == 0.0
+        assert seen == int(((idx >= 0) & (idx < E)).sum())
+        assert (D["recv_src"] >= 0).all()  # rows are dense
+
+
+def pin_rank_combine_bound_and_units(o):
+    rng = _rng(62)
+    T, E, R, K, H = 40, 32, 8, 6, 64
+    idx = W.random_topk(rng, T, E, K, p_neg=0.3)
+    L = o.tc_layout(idx, E, R)
+    RL = o.rank_layout(L["is_token_in_rank"])
+    rows = int(RL["rank_offsets"][-1])
+    offsets, row = _brute_rank(idx, E, R)
+    y = _torch_bf16_bits(rng.standard_normal((rows, H)).astype(np.float32))
+    yf = _bf16_f64(y)
+    for out_dtype in (W.FP32, W.BF16):
+        out = o.rank_combine(y, RL, out_dtype=out_dtype)
+        outf = out.astype(np.float64) if out_dtype == W.FP32 else _bf16_f64(out)
+        for t in range(T):
+            rs = [row[t, r] for r in range(R) if row[t, r] >= 0]
+            exact = yf[rs].sum(axis=0) if rs else np.zeros(H)
+            mag = np.abs(yf[rs]).sum(axis=0) if rs else np.zeros(H)
+            bound = len(rs) * U32 * mag * 1.0001
+            if out_dtype == W.BF16:
+                bound = bound + UBF * np.abs(exact) * 1.0001
+            assert (np.abs(outf[t] - exact) <= bound + 1e-300).all(), t
+            if not rs:
+                assert (outf[t] == 0).all() and not np.signbit(outf[t]).any()
+    ones = np.full((rows, 8), 0x3F80, np.uint16)  # every rank sends back 1.0
+    out = o.rank_combine(ones, RL, out_dtype=W.FP32)
+    assert np.array_equal(out[:, 0], L["is_token_in_rank"].sum(axis=1).astype(np.float32))
+
+
+def pin_rank_combine_order_closed_form(o):
+    """One token in ranks 0, 1, 2 returning 1, 2^-24, -1: ascending-rank fp32
+    addition gives exactly 0 (1 + 2^-24 rounds to 1); any other order that
+    adds 2^-24 last, or first to -1, does not."""
+    idx = np.array([[0, 1, 2]], np.int64)
+    L = o.tc_layout(idx, 3, 3)
+    RL = o.rank_layout(L["is_token_in_rank"])
+    assert RL["rank_row"].tolist() == [[0, 1, 2]]
+    y = _torch_bf16_bits(np.array([[1.0] * 4, [2.0 ** -24] * 4, [-1.0] * 4], np.float32))
+    assert (o.rank_combine(y, RL, out_dtype=W.FP32) == 0.0).all()
+    y = _torch_bf16_bits(np.array([[-1.0] * 4, [2.0 ** -24] * 4, [1.0] * 4], np.float32))
+    assert (o.rank_combine(y, RL, out_dtype=W.FP32) == np.float32(2.0 ** -24)).all()
+
+
+def pin_rank_path_matches_expert_path(o):
+    """Rank dispatch, a per-rank weighted sum over the local experts (each
+    expert returning its input unchanged), then rank combine equals the
+    per-expert dispatch + weighted combine within the fp32 bound: both are
+    sum_k w_k x_t."""
+    inp = W.make_inputs(2, T=64)
+    x, idx, w = inp["x"], inp["topk_idx"], inp["topk_weights"]
+    E, R, K = 256, 8, 8
+    L = o.tc_layout(idx, E, R)
+    RL = o.rank_layout(L["is_token_in_rank"])
+    D = o.rank_dispatch(x, idx, E, R, RL, w)
+    xr = _bf16_f64(D["recv"])
+    yr = (xr * D["recv_topk_weights"].astype(np.float64).sum(axis=1)[:, None]).astype(np.float32)
+    out_rank = o.rank_combine(_torch_bf16_bits(yr), RL, out_dtype=W.FP32).astype(np.float64)
+    out_exp = o.tc_combine(o.tc_dispatch(x, idx, E, L)["recv"], idx, E, L, w, out_dtype=W.FP32).astype(np.float64)
+    xf = _bf16_f64(x)
+    mag = np.abs(xf) * np.abs(w.astype(np.float64)).sum(axis=1)[:, None]
+    bound = (2 * UBF + (K + R + 2) * U32) * mag * 1.0001
+    assert (np.abs(out_rank - out_exp) <= bound + 1e-300).all()
+
+
 # ----------------------------------------------------------- expert choice
 def _brute_ec(ti, T, R):
     E, C = ti.shape

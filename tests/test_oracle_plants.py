@@ -59,6 +59,17 @@ PLANTS = [
     ("mx_block_amax_of_16", "float amax = row_amax(xrow + g * 32, 32);", "float amax = row_amax(xrow + g * 32, 16);", "pin_mx"),
     ("fp4_nibbles_swapped", "if (h % 2 == 0)\n                    q[h / 2] = c;\n                else\n                    q[h / 2] = (uint8_t)(q[h / 2] | (c << 4));",
      "if (h % 2 == 0)\n                    q[h / 2] = (uint8_t)(c << 4);\n                else\n                    q[h / 2] = (uint8_t)(q[h / 2] | c);", "pin_mx"),
+    ("rank_rows_by_token_descending", "    for (int32_t t = 0; t < T; ++t) {\n        for (int32_t r = 0; r < R; ++r) {\n            if (is_token_in_rank[(int64_t)t * R + r]) {",
+     "    for (int32_t t = T - 1; t >= 0; --t) {\n        for (int32_t r = 0; r < R; ++r) {\n            if (is_token_in_rank[(int64_t)t * R + r]) {", "pin_rank"),
+    ("rank_offsets_inclusive", "rank_offsets[r + 1] = rank_offsets[r] + count[r];", "rank_offsets[r + 1] = rank_offsets[r] + count[r] + (r == 0);", "pin_rank"),
+    ("rank_local_id_global", "recv_topk_idx[row * K + k] = local ? e - (int64_t)r * per_rank : -1;",
+     "recv_topk_idx[row * K + k] = local ? e : -1;", "pin_rank_dispatch"),
+    ("rank_weight_of_foreign_expert", "recv_topk_weights[row * K + k] = local ? topk_weights[(int64_t)t * K + k] : 0.0f;",
+     "recv_topk_weights[row * K + k] = topk_weights[(int64_t)t * K + k];", "pin_rank"),
+    ("rank_combine_descending", "        for (int32_t r = 0; r < R; ++r) {\n            int64_t row = rank_row[(int64_t)t * R + r];\n            if (row < 0)\n                continue;\n            for (int32_t h = 0; h < H; ++h)\n                acc[h] = acc[h] +",
+     "        for (int32_t r = R - 1; r >= 0; --r) {\n            int64_t row = rank_row[(int64_t)t * R + r];\n            if (row < 0)\n                continue;\n            for (int32_t h = 0; h < H; ++h)\n                acc[h] = acc[h] +", "pin_rank"),
+    ("rank_combine_skips_last_rank", "            if (row < 0)\n                continue;\n            for (int32_t h = 0; h < H; ++h)\n                acc[h] = acc[h] +",
+     "            if (row < 0 || (r == R - 1 && R > 1))\n                continue;\n            for (int32_t h = 0; h < H; ++h)\n                acc[h] = acc[h] +", "pin_rank"),
     ("quant_dispatch_scale_row_shift", "memcpy((uint8_t*)recv_scales + row * scale_bytes, srow",
      "memcpy((uint8_t*)recv_scales + (row / 2 * 2) * scale_bytes, srow", "pin_quant_dispatch"),
 ]
