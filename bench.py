@@ -55,6 +55,8 @@ def parse():
                     help="with --workloads: just this workload")
     ap.add_argument("--quant", action="store_true",
                     help="with --workloads: also time every quantised dispatch format on the token-choice workloads")
+    ap.add_argument("--ranks", action="store_true",
+                    help="with --workloads: also time the per-rank (deduplicated) dispatch and combine")
     return ap.parse_args()
 
 
@@ -541,6 +543,25 @@ def run_workload_table(args):
             emit(cfg, "combine", timeit(lambda: B.ep_combine(y, rt, lay, w, out, mode=mode,
                                                              max_tokens_per_expert=mt)),
                  n_valid * H * 2 + T * H * 2 + T * K * 16 + E * 4, T)
+            if args.ranks and mode == W.COMPACT:
+                rl = B.RankLayout(rt, device=dev)
+                emit(cfg, "rank_layout", timeit(lambda: B.ep_get_rank_layout(rt, lay, rl)),
+                     T * R + R * 4 + (R + 1) * 4 + T * R * 4, T)
+                B.ep_get_rank_layout(rt, lay, rl)
+                n_rank = int(rl.rank_offsets[-1].item())
+                rrecv = torch.empty((n_rank, H), dtype=torch.bfloat16, device=dev)
+                ridx = torch.empty((n_rank, K), dtype=torch.int64, device=dev)
+                rwt = torch.empty((n_rank, K), dtype=torch.float32, device=dev)
+                emit(cfg, "dispatch_ranks",
+                     timeit(lambda: B.ep_dispatch_ranks(x, rt, lay, rl, rrecv, topk_weights=w, recv_topk_idx=ridx,
+                                                        recv_topk_weights=rwt)),
+                     T * H * 2 + n_rank * H * 2 + n_rank * K * 12 + T * R * 4 + T * K * 12, T)
+                rout = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+                emit(cfg, "combine_ranks", timeit(lambda: B.ep_combine_ranks(rrecv, rt, lay, rl, rout)),
+                     n_rank * H * 2 + T * H * 2 + T * R * 4, T)
+                print(json.dumps({"workload": cfg["name"], "rank_rows": n_rank, "expert_rows": n_valid,
+                                  "rows_saved": round(1 - n_rank / max(n_valid, 1), 3)}), flush=True)
+                del rrecv, ridx, rwt, rout
             if args.quant:
                 del recv
                 for name, dt, code_b, scale_b in QUANT_FORMATS:

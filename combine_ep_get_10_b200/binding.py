@@ -27,7 +27,7 @@ EP_DEVERR_BAD_INDEX, EP_DEVERR_OVERFLOW, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 EXPORTED = ("ep_workspace_bytes", "ep_workspace_init", "ep_get_layout", "ep_dispatch", "ep_combine",
             "ep_dispatch_expert_choice", "ep_combine_expert_choice", "ep_get_device_error", "ep_status_string",
-            "ep_version", "ep_get_layout_no_alloc")
+            "ep_version", "ep_get_layout_no_alloc", "ep_get_rank_layout", "ep_dispatch_ranks", "ep_combine_ranks")
 
 
 class EPError(RuntimeError):
@@ -47,6 +47,10 @@ class LayoutDesc(ctypes.Structure):
                 ("num_tokens_per_rank", ctypes.c_void_p), ("is_token_in_rank", ctypes.c_void_p),
                 ("slot", ctypes.c_void_p), ("token_offsets", ctypes.c_void_p), ("token_slots", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class RankLayoutDesc(ctypes.Structure):
+    _fields_ = [("rank_offsets", ctypes.c_void_p), ("rank_row", ctypes.c_void_p)]
 
 
 _lib = None
@@ -85,6 +89,13 @@ def lib():
         L.ep_version.argtypes = []
         L.ep_get_layout_no_alloc.restype = st
         L.ep_get_layout_no_alloc.argtypes = [RP, LP, P, P]
+        KP = ctypes.POINTER(RankLayoutDesc)
+        L.ep_get_rank_layout.restype = st
+        L.ep_get_rank_layout.argtypes = [RP, LP, KP, P]
+        L.ep_dispatch_ranks.restype = st
+        L.ep_dispatch_ranks.argtypes = [P, i32, RP, LP, KP, i64, P, P, P, P, P, P]
+        L.ep_combine_ranks.restype = st
+        L.ep_combine_ranks.argtypes = [P, i32, i64, RP, LP, KP, P, st, P]
         _lib = L
     return _lib
 
@@ -283,6 +294,42 @@ def ep_get_device_error(layout: Layout, clear: bool = True, stream=None) -> int:
 
 def ep_status_string(status: int) -> str:
     return lib().ep_status_string(status).decode()
+
+
+class RankLayout:
+    """Device buffers of a per-rank layout: rank_offsets [R+1] and
+    rank_row [T, R] (allocated by torch), plus the C descriptor."""
+
+    def __init__(self, routing: Routing, device="cuda"):
+        d = device
+        T, R = routing.desc.num_tokens, routing.desc.num_ranks
+        self.rank_offsets = torch.empty(R + 1, dtype=torch.int32, device=d)
+        self.rank_row = torch.empty((T, R), dtype=torch.int32, device=d)
+        self.desc = RankLayoutDesc(self.rank_offsets.data_ptr(), self.rank_row.data_ptr() if T > 0 else None)
+
+
+def ep_get_rank_layout(routing: Routing, layout: Layout, rank_layout: RankLayout, stream=None) -> None:
+    _check(lib().ep_get_rank_layout(ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                                    ctypes.byref(rank_layout.desc), _stream(stream)), "ep_get_rank_layout")
+
+
+def ep_dispatch_ranks(x: torch.Tensor, routing: Routing, layout: Layout, rank_layout: RankLayout,
+                      recv_x: torch.Tensor, *, num_recv_rows=None, topk_weights=None, recv_topk_idx=None,
+                      recv_topk_weights=None, recv_src=None, stream=None) -> None:
+    rows = recv_x.shape[0] if num_recv_rows is None else int(num_recv_rows)
+    _check(lib().ep_dispatch_ranks(_ptr(x), x.shape[1], ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                                   ctypes.byref(rank_layout.desc), rows, _ptr(topk_weights), _ptr(recv_x),
+                                   _ptr(recv_topk_idx), _ptr(recv_topk_weights), _ptr(recv_src), _stream(stream)),
+           "ep_dispatch_ranks")
+
+
+def ep_combine_ranks(y: torch.Tensor, routing: Routing, layout: Layout, rank_layout: RankLayout, out: torch.Tensor,
+                     *, num_y_rows=None, stream=None) -> None:
+    """out dtype follows `out` (bfloat16 or float32)."""
+    rows = y.shape[0] if num_y_rows is None else int(num_y_rows)
+    _check(lib().ep_combine_ranks(_ptr(y), y.shape[1], rows, ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                                  ctypes.byref(rank_layout.desc), _ptr(out), _dtype_code(out), _stream(stream)),
+           "ep_combine_ranks")
 
 
 def ep_get_layout_no_alloc(routing: Routing, layout: Layout, device_error_flags: torch.Tensor | None = None,

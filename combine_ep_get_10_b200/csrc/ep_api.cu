@@ -319,6 +319,114 @@ ep_status_t ep_combine_expert_choice(const void* y, int32_t hidden, const ep_rou
     return from_cuda(ep::launch_ec_combine(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+
+// Checks shared by the per-rank entry points: routing, the error word of
+// the layout workspace, and a rank layout with both arrays.
+ep_status_t check_rank_call(const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                            const ep_rank_layout_t* rank_layout)
+{
+    ep_status_t st = check_routing(routing);
+    if (st != EP_OK)
+        return st;
+    st = check_workspace(routing, layout, false);
+    if (st != EP_OK)
+        return st;
+    if (rank_layout == nullptr || rank_layout->rank_offsets == nullptr || !aligned(rank_layout->rank_offsets, 4))
+        return EP_ERR_INVALID_ARG;
+    if (routing->num_tokens > 0 && (rank_layout->rank_row == nullptr || !aligned(rank_layout->rank_row, 4)))
+        return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+} // namespace
+
+ep_status_t ep_get_rank_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                               const ep_rank_layout_t* rank_layout, ep_stream_t stream)
+{
+    ep_status_t st = check_rank_call(routing, layout, rank_layout);
+    if (st != EP_OK)
+        return st;
+    if (layout->num_tokens_per_rank == nullptr || !aligned(layout->num_tokens_per_rank, 4) ||
+        (routing->num_tokens > 0 && layout->is_token_in_rank == nullptr))
+        return EP_ERR_INVALID_ARG;
+    ep::RankLayoutLaunch a{layout->is_token_in_rank,
+                           layout->num_tokens_per_rank,
+                           routing->num_tokens,
+                           routing->num_ranks,
+                           rank_layout->rank_offsets,
+                           rank_layout->rank_row};
+    return from_cuda(ep::launch_rank_layout(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_dispatch_ranks(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                              const ep_layout_t* layout, const ep_rank_layout_t* rank_layout, int64_t num_recv_rows,
+                              const float* topk_weights, void* recv_x, int64_t* recv_topk_idx,
+                              float* recv_topk_weights, int32_t* recv_src, ep_stream_t stream)
+{
+    ep_status_t st = check_rank_call(routing, layout, rank_layout);
+    if (st != EP_OK)
+        return st;
+    if (routing->routing != EP_ROUTING_TOPK || hidden < 1 || hidden % 8 != 0 || num_recv_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    const int32_t T = routing->num_tokens;
+    if (T > 0 && (x == nullptr || !aligned(x, 16)))
+        return EP_ERR_INVALID_ARG;
+    if (num_recv_rows > 0 && (recv_x == nullptr || !aligned(recv_x, 16)))
+        return EP_ERR_INVALID_ARG;
+    if (recv_topk_idx != nullptr && !aligned(recv_topk_idx, 8))
+        return EP_ERR_INVALID_ARG;
+    if (recv_topk_weights != nullptr &&
+        (topk_weights == nullptr || !aligned(topk_weights, 4) || !aligned(recv_topk_weights, 4)))
+        return EP_ERR_INVALID_ARG;
+    if (recv_src != nullptr && !aligned(recv_src, 4))
+        return EP_ERR_INVALID_ARG;
+    ep::RankDispatchLaunch a{x,
+                             T,
+                             hidden,
+                             routing->num_topk,
+                             routing->num_experts,
+                             routing->num_ranks,
+                             routing->topk_idx,
+                             topk_weights,
+                             rank_layout->rank_row,
+                             num_recv_rows,
+                             recv_x,
+                             recv_topk_idx,
+                             recv_topk_weights,
+                             recv_src,
+                             ep::error_word(layout->workspace)};
+    return from_cuda(ep::launch_rank_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_combine_ranks(const void* y, int32_t hidden, int64_t num_y_rows, const ep_routing_desc_t* routing,
+                             const ep_layout_t* layout, const ep_rank_layout_t* rank_layout, void* out,
+                             ep_dtype_t out_dtype, ep_stream_t stream)
+{
+    ep_status_t st = check_rank_call(routing, layout, rank_layout);
+    if (st != EP_OK)
+        return st;
+    if (hidden < 1 || hidden % 8 != 0 || num_y_rows < 0 || (out_dtype != EP_BF16 && out_dtype != EP_FP32))
+        return EP_ERR_INVALID_ARG;
+    const int32_t T = routing->num_tokens;
+    if (num_y_rows > 0 && (y == nullptr || !aligned(y, 16)))
+        return EP_ERR_INVALID_ARG;
+    if (T > 0 && (out == nullptr || !aligned(out, 16)))
+        return EP_ERR_INVALID_ARG;
+    if (T == 0)
+        return EP_OK;
+    ep::RankCombineLaunch a{y,
+                            T,
+                            hidden,
+                            routing->num_ranks,
+                            num_y_rows,
+                            rank_layout->rank_row,
+                            out,
+                            static_cast<int32_t>(out_dtype),
+                            ep::error_word(layout->workspace)};
+    return from_cuda(ep::launch_rank_combine(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ep_status_t ep_get_device_error(const ep_layout_t* layout, uint32_t* flags, int clear, ep_stream_t stream)
 {
     if (layout == nullptr || layout->workspace == nullptr || !aligned(layout->workspace, 256) ||

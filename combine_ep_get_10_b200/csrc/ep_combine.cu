@@ -1,7 +1,9 @@
 // ep_combine.cu -- combine (gather-reduce) kernels.
 //
 // Token choice: DeepEP-Ascend README, API Overview, combine and
-// low_latency_combine (the reduce weighted by topk_weights).  Expert choice:
+// low_latency_combine (the reduce weighted by topk_weights); the same
+// kernel reduces the per-rank rows of the deduplicated path (weight 1,
+// ascending rank).  Expert choice:
 // DeepEP issue #595, Solution 1 (the reduce over the slots that picked the
 // token, no [T, K] padding, no cap on their number).  Both skip -1 entries
 // (issue #595, Solution 2).
@@ -75,6 +77,8 @@ struct CombineArgs {
     const int32_t* token_offsets;
     const int32_t* token_slots;
     const float* expert_weights;
+    // per rank: [T, K] rows (K = R), weight 1
+    const int32_t* rank_row;
     void* out;
     uint32_t* err;
     int64_t warp_base; // first (token, segment) item of this launch
@@ -86,13 +90,29 @@ constexpr int kHeavyDeg = 16;
 constexpr int kMaxHeavy = 2048;
 constexpr int kHeavyFirstMaxT = 65536;
 
-template <bool kExpertChoice>
+enum CombineSrc : int {
+    kSrcTopk = 0,  // entries: the token's K (expert, slot) pairs, gate weights
+    kSrcEc = 1,    // entries: the token's CSR slots, expert weights
+    kSrcRanks = 2  // entries: the token's R rank rows, weight 1 (fmaf(1, y, acc) == acc + y)
+};
+
+template <int kSrc>
 __device__ __forceinline__ void entry(const CombineArgs& a, int64_t t, int64_t beg, int j, int64_t& row, float& w,
                                       uint32_t& errbits)
 {
     row = -1;
     w = 0.0f;
-    if (kExpertChoice) {
+    if constexpr (kSrc == kSrcRanks) {
+        const int64_t r = __ldg(a.rank_row + t * a.K + j);
+        if (r < 0)
+            return;
+        if (r >= a.num_y_rows) {
+            errbits |= EP_DEVERR_OVERFLOW;
+            return;
+        }
+        row = r;
+        w = 1.0f;
+    } else if constexpr (kSrc == kSrcEc) {
         const int64_t s = __ldg(a.token_slots + beg + j);
         if (s < 0 || s >= a.num_y_rows) {
             errbits |= EP_DEVERR_OVERFLOW;
@@ -141,9 +161,10 @@ __device__ __forceinline__ void item_token(int64_t g, int64_t heavy_items, int n
     }
 }
 
-template <bool kExpertChoice, bool kOutF32, int kVecPerLane, int kGroup>
+template <int kSrc, bool kOutF32, int kVecPerLane, int kGroup>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 {
+    constexpr bool kExpertChoice = kSrc == kSrcEc;
     constexpr int kSegVec = 32 * kVecPerLane;
     // token choice lists are short (K); expert-choice lists reach E entries
     constexpr int kLookup = kExpertChoice ? 2 : 1;
@@ -242,7 +263,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
                 my_w[i] = 0.0f;
                 const int j = k0 + 32 * i + lane;
                 if (j < n)
-                    entry<kExpertChoice>(a, t, beg, j, my_row[i], my_w[i], errbits);
+                    entry<kSrc>(a, t, beg, j, my_row[i], my_w[i], errbits);
             }
 #pragma unroll
             for (int i = 0; i < kLookup; ++i) {
@@ -333,7 +354,7 @@ int64_t resident_blocks(Kernel kernel, int* cache)
 
 // persistent: one resident wave of warps loops over the (token, segment)
 // items instead of one short-lived block per 8 items
-template <bool kExpertChoice, int kVec, int kGrp>
+template <int kSrc, int kVec, int kGrp>
 cudaError_t launch_combine(CombineArgs k, bool out_f32, bool persistent, cudaStream_t stream)
 {
     constexpr int64_t kMaxBlocks = int64_t{1} << 30;
@@ -342,8 +363,8 @@ cudaError_t launch_combine(CombineArgs k, bool out_f32, bool persistent, cudaStr
     int64_t blocks = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
     if (persistent) {
         static int cache_bf16[64], cache_f32[64];
-        const int64_t res = out_f32 ? resident_blocks(combine_kernel<kExpertChoice, true, kVec, kGrp>, cache_f32)
-                                    : resident_blocks(combine_kernel<kExpertChoice, false, kVec, kGrp>, cache_bf16);
+        const int64_t res = out_f32 ? resident_blocks(combine_kernel<kSrc, true, kVec, kGrp>, cache_f32)
+                                    : resident_blocks(combine_kernel<kSrc, false, kVec, kGrp>, cache_bf16);
         if (res > 0)
             blocks = std::min(blocks, res);
     }
@@ -351,9 +372,9 @@ cudaError_t launch_combine(CombineArgs k, bool out_f32, bool persistent, cudaStr
         k.warp_base = b0 * kWarpsPerCta;
         const unsigned n = static_cast<unsigned>(blocks - b0 < kMaxBlocks ? blocks - b0 : kMaxBlocks);
         if (out_f32)
-            combine_kernel<kExpertChoice, true, kVec, kGrp><<<n, kCombineThreads, 0, stream>>>(k);
+            combine_kernel<kSrc, true, kVec, kGrp><<<n, kCombineThreads, 0, stream>>>(k);
         else
-            combine_kernel<kExpertChoice, false, kVec, kGrp><<<n, kCombineThreads, 0, stream>>>(k);
+            combine_kernel<kSrc, false, kVec, kGrp><<<n, kCombineThreads, 0, stream>>>(k);
         cudaError_t st = cudaGetLastError();
         if (st != cudaSuccess)
             return st;
@@ -381,7 +402,7 @@ cudaError_t launch_tc_combine(const TcCombineLaunch& a, cudaStream_t stream)
     k.topk_weights = a.topk_weights;
     k.out = a.out;
     k.err = a.err;
-    return launch_combine<false, kTcVec, kTcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0, stream);
+    return launch_combine<kSrcTopk, kTcVec, kTcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0, stream);
 }
 
 cudaError_t launch_ec_combine(const EcCombineLaunch& a, cudaStream_t stream)
@@ -398,8 +419,23 @@ cudaError_t launch_ec_combine(const EcCombineLaunch& a, cudaStream_t stream)
     k.out = a.out;
     k.err = a.err;
     k.heavy_first = EP_COMBINE_HEAVY_FIRST && a.T <= kHeavyFirstMaxT ? 1 : 0;
-    return launch_combine<true, kEcVec, kEcGroup>(k, a.out_dtype == EP_FP32,
-                                                  k.heavy_first != 0 || EP_COMBINE_PERSIST_EC != 0, stream);
+    return launch_combine<kSrcEc, kEcVec, kEcGroup>(k, a.out_dtype == EP_FP32,
+                                                    k.heavy_first != 0 || EP_COMBINE_PERSIST_EC != 0, stream);
+}
+
+cudaError_t launch_rank_combine(const RankCombineLaunch& a, cudaStream_t stream)
+{
+    CombineArgs k{};
+    k.y = static_cast<const uint8_t*>(a.y);
+    k.T = a.T;
+    k.H = a.H;
+    k.nvec = a.H / 8;
+    k.num_y_rows = a.num_y_rows;
+    k.K = a.R;
+    k.rank_row = a.rank_row;
+    k.out = a.out;
+    k.err = a.err;
+    return launch_combine<kSrcRanks, kTcVec, kTcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0, stream);
 }
 
 } // namespace ep

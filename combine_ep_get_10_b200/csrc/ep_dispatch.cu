@@ -1,8 +1,8 @@
 // ep_dispatch.cu -- dispatch kernels.
 //
 // bf16 dispatch (token choice: DeepEP-Ascend README, API Overview,
-// dispatch / low_latency_dispatch; expert choice: DeepEP issue #595,
-// Solution 1) is a pure row copy: each source row chunk is read from HBM
+// dispatch / low_latency_dispatch, per expert or deduplicated per rank;
+// expert choice: DeepEP issue #595, Solution 1) is a pure row copy: each source row chunk is read from HBM
 // exactly once by the TMA engine (cp.async.bulk global->shared, completion on
 // an mbarrier) and written to every destination row by bulk stores
 // (cp.async.bulk shared->global), one per destination, issued by different
@@ -80,16 +80,46 @@ struct BulkArgs {
     float* recv_weights;
     const int32_t* token_indices; // expert choice
     int32_t T;
+    const int32_t* rank_row;      // per rank: [T, R] destination rows
+    int32_t R;
+    int64_t* recv_topk_idx;
+    float* recv_topk_weights;
     uint32_t* err;
     int64_t item_base; // first item of this launch
 };
 
-// One warp per (row, chunk) item.  kExpertChoice: item row = slot s, source
-// token = token_indices[s], one destination (row s).  Otherwise item row =
-// token t, destinations = its K routed pairs.
-template <bool kExpertChoice>
+enum BulkSrc : int {
+    kSrcTopk = 0,  // item row = token t; destinations = its K routed pairs
+    kSrcEc = 1,    // item row = slot s; source token_indices[s]; destination row s
+    kSrcRanks = 2  // item row = token t; destinations = its ranks' rows
+};
+
+// Top-k entries of token t as rank r sees them (per-rank dispatch): local
+// expert id and weight for the experts of rank r, -1 and 0 for the others.
+__device__ __forceinline__ void write_rank_topk(const BulkArgs& a, int64_t t, int lane)
+{
+    const int K = a.map.K;
+    const int per_rank = a.map.E / a.R;
+    for (int j = lane; j < a.R * K; j += 32) {
+        const int r = j / K;
+        const int k = j - r * K;
+        const int64_t row = __ldg(a.rank_row + t * a.R + r);
+        if (row < 0 || row >= a.map.num_rows)
+            continue;
+        const int64_t e = __ldg(a.map.topk_idx + t * K + k);
+        const bool local = e >= 0 && e < a.map.E && e / per_rank == r;
+        if (a.recv_topk_idx != nullptr)
+            a.recv_topk_idx[row * K + k] = local ? e - static_cast<int64_t>(r) * per_rank : -1;
+        if (a.recv_topk_weights != nullptr)
+            a.recv_topk_weights[row * K + k] = local ? __ldg(a.topk_weights + t * K + k) : 0.0f;
+    }
+}
+
+// One warp per (row, chunk) item; kSrc says what an item row is.
+template <int kSrc>
 __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
 {
+    constexpr bool kExpertChoice = kSrc == kSrcEc;
     __shared__ __align__(8) uint64_t bar;
     extern __shared__ __align__(128) uint8_t buf[];
     const int lane = threadIdx.x;
@@ -121,8 +151,16 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
     }
     // destination rows of the first 32 pairs while the load is in flight
     int64_t dst_row = -1;
-    if (kExpertChoice) {
+    if constexpr (kSrc == kSrcEc) {
         dst_row = lane == 0 ? r : -1;
+    } else if constexpr (kSrc == kSrcRanks) {
+        if (lane < a.R) {
+            dst_row = __ldg(a.rank_row + r * a.R + lane);
+            if (dst_row >= a.map.num_rows) {
+                errbits |= EP_DEVERR_OVERFLOW;
+                dst_row = -1;
+            }
+        }
     } else if (lane < a.map.K) {
         dst_row = a.map.row(r, lane, errbits);
     }
@@ -131,7 +169,7 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
     if (ok) {
         if (dst_row >= 0)
             bulk_store_s2g(a.dst + dst_row * a.row_bytes + off, buf, bytes);
-        if (!kExpertChoice) {
+        if constexpr (kSrc == kSrcTopk) {
             for (int k = lane + 32; k < a.map.K; k += 32) {
                 const int64_t rk = a.map.row(r, k, errbits);
                 if (rk >= 0)
@@ -141,7 +179,15 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
         bulk_commit();
         bulk_wait_read_all();
     }
-    if (!kExpertChoice && c == 0 && (a.recv_src != nullptr || a.recv_weights != nullptr)) {
+    if constexpr (kSrc == kSrcRanks) {
+        if (c == 0) {
+            if (dst_row >= 0 && a.recv_src != nullptr)
+                a.recv_src[dst_row] = static_cast<int32_t>(r);
+            if (a.recv_topk_idx != nullptr || a.recv_topk_weights != nullptr)
+                write_rank_topk(a, r, lane);
+        }
+    }
+    if (kSrc == kSrcTopk && c == 0 && (a.recv_src != nullptr || a.recv_weights != nullptr)) {
         uint32_t ignored = 0;
         for (int k = lane; k < a.map.K; k += 32) {
             const int64_t rk = k < 32 ? dst_row : a.map.row(r, k, ignored);
@@ -422,13 +468,13 @@ cudaError_t launch_quant(const QuantArgs& a, int32_t T, int32_t K, cudaStream_t 
 
 constexpr int64_t kMaxGrid = int64_t{1} << 30;
 
-template <bool kExpertChoice>
+template <int kSrc>
 cudaError_t launch_bulk(BulkArgs k, int64_t items, cudaStream_t stream)
 {
     for (int64_t base = 0; base < items; base += kMaxGrid) {
         k.item_base = base;
         const unsigned n = static_cast<unsigned>(std::min(kMaxGrid, items - base));
-        bulk_dispatch_kernel<kExpertChoice><<<n, 32, static_cast<size_t>(k.chunk_bytes), stream>>>(k);
+        bulk_dispatch_kernel<kSrc><<<n, 32, static_cast<size_t>(k.chunk_bytes), stream>>>(k);
         cudaError_t st = cudaGetLastError();
         if (st != cudaSuccess)
             return st;
@@ -476,7 +522,7 @@ cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream)
     k.recv_src = a.recv_src;
     k.recv_weights = a.recv_weights;
     k.err = a.err;
-    return launch_bulk<false>(k, static_cast<int64_t>(a.T) * k.nchunks, stream);
+    return launch_bulk<kSrcTopk>(k, static_cast<int64_t>(a.T) * k.nchunks, stream);
 }
 
 cudaError_t launch_ec_dispatch(const EcDispatchLaunch& a, cudaStream_t stream)
@@ -492,7 +538,33 @@ cudaError_t launch_ec_dispatch(const EcDispatchLaunch& a, cudaStream_t stream)
     k.token_indices = a.token_indices;
     k.T = a.T;
     k.err = a.err;
-    return launch_bulk<true>(k, S * k.nchunks, stream);
+    return launch_bulk<kSrcEc>(k, S * k.nchunks, stream);
+}
+
+cudaError_t launch_rank_dispatch(const RankDispatchLaunch& a, cudaStream_t stream)
+{
+    if (a.T == 0)
+        return cudaSuccess;
+    BulkArgs k{};
+    k.src = static_cast<const uint8_t*>(a.x);
+    k.dst = static_cast<uint8_t*>(a.recv_x);
+    k.row_bytes = static_cast<int64_t>(a.H) * 2;
+    k.nchunks = static_cast<int32_t>((k.row_bytes + kChunkTarget - 1) / kChunkTarget);
+    k.chunk_bytes = ((k.row_bytes / k.nchunks + 15) / 16) * 16;
+    k.nchunks = static_cast<int32_t>((k.row_bytes + k.chunk_bytes - 1) / k.chunk_bytes);
+    k.map.topk_idx = a.topk_idx;
+    k.map.K = a.K;
+    k.map.E = a.E;
+    k.map.num_rows = a.num_rows;
+    k.topk_weights = a.topk_weights;
+    k.recv_src = a.recv_src;
+    k.rank_row = a.rank_row;
+    k.R = a.R;
+    k.recv_topk_idx = a.recv_topk_idx;
+    k.recv_topk_weights = a.recv_topk_weights;
+    k.T = a.T;
+    k.err = a.err;
+    return launch_bulk<kSrcRanks>(k, static_cast<int64_t>(a.T) * k.nchunks, stream);
 }
 
 } // namespace ep

@@ -49,6 +49,15 @@ struct EcLayoutLaunch {
 size_t ec_layout_workspace_bytes(int64_t T, int64_t E, int64_t C);
 cudaError_t launch_ec_layout(const EcLayoutLaunch& a, cudaStream_t stream);
 
+struct RankLayoutLaunch {
+    const uint8_t* in_rank;
+    const int32_t* rank_counts;
+    int32_t T, R;
+    int32_t* rank_offsets;
+    int32_t* rank_row;
+};
+cudaError_t launch_rank_layout(const RankLayoutLaunch& a, cudaStream_t stream);
+
 // --------------------------------------------------------------- dispatch
 // Token-choice destination rows (shared by dispatch and combine).
 struct TcRows {
@@ -82,6 +91,21 @@ struct EcDispatchLaunch {
 };
 cudaError_t launch_ec_dispatch(const EcDispatchLaunch& a, cudaStream_t stream);
 
+struct RankDispatchLaunch {
+    const void* x;
+    int32_t T, H, K, E, R;
+    const int64_t* topk_idx;
+    const float* topk_weights;
+    const int32_t* rank_row;
+    int64_t num_rows;
+    void* recv_x;
+    int64_t* recv_topk_idx;
+    float* recv_topk_weights;
+    int32_t* recv_src;
+    uint32_t* err;
+};
+cudaError_t launch_rank_dispatch(const RankDispatchLaunch& a, cudaStream_t stream);
+
 // ---------------------------------------------------------------- combine
 struct TcCombineLaunch {
     const void* y;
@@ -106,5 +130,16 @@ struct EcCombineLaunch {
     uint32_t* err;
 };
 cudaError_t launch_ec_combine(const EcCombineLaunch& a, cudaStream_t stream);
+
+struct RankCombineLaunch {
+    const void* y;
+    int32_t T, H, R;
+    int64_t num_y_rows;
+    const int32_t* rank_row;
+    void* out;
+    int32_t out_dtype;
+    uint32_t* err;
+};
+cudaError_t launch_rank_combine(const RankCombineLaunch& a, cudaStream_t stream);
 
 } // namespace ep

@@ -227,6 +227,52 @@ EP_API ep_status_t ep_combine_expert_choice(const void* y, int32_t hidden, const
                                      const ep_layout_t* layout, const float* expert_weights, void* out,
                                      ep_dtype_t out_dtype, ep_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Per-rank (deduplicated) path: [README] "API Overview", normal-mode
+ * dispatch "to expert ranks" (received tokens plus their top-k information)
+ * and combine "(reduce) tokens from dispatch" with the dispatch handle.
+ * A token is copied once to every logical rank r with
+ * is_token_in_rank[t, r] = 1, instead of once per (token, expert) pair.
+ * Rank r's rows are its tokens in ascending token order; the ranks' row
+ * ranges are laid end to end in one buffer of rank_offsets[R] rows.
+ *   rank_offsets  int32 [R+1]  exclusive scan of num_tokens_per_rank
+ *   rank_row      int32 [T, R] row of token t in rank r's range, -1 if the
+ *                              token does not go to rank r
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    int32_t* rank_offsets;
+    int32_t* rank_row;
+} ep_rank_layout_t;
+
+/* Rank layout from the is_token_in_rank and num_tokens_per_rank that
+ * ep_get_layout wrote for the same routing (either routing kind). */
+EP_API ep_status_t ep_get_rank_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                                      const ep_rank_layout_t* rank_layout, ep_stream_t stream);
+
+/* Per-rank dispatch (TOPK routing): recv_x[rank_row[t, r]] = x[t] for every
+ * rank of every token, and, per received row, the token's K entries as the
+ * rank sees them:
+ *   recv_topk_idx     optional int64 [rows, K]: e - r*E/R for an expert e of
+ *                     rank r, else -1
+ *   recv_topk_weights optional fp32 [rows, K]: topk_weights[t, k] for those
+ *                     entries, else 0 (needs topk_weights)
+ *   recv_src          optional int32 [rows]: source token
+ * x bf16 [T, H], recv_x bf16 [num_recv_rows, H], both 16-byte aligned,
+ * H % 8 == 0.  Rows >= num_recv_rows are skipped with EP_DEVERR_OVERFLOW. */
+EP_API ep_status_t ep_dispatch_ranks(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                     const ep_layout_t* layout, const ep_rank_layout_t* rank_layout,
+                                     int64_t num_recv_rows, const float* topk_weights, void* recv_x,
+                                     int64_t* recv_topk_idx, float* recv_topk_weights, int32_t* recv_src,
+                                     ep_stream_t stream);
+
+/* Rank-level combine: out[t] = sum over the token's ranks r in ascending
+ * order of y[rank_row[t, r]], fp32 additions from 0 (the ranks have applied
+ * the gate weights), written as fp32 or rounded once (RNE) to bf16; a token
+ * with no rank gets +0.  y bf16 [num_y_rows, H]; out [T, H]. */
+EP_API ep_status_t ep_combine_ranks(const void* y, int32_t hidden, int64_t num_y_rows, const ep_routing_desc_t* routing,
+                                    const ep_layout_t* layout, const ep_rank_layout_t* rank_layout, void* out,
+                                    ep_dtype_t out_dtype, ep_stream_t stream);
+
 /* ep_get_layout for callers that cannot allocate device memory.  The pages
  * have no counterpart: this is a deployment variant of the layout call.
  *
