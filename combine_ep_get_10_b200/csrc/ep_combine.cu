@@ -18,6 +18,7 @@
 // a producer warp streaming row chunks into a shared-memory ring -- measured
 // no faster at 4096 tokens and slower under expert-choice skew.)
 #include <algorithm>
+#include <type_traits>
 
 #include "ep_device.cuh"
 #include "ep_internal.h"
@@ -49,19 +50,30 @@ constexpr int kTcGroup = EP_COMBINE_GROUP;
 #ifndef EP_COMBINE_EC_GROUP
 #define EP_COMBINE_EC_GROUP 8
 #endif
-// token choice: uniform items, so one resident wave of persistent warps;
-// expert choice: item cost varies by 100x, so blocks are scheduled dynamically
+// token choice: uniform items, so one resident wave of persistent warps
 #ifndef EP_COMBINE_PERSIST_TC
 #define EP_COMBINE_PERSIST_TC 1
-#endif
-#ifndef EP_COMBINE_PERSIST_EC
-#define EP_COMBINE_PERSIST_EC 0
 #endif
 #ifndef EP_COMBINE_HEAVY_FIRST
 #define EP_COMBINE_HEAVY_FIRST 1
 #endif
 constexpr int kEcVec = EP_COMBINE_EC_VEC;
 constexpr int kEcGroup = EP_COMBINE_EC_GROUP;
+// expert choice, heavy tokens: narrower segments and longer groups keep more
+// loads in flight on the long lists
+#ifndef EP_COMBINE_HEAVY_VEC
+#define EP_COMBINE_HEAVY_VEC 2
+#endif
+#ifndef EP_COMBINE_HEAVY_GROUP
+#define EP_COMBINE_HEAVY_GROUP 8
+#endif
+#ifndef EP_COMBINE_EC_RUN
+#define EP_COMBINE_EC_RUN 32
+#endif
+constexpr int kHeavyVec = EP_COMBINE_HEAVY_VEC;
+constexpr int kHeavyGroup = EP_COMBINE_HEAVY_GROUP;
+constexpr int kEcRun = EP_COMBINE_EC_RUN; // tokens per light item
+static_assert(kEcRun >= 1 && kEcRun <= 32, "a light item's tokens are held one per lane");
 
 struct CombineArgs {
     const uint8_t* y;
@@ -89,6 +101,8 @@ struct CombineArgs {
 constexpr int kHeavyDeg = 16;
 constexpr int kMaxHeavy = 2048;
 constexpr int kHeavyFirstMaxT = 65536;
+// 16-byte vectors of CSR bounds each thread loads per round of the heavy listing
+constexpr int kHeavyVecs = 8;
 
 enum CombineSrc : int {
     kSrcTopk = 0,  // entries: the token's K (expert, slot) pairs, gate weights
@@ -147,184 +161,271 @@ __device__ __forceinline__ void entry(const CombineArgs& a, int64_t t, int64_t b
     }
 }
 
-// Expert choice: virtual item g -> (token, segment); the first heavy_items
-// items are the listed heavy tokens' segments, then every token in order.
-__device__ __forceinline__ void item_token(int64_t g, int64_t heavy_items, int nseg, const int* heavy, int64_t& t,
-                                           int& seg)
+// out[t, segment seg] = sum over the token's n entries (ascending) of
+// w * y[row], one warp.  A segment is kVecPerLane 16-byte vectors per lane;
+// entries are looked up kLookup * 32 at a time (all of their loads in
+// flight), broadcast by shuffles and folded kGroup at a time, every 16-byte
+// load of a group issued before its FMAs.
+template <int kSrc, bool kOutF32, int kVecPerLane, int kGroup, int kLookup>
+__device__ __forceinline__ void reduce_segment(const CombineArgs& a, int64_t t, int seg, int64_t beg, int n, int lane,
+                                               uint32_t& errbits)
 {
-    if (g < heavy_items) {
-        t = heavy[g / nseg];
-        seg = static_cast<int>(g % nseg);
-    } else {
-        t = (g - heavy_items) / nseg;
-        seg = static_cast<int>((g - heavy_items) - t * nseg);
-    }
-}
-
-template <int kSrc, bool kOutF32, int kVecPerLane, int kGroup>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
-{
-    constexpr bool kExpertChoice = kSrc == kSrcEc;
     constexpr int kSegVec = 32 * kVecPerLane;
-    // token choice lists are short (K); expert-choice lists reach E entries
-    constexpr int kLookup = kExpertChoice ? 2 : 1;
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarpsPerCta;
-    uint32_t errbits = 0;
-
-    // Expert choice, heavy first: every CTA lists, in token order, the tokens
-    // with at least kHeavyDeg picks (the same list in every CTA); warps take
-    // their items before all others, so the long lists start in the first
-    // wave and overlap the light work instead of trailing it.
-    __shared__ int s_heavy[kMaxHeavy];
-    __shared__ uint32_t s_flags[kHeavyFirstMaxT / 32];
-    __shared__ int s_wbase[kWarpsPerCta + 1];
-    int n_heavy = 0;
-    if (kExpertChoice && a.heavy_first) {
-        const int64_t per_warp = ((static_cast<int64_t>(a.T) + kWarpsPerCta * 32 - 1) / (kWarpsPerCta * 32)) * 32;
-        const int64_t w0 = min(static_cast<int64_t>(a.T), warp * per_warp);
-        const int64_t w1 = min(static_cast<int64_t>(a.T), w0 + per_warp);
-        int cnt = 0;
-        for (int64_t base = w0; base < w1; base += 32) {
-            const int64_t t = base + lane;
-            const bool heavy = t < w1 && __ldg(a.token_offsets + t + 1) - __ldg(a.token_offsets + t) >= kHeavyDeg;
-            const uint32_t bits = __ballot_sync(kFullMask, heavy);
-            if (lane == 0)
-                s_flags[base / 32] = bits;
-            cnt += __popc(bits);
-        }
-        if (lane == 0)
-            s_wbase[warp + 1] = cnt;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            s_wbase[0] = 0;
-            for (int w = 0; w < kWarpsPerCta; ++w)
-                s_wbase[w + 1] += s_wbase[w];
-        }
-        __syncthreads();
-        n_heavy = s_wbase[kWarpsPerCta];
-        if (n_heavy <= kMaxHeavy) {
-            int pos = s_wbase[warp];
-            for (int64_t base = w0; base < w1; base += 32) {
-                const uint32_t bits = s_flags[base / 32];
-                if ((bits >> lane) & 1u)
-                    s_heavy[pos + __popc(bits & ((1u << lane) - 1u))] = static_cast<int>(base + lane);
-                pos += __popc(bits);
-            }
-        } else {
-            n_heavy = 0; // too many to list: plain token order
-        }
-        __syncthreads();
+    int v[kVecPerLane];
+    bool vin[kVecPerLane];
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j) {
+        v[j] = seg * kSegVec + j * 32 + lane;
+        vin[j] = v[j] < a.nvec;
     }
-    const int64_t heavy_items = static_cast<int64_t>(n_heavy) * a.nseg;
-    const int64_t items = heavy_items + static_cast<int64_t>(a.T) * a.nseg;
-    for (int64_t gw = a.warp_base + static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + warp; gw < items;
-         gw += stride) {
-        int64_t t;
-        int seg;
-        int64_t beg = 0;
-        int n;
-        if constexpr (kExpertChoice) {
-            item_token(gw, heavy_items, a.nseg, s_heavy, t, seg);
-            beg = __ldg(a.token_offsets + t);
-            n = __ldg(a.token_offsets + t + 1) - static_cast<int>(beg);
-        } else {
-            t = gw / a.nseg;
-            seg = static_cast<int>(gw - t * a.nseg);
-            n = a.K;
-        }
-        if (kExpertChoice && n_heavy > 0 && gw >= heavy_items && n >= kHeavyDeg)
-            continue; // done in the heavy phase
+    float acc[kVecPerLane][8];
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            acc[j][i] = 0.0f;
 
-        int v[kVecPerLane];
-        bool vin[kVecPerLane];
+    // expert-choice rows are slot ids below E*C < 2^31: 32-bit row registers
+    using RowT = typename std::conditional<kSrc == kSrcEc, int32_t, int64_t>::type;
+    const int64_t row_bytes = static_cast<int64_t>(a.H) * 2;
+    for (int k0 = 0; k0 < n; k0 += 32 * kLookup) {
+        RowT my_row[kLookup];
+        float my_w[kLookup];
 #pragma unroll
-        for (int j = 0; j < kVecPerLane; ++j) {
-            v[j] = seg * kSegVec + j * 32 + lane;
-            vin[j] = v[j] < a.nvec;
-        }
-        float acc[kVecPerLane][8];
-#pragma unroll
-        for (int j = 0; j < kVecPerLane; ++j)
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                acc[j][i] = 0.0f;
-
-        const int64_t row_bytes = static_cast<int64_t>(a.H) * 2;
-        // entries are looked up kLookup at a time (all of their loads in flight),
-        // then folded kGroup at a time in ascending order
-        for (int k0 = 0; k0 < n; k0 += 32 * kLookup) {
-            int64_t my_row[kLookup];
-            float my_w[kLookup];
-#pragma unroll
-            for (int i = 0; i < kLookup; ++i) {
-                my_row[i] = -1;
-                my_w[i] = 0.0f;
-                const int j = k0 + 32 * i + lane;
-                if (j < n)
-                    entry<kSrc>(a, t, beg, j, my_row[i], my_w[i], errbits);
+        for (int i = 0; i < kLookup; ++i) {
+            my_row[i] = -1;
+            my_w[i] = 0.0f;
+            const int j = k0 + 32 * i + lane;
+            if (j < n) {
+                int64_t r = -1;
+                entry<kSrc>(a, t, beg, j, r, my_w[i], errbits);
+                my_row[i] = static_cast<RowT>(r);
             }
+        }
 #pragma unroll
-            for (int i = 0; i < kLookup; ++i) {
-                const int kb = k0 + 32 * i;
-                if (kb >= n)
-                    break; // warp-uniform
-                const int m = min(32, n - kb);
-                for (int g0 = 0; g0 < m; g0 += kGroup) {
-                    int64_t rows[kGroup];
-                    float ws[kGroup];
+        for (int i = 0; i < kLookup; ++i) {
+            const int kb = k0 + 32 * i;
+            if (kb >= n)
+                break; // warp-uniform
+            const int m = min(32, n - kb);
+            for (int g0 = 0; g0 < m; g0 += kGroup) {
+                RowT rows[kGroup];
+                float ws[kGroup];
 #pragma unroll
-                    for (int g = 0; g < kGroup; ++g) {
-                        const int src = (g0 + g) & 31;
-                        rows[g] = __shfl_sync(kFullMask, my_row[i], src);
-                        ws[g] = __shfl_sync(kFullMask, my_w[i], src);
-                        if (g0 + g >= m)
-                            rows[g] = -1;
-                    }
-                    uint4 d[kGroup][kVecPerLane];
+                for (int g = 0; g < kGroup; ++g) {
+                    const int src = (g0 + g) & 31;
+                    rows[g] = __shfl_sync(kFullMask, my_row[i], src);
+                    ws[g] = __shfl_sync(kFullMask, my_w[i], src);
+                    if (g0 + g >= m)
+                        rows[g] = -1;
+                }
+                uint4 d[kGroup][kVecPerLane];
 #pragma unroll
-                    for (int g = 0; g < kGroup; ++g)
+                for (int g = 0; g < kGroup; ++g)
 #pragma unroll
-                        for (int j = 0; j < kVecPerLane; ++j)
-                            d[g][j] = (rows[g] >= 0 && vin[j])
-                                          ? ld_nc_v4(a.y + rows[g] * row_bytes + static_cast<int64_t>(v[j]) * 16)
-                                          : make_uint4(0, 0, 0, 0);
+                    for (int j = 0; j < kVecPerLane; ++j)
+                        d[g][j] = (rows[g] >= 0 && vin[j])
+                                      ? ld_nc_v4(a.y + static_cast<int64_t>(rows[g]) * row_bytes +
+                                                 static_cast<int64_t>(v[j]) * 16)
+                                      : make_uint4(0, 0, 0, 0);
 #pragma unroll
-                    for (int g = 0; g < kGroup; ++g) {
-                        if (rows[g] < 0)
-                            continue;
+                for (int g = 0; g < kGroup; ++g) {
+                    if (rows[g] < 0)
+                        continue;
 #pragma unroll
-                        for (int j = 0; j < kVecPerLane; ++j) {
-                            acc[j][0] = fmaf(ws[g], bf16_lo(d[g][j].x), acc[j][0]);
-                            acc[j][1] = fmaf(ws[g], bf16_hi(d[g][j].x), acc[j][1]);
-                            acc[j][2] = fmaf(ws[g], bf16_lo(d[g][j].y), acc[j][2]);
-                            acc[j][3] = fmaf(ws[g], bf16_hi(d[g][j].y), acc[j][3]);
-                            acc[j][4] = fmaf(ws[g], bf16_lo(d[g][j].z), acc[j][4]);
-                            acc[j][5] = fmaf(ws[g], bf16_hi(d[g][j].z), acc[j][5]);
-                            acc[j][6] = fmaf(ws[g], bf16_lo(d[g][j].w), acc[j][6]);
-                            acc[j][7] = fmaf(ws[g], bf16_hi(d[g][j].w), acc[j][7]);
-                        }
+                    for (int j = 0; j < kVecPerLane; ++j) {
+                        acc[j][0] = fmaf(ws[g], bf16_lo(d[g][j].x), acc[j][0]);
+                        acc[j][1] = fmaf(ws[g], bf16_hi(d[g][j].x), acc[j][1]);
+                        acc[j][2] = fmaf(ws[g], bf16_lo(d[g][j].y), acc[j][2]);
+                        acc[j][3] = fmaf(ws[g], bf16_hi(d[g][j].y), acc[j][3]);
+                        acc[j][4] = fmaf(ws[g], bf16_lo(d[g][j].z), acc[j][4]);
+                        acc[j][5] = fmaf(ws[g], bf16_hi(d[g][j].z), acc[j][5]);
+                        acc[j][6] = fmaf(ws[g], bf16_lo(d[g][j].w), acc[j][6]);
+                        acc[j][7] = fmaf(ws[g], bf16_hi(d[g][j].w), acc[j][7]);
                     }
                 }
             }
         }
+    }
 
 #pragma unroll
-        for (int j = 0; j < kVecPerLane; ++j) {
-            if (!vin[j])
-                continue;
-            if (kOutF32) {
-                float* o = static_cast<float*>(a.out) + t * a.H + static_cast<int64_t>(v[j]) * 8;
-                st_cs_v4(o, make_uint4(__float_as_uint(acc[j][0]), __float_as_uint(acc[j][1]), __float_as_uint(acc[j][2]),
-                                       __float_as_uint(acc[j][3])));
-                st_cs_v4(o + 4, make_uint4(__float_as_uint(acc[j][4]), __float_as_uint(acc[j][5]),
-                                           __float_as_uint(acc[j][6]), __float_as_uint(acc[j][7])));
-            } else {
-                uint8_t* o = static_cast<uint8_t*>(a.out) + t * row_bytes + static_cast<int64_t>(v[j]) * 16;
-                st_cs_v4(o, make_uint4(pack_bf16x2(acc[j][0], acc[j][1]), pack_bf16x2(acc[j][2], acc[j][3]),
-                                       pack_bf16x2(acc[j][4], acc[j][5]), pack_bf16x2(acc[j][6], acc[j][7])));
+    for (int j = 0; j < kVecPerLane; ++j) {
+        if (!vin[j])
+            continue;
+        if (kOutF32) {
+            float* o = static_cast<float*>(a.out) + t * a.H + static_cast<int64_t>(v[j]) * 8;
+            st_cs_v4(o, make_uint4(__float_as_uint(acc[j][0]), __float_as_uint(acc[j][1]), __float_as_uint(acc[j][2]),
+                                   __float_as_uint(acc[j][3])));
+            st_cs_v4(o + 4, make_uint4(__float_as_uint(acc[j][4]), __float_as_uint(acc[j][5]),
+                                       __float_as_uint(acc[j][6]), __float_as_uint(acc[j][7])));
+        } else {
+            uint8_t* o = static_cast<uint8_t*>(a.out) + t * row_bytes + static_cast<int64_t>(v[j]) * 16;
+            st_cs_v4(o, make_uint4(pack_bf16x2(acc[j][0], acc[j][1]), pack_bf16x2(acc[j][2], acc[j][3]),
+                                   pack_bf16x2(acc[j][4], acc[j][5]), pack_bf16x2(acc[j][6], acc[j][7])));
+        }
+    }
+}
+
+// Token choice and per-rank rows: one warp per (token, segment) item; the
+// items are taken with a fixed stride by a persistent grid (uniform cost).
+template <int kSrc, bool kOutF32, int kVecPerLane, int kGroup>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarpsPerCta;
+    uint32_t errbits = 0;
+    const int64_t items = static_cast<int64_t>(a.T) * a.nseg;
+    for (int64_t gw = a.warp_base + static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + warp; gw < items;
+         gw += stride) {
+        const int64_t t = gw / a.nseg;
+        const int seg = static_cast<int>(gw - t * a.nseg);
+        reduce_segment<kSrc, kOutF32, kVecPerLane, kGroup, 1>(a, t, seg, 0, a.K, lane, errbits);
+    }
+    const uint32_t any = __reduce_or_sync(kFullMask, errbits);
+    if (lane == 0)
+        flag_error(a.err, any);
+}
+
+// Expert choice.  A few tokens are picked by up to all E experts and most by
+// none, so the work per token varies by 100x.  Every CTA first lists, in
+// token order, the tokens with at least kHeavyDeg picks (the same list in
+// every CTA).  The items are then: one per (heavy token, segment), followed
+// by one per (run of 32 tokens, segment).  A run item reads the 32 tokens'
+// CSR bounds with one load per lane and walks the tokens: unpicked ones just
+// store zeros, heavy ones are skipped (done as heavy items), the rest are
+// reduced.  Items go to warps in warp-major order (warp w of every CTA before
+// warp w + 1), so the heavy items, which come first, spread over all SMs.
+template <bool kOutF32>
+__global__ void __launch_bounds__(kCombineThreads) ec_combine_kernel(CombineArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    uint32_t errbits = 0;
+
+    __shared__ int s_heavy[kMaxHeavy];
+    __shared__ uint32_t s_flags[kHeavyFirstMaxT / 32];
+    __shared__ int s_wsum[kWarpsPerCta];
+    int n_heavy = 0;
+    if (a.heavy_first) {
+        // Every CTA reads the whole CSR bound array once, coalesced and all at
+        // once (16-byte vectors, kHeavyVecs per thread, plus the bound after
+        // each vector), flags the heavy tokens in a shared bit mask, then
+        // lists them in token order (count per 32-token word, CTA scan).
+        const int tid = threadIdx.x;
+        const int nwords = (a.T + 31) / 32;
+        for (int i = tid; i < nwords; i += kCombineThreads)
+            s_flags[i] = 0u;
+        __syncthreads();
+        // 4 bounds per 16-byte vector (1 when the array is not 16-byte aligned),
+        // kHeavyVecs vectors per thread per round, all loads of a round at once
+        const int per = (reinterpret_cast<uintptr_t>(a.token_offsets) & 15u) == 0 ? 4 : 1;
+        const int nv = (a.T + per - 1) / per; // vectors holding bounds 0 .. T-1
+        for (int base = 0; base < nv; base += kHeavyVecs * kCombineThreads) {
+            int4 q[kHeavyVecs];
+            int nxt[kHeavyVecs];
+#pragma unroll
+            for (int k = 0; k < kHeavyVecs; ++k) {
+                const int v = base + k * kCombineThreads + tid;
+                q[k] = make_int4(0, 0, 0, 0);
+                nxt[k] = 0;
+                if (v < nv) {
+                    const int b = per * v;
+                    if (per == 4 && b + 3 <= a.T) {
+                        q[k] = __ldg(reinterpret_cast<const int4*>(a.token_offsets) + v);
+                    } else { // the array's last bounds: no read past index T
+                        q[k].x = __ldg(a.token_offsets + b);
+                        if (per == 4) {
+                            q[k].y = b + 1 <= a.T ? __ldg(a.token_offsets + b + 1) : 0;
+                            q[k].z = b + 2 <= a.T ? __ldg(a.token_offsets + b + 2) : 0;
+                        }
+                    }
+                    nxt[k] = __ldg(a.token_offsets + min(b + per, a.T));
+                }
             }
+#pragma unroll
+            for (int k = 0; k < kHeavyVecs; ++k) {
+                const int v = base + k * kCombineThreads + tid;
+                if (v >= nv)
+                    continue;
+                const int o[5] = {q[k].x, q[k].y, q[k].z, q[k].w, nxt[k]};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int t = per * v + j;
+                    if (j < per && t < a.T && (j + 1 < per ? o[j + 1] : o[4]) - o[j] >= kHeavyDeg)
+                        atomicOr(&s_flags[t / 32], 1u << (t % 32));
+                }
+            }
+        }
+        __syncthreads();
+        // words w0 .. w1 of this thread, scanned over the CTA
+        const int wpt = (nwords + kCombineThreads - 1) / kCombineThreads;
+        const int w0 = min(nwords, tid * wpt);
+        const int w1 = min(nwords, w0 + wpt);
+        int cnt = 0;
+        for (int w = w0; w < w1; ++w)
+            cnt += __popc(s_flags[w]);
+        int inc = cnt;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int v = __shfl_up_sync(kFullMask, inc, d);
+            if (lane >= d)
+                inc += v;
+        }
+        if (lane == 31)
+            s_wsum[warp] = inc;
+        __syncthreads();
+        int before = 0;
+        n_heavy = 0;
+        for (int w = 0; w < kWarpsPerCta; ++w) {
+            before += w < warp ? s_wsum[w] : 0;
+            n_heavy += s_wsum[w];
+        }
+        if (n_heavy <= kMaxHeavy) {
+            int pos = before + inc - cnt;
+            for (int w = w0; w < w1; ++w) {
+                uint32_t bits = s_flags[w];
+                while (bits) {
+                    const int i = __ffs(bits) - 1;
+                    bits &= bits - 1u;
+                    s_heavy[pos++] = w * 32 + i;
+                }
+            }
+        } else {
+            n_heavy = 0; // too many to list: every token goes through the runs
+        }
+        __syncthreads();
+    }
+    const int nseg_h = (a.nvec + 32 * kHeavyVec - 1) / (32 * kHeavyVec);
+    const int64_t heavy_items = static_cast<int64_t>(n_heavy) * nseg_h;
+    const int64_t runs = (static_cast<int64_t>(a.T) + kEcRun - 1) / kEcRun;
+    const int64_t items = heavy_items + runs * a.nseg;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerCta;
+    for (int64_t it = a.warp_base + static_cast<int64_t>(warp) * gridDim.x + blockIdx.x; it < items; it += nwarps) {
+        if (it < heavy_items) {
+            const int64_t t = s_heavy[it / nseg_h];
+            const int seg = static_cast<int>(it % nseg_h);
+            const int beg = __ldg(a.token_offsets + t);
+            const int n = __ldg(a.token_offsets + t + 1) - beg;
+            reduce_segment<kSrcEc, kOutF32, kHeavyVec, kHeavyGroup, 2>(a, t, seg, beg, n, lane, errbits);
+            continue;
+        }
+        // a run of up to kEcRun tokens; lane j holds the CSR bounds of its j-th token
+        const int64_t r = (it - heavy_items) / a.nseg;
+        const int seg = static_cast<int>((it - heavy_items) - r * a.nseg);
+        const int64_t t0 = r * kEcRun;
+        const int cnt = static_cast<int>(min(static_cast<int64_t>(kEcRun), a.T - t0));
+        int my_beg = 0, my_n = 0;
+        if (lane < cnt) {
+            my_beg = __ldg(a.token_offsets + t0 + lane);
+            my_n = __ldg(a.token_offsets + t0 + lane + 1) - my_beg;
+        }
+        for (int j = 0; j < cnt; ++j) {
+            const int n = __shfl_sync(kFullMask, my_n, j);
+            const int beg = __shfl_sync(kFullMask, my_beg, j);
+            if (n_heavy > 0 && n >= kHeavyDeg)
+                continue; // done as a heavy item
+            reduce_segment<kSrcEc, kOutF32, kEcVec, kEcGroup, 2>(a, t0 + j, seg, beg, n, lane, errbits);
         }
     }
     const uint32_t any = __reduce_or_sync(kFullMask, errbits);
@@ -382,6 +483,25 @@ cudaError_t launch_combine(CombineArgs k, bool out_f32, bool persistent, cudaStr
     return cudaSuccess;
 }
 
+// Expert choice: one resident wave of warps over the heavy and run items.
+cudaError_t launch_ec(CombineArgs k, bool out_f32, cudaStream_t stream)
+{
+    k.nseg = (k.nvec + 32 * kEcVec - 1) / (32 * kEcVec);
+    const int64_t runs = (static_cast<int64_t>(k.T) + kEcRun - 1) / kEcRun;
+    const int64_t items = std::max<int64_t>(1, runs * k.nseg);
+    static int cache_bf16[64], cache_f32[64];
+    const int64_t res = out_f32 ? resident_blocks(ec_combine_kernel<true>, cache_f32)
+                                : resident_blocks(ec_combine_kernel<false>, cache_bf16);
+    int64_t blocks = res > 0 ? res : (items + kWarpsPerCta - 1) / kWarpsPerCta;
+    blocks = std::min<int64_t>(blocks, int64_t{1} << 30);
+    k.warp_base = 0;
+    if (out_f32)
+        ec_combine_kernel<true><<<static_cast<unsigned>(blocks), kCombineThreads, 0, stream>>>(k);
+    else
+        ec_combine_kernel<false><<<static_cast<unsigned>(blocks), kCombineThreads, 0, stream>>>(k);
+    return cudaGetLastError();
+}
+
 } // namespace
 
 cudaError_t launch_tc_combine(const TcCombineLaunch& a, cudaStream_t stream)
@@ -419,8 +539,9 @@ cudaError_t launch_ec_combine(const EcCombineLaunch& a, cudaStream_t stream)
     k.out = a.out;
     k.err = a.err;
     k.heavy_first = EP_COMBINE_HEAVY_FIRST && a.T <= kHeavyFirstMaxT ? 1 : 0;
-    return launch_combine<kSrcEc, kEcVec, kEcGroup>(k, a.out_dtype == EP_FP32,
-                                                    k.heavy_first != 0 || EP_COMBINE_PERSIST_EC != 0, stream);
+    if (a.T == 0)
+        return cudaSuccess;
+    return launch_ec(k, a.out_dtype == EP_FP32, stream);
 }
 
 cudaError_t launch_rank_combine(const RankCombineLaunch& a, cudaStream_t stream)
