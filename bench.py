@@ -57,6 +57,9 @@ def parse():
                     help="with --workloads: also time every quantised dispatch format on the token-choice workloads")
     ap.add_argument("--ranks", action="store_true",
                     help="with --workloads: also time the per-rank (deduplicated) dispatch and combine")
+    ap.add_argument("--rounds", type=int, default=0,
+                    help="with --workloads: also time the whole batch in rounds of this many tokens "
+                         "(per-round layout, dispatch and combine; receive buffer of one round)")
     return ap.parse_args()
 
 
@@ -543,6 +546,26 @@ def run_workload_table(args):
             emit(cfg, "combine", timeit(lambda: B.ep_combine(y, rt, lay, w, out, mode=mode,
                                                              max_tokens_per_expert=mt)),
                  n_valid * H * 2 + T * H * 2 + T * K * 16 + E * 4, T)
+            if args.rounds and mode == W.COMPACT and args.rounds < T:
+                P = args.rounds
+                rnd = [(t0, min(T, t0 + P)) for t0 in range(0, T, P)]
+                rr = [rt.tokens(t0, t1) for t0, t1 in rnd]
+                rl = [B.Layout(r, device=dev) for r in rr]
+                rbuf = torch.empty((P * K, H), dtype=torch.bfloat16, device=dev)
+                rout = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+
+                def all_rounds():
+                    for (t0, t1), r, l in zip(rnd, rr, rl):
+                        B.ep_get_layout(r, l)
+                        B.ep_dispatch(x[t0:t1], r, l, rbuf, num_recv_rows=P * K)
+                        B.ep_combine(rbuf, r, l, w[t0:t1], rout[t0:t1], num_y_rows=P * K)
+
+                us = timeit(all_rounds)
+                nb = (T * K * 12 + T * R + (E * 8 + R * 4) * len(rnd)  # layouts
+                      + T * H * 2 + n_valid * H * 2 + T * K * 12 + E * 4 * len(rnd)  # dispatches
+                      + n_valid * H * 2 + T * H * 2 + T * K * 16)  # combines
+                emit(cfg, "rounds_%dx%d_layout_dispatch_combine" % (len(rnd), P), us, nb, T)
+                del rbuf, rout
             if args.ranks and mode == W.COMPACT:
                 rl = B.RankLayout(rt, device=dev)
                 emit(cfg, "rank_layout", timeit(lambda: B.ep_get_rank_layout(rt, lay, rl)),

@@ -241,6 +241,18 @@ def layout_tokens(layout: Layout, routing: Routing, t0: int, t1: int) -> LayoutV
     return LayoutView(layout, t0, routing.desc.num_topk)
 
 
+def token_rounds(num_tokens: int, per_round_tokens: int) -> list[tuple[int, int]]:
+    """Token ranges [t0, t1) of a long batch processed in rounds of at most
+    per_round_tokens tokens (the README's "ant moving home" long-sequence
+    mode: DEEPEP_NORMAL_LONG_SEQ_PER_ROUND_TOKENS tokens per round).  Each
+    round is an independent layout -> dispatch -> (experts) -> combine on
+    Routing.tokens(t0, t1), so the receive buffers need only
+    per_round_tokens * K rows; per-token results equal the one-shot ones."""
+    if num_tokens < 0 or per_round_tokens < 1:
+        raise ValueError("num_tokens >= 0 and per_round_tokens >= 1")
+    return [(t0, min(num_tokens, t0 + per_round_tokens)) for t0 in range(0, num_tokens, per_round_tokens)]
+
+
 def ep_get_layout(routing: Routing, layout: Layout, stream=None) -> Layout:
     _check(lib().ep_get_layout(ctypes.byref(routing.desc), ctypes.byref(layout.desc), _stream(stream)),
            "ep_get_layout")

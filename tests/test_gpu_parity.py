@@ -437,3 +437,43 @@ def test_device_error_word_clears():
     _, lay, flags = gpu_tc_layout(idx, 4, 2)
     assert flags == B.EP_DEVERR_BAD_INDEX
     assert B.ep_get_device_error(lay) == 0  # cleared by the previous read
+
+
+def test_long_sequence_in_rounds():
+    """Long-sequence rounds ("ant moving home"): 32768 tokens of the skewed
+    routing in rounds of 8192, each with its own layout and a receive buffer
+    of 8192 * K rows; the combined output equals the one-shot oracle combine
+    (identity experts), checked on sampled tokens, and each round's buffer
+    holds exactly that round's routed pairs."""
+    inp = W.make_inputs(5, T=32768)
+    c = inp["cfg"]
+    x, idx, w = inp["x"], inp["topk_idx"], inp["topk_weights"]
+    T, H, E, R, K = idx.shape[0], c["H"], c["E"], c["R"], c["K"]
+    P = 8192
+    xd, idxd, wd = to_dev(x, bf16=True), to_dev(idx), to_dev(w)
+    routing = B.Routing.topk(idxd, E, R)
+    recv = torch.empty((P * K, H), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    rounds = B.token_rounds(T, P)
+    assert len(rounds) == 4
+    for t0, t1 in rounds:
+        r = routing.tokens(t0, t1)
+        lay = B.Layout(r)
+        B.ep_get_layout(r, lay)
+        n = int(lay.expert_offsets[-1].item())
+        assert n == int((idx[t0:t1] >= 0).sum()) <= P * K
+        B.ep_dispatch(xd[t0:t1], r, lay, recv, num_recv_rows=n)
+        B.ep_combine(recv, r, lay, wd[t0:t1], out[t0:t1], num_y_rows=n)
+        assert B.ep_get_device_error(lay) == 0
+    tokens = np.sort(rng(17).choice(T, size=256, replace=False)).astype(np.int32)
+    # per sampled token, the one-shot path restricted to that token (its
+    # combine reads only its own pairs' rows, which identity experts fill
+    # with x[t]): the oracle's dispatch + combine of that one-token routing
+    ref = np.empty((tokens.size, H), np.uint16)
+    for i, t in enumerate(tokens):
+        l1 = oracle.tc_layout(idx[t:t + 1], E, R)
+        y1 = oracle.tc_dispatch(x[t:t + 1], idx[t:t + 1], E, l1)["recv"]
+        ref[i] = oracle.tc_combine(y1, idx[t:t + 1], E, l1, w[t:t + 1], out_dtype=W.BF16)[0]
+    got = host(out[torch.from_numpy(tokens).cuda()])
+    assert_combine_close(got, ref, True, "rounds")
+    assert exact_fraction(got, ref) == 1.0
