@@ -2,18 +2,19 @@
 //
 // bf16 dispatch (token choice: DeepEP-Ascend README, API Overview,
 // dispatch / low_latency_dispatch, per expert or deduplicated per rank;
-// expert choice: DeepEP issue #595, Solution 1) is a pure row copy: each source row chunk is read from HBM
-// exactly once by the TMA engine (cp.async.bulk global->shared, completion on
-// an mbarrier) and written to every destination row by bulk stores
-// (cp.async.bulk shared->global), one per destination, issued by different
-// lanes.  A CTA is one warp and moves one (row, chunk) item; up to 28 CTAs
-// per SM keep ~200 KB of copies in flight per SM and the block scheduler
-// balances the tail.  (A persistent variant streaming each CTA's items
-// through a 3-4 stage ring measured 10-15% slower.)
+// expert choice: DeepEP issue #595, Solution 1) is a pure row copy: each
+// source row chunk (a whole row up to 16 KB) is read from HBM exactly once by
+// the TMA engine (cp.async.bulk global->shared, completion on an mbarrier)
+// and written to every destination row by bulk stores (cp.async.bulk
+// shared->global), one per destination, issued by different lanes.  A CTA is
+// one warp and moves one (row, chunk) item; up to 14 CTAs of 16 KB per SM
+// keep ~200 KB of copies in flight per SM and the block scheduler balances
+// the tail.  (8 KB chunks measured 2% slower on 14 KB rows; a persistent
+// variant streaming each CTA's items through a 3-4 stage ring 10-15% slower.)
 //
 // Quantised dispatch (README, "Quantization Modes in Normal Dispatch": FP8
 // with one fp32 scale per 128 channels, per-token INT8 and FP8, MX FP8/FP4
-// with an e8m0 scale per 32): one CTA per token holds the row in registers
+// with an e8m0 scale per 32): one CTA per token stages the row in shared memory
 // (all loads issued at once), reduces the amax over each scale group by
 // shuffles (or over the CTA for per-token scales), encodes every element once
 // with the cvt.rn.satfinite packing instructions, and stores the code runs
@@ -28,7 +29,7 @@ namespace ep {
 namespace {
 
 #ifndef EP_DISPATCH_CHUNK
-#define EP_DISPATCH_CHUNK 8192
+#define EP_DISPATCH_CHUNK 16384
 #endif
 
 constexpr int64_t kChunkTarget = EP_DISPATCH_CHUNK; // bytes per bulk-copy item

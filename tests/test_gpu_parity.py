@@ -172,10 +172,10 @@ def test_tc_dispatch_fp8_padded_decode():
 @pytest.mark.parametrize("mode,mt,dtype", [(W.PADDED, 3, W.BF16), (W.PADDED, 5, W.FP8_E4M3), (W.COMPACT, 0, W.FP8_E4M3)])
 def test_tc_dispatch_small_edges(mode, mt, dtype):
     """Padded overflow (flagged, skipped), duplicates, -1, K > 32, FP8 compact,
-    a ragged two-chunk row (H = 4104 -> 8208-byte rows), and special values."""
+    a ragged two-chunk row (H = 8264 -> 16528-byte rows), and special values."""
     r = rng(77)
     T, E, R, K = 45, 12, 3, 36
-    H = 4104 if dtype == W.BF16 else 384
+    H = 8264 if dtype == W.BF16 else 384
     idx = W.random_topk(r, T, E, K, p_neg=0.2, allow_dup=True, p_bad=0.02)
     xf = r.standard_normal((T, H)).astype(np.float32) * np.float32(3.0)
     xf[0, :128] = 0.0  # an all-zero group
