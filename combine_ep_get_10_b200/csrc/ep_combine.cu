@@ -294,8 +294,10 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 // by one per (run of 32 tokens, segment).  A run item reads the 32 tokens'
 // CSR bounds with one load per lane and walks the tokens: unpicked ones just
 // store zeros, heavy ones are skipped (done as heavy items), the rest are
-// reduced.  Items go to warps in warp-major order (warp w of every CTA before
-// warp w + 1), so the heavy items, which come first, spread over all SMs.
+// reduced.  Warps are numbered warp-major (warp w of every CTA before warp
+// w + 1): heavy items go to the first warps, so they spread over all SMs, and
+// light items to the last warps first, so the long lists get no light work
+// unless there are more items than warps.
 template <bool kOutF32>
 __global__ void __launch_bounds__(kCombineThreads) ec_combine_kernel(CombineArgs a)
 {
@@ -401,18 +403,22 @@ __global__ void __launch_bounds__(kCombineThreads) ec_combine_kernel(CombineArgs
     const int64_t runs = (static_cast<int64_t>(a.T) + kEcRun - 1) / kEcRun;
     const int64_t items = heavy_items + runs * a.nseg;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerCta;
-    for (int64_t it = a.warp_base + static_cast<int64_t>(warp) * gridDim.x + blockIdx.x; it < items; it += nwarps) {
-        if (it < heavy_items) {
-            const int64_t t = s_heavy[it / nseg_h];
-            const int seg = static_cast<int>(it % nseg_h);
-            const int beg = __ldg(a.token_offsets + t);
-            const int n = __ldg(a.token_offsets + t + 1) - beg;
-            reduce_segment<kSrcEc, kOutF32, kHeavyVec, kHeavyGroup, 2>(a, t, seg, beg, n, lane, errbits);
-            continue;
-        }
+    const int64_t g = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x; // warp-major
+    // heavy items from the first warps, light items from the last warps
+    // backwards, so a warp with a long list gets light work only when there
+    // are more items than warps
+    for (int64_t it = g; it < heavy_items; it += nwarps) {
+        const int64_t t = s_heavy[it / nseg_h];
+        const int seg = static_cast<int>(it % nseg_h);
+        const int beg = __ldg(a.token_offsets + t);
+        const int n = __ldg(a.token_offsets + t + 1) - beg;
+        reduce_segment<kSrcEc, kOutF32, kHeavyVec, kHeavyGroup, 2>(a, t, seg, beg, n, lane, errbits);
+    }
+    const int64_t light_items = items - heavy_items;
+    for (int64_t it = nwarps - 1 - g; it < light_items; it += nwarps) {
         // a run of up to kEcRun tokens; lane j holds the CSR bounds of its j-th token
-        const int64_t r = (it - heavy_items) / a.nseg;
-        const int seg = static_cast<int>((it - heavy_items) - r * a.nseg);
+        const int64_t r = it / a.nseg;
+        const int seg = static_cast<int>(it - r * a.nseg);
         const int64_t t0 = r * kEcRun;
         const int cnt = static_cast<int>(min(static_cast<int64_t>(kEcRun), a.T - t0));
         int my_beg = 0, my_n = 0;

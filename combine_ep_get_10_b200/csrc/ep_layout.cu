@@ -358,7 +358,10 @@ constexpr int kGridWarps = kGridThreads / 32;
 constexpr int kGridPrefetch = 8;                          // 32-pair steps per warp in registers
 constexpr int64_t kGridIds = kGridWarps * kGridPrefetch * 32; // pairs per CTA staged in shared memory
 constexpr int kGridMaxBlocks = 64;                      // workspace holds this many CTAs' totals
-constexpr int64_t kGridPairsPerCta = 1024;
+#ifndef EP_LAYOUT_GRID_PAIRS_PER_CTA
+#define EP_LAYOUT_GRID_PAIRS_PER_CTA 1024
+#endif
+constexpr int64_t kGridPairsPerCta = EP_LAYOUT_GRID_PAIRS_PER_CTA;
 
 struct GridBar {
     uint32_t* arrive;
