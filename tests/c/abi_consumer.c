@@ -88,9 +88,11 @@ static int gpu_mode(void)
     r.num_topk = K;
     r.num_experts = E;
     r.num_ranks = R;
-    size_t ws = ep_workspace_bytes(&r);
     CHECK(cudaMalloc(&d_idx, sizeof idx) == 0 && cudaMalloc(&d_w, sizeof w) == 0 && cudaMalloc(&d_x, sizeof x) == 0,
           "cudaMalloc");
+    r.topk_idx = (const int64_t*)d_idx;
+    size_t ws = ep_workspace_bytes(&r);
+    CHECK(ws >= 256, "workspace bytes");
     CHECK(cudaMalloc(&d_recv, T * K * H * 2) == 0 && cudaMalloc(&d_out, T * H * 4) == 0 && cudaMalloc(&d_ws, ws) == 0,
           "cudaMalloc");
     CHECK(cudaMalloc((void**)&d_cnt, E * 4) == 0 && cudaMalloc((void**)&d_off, (E + 1) * 4) == 0 &&
@@ -101,7 +103,6 @@ static int gpu_mode(void)
               cudaMemcpy(d_x, x, sizeof x, H2D) == 0,
           "copy in");
     CHECK(ep_workspace_init(d_ws, ws, NULL) == EP_OK, "workspace init");
-    r.topk_idx = (const int64_t*)d_idx;
     ep_layout_t l;
     memset(&l, 0, sizeof l);
     l.num_tokens_per_expert = d_cnt;
