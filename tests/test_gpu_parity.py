@@ -477,3 +477,24 @@ def test_long_sequence_in_rounds():
     got = host(out[torch.from_numpy(tokens).cuda()])
     assert_combine_close(got, ref, True, "rounds")
     assert exact_fraction(got, ref) == 1.0
+
+
+def test_combine_into_pinned_host_memory():
+    """`out` may be pinned host memory (mapped under unified addressing): the
+    combine's stores then cross PCIe directly, and the bytes equal those of
+    a device output."""
+    inp = inputs(2, T=512)
+    c = inp["cfg"]
+    x, idx, w = inp["x"], inp["topk_idx"], inp["topk_weights"]
+    routing, lay, _ = gpu_tc_layout(idx, c["E"], c["R"])
+    n = int(host(lay.expert_offsets)[-1])
+    recv = torch.empty((n, c["H"]), dtype=torch.bfloat16, device="cuda")
+    B.ep_dispatch(to_dev(x, bf16=True), routing, lay, recv)
+    wd = to_dev(w)
+    out_d = torch.empty((512, c["H"]), dtype=torch.bfloat16, device="cuda")
+    out_h = torch.zeros((512, c["H"]), dtype=torch.bfloat16).pin_memory()
+    B.ep_combine(recv, routing, lay, wd, out_d)
+    B.ep_combine(recv, routing, lay, wd, out_h)
+    torch.cuda.synchronize()
+    assert B.ep_get_device_error(lay) == 0
+    assert torch.equal(out_d.cpu().view(torch.int16), out_h.view(torch.int16))
