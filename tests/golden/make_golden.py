@@ -62,8 +62,36 @@ def workload4_small():
             "combine_fp32": digest(C)}
 
 
+def workload3_quant_formats():
+    """Every quantised dispatch format on 16 decode tokens, compact rows."""
+    inp = W.make_inputs(3, T=16)
+    x, idx = inp["x"], inp["topk_idx"]
+    L = oracle.tc_layout(idx, 256, 8)
+    out = {}
+    for name, dt in (("int8_per_token", oracle.INT8_PER_TOKEN), ("fp8_per_token", oracle.FP8_E4M3_PER_TOKEN),
+                     ("mxfp8_e4m3", oracle.MXFP8_E4M3), ("mxfp8_e5m2", oracle.MXFP8_E5M2),
+                     ("mxfp4_e2m1", oracle.MXFP4_E2M1)):
+        D = oracle.tc_dispatch(x, idx, 256, L, out_dtype=dt)
+        out[name] = {"codes": digest(D["recv"]), "scales": digest(D["recv_scales"])}
+    return out
+
+
+def workload1_ranks():
+    """The per-rank (deduplicated) path on workload 1."""
+    inp = W.make_inputs(1)
+    x, idx, w = inp["x"], inp["topk_idx"], inp["topk_weights"]
+    L = oracle.tc_layout(idx, 8, 2)
+    RL = oracle.rank_layout(L["is_token_in_rank"])
+    D = oracle.rank_dispatch(x, idx, 8, 2, RL, w, want_src=True)
+    C = oracle.rank_combine(D["recv"], RL, out_dtype=oracle.FP32)
+    return {"rank_offsets": RL["rank_offsets"].tolist(), "rank_row": digest(RL["rank_row"]),
+            "recv": digest(D["recv"]), "recv_topk_idx": digest(D["recv_topk_idx"]),
+            "recv_topk_weights": digest(D["recv_topk_weights"]), "combine_fp32": digest(C)}
+
+
 def compute():
-    return {"workload1": workload1(), "workload3_T16": workload3_small(), "workload4_T512": workload4_small()}
+    return {"workload1": workload1(), "workload3_T16": workload3_small(), "workload4_T512": workload4_small(),
+            "workload3_T16_quant": workload3_quant_formats(), "workload1_ranks": workload1_ranks()}
 
 
 if __name__ == "__main__":
