@@ -531,6 +531,11 @@ def run_workload_table(args):
                 emit(cfg, "dispatch_fp8", timeit(lambda: B.ep_dispatch(x, rt, lay, recv, mode=mode,
                                                                        max_tokens_per_expert=mt, recv_scales=sc)),
                      T * H * 2 + n_valid * (H + H // 128 * 4) + meta, T)
+                if mode == W.PADDED:  # layout + padded FP8 dispatch in one call
+                    emit(cfg, "low_latency_layout_dispatch_fp8",
+                         timeit(lambda: B.ep_dispatch_low_latency(x, rt, lay, recv, max_tokens_per_expert=mt,
+                                                                  recv_scales=sc)),
+                         T * K * 12 + T * R + E * 8 + R * 4 + T * H * 2 + n_valid * (H + H // 128 * 4), T)
                 y = torch.zeros((rows, H), dtype=torch.bfloat16, device=dev)
             else:
                 recv = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)

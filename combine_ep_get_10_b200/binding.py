@@ -27,7 +27,8 @@ EP_DEVERR_BAD_INDEX, EP_DEVERR_OVERFLOW, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 EXPORTED = ("ep_workspace_bytes", "ep_workspace_init", "ep_get_layout", "ep_dispatch", "ep_combine",
             "ep_dispatch_expert_choice", "ep_combine_expert_choice", "ep_get_device_error", "ep_status_string",
-            "ep_version", "ep_get_layout_no_alloc", "ep_get_rank_layout", "ep_dispatch_ranks", "ep_combine_ranks")
+            "ep_version", "ep_get_layout_no_alloc", "ep_get_rank_layout", "ep_dispatch_ranks", "ep_combine_ranks",
+            "ep_dispatch_low_latency")
 
 
 class EPError(RuntimeError):
@@ -96,6 +97,8 @@ def lib():
         L.ep_dispatch_ranks.argtypes = [P, i32, RP, LP, KP, i64, P, P, P, P, P, P]
         L.ep_combine_ranks.restype = st
         L.ep_combine_ranks.argtypes = [P, i32, i64, RP, LP, KP, P, st, P]
+        L.ep_dispatch_low_latency.restype = st
+        L.ep_dispatch_low_latency.argtypes = [P, i32, RP, LP, i32, st, P, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -269,6 +272,18 @@ def ep_dispatch(x: torch.Tensor, routing: Routing, layout: Layout, recv_x: torch
     _check(lib().ep_dispatch(_ptr(x), x.shape[1], ctypes.byref(routing.desc), ctypes.byref(layout.desc), int(mode),
                              int(max_tokens_per_expert), rows, out_dtype, _ptr(topk_weights), _ptr(recv_x),
                              _ptr(recv_scales), _ptr(recv_src), _ptr(recv_weights), _stream(stream)), "ep_dispatch")
+
+
+def ep_dispatch_low_latency(x: torch.Tensor, routing: Routing, layout: Layout, recv_x: torch.Tensor, *,
+                            max_tokens_per_expert: int, out_dtype=None, topk_weights=None, recv_scales=None,
+                            recv_src=None, recv_weights=None, stream=None) -> None:
+    """ep_get_layout + padded ep_dispatch in one launch for small batches
+    (layout outputs land in `layout`); out_dtype as for ep_dispatch."""
+    out_dtype = _dtype_code(recv_x) if out_dtype is None else int(out_dtype)
+    _check(lib().ep_dispatch_low_latency(_ptr(x), x.shape[1], ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                                         int(max_tokens_per_expert), out_dtype, _ptr(topk_weights), _ptr(recv_x),
+                                         _ptr(recv_scales), _ptr(recv_src), _ptr(recv_weights), _stream(stream)),
+           "ep_dispatch_low_latency")
 
 
 def ep_combine(y: torch.Tensor, routing: Routing, layout: Layout, topk_weights: torch.Tensor, out: torch.Tensor, *,

@@ -175,10 +175,14 @@ ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* l
     return from_cuda(ep::launch_ec_layout(a, s));
 }
 
-ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing, const ep_layout_t* layout,
-                        ep_buffer_mode_t mode, int32_t max_tokens_per_expert, int64_t num_recv_rows,
-                        ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, void* recv_scales,
-                        int32_t* recv_src, float* recv_weights, ep_stream_t stream)
+namespace {
+
+// Host-side checks of a token-choice dispatch call (ep_dispatch and the
+// dispatch half of ep_dispatch_low_latency).
+ep_status_t check_dispatch_args(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                const ep_layout_t* layout, ep_buffer_mode_t mode, int32_t max_tokens_per_expert,
+                                int64_t num_recv_rows, ep_dtype_t out_dtype, const float* topk_weights, void* recv_x,
+                                void* recv_scales, int32_t* recv_src, float* recv_weights)
 {
     ep_status_t st = check_routing(routing);
     if (st != EP_OK)
@@ -212,6 +216,21 @@ ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* 
         return EP_ERR_INVALID_ARG;
     if (recv_src != nullptr && !aligned(recv_src, 4))
         return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+} // namespace
+
+ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                        ep_buffer_mode_t mode, int32_t max_tokens_per_expert, int64_t num_recv_rows,
+                        ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, void* recv_scales,
+                        int32_t* recv_src, float* recv_weights, ep_stream_t stream)
+{
+    ep_status_t st = check_dispatch_args(x, hidden, routing, layout, mode, max_tokens_per_expert, num_recv_rows,
+                                         out_dtype, topk_weights, recv_x, recv_scales, recv_src, recv_weights);
+    if (st != EP_OK)
+        return st;
+    const int32_t T = routing->num_tokens;
     ep::TcDispatchLaunch a{x,
                            T,
                            hidden,
@@ -224,6 +243,66 @@ ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* 
                            recv_weights,
                            ep::error_word(layout->workspace)};
     return from_cuda(ep::launch_tc_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_dispatch_low_latency(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                    const ep_layout_t* layout, int32_t max_tokens_per_expert, ep_dtype_t out_dtype,
+                                    const float* topk_weights, void* recv_x, void* recv_scales, int32_t* recv_src,
+                                    float* recv_weights, ep_stream_t stream)
+{
+    ep_status_t st = check_routing(routing);
+    if (st != EP_OK)
+        return st;
+    if (routing->routing != EP_ROUTING_TOPK)
+        return EP_ERR_INVALID_ARG;
+    st = check_workspace(routing, layout, true); // the unfused fallback runs ep_get_layout
+    if (st != EP_OK)
+        return st;
+    if (max_tokens_per_expert < 1)
+        return EP_ERR_INVALID_ARG;
+    const int32_t T = routing->num_tokens, K = routing->num_topk, E = routing->num_experts, R = routing->num_ranks;
+    if (E > ep::kMaxTopkLayoutExperts)
+        return EP_ERR_UNSUPPORTED;
+    if (layout->num_tokens_per_expert == nullptr || layout->num_tokens_per_rank == nullptr ||
+        layout->expert_offsets == nullptr || !aligned(layout->num_tokens_per_expert, 4) ||
+        !aligned(layout->num_tokens_per_rank, 4) || !aligned(layout->expert_offsets, 4))
+        return EP_ERR_INVALID_ARG;
+    if (T > 0 && (layout->is_token_in_rank == nullptr || layout->slot == nullptr || !aligned(layout->slot, 4)))
+        return EP_ERR_INVALID_ARG;
+    const int64_t rows = static_cast<int64_t>(E) * max_tokens_per_expert;
+    st = check_dispatch_args(x, hidden, routing, layout, EP_LAYOUT_PADDED, max_tokens_per_expert, rows, out_dtype,
+                             topk_weights, recv_x, recv_scales, recv_src, recv_weights);
+    if (st != EP_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (ep::ll_fusable(T, K, E, hidden, static_cast<int>(out_dtype))) {
+        ep::LowLatencyLaunch a{x,
+                               T,
+                               hidden,
+                               K,
+                               E,
+                               R,
+                               max_tokens_per_expert,
+                               routing->topk_idx,
+                               static_cast<int32_t>(out_dtype),
+                               topk_weights,
+                               recv_x,
+                               recv_scales,
+                               recv_src,
+                               recv_weights,
+                               layout->slot,
+                               layout->is_token_in_rank,
+                               layout->num_tokens_per_expert,
+                               layout->expert_offsets,
+                               layout->num_tokens_per_rank,
+                               ep::error_word(layout->workspace)};
+        return from_cuda(ep::launch_ll_dispatch(a, s));
+    }
+    st = ep_get_layout(routing, layout, stream);
+    if (st != EP_OK)
+        return st;
+    return ep_dispatch(x, hidden, routing, layout, EP_LAYOUT_PADDED, max_tokens_per_expert, rows, out_dtype,
+                       topk_weights, recv_x, recv_scales, recv_src, recv_weights, stream);
 }
 
 ep_status_t ep_combine(const void* y, int32_t hidden, int64_t num_y_rows, const ep_routing_desc_t* routing,

@@ -214,7 +214,8 @@ enum QuantFmt : int {
     kQFp8Tok = EP_FP8_E4M3_PER_TOKEN, // e4m3, fp32 scale per row
     kQMxE4m3 = EP_MXFP8_E4M3,       // e4m3, e8m0 scale per 32
     kQMxE5m2 = EP_MXFP8_E5M2,       // e5m2, e8m0 scale per 32
-    kQMxE2m1 = EP_MXFP4_E2M1        // e2m1 x2, e8m0 scale per 32
+    kQMxE2m1 = EP_MXFP4_E2M1,       // e2m1 x2, e8m0 scale per 32
+    kQBf16 = EP_BF16                // bf16 copy (fused low-latency dispatch only)
 };
 
 struct QuantArgs {
@@ -227,7 +228,19 @@ struct QuantArgs {
     int32_t* recv_src;
     float* recv_weights;
     uint32_t* err;
+    // fused low-latency mode: the layout is computed in the same launch
+    int32_t T, R;
+    int32_t* slot;
+    uint8_t* in_rank;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* rank_counts;
 };
+
+// fused low-latency dispatch limits: a CTA scans the ids of all earlier pairs
+constexpr int kFusedMaxPairs = 8192;
+constexpr int kFusedMaxK = 32;
+constexpr int kFusedMaxE = 1024;
 
 constexpr int kQuantThreads = 128; // threads per token CTA
 
@@ -289,11 +302,156 @@ __device__ __forceinline__ uint2 encode8(uint4 r, float mul)
 // are written with 8-byte stores instead.  Registers stay low, so many CTAs
 // (and their row loads) are resident per SM.
 //   shared memory: x row [2H] | codes [code_row] | scales [scale_row -> 16] | rows [K]
-template <int kFmt>
+// Shared-memory bytes of one token CTA: x row | codes | scales | rows [K]
+// (| fused layout: expert -> k mask [E], histogram [E], per-token rank bits
+// [T], small arrays [4 x 32]).
+__host__ __device__ inline size_t quant_smem_bytes(int fmt, int H, int K, int E, int T, bool fused)
+{
+    const size_t nvec = static_cast<size_t>(H) / 8;
+    const bool mx = fmt == kQMxE4m3 || fmt == kQMxE5m2 || fmt == kQMxE2m1;
+    const size_t code_row = fmt == kQBf16 ? 0 : nvec * (fmt == kQMxE2m1 ? 4 : 8);
+    const size_t scale_row =
+        fmt == kQBf16 ? 0 : (mx ? nvec / 4 : ((fmt == kQInt8Tok || fmt == kQFp8Tok) ? 4 : nvec / 16 * 4));
+    size_t n = nvec * 16 + code_row + ((scale_row + 15) & ~static_cast<size_t>(15)) + sizeof(int64_t) * K;
+    if (fused)
+        n += sizeof(uint32_t) * (2 * static_cast<size_t>(E) + static_cast<size_t>(T) + 4 * 32);
+    return n;
+}
+
+// Fused low-latency layout of token t (padded rows e * max_tokens + slot).
+// The slot of pair (t, k) is the number of earlier pairs (token-major) routed
+// to the same expert: the CTA counts them itself over the ids of tokens
+// 0..t, with a shared expert -> k mask.  The last token's CTA scans every id
+// anyway, so it also builds the per-expert histogram (counts, offsets by a
+// CTA scan) and each token's rank bits (per-rank token counts).  No
+// inter-CTA synchronisation: every output is computed from topk_idx alone.
+__device__ __forceinline__ void fused_layout(const QuantArgs& a, int64_t t, int64_t* rows, uint32_t* sm,
+                                             uint32_t& errbits)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int K = a.map.K, E = a.map.E;
+    const bool last = t == a.T - 1;
+    const int per_rank = E / a.R;
+    uint32_t* s_kmask = sm;             // [E] which of this token's k route to expert e
+    uint32_t* s_hist = sm + E;          // [E] last CTA: pairs per expert
+    uint32_t* s_tmask = sm + 2 * E;     // [T] last CTA: rank bits per token
+    int* s_cnt = reinterpret_cast<int*>(s_tmask + a.T); // [32] earlier pairs per k
+    int* s_e = s_cnt + 32;              // [32] this token's ids (-1 if not routed)
+    int* s_rank = s_cnt + 64;           // [32] last CTA: tokens per rank
+    int* s_wsum = s_cnt + 96;           // [32] last CTA: scan scratch
+    for (int i = tid; i < E; i += kQuantThreads) {
+        s_kmask[i] = 0u;
+        s_hist[i] = 0u;
+    }
+    if (last)
+        for (int i = tid; i < a.T; i += kQuantThreads)
+            s_tmask[i] = 0u;
+    if (tid < 32) {
+        s_cnt[tid] = 0;
+        s_rank[tid] = 0;
+    }
+    __syncthreads();
+    if (tid < K) {
+        const int64_t e = __ldg(a.map.topk_idx + t * K + tid);
+        const bool ok = e >= 0 && e < E;
+        if (!ok && e != -1)
+            errbits |= EP_DEVERR_BAD_INDEX;
+        s_e[tid] = ok ? static_cast<int>(e) : -1;
+        if (ok)
+            atomicOr(&s_kmask[e], 1u << tid);
+    }
+    __syncthreads();
+    const int64_t lim = last ? static_cast<int64_t>(a.T) * K : t * K + K;
+#pragma unroll 4
+    for (int64_t p = tid; p < lim; p += kQuantThreads) {
+        const int64_t e = __ldg(a.map.topk_idx + p);
+        if (e < 0 || e >= E)
+            continue;
+        uint32_t m = s_kmask[e];
+        while (m) {
+            const int k = __ffs(m) - 1;
+            m &= m - 1u;
+            if (p < t * K + k)
+                atomicAdd(&s_cnt[k], 1);
+        }
+        if (last) {
+            atomicAdd(&s_hist[e], 1u);
+            atomicOr(&s_tmask[p / K], 1u << static_cast<uint32_t>(e / per_rank));
+        }
+    }
+    __syncthreads();
+    if (tid < K) {
+        const int e = s_e[tid];
+        const int sl = e >= 0 ? s_cnt[tid] : -1;
+        a.slot[t * K + tid] = sl;
+        int64_t rk = -1;
+        if (e >= 0) {
+            if (sl < a.map.max_tokens)
+                rk = static_cast<int64_t>(e) * a.map.max_tokens + sl;
+            else
+                errbits |= EP_DEVERR_OVERFLOW;
+        }
+        rows[tid] = rk;
+        if (rk >= 0) {
+            if (a.recv_src != nullptr)
+                a.recv_src[rk] = static_cast<int32_t>(t);
+            if (a.recv_weights != nullptr)
+                a.recv_weights[rk] = __ldg(a.topk_weights + t * K + tid);
+        }
+    }
+    if (tid < a.R) {
+        bool in = false;
+        for (int k = 0; k < K; ++k)
+            in |= s_e[k] >= 0 && s_e[k] / per_rank == tid;
+        a.in_rank[t * a.R + tid] = in ? 1 : 0;
+    }
+    if (last) {
+        for (int64_t u = tid; u < a.T; u += kQuantThreads) {
+            uint32_t m = s_tmask[u];
+            while (m) {
+                const int r = __ffs(m) - 1;
+                m &= m - 1u;
+                atomicAdd(&s_rank[r], 1);
+            }
+        }
+        // counts and offsets: thread i owns experts [i*epc, (i+1)*epc)
+        const int epc = (E + kQuantThreads - 1) / kQuantThreads;
+        const int e0 = min(E, tid * epc), e1 = min(E, e0 + epc);
+        int sum = 0;
+        for (int e = e0; e < e1; ++e)
+            sum += static_cast<int>(s_hist[e]);
+        int inc = sum;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int v = __shfl_up_sync(kFullMask, inc, d);
+            if (lane >= d)
+                inc += v;
+        }
+        if (lane == 31)
+            s_wsum[warp] = inc;
+        __syncthreads();
+        int run = inc - sum;
+        for (int w = 0; w < warp; ++w)
+            run += s_wsum[w];
+        for (int e = e0; e < e1; ++e) {
+            const int c = static_cast<int>(s_hist[e]);
+            a.counts[e] = c;
+            a.offsets[e] = run;
+            run += c;
+        }
+        if (tid == kQuantThreads - 1)
+            a.offsets[E] = run; // the last thread's run ends at the total
+        if (tid < a.R)
+            a.rank_counts[tid] = s_rank[tid];
+    }
+}
+
+template <int kFmt, bool kFused>
 __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs a)
 {
     constexpr bool kMx = kFmt == kQMxE4m3 || kFmt == kQMxE5m2 || kFmt == kQMxE2m1;
     constexpr bool kPerToken = kFmt == kQInt8Tok || kFmt == kQFp8Tok;
+    constexpr bool kCopy = kFmt == kQBf16;
     constexpr int kGroupLanes = kFmt == kQFp8G128 ? 16 : 4; // group modes only
     constexpr int kCodeBytes = kFmt == kQMxE2m1 ? 4 : 8;  // bytes per 8 channels
     extern __shared__ __align__(128) uint8_t qsmem[];
@@ -303,11 +461,11 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
     const int tid = threadIdx.x;
     const int nvec = a.H / 8;
     const int row_bytes = a.H * 2;
-    const int code_row = nvec * kCodeBytes;
-    const int scale_row = kMx ? nvec / 4 : (kPerToken ? 4 : nvec / 16 * 4);
+    const int code_row = kCopy ? row_bytes : nvec * kCodeBytes;
+    const int scale_row = kCopy ? 0 : (kMx ? nvec / 4 : (kPerToken ? 4 : nvec / 16 * 4));
     uint8_t* s_x = qsmem;
-    uint8_t* s_codes = qsmem + row_bytes;
-    uint8_t* s_scales = s_codes + code_row;
+    uint8_t* s_codes = kCopy ? s_x : qsmem + row_bytes;
+    uint8_t* s_scales = qsmem + row_bytes + (kCopy ? 0 : code_row);
     int64_t* rows = reinterpret_cast<int64_t*>(s_scales + ((scale_row + 15) & ~15));
 
     if (tid == 0) {
@@ -318,19 +476,23 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
                       static_cast<uint32_t>(row_bytes), &bar);
     }
     uint32_t errbits = 0;
-    for (int k = tid; k < a.map.K; k += kQuantThreads) {
-        const int64_t rk = a.map.row(t, k, errbits);
-        rows[k] = rk;
-        if (rk >= 0) {
-            if (a.recv_src != nullptr)
-                a.recv_src[rk] = static_cast<int32_t>(t);
-            if (a.recv_weights != nullptr)
-                a.recv_weights[rk] = __ldg(a.topk_weights + t * a.map.K + k);
+    if constexpr (kFused) {
+        fused_layout(a, t, rows, reinterpret_cast<uint32_t*>(rows + a.map.K), errbits);
+    } else {
+        for (int k = tid; k < a.map.K; k += kQuantThreads) {
+            const int64_t rk = a.map.row(t, k, errbits);
+            rows[k] = rk;
+            if (rk >= 0) {
+                if (a.recv_src != nullptr)
+                    a.recv_src[rk] = static_cast<int32_t>(t);
+                if (a.recv_weights != nullptr)
+                    a.recv_weights[rk] = __ldg(a.topk_weights + t * a.map.K + k);
+            }
         }
     }
     if (errbits)
         flag_error(a.err, errbits);
-    __syncthreads(); // barrier initialised before anyone waits on it
+    __syncthreads(); // barrier initialised (and rows written) before anyone reads them
     if (!mbar_wait_bounded(&bar, 0, a.err))
         return;
 
@@ -360,7 +522,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
     }
 
     // uniform trip count: every lane takes part in the group shuffles
-    for (int base = 0; base < nvec; base += kQuantThreads) {
+    for (int base = 0; !kCopy && base < nvec; base += kQuantThreads) {
         const int v = base + tid;
         const bool active = v < nvec; // a scale group is all-in or all-out
         const uint4 raw = active ? *reinterpret_cast<const uint4*>(s_x + v * 16) : make_uint4(0, 0, 0, 0);
@@ -403,7 +565,8 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
     __syncthreads();
 
     const bool bulk_codes = (code_row & 15) == 0;
-    const bool bulk_scales = (scale_row & 15) == 0 && (reinterpret_cast<uintptr_t>(a.scales) & 15) == 0;
+    const bool bulk_scales =
+        kCopy || ((scale_row & 15) == 0 && (reinterpret_cast<uintptr_t>(a.scales) & 15) == 0);
     if (bulk_codes) {
         bool issued = false;
         for (int k = tid; k < a.map.K; k += kQuantThreads) {
@@ -411,7 +574,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
             if (rk < 0)
                 continue;
             bulk_store_s2g(a.recv + rk * code_row, s_codes, static_cast<uint32_t>(code_row));
-            if (bulk_scales)
+            if (bulk_scales && !kCopy)
                 bulk_store_s2g(static_cast<uint8_t*>(a.scales) + rk * scale_row, s_scales,
                                static_cast<uint32_t>(scale_row));
             issued = true;
@@ -428,7 +591,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
                 st_v2(dst + i * 8, *reinterpret_cast<const uint2*>(s_codes + i * 8));
         }
     }
-    if (!(bulk_codes && bulk_scales)) {
+    if (!kCopy && !(bulk_codes && bulk_scales)) {
         // scales by plain stores (per-token: 4 bytes; rows not 16-byte multiples)
         for (int k = 0; k < a.map.K; ++k) {
             const int64_t rk = rows[k];
@@ -448,23 +611,43 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
         bulk_wait_read_all(); // shared memory must outlive the copies' reads
 }
 
-template <int kFmt>
+template <int kFmt, bool kFused>
 cudaError_t launch_quant(const QuantArgs& a, int32_t T, int32_t K, cudaStream_t stream)
 {
-    const size_t nvec = static_cast<size_t>(a.H) / 8;
-    const bool mx = kFmt == kQMxE4m3 || kFmt == kQMxE5m2 || kFmt == kQMxE2m1;
-    const size_t code_row = nvec * (kFmt == kQMxE2m1 ? 4 : 8);
-    const size_t scale_row = mx ? nvec / 4 : ((kFmt == kQInt8Tok || kFmt == kQFp8Tok) ? 4 : nvec / 16 * 4);
-    const size_t smem = nvec * 16 + code_row + ((scale_row + 15) & ~static_cast<size_t>(15)) + sizeof(int64_t) * K;
+    const size_t smem = quant_smem_bytes(kFmt, a.H, K, a.map.E, kFused ? T : 0, kFused);
     if (smem > 48 * 1024) {
-        cudaError_t st = cudaFuncSetAttribute(quant_dispatch_kernel<kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(smem));
+        cudaError_t st = cudaFuncSetAttribute(quant_dispatch_kernel<kFmt, kFused>,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (st != cudaSuccess)
             return st;
     }
-    const int nthr = kQuantThreads;
-    quant_dispatch_kernel<kFmt><<<T, nthr, smem, stream>>>(a);
+    quant_dispatch_kernel<kFmt, kFused><<<T, kQuantThreads, smem, stream>>>(a);
     return cudaGetLastError();
+}
+
+template <bool kFused>
+cudaError_t launch_quant_fmt(int fmt, const QuantArgs& k, int32_t T, int32_t K, cudaStream_t stream)
+{
+    switch (fmt) {
+    case EP_FP8_E4M3:
+        return launch_quant<kQFp8G128, kFused>(k, T, K, stream);
+    case EP_INT8_PER_TOKEN:
+        return launch_quant<kQInt8Tok, kFused>(k, T, K, stream);
+    case EP_FP8_E4M3_PER_TOKEN:
+        return launch_quant<kQFp8Tok, kFused>(k, T, K, stream);
+    case EP_MXFP8_E4M3:
+        return launch_quant<kQMxE4m3, kFused>(k, T, K, stream);
+    case EP_MXFP8_E5M2:
+        return launch_quant<kQMxE5m2, kFused>(k, T, K, stream);
+    case EP_MXFP4_E2M1:
+        return launch_quant<kQMxE2m1, kFused>(k, T, K, stream);
+    case EP_BF16:
+        if constexpr (kFused)
+            return launch_quant<kQBf16, true>(k, T, K, stream);
+        return cudaErrorInvalidValue;
+    default:
+        return cudaErrorInvalidValue;
+    }
 }
 
 constexpr int64_t kMaxGrid = int64_t{1} << 30;
@@ -485,6 +668,36 @@ cudaError_t launch_bulk(BulkArgs k, int64_t items, cudaStream_t stream)
 
 } // namespace
 
+bool ll_fusable(int32_t T, int32_t K, int32_t E, int32_t H, int out_dtype)
+{
+    return T > 0 && static_cast<int64_t>(T) * K <= kFusedMaxPairs && K <= kFusedMaxK && E <= kFusedMaxE &&
+           quant_smem_bytes(out_dtype, H, K, E, T, true) <= 200 * 1024;
+}
+
+cudaError_t launch_ll_dispatch(const LowLatencyLaunch& a, cudaStream_t stream)
+{
+    RowMap m{a.topk_idx, nullptr, nullptr, a.K, a.E, EP_LAYOUT_PADDED, a.max_tokens,
+             static_cast<int64_t>(a.E) * a.max_tokens};
+    QuantArgs k{};
+    k.x = static_cast<const uint16_t*>(a.x);
+    k.H = a.H;
+    k.map = m;
+    k.recv = static_cast<uint8_t*>(a.recv_x);
+    k.scales = a.recv_scales;
+    k.topk_weights = a.topk_weights;
+    k.recv_src = a.recv_src;
+    k.recv_weights = a.recv_weights;
+    k.err = a.err;
+    k.T = a.T;
+    k.R = a.R;
+    k.slot = a.slot;
+    k.in_rank = a.in_rank;
+    k.counts = a.counts;
+    k.offsets = a.offsets;
+    k.rank_counts = a.rank_counts;
+    return launch_quant_fmt<true>(a.out_dtype, k, a.T, a.K, stream);
+}
+
 cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream)
 {
     if (a.T == 0)
@@ -492,24 +705,17 @@ cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream)
     RowMap m{a.rows.topk_idx, a.rows.slot, a.rows.offsets, a.rows.K, a.rows.E, a.rows.mode, a.rows.max_tokens,
              a.rows.num_rows};
     if (a.out_dtype != EP_BF16) {
-        QuantArgs k{static_cast<const uint16_t*>(a.x), a.H, m, static_cast<uint8_t*>(a.recv_x), a.recv_scales,
-                    a.topk_weights, a.recv_src, a.recv_weights, a.err};
-        switch (a.out_dtype) {
-        case EP_FP8_E4M3:
-            return launch_quant<kQFp8G128>(k, a.T, a.rows.K, stream);
-        case EP_INT8_PER_TOKEN:
-            return launch_quant<kQInt8Tok>(k, a.T, a.rows.K, stream);
-        case EP_FP8_E4M3_PER_TOKEN:
-            return launch_quant<kQFp8Tok>(k, a.T, a.rows.K, stream);
-        case EP_MXFP8_E4M3:
-            return launch_quant<kQMxE4m3>(k, a.T, a.rows.K, stream);
-        case EP_MXFP8_E5M2:
-            return launch_quant<kQMxE5m2>(k, a.T, a.rows.K, stream);
-        case EP_MXFP4_E2M1:
-            return launch_quant<kQMxE2m1>(k, a.T, a.rows.K, stream);
-        default:
-            return cudaErrorInvalidValue;
-        }
+        QuantArgs k{};
+        k.x = static_cast<const uint16_t*>(a.x);
+        k.H = a.H;
+        k.map = m;
+        k.recv = static_cast<uint8_t*>(a.recv_x);
+        k.scales = a.recv_scales;
+        k.topk_weights = a.topk_weights;
+        k.recv_src = a.recv_src;
+        k.recv_weights = a.recv_weights;
+        k.err = a.err;
+        return launch_quant_fmt<false>(a.out_dtype, k, a.T, a.rows.K, stream);
     }
     BulkArgs k{};
     k.src = static_cast<const uint8_t*>(a.x);

@@ -82,6 +82,28 @@ struct TcDispatchLaunch {
 };
 cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream);
 
+// Fused low-latency dispatch: the token-choice layout and a padded dispatch
+// (bf16 or any quantised format) in one launch, for small batches.
+struct LowLatencyLaunch {
+    const void* x;
+    int32_t T, H, K, E, R, max_tokens;
+    const int64_t* topk_idx;
+    int32_t out_dtype;
+    const float* topk_weights;
+    void* recv_x;
+    void* recv_scales;
+    int32_t* recv_src;
+    float* recv_weights;
+    int32_t* slot;
+    uint8_t* in_rank;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* rank_counts;
+    uint32_t* err;
+};
+bool ll_fusable(int32_t T, int32_t K, int32_t E, int32_t H, int out_dtype);
+cudaError_t launch_ll_dispatch(const LowLatencyLaunch& a, cudaStream_t stream);
+
 struct EcDispatchLaunch {
     const void* x;
     int32_t T, H, E, C;

@@ -198,6 +198,23 @@ EP_API ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_d
                         ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, void* recv_scales,
                         int32_t* recv_src, float* recv_weights, ep_stream_t stream);
 
+/* Low-latency dispatch ([README] API Overview: low_latency_dispatch, which
+ * takes topk_idx and num_max_dispatch_tokens_per_rank and needs no separate
+ * layout call): exactly ep_get_layout(routing, layout) followed by
+ * ep_dispatch(..., EP_LAYOUT_PADDED, max_tokens_per_expert,
+ * num_recv_rows = E * max_tokens_per_expert, out_dtype, ...), with the same
+ * outputs, arguments and errors, but in ONE launch when T * K <= 8192,
+ * K <= 32 and E <= 1024 (each token's CTA counts the earlier pairs of its
+ * experts itself; the last token's CTA forms the counts, offsets and
+ * per-rank totals).  Larger batches take the two-call path.  out_dtype may
+ * be EP_BF16 or any quantised format; layout->workspace must have
+ * ep_workspace_bytes() bytes. */
+EP_API ep_status_t ep_dispatch_low_latency(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                           const ep_layout_t* layout, int32_t max_tokens_per_expert,
+                                           ep_dtype_t out_dtype, const float* topk_weights, void* recv_x,
+                                           void* recv_scales, int32_t* recv_src, float* recv_weights,
+                                           ep_stream_t stream);
+
 /* Token-choice combine ([README] API Overview: combine / low_latency_combine,
  * the weighted reduce; [EC] Solution 2: -1 slots are skipped).
  *   out[t] = sum over k = 0..K-1 of topk_weights[t,k] * y[row(t,k)], over the

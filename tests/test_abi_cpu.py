@@ -127,6 +127,27 @@ def test_dispatch_and_combine_reject_bad_args(L):
     assert L.ep_combine_expert_choice(0x2000, 256, ctypes.byref(ec), ctypes.byref(lay), None, 0x5000, 0, None) == 1
 
 
+def test_low_latency_dispatch_rejects_bad_args(L):
+    d = _topk_desc()
+    ws = L.ep_workspace_bytes(ctypes.byref(d))
+    lay = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x100000, ws)
+
+    def ll(desc=d, layout=lay, hidden=256, mt=4, dt=B.EP_BF16, x=0x2000, recv=0x4000, sc=None):
+        return L.ep_dispatch_low_latency(x, hidden, ctypes.byref(desc), ctypes.byref(layout), mt, dt, None, recv,
+                                         sc, None, None, None)
+
+    assert ll(mt=0) == 1  # padded rows need max_tokens >= 1
+    assert ll(desc=_ec_desc()) == 1  # token choice only
+    assert ll(hidden=12) == 1
+    assert ll(dt=B.EP_FP32) == 1
+    assert ll(dt=B.EP_MXFP8_E4M3, sc=None) == 1  # scales required
+    assert ll(x=0x2008) == 1
+    small = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x100000, 256)
+    assert ll(layout=small) == 4  # needs the full layout workspace (the two-call path may run)
+    assert ll(desc=_topk_desc(E=2048, R=1), layout=B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None,
+                                                                  0x100000, 1 << 24)) == 6
+
+
 def test_device_error_rejects_missing_workspace(L):
     lay = B.LayoutDesc(None, None, None, None, None, None, None, None, 0)
     flags = ctypes.c_uint32(0)
