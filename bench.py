@@ -532,10 +532,35 @@ def run_workload_table(args):
                                                                        max_tokens_per_expert=mt, recv_scales=sc)),
                      T * H * 2 + n_valid * (H + H // 128 * 4) + meta, T)
                 if mode == W.PADDED:  # layout + padded FP8 dispatch in one call
+                    ll_bytes = T * K * 12 + T * R + E * 8 + R * 4 + T * H * 2 + n_valid * (H + H // 128 * 4)
                     emit(cfg, "low_latency_layout_dispatch_fp8",
                          timeit(lambda: B.ep_dispatch_low_latency(x, rt, lay, recv, max_tokens_per_expert=mt,
-                                                                  recv_scales=sc)),
-                         T * K * 12 + T * R + E * 8 + R * 4 + T * H * 2 + n_valid * (H + H // 128 * 4), T)
+                                                                  recv_scales=sc)), ll_bytes, T)
+                    # the decode step (fused dispatch + padded combine) replayed from a CUDA graph
+                    yy = torch.zeros((rows, H), dtype=torch.bfloat16, device=dev)
+                    oo = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+                    gs = torch.cuda.Stream(dev)
+
+                    def decode_step():
+                        B.ep_dispatch_low_latency(x, rt, lay, recv, max_tokens_per_expert=mt, recv_scales=sc,
+                                                  stream=gs)
+                        B.ep_combine(yy, rt, lay, w, oo, mode=mode, max_tokens_per_expert=mt, stream=gs)
+
+                    gs.wait_stream(torch.cuda.current_stream(dev))
+                    decode_step()
+                    torch.cuda.synchronize(dev)
+                    graph = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(graph, stream=gs):
+                        decode_step()
+                    step_bytes_ll = ll_bytes + n_valid * H * 2 + T * H * 2 + T * K * 16 + E * 4
+                    emit(cfg, "decode_step_eager (fused dispatch + combine)",
+                         timeit(lambda: (B.ep_dispatch_low_latency(x, rt, lay, recv, max_tokens_per_expert=mt,
+                                                                   recv_scales=sc),
+                                         B.ep_combine(yy, rt, lay, w, oo, mode=mode, max_tokens_per_expert=mt))),
+                         step_bytes_ll, T)
+                    emit(cfg, "decode_step_cuda_graph (fused dispatch + combine)", timeit(graph.replay),
+                         step_bytes_ll, T)
+                    del graph
                 y = torch.zeros((rows, H), dtype=torch.bfloat16, device=dev)
             else:
                 recv = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)
