@@ -404,6 +404,8 @@ EC_EDGE = [
     (3000, 4, 5, 1, 64, 0.0, 0.0, 4),   # most tokens unpicked
     (1, 3, 2, 3, 8, 0.5, 0.0, 5),
     (20000, 2, 700, 1, 8, 0.0, 0.0, 6),  # scan over several 8192-token passes
+    (3000, 64, 1024, 4, 64, 0.0, 0.0, 7),  # ~3000 tokens with >= 16 picks: more than the combine lists
+    (70000, 2, 1000, 1, 8, 0.0, 0.0, 8),  # T above the combine's heavy-listing limit
 ]
 
 
