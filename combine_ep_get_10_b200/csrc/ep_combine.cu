@@ -98,7 +98,10 @@ struct CombineArgs {
 };
 
 // expert choice, heavy first (see combine_kernel)
-constexpr int kHeavyDeg = 16;
+#ifndef EP_COMBINE_EC_HEAVY_DEG
+#define EP_COMBINE_EC_HEAVY_DEG 16
+#endif
+constexpr int kHeavyDeg = EP_COMBINE_EC_HEAVY_DEG; // picks that make a token "heavy"
 constexpr int kMaxHeavy = 2048;
 constexpr int kHeavyFirstMaxT = 65536;
 // 16-byte vectors of CSR bounds each thread loads per round of the heavy listing
