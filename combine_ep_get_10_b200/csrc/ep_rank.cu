@@ -57,13 +57,21 @@ __global__ void __launch_bounds__(kRankThreads) rank_layout_kernel(RankLayoutLau
     for (int i = tid; i < kRankWarps * 33; i += kRankThreads)
         (&s_wpre[0][0])[i] = 0;
     __syncthreads();
-    // tokens of the earlier tiles, per rank
-    for (int64_t base = 0; base < tile; base += kRankThreads) {
-        const uint32_t mask = token_mask(a.in_rank, base + tid, R);
+    // tokens of the earlier tiles, per rank (four tiles' masks loaded at once)
+    for (int64_t base = 0; base < tile; base += 4 * kRankThreads) {
+        uint32_t m4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t u = base + i * kRankThreads + tid;
+            m4[i] = u < tile ? token_mask(a.in_rank, u, R) : 0u;
+        }
         for (int r = 0; r < R; ++r) {
-            const uint32_t b = __ballot_sync(kFullMask, (mask >> r) & 1u);
+            int c = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                c += __popc(__ballot_sync(kFullMask, (m4[i] >> r) & 1u));
             if (lane == 0)
-                s_wpre[warp][r] += __popc(b);
+                s_wpre[warp][r] += c;
         }
     }
     __syncthreads();
