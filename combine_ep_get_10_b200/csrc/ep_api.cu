@@ -4,10 +4,22 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "ep.h"
 #include "ep_internal.h"
 
 namespace {
+
+// An NVTX range named after the entry point, around the whole call (checks
+// and launches), so that profilers can attribute kernels to ABI calls.  With
+// no tool attached the push and pop return at once.
+struct CallRange {
+    explicit CallRange(const char* name) { nvtxRangePushA(name); }
+    ~CallRange() { nvtxRangePop(); }
+    CallRange(const CallRange&) = delete;
+    CallRange& operator=(const CallRange&) = delete;
+};
 
 using ep::kWorkspaceHeaderBytes;
 
@@ -115,6 +127,7 @@ size_t ep_workspace_bytes(const ep_routing_desc_t* routing)
 
 ep_status_t ep_workspace_init(void* workspace, size_t bytes, ep_stream_t stream)
 {
+    CallRange range_("ep_workspace_init");
     if (workspace == nullptr || !aligned(workspace, 256) || bytes < kWorkspaceHeaderBytes)
         return EP_ERR_WORKSPACE;
     return from_cuda(cudaMemsetAsync(workspace, 0, bytes, reinterpret_cast<cudaStream_t>(stream)));
@@ -122,6 +135,7 @@ ep_status_t ep_workspace_init(void* workspace, size_t bytes, ep_stream_t stream)
 
 ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream)
 {
+    CallRange range_("ep_get_layout");
     ep_status_t st = check_routing(routing);
     if (st != EP_OK)
         return st;
@@ -226,6 +240,7 @@ ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* 
                         ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, void* recv_scales,
                         int32_t* recv_src, float* recv_weights, ep_stream_t stream)
 {
+    CallRange range_("ep_dispatch");
     ep_status_t st = check_dispatch_args(x, hidden, routing, layout, mode, max_tokens_per_expert, num_recv_rows,
                                          out_dtype, topk_weights, recv_x, recv_scales, recv_src, recv_weights);
     if (st != EP_OK)
@@ -250,6 +265,7 @@ ep_status_t ep_dispatch_low_latency(const void* x, int32_t hidden, const ep_rout
                                     const float* topk_weights, void* recv_x, void* recv_scales, int32_t* recv_src,
                                     float* recv_weights, ep_stream_t stream)
 {
+    CallRange range_("ep_dispatch_low_latency");
     ep_status_t st = check_routing(routing);
     if (st != EP_OK)
         return st;
@@ -309,6 +325,7 @@ ep_status_t ep_combine(const void* y, int32_t hidden, int64_t num_y_rows, const 
                        const ep_layout_t* layout, ep_buffer_mode_t mode, int32_t max_tokens_per_expert,
                        const float* topk_weights, void* out, ep_dtype_t out_dtype, ep_stream_t stream)
 {
+    CallRange range_("ep_combine");
     ep_status_t st = check_routing(routing);
     if (st != EP_OK)
         return st;
@@ -341,6 +358,7 @@ ep_status_t ep_combine(const void* y, int32_t hidden, int64_t num_y_rows, const 
 ep_status_t ep_dispatch_expert_choice(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
                                       const ep_layout_t* layout, void* recv_x, ep_stream_t stream)
 {
+    CallRange range_("ep_dispatch_expert_choice");
     ep_status_t st = check_routing(routing);
     if (st != EP_OK)
         return st;
@@ -368,6 +386,7 @@ ep_status_t ep_combine_expert_choice(const void* y, int32_t hidden, const ep_rou
                                      const ep_layout_t* layout, const float* expert_weights, void* out,
                                      ep_dtype_t out_dtype, ep_stream_t stream)
 {
+    CallRange range_("ep_combine_expert_choice");
     ep_status_t st = check_routing(routing);
     if (st != EP_OK)
         return st;
@@ -423,6 +442,7 @@ ep_status_t check_rank_call(const ep_routing_desc_t* routing, const ep_layout_t*
 ep_status_t ep_get_rank_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout,
                                const ep_rank_layout_t* rank_layout, ep_stream_t stream)
 {
+    CallRange range_("ep_get_rank_layout");
     ep_status_t st = check_rank_call(routing, layout, rank_layout);
     if (st != EP_OK)
         return st;
@@ -443,6 +463,7 @@ ep_status_t ep_dispatch_ranks(const void* x, int32_t hidden, const ep_routing_de
                               const float* topk_weights, void* recv_x, int64_t* recv_topk_idx,
                               float* recv_topk_weights, int32_t* recv_src, ep_stream_t stream)
 {
+    CallRange range_("ep_dispatch_ranks");
     ep_status_t st = check_rank_call(routing, layout, rank_layout);
     if (st != EP_OK)
         return st;
@@ -482,6 +503,7 @@ ep_status_t ep_combine_ranks(const void* y, int32_t hidden, int64_t num_y_rows, 
                              const ep_layout_t* layout, const ep_rank_layout_t* rank_layout, void* out,
                              ep_dtype_t out_dtype, ep_stream_t stream)
 {
+    CallRange range_("ep_combine_ranks");
     ep_status_t st = check_rank_call(routing, layout, rank_layout);
     if (st != EP_OK)
         return st;
@@ -508,6 +530,7 @@ ep_status_t ep_combine_ranks(const void* y, int32_t hidden, int64_t num_y_rows, 
 
 ep_status_t ep_get_device_error(const ep_layout_t* layout, uint32_t* flags, int clear, ep_stream_t stream)
 {
+    CallRange range_("ep_get_device_error");
     if (layout == nullptr || layout->workspace == nullptr || !aligned(layout->workspace, 256) ||
         layout->workspace_bytes < kWorkspaceHeaderBytes)
         return EP_ERR_WORKSPACE;
