@@ -433,7 +433,9 @@ def run_ours(args):
             "kernels_gbs": {k: nbytes[k] / (k_ms[k] * 1e-3) / 1e9 for k in k_ms},
             "algorithmic_bytes_per_step": nbytes,
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_source": peak_kind, "traffic": traffic},
+                         "frac": achieved / peak, "peak_source": peak_kind, "traffic": traffic,
+                         "frac_of_nominal_8000_gbs": achieved / 8000.0,
+                         "step_frac": value / peak},
             "gpu_launches": 3 * K_steps,
             "e2e": {"value": step_bytes * e2e_steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "tokens_per_s": T * e2e_steps * world / (e2e_ms * 1e-3), "steps": e2e_steps,
