@@ -18,6 +18,7 @@
 // a producer warp streaming row chunks into a shared-memory ring -- measured
 // no faster at 4096 tokens and slower under expert-choice skew.)
 #include <algorithm>
+#include <atomic>
 #include <type_traits>
 
 #include "ep_device.cuh"
@@ -443,23 +444,26 @@ __global__ void __launch_bounds__(kCombineThreads) ec_combine_kernel(CombineArgs
 }
 
 // Blocks of 256 threads of `kernel` resident on the whole device (SMs x
-// blocks per SM), cached per device in `cache`.
+// blocks per SM), cached per device in `cache` (host threads may race to
+// fill an entry; they store the same value).
 template <typename Kernel>
-int64_t resident_blocks(Kernel kernel, int* cache)
+int64_t resident_blocks(Kernel kernel, std::atomic<int>* cache)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return 0;
-    if (cache[dev] == 0) {
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         int sms = 0, per_sm = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kCombineThreads, 0) != cudaSuccess) {
             cudaGetLastError();
             return 0;
         }
-        cache[dev] = sms * std::max(per_sm, 1);
+        n = sms * std::max(per_sm, 1);
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 // persistent: one resident wave of warps loops over the (token, segment)
@@ -472,7 +476,7 @@ cudaError_t launch_combine(CombineArgs k, bool out_f32, bool persistent, cudaStr
     const int64_t warps = static_cast<int64_t>(k.T) * k.nseg;
     int64_t blocks = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
     if (persistent) {
-        static int cache_bf16[64], cache_f32[64];
+        static std::atomic<int> cache_bf16[64], cache_f32[64];
         const int64_t res = out_f32 ? resident_blocks(combine_kernel<kSrc, true, kVec, kGrp>, cache_f32)
                                     : resident_blocks(combine_kernel<kSrc, false, kVec, kGrp>, cache_bf16);
         if (res > 0)
@@ -498,7 +502,7 @@ cudaError_t launch_ec(CombineArgs k, bool out_f32, cudaStream_t stream)
     k.nseg = (k.nvec + 32 * kEcVec - 1) / (32 * kEcVec);
     const int64_t runs = (static_cast<int64_t>(k.T) + kEcRun - 1) / kEcRun;
     const int64_t items = std::max<int64_t>(1, runs * k.nseg);
-    static int cache_bf16[64], cache_f32[64];
+    static std::atomic<int> cache_bf16[64], cache_f32[64];
     const int64_t res = out_f32 ? resident_blocks(ec_combine_kernel<true>, cache_f32)
                                 : resident_blocks(ec_combine_kernel<false>, cache_bf16);
     int64_t blocks = res > 0 ? res : (items + kWarpsPerCta - 1) / kWarpsPerCta;

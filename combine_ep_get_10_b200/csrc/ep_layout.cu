@@ -18,6 +18,7 @@
 // then each token's slot list is put in ascending order by a warp that ranks
 // every entry against the others (slot ids are distinct).
 #include <algorithm>
+#include <atomic>
 
 #include <cooperative_groups.h>
 
@@ -996,8 +997,10 @@ __global__ void __launch_bounds__(kEcClusterThreads, 1) ec_layout_cluster_kernel
     }
 }
 
-int cluster_limit_cache[64];
-size_t smem_attr_cache[64];
+// per-device caches of driver queries (host threads may race to fill an
+// entry; they store the same value)
+std::atomic<int> cluster_limit_cache[64];
+std::atomic<size_t> smem_attr_cache[64];
 
 // Kernel attributes (dynamic shared memory limit, 16-CTA clusters) are set
 // once per device and shared-memory size; later calls skip the driver calls.
@@ -1007,7 +1010,7 @@ cudaError_t prepare_layout_kernel(size_t smem)
     cudaError_t st = cudaGetDevice(&dev);
     if (st != cudaSuccess)
         return st;
-    if (dev >= 0 && dev < 64 && smem_attr_cache[dev] >= smem)
+    if (dev >= 0 && dev < 64 && smem_attr_cache[dev].load(std::memory_order_relaxed) >= smem)
         return cudaSuccess;
     const size_t want = std::max<size_t>(smem, sizeof(int32_t) * (kLayoutWarps * 256 + 3 * 256 + 64 + 2 * kSmemIds));
     st = cudaFuncSetAttribute(tc_layout_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1018,7 +1021,7 @@ cudaError_t prepare_layout_kernel(size_t smem)
     if (st != cudaSuccess)
         return st;
     if (dev >= 0 && dev < 64)
-        smem_attr_cache[dev] = want;
+        smem_attr_cache[dev].store(want, std::memory_order_relaxed);
     return cudaSuccess;
 }
 
@@ -1027,7 +1030,7 @@ int max_layout_cluster(size_t smem_bytes)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return 8;
-    int cached = cluster_limit_cache[dev];
+    int cached = cluster_limit_cache[dev].load(std::memory_order_relaxed);
     if (cached > 0)
         return cached;
     int best = 8;
@@ -1046,11 +1049,11 @@ int max_layout_cluster(size_t smem_bytes)
     if (cudaOccupancyMaxActiveClusters(&n, tc_layout_cluster_kernel, &cfg) == cudaSuccess && n >= 1)
         best = 16;
     cudaGetLastError();
-    cluster_limit_cache[dev] = best;
+    cluster_limit_cache[dev].store(best, std::memory_order_relaxed);
     return best;
 }
 
-int ec_cluster_limit_cache[64];
+std::atomic<int> ec_cluster_limit_cache[64];
 
 // 16-CTA clusters of the expert-choice kernel fit on this device (else 8).
 int max_ec_cluster()
@@ -1058,8 +1061,9 @@ int max_ec_cluster()
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return 8;
-    if (ec_cluster_limit_cache[dev] > 0)
-        return ec_cluster_limit_cache[dev];
+    const int cached_ec = ec_cluster_limit_cache[dev].load(std::memory_order_relaxed);
+    if (cached_ec > 0)
+        return cached_ec;
     int best = 8;
     const size_t smem = ec_cluster_smem_bytes(kEcClusterMaxT, kEcClusterSlotsPerCta, kEcClusterMaxE);
     if (cudaFuncSetAttribute(ec_layout_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1082,7 +1086,7 @@ int max_ec_cluster()
             best = 16;
     }
     cudaGetLastError();
-    ec_cluster_limit_cache[dev] = best;
+    ec_cluster_limit_cache[dev].store(best, std::memory_order_relaxed);
     return best;
 }
 
@@ -1093,7 +1097,7 @@ size_t tc_layout_workspace_bytes(int64_t E)
     return kWorkspaceHeaderBytes + sizeof(int32_t) * static_cast<size_t>(kGridMaxBlocks) * (E + 32);
 }
 
-int grid_blocks_cache[64];
+std::atomic<int> grid_blocks_cache[64];
 
 cudaError_t launch_tc_layout_grid(const TcArgs& k, void* workspace, cudaStream_t stream)
 {
@@ -1102,7 +1106,7 @@ cudaError_t launch_tc_layout_grid(const TcArgs& k, void* workspace, cudaStream_t
     if (st != cudaSuccess)
         return st;
     const size_t smem = sizeof(int32_t) * (static_cast<size_t>(kGridWarps) * k.E + 64 + 2 * kGridIds + 4);
-    int resident = dev >= 0 && dev < 64 ? grid_blocks_cache[dev] : 0;
+    int resident = dev >= 0 && dev < 64 ? grid_blocks_cache[dev].load(std::memory_order_relaxed) : 0;
     if (resident == 0) {
         const size_t max_smem = sizeof(int32_t) * (static_cast<size_t>(kGridWarps) * kMaxTopkLayoutExperts + 64 +
                                                    2 * kGridIds + 4);
@@ -1118,7 +1122,7 @@ cudaError_t launch_tc_layout_grid(const TcArgs& k, void* workspace, cudaStream_t
             return st;
         resident = std::max(1, sms * per_sm);
         if (dev >= 0 && dev < 64)
-            grid_blocks_cache[dev] = resident;
+            grid_blocks_cache[dev].store(resident, std::memory_order_relaxed);
     }
     const int64_t pairs = static_cast<int64_t>(k.T) * k.K;
     const int G = static_cast<int>(std::min<int64_t>(
@@ -1193,7 +1197,7 @@ size_t ec_layout_workspace_bytes(int64_t T, int64_t E, int64_t C)
     return kWorkspaceHeaderBytes + ((arrays + 255) / 256) * 256;
 }
 
-int ec_smem_attr_dev[64];
+std::atomic<int> ec_smem_attr_dev[64];
 
 cudaError_t launch_ec_layout_cluster(const EcLayoutLaunch& a, cudaStream_t stream, bool& launched)
 {
