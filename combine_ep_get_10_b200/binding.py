@@ -116,7 +116,14 @@ def _check(status: int, what: str) -> None:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device (or pinned host) address of a dense row-major tensor; the C ABI
+    takes plain pointers, so strided views are refused here."""
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("the C ABI takes dense row-major tensors; got a strided view of shape %s"
+                         % (tuple(t.shape),))
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream):
