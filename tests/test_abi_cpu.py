@@ -152,3 +152,14 @@ def test_device_error_rejects_missing_workspace(L):
     lay = B.LayoutDesc(None, None, None, None, None, None, None, None, 0)
     flags = ctypes.c_uint32(0)
     assert L.ep_get_device_error(ctypes.byref(lay), ctypes.byref(flags), 1, None) == 4
+
+
+def test_token_rounds_cover_the_batch_in_order():
+    assert B.token_rounds(0, 8) == []
+    assert B.token_rounds(10, 4) == [(0, 4), (4, 8), (8, 10)]
+    assert B.token_rounds(8192, 8192) == [(0, 8192)]
+    r = B.token_rounds(131072, 8192)
+    assert len(r) == 16 and r[0] == (0, 8192) and r[-1] == (122880, 131072)
+    assert all(b0 == a1 for (_, a1), (b0, _) in zip(r, r[1:]))
+    with pytest.raises(ValueError):
+        B.token_rounds(10, 0)
