@@ -105,6 +105,43 @@ struct CombineArgs {
 constexpr int kHeavyDeg = EP_COMBINE_EC_HEAVY_DEG; // picks that make a token "heavy"
 constexpr int kMaxHeavy = 2048;
 constexpr int kHeavyFirstMaxT = 65536;
+// heavy tokens listed by degree class, longest lists first (1: token order)
+#ifndef EP_COMBINE_HEAVY_SORT
+#define EP_COMBINE_HEAVY_SORT 1
+#endif
+constexpr int kHeavyClasses = EP_COMBINE_HEAVY_SORT ? 3 : 1;
+// entries a heavy item looks up at once, in units of 32
+#ifndef EP_COMBINE_HEAVY_LOOKUP
+#define EP_COMBINE_HEAVY_LOOKUP 1
+#endif
+constexpr int kHeavyLookup = EP_COMBINE_HEAVY_LOOKUP;
+// light runs: one list over the run's tokens (1) or one token at a time (0)
+#ifndef EP_COMBINE_EC_FLAT
+#define EP_COMBINE_EC_FLAT 1
+#endif
+#ifndef EP_COMBINE_EC_LOOKUP
+#define EP_COMBINE_EC_LOOKUP 1
+#endif
+constexpr int kEcLookup = EP_COMBINE_EC_LOOKUP;
+// resident CTAs per SM the expert-choice kernel is compiled for
+#ifndef EP_COMBINE_EC_MINB
+#define EP_COMBINE_EC_MINB 2
+#endif
+constexpr int kEcMinBlocks = EP_COMBINE_EC_MINB;
+// heavy items: lookups pipelined (reduce_heavy) or not (reduce_segment)
+#ifndef EP_COMBINE_HEAVY_PIPE
+#define EP_COMBINE_HEAVY_PIPE 1
+#endif
+// the longest lists (>= 4 kHeavyDeg picks, when listed by class) take
+// narrower segments and longer groups: twice the warps, half the rounds
+#ifndef EP_COMBINE_HEAVY0_VEC
+#define EP_COMBINE_HEAVY0_VEC 1
+#endif
+#ifndef EP_COMBINE_HEAVY0_GROUP
+#define EP_COMBINE_HEAVY0_GROUP 16
+#endif
+constexpr int kHeavy0Vec = EP_COMBINE_HEAVY0_VEC;
+constexpr int kHeavy0Group = EP_COMBINE_HEAVY0_GROUP;
 // 16-byte vectors of CSR bounds each thread loads per round of the heavy listing
 constexpr int kHeavyVecs = 8;
 
@@ -270,6 +307,271 @@ __device__ __forceinline__ void reduce_segment(const CombineArgs& a, int64_t t, 
     }
 }
 
+// out[t, segment] <- acc (kVecPerLane 16-byte vectors per lane, as in
+// reduce_segment)
+template <bool kOutF32, int kVecPerLane>
+__device__ __forceinline__ void store_segment(const CombineArgs& a, int64_t t, const int (&v)[kVecPerLane],
+                                              const bool (&vin)[kVecPerLane], const float (&acc)[kVecPerLane][8])
+{
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j) {
+        if (!vin[j])
+            continue;
+        if (kOutF32) {
+            float* o = static_cast<float*>(a.out) + t * a.H + static_cast<int64_t>(v[j]) * 8;
+            st_cs_v4(o, make_uint4(__float_as_uint(acc[j][0]), __float_as_uint(acc[j][1]), __float_as_uint(acc[j][2]),
+                                   __float_as_uint(acc[j][3])));
+            st_cs_v4(o + 4, make_uint4(__float_as_uint(acc[j][4]), __float_as_uint(acc[j][5]),
+                                       __float_as_uint(acc[j][6]), __float_as_uint(acc[j][7])));
+        } else {
+            uint8_t* o = static_cast<uint8_t*>(a.out) + t * static_cast<int64_t>(a.H) * 2 + static_cast<int64_t>(v[j]) * 16;
+            st_cs_v4(o, make_uint4(pack_bf16x2(acc[j][0], acc[j][1]), pack_bf16x2(acc[j][2], acc[j][3]),
+                                   pack_bf16x2(acc[j][4], acc[j][5]), pack_bf16x2(acc[j][6], acc[j][7])));
+        }
+    }
+}
+
+// Expert choice, a run of light tokens t0 .. t0 + cnt - 1 (cnt <= 32, lane j
+// holds token j's CSR bounds), one segment.  The entries of the run's tokens
+// (skipping heavy ones when skip_heavy) make one list in token order, each
+// token's CSR slots in order.  Lanes look the list up kLookup * 32 entries at
+// a time; the warp folds it kGroup entries at a time with every load of a
+// group issued together, also when the group spans tokens, so a run costs
+// one load round per kGroup entries instead of one per token.  A token's
+// accumulators start from zero at its first entry and are stored after its
+// last: each token's sum is the fmaf chain over its own entries in ascending
+// CSR order, as in reduce_segment.  Tokens without entries store zeros.
+template <bool kOutF32, int kVecPerLane, int kGroup, int kLookup>
+__device__ __forceinline__ void reduce_run(const CombineArgs& a, int64_t t0, int cnt, int seg, bool skip_heavy,
+                                           int lane, uint32_t& errbits)
+{
+    constexpr int kSegVec = 32 * kVecPerLane;
+    int v[kVecPerLane];
+    bool vin[kVecPerLane];
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j) {
+        v[j] = seg * kSegVec + j * 32 + lane;
+        vin[j] = v[j] < a.nvec;
+    }
+    float acc[kVecPerLane][8];
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            acc[j][i] = 0.0f;
+
+    int my_beg = 0, my_n = 0;
+    if (lane < cnt) {
+        my_beg = __ldg(a.token_offsets + t0 + lane);
+        my_n = __ldg(a.token_offsets + t0 + lane + 1) - my_beg;
+    }
+    const bool mine = lane < cnt && !(skip_heavy && my_n >= kHeavyDeg);
+    const int my_cnt = mine ? max(my_n, 0) : 0;
+    uint32_t zeros = __ballot_sync(kFullMask, mine && my_cnt == 0);
+    while (zeros) { // warp-uniform
+        const int j = __ffs(zeros) - 1;
+        zeros &= zeros - 1u;
+        store_segment<kOutF32, kVecPerLane>(a, t0 + j, v, vin, acc);
+    }
+    int incl = my_cnt; // list positions up to and including this lane's token
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(kFullMask, incl, d);
+        if (lane >= d)
+            incl += o;
+    }
+    const int total = __shfl_sync(kFullMask, incl, 31);
+    const int my_start = incl - my_cnt;
+
+    int cur = -1; // lane (token) whose sum is open
+    for (int c0 = 0; c0 < total; c0 += 32 * kLookup) {
+        int32_t my_row[kLookup];
+        float my_w[kLookup];
+        int my_tok[kLookup];
+        uint32_t first[kLookup]; // bit g: list position 32 * i + g opens a token
+#pragma unroll
+        for (int i = 0; i < kLookup; ++i) {
+            const int e = c0 + 32 * i + lane;
+            // owner of list position e: the number of lanes whose entries end
+            // at or before e (incl is non-decreasing over the lanes)
+            int j = 0;
+#pragma unroll
+            for (int step = 16; step >= 1; step >>= 1) {
+                const int end = __shfl_sync(kFullMask, incl, j + step - 1);
+                if (end <= e)
+                    j += step;
+            }
+            const int jbeg = __shfl_sync(kFullMask, my_beg, j);
+            const int jstart = __shfl_sync(kFullMask, my_start, j);
+            my_tok[i] = j;
+            first[i] = __ballot_sync(kFullMask, e < total && e == jstart);
+            my_row[i] = -1;
+            my_w[i] = 0.0f;
+            if (e < total) {
+                const int32_t s = __ldg(a.token_slots + jbeg + (e - jstart));
+                if (s < 0 || s >= a.num_y_rows) {
+                    errbits |= EP_DEVERR_OVERFLOW;
+                } else {
+                    my_row[i] = s;
+                    my_w[i] = __ldg(a.expert_weights + s);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kLookup; ++i) {
+            const int kb = c0 + 32 * i;
+            if (kb >= total)
+                break; // warp-uniform
+            const int m = min(32, total - kb);
+            for (int g0 = 0; g0 < m; g0 += kGroup) {
+                int32_t rows[kGroup];
+                float ws[kGroup];
+#pragma unroll
+                for (int g = 0; g < kGroup; ++g) {
+                    const int src = (g0 + g) & 31;
+                    rows[g] = __shfl_sync(kFullMask, my_row[i], src);
+                    ws[g] = __shfl_sync(kFullMask, my_w[i], src);
+                    if (g0 + g >= m)
+                        rows[g] = -1;
+                }
+                uint4 d[kGroup][kVecPerLane];
+#pragma unroll
+                for (int g = 0; g < kGroup; ++g)
+#pragma unroll
+                    for (int j = 0; j < kVecPerLane; ++j)
+                        d[g][j] = (rows[g] >= 0 && vin[j])
+                                      ? ld_nc_v4(a.y + static_cast<int64_t>(rows[g]) * a.H * 2 +
+                                                 static_cast<int64_t>(v[j]) * 16)
+                                      : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int g = 0; g < kGroup; ++g) {
+                    if (g0 + g >= m)
+                        break; // warp-uniform
+                    if ((first[i] >> ((g0 + g) & 31)) & 1u) { // warp-uniform: a token opens, the open one ended
+                        if (cur >= 0)
+                            store_segment<kOutF32, kVecPerLane>(a, t0 + cur, v, vin, acc);
+#pragma unroll
+                        for (int j = 0; j < kVecPerLane; ++j)
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                acc[j][q] = 0.0f;
+                        cur = __shfl_sync(kFullMask, my_tok[i], (g0 + g) & 31);
+                    }
+                    if (rows[g] < 0)
+                        continue;
+#pragma unroll
+                    for (int j = 0; j < kVecPerLane; ++j) {
+                        acc[j][0] = fmaf(ws[g], bf16_lo(d[g][j].x), acc[j][0]);
+                        acc[j][1] = fmaf(ws[g], bf16_hi(d[g][j].x), acc[j][1]);
+                        acc[j][2] = fmaf(ws[g], bf16_lo(d[g][j].y), acc[j][2]);
+                        acc[j][3] = fmaf(ws[g], bf16_hi(d[g][j].y), acc[j][3]);
+                        acc[j][4] = fmaf(ws[g], bf16_lo(d[g][j].z), acc[j][4]);
+                        acc[j][5] = fmaf(ws[g], bf16_hi(d[g][j].z), acc[j][5]);
+                        acc[j][6] = fmaf(ws[g], bf16_lo(d[g][j].w), acc[j][6]);
+                        acc[j][7] = fmaf(ws[g], bf16_hi(d[g][j].w), acc[j][7]);
+                    }
+                }
+            }
+        }
+    }
+    if (cur >= 0)
+        store_segment<kOutF32, kVecPerLane>(a, t0 + cur, v, vin, acc);
+}
+
+// Expert choice, one heavy token's segment: the same fmaf chain as
+// reduce_segment (entries in ascending CSR order, from zero), with the
+// entry lookups taken off the chain: the slots of the next 32 entries are in
+// flight while the current 32 are folded, and their weights are fetched
+// while the first group of the current 32 is in flight, so a long list costs
+// one load round per kGroup entries plus two at the start.
+template <bool kOutF32, int kVecPerLane, int kGroup>
+__device__ __forceinline__ void reduce_heavy(const CombineArgs& a, int64_t t, int seg, int beg, int n, int lane,
+                                             uint32_t& errbits)
+{
+    constexpr int kSegVec = 32 * kVecPerLane;
+    static_assert(32 % kGroup == 0, "a group never straddles two lookups");
+    int v[kVecPerLane];
+    bool vin[kVecPerLane];
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j) {
+        v[j] = seg * kSegVec + j * 32 + lane;
+        vin[j] = v[j] < a.nvec;
+    }
+    float acc[kVecPerLane][8];
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            acc[j][i] = 0.0f;
+
+    const int64_t row_bytes = static_cast<int64_t>(a.H) * 2;
+    // slot of entry j (-1 past the list); a slot outside y is flagged and skipped
+    auto slot_at = [&](int j) -> int32_t { return j < n ? __ldg(a.token_slots + beg + j) : -1; };
+    auto valid = [&](int j, int32_t s) -> bool {
+        if (j >= n)
+            return false;
+        if (s < 0 || s >= a.num_y_rows) {
+            errbits |= EP_DEVERR_OVERFLOW;
+            return false;
+        }
+        return true;
+    };
+    int32_t s_cur = slot_at(lane);
+    int32_t s_nxt = slot_at(32 + lane);
+    int32_t r_cur = valid(lane, s_cur) ? s_cur : -1;
+    float w_cur = r_cur >= 0 ? __ldg(a.expert_weights + r_cur) : 0.0f;
+    for (int k0 = 0; k0 < n; k0 += 32) {
+        const int m = min(32, n - k0);
+        int32_t r_nxt = -1, s_after = -1;
+        float w_nxt = 0.0f;
+        for (int g0 = 0; g0 < m; g0 += kGroup) {
+            int32_t rows[kGroup];
+            float ws[kGroup];
+#pragma unroll
+            for (int g = 0; g < kGroup; ++g) {
+                rows[g] = __shfl_sync(kFullMask, r_cur, g0 + g);
+                ws[g] = __shfl_sync(kFullMask, w_cur, g0 + g);
+                if (g0 + g >= m)
+                    rows[g] = -1;
+            }
+            uint4 d[kGroup][kVecPerLane];
+#pragma unroll
+            for (int g = 0; g < kGroup; ++g)
+#pragma unroll
+                for (int j = 0; j < kVecPerLane; ++j)
+                    d[g][j] = (rows[g] >= 0 && vin[j])
+                                  ? ld_nc_v4(a.y + static_cast<int64_t>(rows[g]) * row_bytes +
+                                             static_cast<int64_t>(v[j]) * 16)
+                                  : make_uint4(0, 0, 0, 0);
+            if (g0 == 0) { // the next 32 entries' weights, and the slots of the 32 after them
+                r_nxt = valid(k0 + 32 + lane, s_nxt) ? s_nxt : -1;
+                w_nxt = r_nxt >= 0 ? __ldg(a.expert_weights + r_nxt) : 0.0f;
+                s_after = slot_at(k0 + 64 + lane);
+            }
+#pragma unroll
+            for (int g = 0; g < kGroup; ++g) {
+                if (rows[g] < 0)
+                    continue;
+#pragma unroll
+                for (int j = 0; j < kVecPerLane; ++j) {
+                    acc[j][0] = fmaf(ws[g], bf16_lo(d[g][j].x), acc[j][0]);
+                    acc[j][1] = fmaf(ws[g], bf16_hi(d[g][j].x), acc[j][1]);
+                    acc[j][2] = fmaf(ws[g], bf16_lo(d[g][j].y), acc[j][2]);
+                    acc[j][3] = fmaf(ws[g], bf16_hi(d[g][j].y), acc[j][3]);
+                    acc[j][4] = fmaf(ws[g], bf16_lo(d[g][j].z), acc[j][4]);
+                    acc[j][5] = fmaf(ws[g], bf16_hi(d[g][j].z), acc[j][5]);
+                    acc[j][6] = fmaf(ws[g], bf16_lo(d[g][j].w), acc[j][6]);
+                    acc[j][7] = fmaf(ws[g], bf16_hi(d[g][j].w), acc[j][7]);
+                }
+            }
+        }
+        r_cur = r_nxt;
+        w_cur = w_nxt;
+        s_nxt = s_after;
+    }
+    store_segment<kOutF32, kVecPerLane>(a, t, v, vin, acc);
+}
+
 // Token choice and per-rank rows: one warp per (token, segment) item; the
 // items are taken with a fixed stride by a persistent grid (uniform cost).
 template <int kSrc, bool kOutF32, int kVecPerLane, int kGroup>
@@ -292,36 +594,40 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 }
 
 // Expert choice.  A few tokens are picked by up to all E experts and most by
-// none, so the work per token varies by 100x.  Every CTA first lists, in
-// token order, the tokens with at least kHeavyDeg picks (the same list in
-// every CTA).  The items are then: one per (heavy token, segment), followed
-// by one per (run of 32 tokens, segment).  A run item reads the 32 tokens'
-// CSR bounds with one load per lane and walks the tokens: unpicked ones just
-// store zeros, heavy ones are skipped (done as heavy items), the rest are
-// reduced.  Warps are numbered warp-major (warp w of every CTA before warp
-// w + 1): heavy items go to the first warps, so they spread over all SMs, and
-// light items to the last warps first, so the long lists get no light work
-// unless there are more items than warps.
+// none, so the work per token varies by 100x.  Every CTA first lists the
+// tokens with at least kHeavyDeg picks (the same list in every CTA): by
+// degree class, longest first (>= 4x, >= 2x, >= 1x kHeavyDeg), in token
+// order inside a class.  The items are then: one per (heavy token, segment),
+// followed by one per (run of kEcRun tokens, segment); a run item folds its
+// light tokens' entries as one list (reduce_run) and leaves the heavy tokens
+// to the heavy items.  Warps are numbered warp-major (warp w of every CTA
+// before warp w + 1): heavy items go to the first warps, so they spread over
+// all SMs, and light items to the last warps first, so that when there are
+// more items than warps the extra light work lands on the warps holding the
+// shortest heavy lists.
 template <bool kOutF32>
-__global__ void __launch_bounds__(kCombineThreads) ec_combine_kernel(CombineArgs a)
+__global__ void __launch_bounds__(kCombineThreads, kEcMinBlocks) ec_combine_kernel(CombineArgs a)
 {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     uint32_t errbits = 0;
 
     __shared__ int s_heavy[kMaxHeavy];
-    __shared__ uint32_t s_flags[kHeavyFirstMaxT / 32];
+    __shared__ uint32_t s_flags[kHeavyClasses][kHeavyFirstMaxT / 32];
     __shared__ int s_wsum[kWarpsPerCta];
-    int n_heavy = 0;
+    int n_heavy = 0, n_long = 0;
     if (a.heavy_first) {
         // Every CTA reads the whole CSR bound array once, coalesced and all at
         // once (16-byte vectors, kHeavyVecs per thread, plus the bound after
-        // each vector), flags the heavy tokens in a shared bit mask, then
-        // lists them in token order (count per 32-token word, CTA scan).
+        // each vector), flags the heavy tokens in one shared bit mask per
+        // degree class, then lists them class by class (count per 32-token
+        // word, CTA scan).
         const int tid = threadIdx.x;
         const int nwords = (a.T + 31) / 32;
         for (int i = tid; i < nwords; i += kCombineThreads)
-            s_flags[i] = 0u;
+#pragma unroll
+            for (int c = 0; c < kHeavyClasses; ++c)
+                s_flags[c][i] = 0u;
         __syncthreads();
         // 4 bounds per 16-byte vector (1 when the array is not 16-byte aligned),
         // kHeavyVecs vectors per thread per round, all loads of a round at once
@@ -358,52 +664,64 @@ __global__ void __launch_bounds__(kCombineThreads) ec_combine_kernel(CombineArgs
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int t = per * v + j;
-                    if (j < per && t < a.T && (j + 1 < per ? o[j + 1] : o[4]) - o[j] >= kHeavyDeg)
-                        atomicOr(&s_flags[t / 32], 1u << (t % 32));
+                    const int deg = (j + 1 < per ? o[j + 1] : o[4]) - o[j];
+                    if (j < per && t < a.T && deg >= kHeavyDeg) {
+                        const int c = kHeavyClasses == 1 ? 0 : deg >= 4 * kHeavyDeg ? 0 : deg >= 2 * kHeavyDeg ? 1 : 2;
+                        atomicOr(&s_flags[c][t / 32], 1u << (t % 32));
+                    }
                 }
             }
         }
         __syncthreads();
-        // words w0 .. w1 of this thread, scanned over the CTA
+        // words w0 .. w1 of this thread, scanned over the CTA, class by class
         const int wpt = (nwords + kCombineThreads - 1) / kCombineThreads;
         const int w0 = min(nwords, tid * wpt);
         const int w1 = min(nwords, w0 + wpt);
-        int cnt = 0;
-        for (int w = w0; w < w1; ++w)
-            cnt += __popc(s_flags[w]);
-        int inc = cnt;
+        int listed = 0;
+#pragma unroll 1
+        for (int c = 0; c < kHeavyClasses; ++c) {
+            if (c == 1)
+                n_long = listed; // class 0: the longest lists
+            int cnt = 0;
+            for (int w = w0; w < w1; ++w)
+                cnt += __popc(s_flags[c][w]);
+            int inc = cnt;
 #pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int v = __shfl_up_sync(kFullMask, inc, d);
-            if (lane >= d)
-                inc += v;
-        }
-        if (lane == 31)
-            s_wsum[warp] = inc;
-        __syncthreads();
-        int before = 0;
-        n_heavy = 0;
-        for (int w = 0; w < kWarpsPerCta; ++w) {
-            before += w < warp ? s_wsum[w] : 0;
-            n_heavy += s_wsum[w];
-        }
-        if (n_heavy <= kMaxHeavy) {
-            int pos = before + inc - cnt;
-            for (int w = w0; w < w1; ++w) {
-                uint32_t bits = s_flags[w];
-                while (bits) {
-                    const int i = __ffs(bits) - 1;
-                    bits &= bits - 1u;
-                    s_heavy[pos++] = w * 32 + i;
+            for (int d = 1; d < 32; d <<= 1) {
+                const int v = __shfl_up_sync(kFullMask, inc, d);
+                if (lane >= d)
+                    inc += v;
+            }
+            if (lane == 31)
+                s_wsum[warp] = inc;
+            __syncthreads();
+            int before = 0, n_c = 0;
+            for (int w = 0; w < kWarpsPerCta; ++w) {
+                before += w < warp ? s_wsum[w] : 0;
+                n_c += s_wsum[w];
+            }
+            if (listed + n_c <= kMaxHeavy) {
+                int pos = listed + before + inc - cnt;
+                for (int w = w0; w < w1; ++w) {
+                    uint32_t bits = s_flags[c][w];
+                    while (bits) {
+                        const int i = __ffs(bits) - 1;
+                        bits &= bits - 1u;
+                        s_heavy[pos++] = w * 32 + i;
+                    }
                 }
             }
-        } else {
-            n_heavy = 0; // too many to list: every token goes through the runs
+            listed += n_c;
+            __syncthreads(); // s_wsum is reused by the next class
         }
-        __syncthreads();
+        n_heavy = listed <= kMaxHeavy ? listed : 0; // too many to list: every token goes through the runs
+        if (n_heavy == 0 || kHeavyClasses == 1)
+            n_long = 0;
     }
     const int nseg_h = (a.nvec + 32 * kHeavyVec - 1) / (32 * kHeavyVec);
-    const int64_t heavy_items = static_cast<int64_t>(n_heavy) * nseg_h;
+    const int nseg_l = (a.nvec + 32 * kHeavy0Vec - 1) / (32 * kHeavy0Vec);
+    const int64_t long_items = static_cast<int64_t>(n_long) * nseg_l;
+    const int64_t heavy_items = long_items + static_cast<int64_t>(n_heavy - n_long) * nseg_h;
     const int64_t runs = (static_cast<int64_t>(a.T) + kEcRun - 1) / kEcRun;
     const int64_t items = heavy_items + runs * a.nseg;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerCta;
@@ -412,19 +730,35 @@ __global__ void __launch_bounds__(kCombineThreads) ec_combine_kernel(CombineArgs
     // backwards, so a warp with a long list gets light work only when there
     // are more items than warps
     for (int64_t it = g; it < heavy_items; it += nwarps) {
-        const int64_t t = s_heavy[it / nseg_h];
-        const int seg = static_cast<int>(it % nseg_h);
+        const bool is_long = it < long_items;
+        const int64_t k = is_long ? it : it - long_items;
+        const int ns = is_long ? nseg_l : nseg_h;
+        const int64_t t = s_heavy[(is_long ? 0 : n_long) + k / ns];
+        const int seg = static_cast<int>(k % ns);
         const int beg = __ldg(a.token_offsets + t);
         const int n = __ldg(a.token_offsets + t + 1) - beg;
-        reduce_segment<kSrcEc, kOutF32, kHeavyVec, kHeavyGroup, 2>(a, t, seg, beg, n, lane, errbits);
+#if EP_COMBINE_HEAVY_PIPE
+        if (is_long)
+            reduce_heavy<kOutF32, kHeavy0Vec, kHeavy0Group>(a, t, seg, beg, n, lane, errbits);
+        else
+            reduce_heavy<kOutF32, kHeavyVec, kHeavyGroup>(a, t, seg, beg, n, lane, errbits);
+#else
+        if (is_long)
+            reduce_segment<kSrcEc, kOutF32, kHeavy0Vec, kHeavy0Group, kHeavyLookup>(a, t, seg, beg, n, lane, errbits);
+        else
+            reduce_segment<kSrcEc, kOutF32, kHeavyVec, kHeavyGroup, kHeavyLookup>(a, t, seg, beg, n, lane, errbits);
+#endif
     }
     const int64_t light_items = items - heavy_items;
     for (int64_t it = nwarps - 1 - g; it < light_items; it += nwarps) {
-        // a run of up to kEcRun tokens; lane j holds the CSR bounds of its j-th token
         const int64_t r = it / a.nseg;
         const int seg = static_cast<int>(it - r * a.nseg);
         const int64_t t0 = r * kEcRun;
         const int cnt = static_cast<int>(min(static_cast<int64_t>(kEcRun), a.T - t0));
+#if EP_COMBINE_EC_FLAT
+        reduce_run<kOutF32, kEcVec, kEcGroup, kEcLookup>(a, t0, cnt, seg, n_heavy > 0, lane, errbits);
+#else
+        // lane j holds the CSR bounds of the run's j-th token; one token at a time
         int my_beg = 0, my_n = 0;
         if (lane < cnt) {
             my_beg = __ldg(a.token_offsets + t0 + lane);
@@ -437,6 +771,7 @@ __global__ void __launch_bounds__(kCombineThreads) ec_combine_kernel(CombineArgs
                 continue; // done as a heavy item
             reduce_segment<kSrcEc, kOutF32, kEcVec, kEcGroup, 2>(a, t0 + j, seg, beg, n, lane, errbits);
         }
+#endif
     }
     const uint32_t any = __reduce_or_sync(kFullMask, errbits);
     if (lane == 0)

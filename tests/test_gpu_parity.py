@@ -406,6 +406,7 @@ EC_EDGE = [
     (20000, 2, 700, 1, 8, 0.0, 0.0, 6),  # scan over several 8192-token passes
     (3000, 64, 1024, 4, 64, 0.0, 0.0, 7),  # ~3000 tokens with >= 16 picks: more than the combine lists
     (70000, 2, 1000, 1, 8, 0.0, 0.0, 8),  # T above the combine's heavy-listing limit
+    (100, 128, 64, 1, 1000, 0.0, 0.0, 9),  # lists of ~80 picks: the narrow heavy segments, ragged hidden
 ]
 
 
@@ -432,6 +433,29 @@ def test_ec_edges(case):
         ref = oracle.ec_combine(y, ref_l, ew, T, out_dtype=dt)
         assert_combine_close(host(out), ref, bf, "ec edges")
         assert exact_fraction(host(out), ref) == 1.0
+
+
+@pytest.mark.parametrize("T,E,C,H", [(600, 96, 64, 1000), (1000, 128, 64, 264)])
+def test_ec_skewed_mixed(T, E, C, H):
+    """The workload's skewed expert-choice router at a size the oracle checks
+    whole: unpicked tokens, light tokens and heavy ones of every degree class
+    (>= 64, 32-63, 16-31 picks) in one launch, ragged hidden sizes."""
+    r = rng(T)
+    ti, ew = W.route_expert_choice(r, T, E, C)
+    deg = np.bincount(ti[ti >= 0].ravel(), minlength=T)
+    assert (deg >= 64).any() and ((deg >= 32) & (deg < 64)).any() and ((deg >= 16) & (deg < 32)).any()
+    assert ((deg > 0) & (deg < 16)).any() and (deg == 0).any()
+    ref_l = oracle.ec_layout(ti, T, 2)
+    routing, lay, flags = gpu_ec_layout(ti, T, 2)
+    assert flags == 0
+    y = W.to_bf16_bits(r.standard_normal((E * C, H)).astype(np.float32))
+    for dt, bf in ((W.FP32, False), (W.BF16, True)):
+        out = torch.empty((T, H), dtype=torch.float32 if dt == W.FP32 else torch.bfloat16, device="cuda")
+        B.ep_combine_expert_choice(to_dev(y, bf16=True), routing, lay, to_dev(ew), out)
+        ref = oracle.ec_combine(y, ref_l, ew, T, out_dtype=dt)
+        assert_combine_close(host(out), ref, bf, "ec skewed")
+        assert exact_fraction(host(out), ref) == 1.0
+    assert B.ep_get_device_error(lay) == 0
 
 
 def test_device_error_word_clears():
