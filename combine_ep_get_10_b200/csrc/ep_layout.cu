@@ -528,7 +528,7 @@ __global__ void __launch_bounds__(kGridThreads) tc_layout_grid_kernel(TcArgs a, 
 
     // phase 3: base per expert = totals of the CTAs before this one; CTA 0
     // also forms the counts, offsets and rank totals
-    constexpr int kUnroll = 16;
+    constexpr int kUnroll = kGridMaxBlocks; // every CTA's total in flight at once
     int carry = 0;
     for (int e0 = 0; e0 < a.E; e0 += kGridThreads) {
         const int e = e0 + tid;
@@ -563,9 +563,14 @@ __global__ void __launch_bounds__(kGridThreads) tc_layout_grid_kernel(TcArgs a, 
         if (tid == 0)
             a.offsets[a.E] = carry;
         if (tid < a.R) {
+            int v[kGridMaxBlocks];
+#pragma unroll
+            for (int j = 0; j < kGridMaxBlocks; ++j)
+                v[j] = j < G ? __ldcg(tile_ranks + j * 32 + tid) : 0;
             int n = 0;
-            for (int j = 0; j < G; ++j)
-                n += __ldcg(tile_ranks + j * 32 + tid);
+#pragma unroll
+            for (int j = 0; j < kGridMaxBlocks; ++j)
+                n += v[j];
             a.rank_counts[tid] = n;
         }
     }
@@ -812,10 +817,22 @@ __global__ void __launch_bounds__(kEcClusterThreads, 1) ec_layout_cluster_kernel
     const int64_t s0 = min(S, static_cast<int64_t>(b) * spc);
     const int64_t s1 = min(S, s0 + spc);
     bool bad = false;
-    for (int64_t sb = s0 + (tid & ~31); sb < s1; sb += kEcClusterThreads) {
+    // every id of this thread in flight at once (spc <= kEcClusterSlotsPerCta)
+    constexpr int kIdsPerThread = static_cast<int>(kEcClusterSlotsPerCta / kEcClusterThreads);
+    int tids[kIdsPerThread];
+#pragma unroll
+    for (int i = 0; i < kIdsPerThread; ++i) {
+        const int64_t s = s0 + (tid & ~31) + static_cast<int64_t>(i) * kEcClusterThreads + lane;
+        tids[i] = s < s1 ? __ldg(a.ti + s) : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < kIdsPerThread; ++i) {
+        const int64_t sb = s0 + (tid & ~31) + static_cast<int64_t>(i) * kEcClusterThreads;
+        if (sb >= s1)
+            break; // warp-uniform
         const int64_t s = sb + lane;
         const bool in = s < s1;
-        const int t = in ? __ldg(a.ti + s) : -1;
+        const int t = tids[i];
         const bool good = in && t >= 0 && t < a.T;
         bad |= in && !good && t != -1;
         const int e = in ? static_cast<int>(s / a.C) : -1;
@@ -912,9 +929,14 @@ __global__ void __launch_bounds__(kEcClusterThreads, 1) ec_layout_cluster_kernel
     const int e_own = tid;
     if (b == 0) {
         for (int e = tid; e < a.E; e += kEcClusterThreads) {
+            int v[kMaxCluster];
+#pragma unroll
+            for (int j = 0; j < kMaxCluster; ++j)
+                v[j] = j < cs ? cluster.map_shared_rank(pcount, j)[e] : 0;
             int n = 0;
-            for (int j = 0; j < cs; ++j)
-                n += cluster.map_shared_rank(pcount, j)[e];
+#pragma unroll
+            for (int j = 0; j < kMaxCluster; ++j)
+                n += v[j];
             if (e == e_own)
                 ecount = n;
             else
