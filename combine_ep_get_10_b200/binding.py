@@ -17,6 +17,8 @@ LIB_PATH = os.path.join(_HERE, "libep_b200.so")
 
 # enums of include/ep.h
 EP_OK = 0
+EP_ERR_INVALID_ARG, EP_ERR_BAD_INDEX, EP_ERR_OVERFLOW, EP_ERR_WORKSPACE = 1, 2, 3, 4
+EP_ERR_CUDA, EP_ERR_UNSUPPORTED, EP_ERR_TIMEOUT = 5, 6, 7
 STATUS_NAMES = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_BAD_INDEX", 3: "EP_ERR_OVERFLOW",
                 4: "EP_ERR_WORKSPACE", 5: "EP_ERR_CUDA", 6: "EP_ERR_UNSUPPORTED", 7: "EP_ERR_TIMEOUT"}
 EP_BF16, EP_FP32, EP_FP8_E4M3 = 0, 1, 2
@@ -193,7 +195,7 @@ class Routing:
 def ep_workspace_bytes(routing: Routing) -> int:
     n = lib().ep_workspace_bytes(ctypes.byref(routing.desc))
     if n == 0:
-        raise EPError(1, "ep_workspace_bytes")
+        raise EPError(EP_ERR_INVALID_ARG, "ep_workspace_bytes")
     return int(n)
 
 
@@ -321,7 +323,7 @@ def ep_get_device_error(layout: Layout, clear: bool = True, stream=None) -> int:
     flags = ctypes.c_uint32(0)
     st = lib().ep_get_device_error(ctypes.byref(layout.desc), ctypes.byref(flags), 1 if clear else 0,
                                    _stream(stream))
-    if st not in (EP_OK, 2, 3, 7):
+    if st not in (EP_OK, EP_ERR_BAD_INDEX, EP_ERR_OVERFLOW, EP_ERR_TIMEOUT):  # these report the flags
         raise EPError(st, "ep_get_device_error")
     return int(flags.value)
 

@@ -163,3 +163,18 @@ def test_token_rounds_cover_the_batch_in_order():
     assert all(b0 == a1 for (_, a1), (b0, _) in zip(r, r[1:]))
     with pytest.raises(ValueError):
         B.token_rounds(10, 0)
+
+
+def test_binding_constants_match_the_header():
+    """Every enum value and device-error bit of include/ep.h has the same value
+    in the binding (the binding marshals them as plain ints)."""
+    here = os.path.dirname(os.path.abspath(__file__))
+    text = open(os.path.join(here, "..", "include", "ep.h")).read()
+    values = {m.group(1): int(m.group(2), 0) for m in re.finditer(r"\b(EP_[A-Z0-9_]+) = (\d+)\b", text)}
+    values.update({m.group(1): int(m.group(2), 16) for m in
+                   re.finditer(r"#define (EP_DEVERR_[A-Z_]+) 0x([0-9a-fA-F]+)u", text)})
+    assert len(values) >= 22, sorted(values)
+    for name, v in values.items():
+        assert getattr(B, name) == v, name
+    for v, name in B.STATUS_NAMES.items():
+        assert values[name] == v
