@@ -190,3 +190,49 @@ def test_quant_dispatch_rejects_bad_shapes():
         B.ep_dispatch(torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda"), routing, lay, codes,
                       recv_scales=sc[1:], out_dtype=W.FP8_E4M3_PER_TOKEN)
     assert ei.value.status == 1
+
+
+def _codec_sweep_rows(H=7168):
+    """bf16 rows for an exhaustive codec check: groups of 128 channels that
+    hold one amax value and 127 others bounded by it, such that every finite
+    bf16 value of magnitude <= amax appears (both signs) under every amax of
+    the sweep (each exponent field 0..254, subnormal amax included, positive
+    and negative amax).  2^24 values and more; padded with zero groups."""
+    mags = np.arange(0x7F80, dtype=np.uint16)  # finite magnitudes, as bits
+    groups = []
+    for e in range(255):
+        m = (e * 37 + 1) % 128 or 1
+        amax = np.uint16((e << 7) | m)
+        for sign in (0, 0x8000):
+            vals = mags[mags <= amax]
+            vals = np.concatenate([vals, vals | 0x8000]).astype(np.uint16)
+            ng = (len(vals) + 126) // 127
+            vals = np.concatenate([vals, np.zeros(ng * 127 - len(vals), np.uint16)]).reshape(ng, 127)
+            g = np.empty((ng, 128), np.uint16)
+            g[:, 0] = amax | sign
+            g[:, 1:] = vals
+            groups.append(g)
+    g = np.concatenate(groups)
+    n_values = g.size
+    per = H // 128
+    T = (g.shape[0] + per - 1) // per
+    g = np.concatenate([g, np.zeros((T * per - g.shape[0], 128), np.uint16)])
+    return g.reshape(T, H), n_values
+
+
+@pytest.mark.parametrize("dt", [W.FP8_E4M3, W.MXFP8_E4M3, W.MXFP8_E5M2, W.MXFP4_E2M1], ids=lambda d: NAMES[d])
+def test_codec_every_bf16_under_a_sweep_of_scales(dt):
+    """The device conversion against the oracle codec on more than 2^24
+    values: every finite bf16 input under every exponent of the group amax,
+    codes and scales bit for bit (the 128-channel FP8 scale reaches the fp32
+    overflow of 448 / amax for subnormal amax)."""
+    x, n_values = _codec_sweep_rows()
+    assert n_values >= 1 << 24
+    T = x.shape[0]
+    idx = (np.arange(T, dtype=np.int64) % 4).reshape(T, 1)
+    ref, _, g_codes, g_scales, flags, _, _ = _run(x, idx, 4, 1, dt)
+    assert flags == 0
+    r_codes, r_scales = _host_bytes(ref, dt, T, x.shape[1])
+    bad = np.argwhere(g_codes != r_codes)
+    assert bad.size == 0, ("codes differ", bad[:5], g_codes[tuple(bad[0])], r_codes[tuple(bad[0])])
+    assert np.array_equal(g_scales, r_scales), "scales differ"
