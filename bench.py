@@ -202,6 +202,16 @@ def max_over_ranks(value, world, device=None):
     return float(t.item())
 
 
+def host_cores():
+    """Cores of this host (the oracle itself runs on one thread): what the OS
+    reports and what this process may use."""
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        usable = None
+    return {"cpu_count": os.cpu_count(), "usable": usable}
+
+
 def cpu_oracle_run(cfg_id, seed, n_tokens, reps_budget_s, min_reps=1):
     """Time the CPU oracle (single thread) on the first n_tokens tokens of the
     workload: layout + dispatch + combine, as a bounded sample."""
@@ -265,7 +275,8 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": {"workload": cfg["name"], "sample_tokens": n_tok},
             "tokens_per_s": n_tok * args.steps / dt,
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+                             "host_cores": host_cores()},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -463,6 +474,7 @@ def run_ours(args):
             times, b = cpu_oracle_run(args.workload, seed, n_tok, reps_budget_s=10.0)
             med = statistics.median(times)
             line["cpu_baseline"] = {"value": b / med / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                    "host_cores": host_cores(),
                                     "sample": "first %d of %d tokens, layout+dispatch+combine, median of %d reps"
                                               % (n_tok, T, len(times)),
                                     "tokens_per_s": n_tok / med}

@@ -15,7 +15,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libep_b200.so")
 
-# enums of include/ep.h
+# ABI version and enums of include/ep.h
+EP_ABI_VERSION = 2  # the structures below follow this version of the header
 EP_OK = 0
 EP_ERR_INVALID_ARG, EP_ERR_BAD_INDEX, EP_ERR_OVERFLOW, EP_ERR_WORKSPACE = 1, 2, 3, 4
 EP_ERR_CUDA, EP_ERR_UNSUPPORTED, EP_ERR_TIMEOUT = 5, 6, 7
@@ -49,7 +50,8 @@ class LayoutDesc(ctypes.Structure):
     _fields_ = [("num_tokens_per_expert", ctypes.c_void_p), ("expert_offsets", ctypes.c_void_p),
                 ("num_tokens_per_rank", ctypes.c_void_p), ("is_token_in_rank", ctypes.c_void_p),
                 ("slot", ctypes.c_void_p), ("token_offsets", ctypes.c_void_p), ("token_slots", ctypes.c_void_p),
-                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("num_valid_host", ctypes.c_void_p)]
 
 
 class RankLayoutDesc(ctypes.Structure):
@@ -101,6 +103,9 @@ def lib():
         L.ep_combine_ranks.argtypes = [P, i32, i64, RP, LP, KP, P, st, P]
         L.ep_dispatch_low_latency.restype = st
         L.ep_dispatch_low_latency.argtypes = [P, i32, RP, LP, i32, st, P, P, P, P, P, P]
+        if L.ep_version() != EP_ABI_VERSION:
+            raise ImportError("libep_b200.so has ABI version %d, the binding expects %d; rebuild it"
+                              % (L.ep_version(), EP_ABI_VERSION))
         _lib = L
     return _lib
 
@@ -206,9 +211,13 @@ def ep_workspace_init(workspace: torch.Tensor, stream=None) -> None:
 
 class Layout:
     """Device buffers of one layout (allocated by torch, i.e. by the caller
-    of the C ABI) plus the C descriptor pointing at them."""
+    of the C ABI) plus the C descriptor pointing at them.  With
+    report_num_valid=True a pinned host int32 is attached as num_valid_host:
+    every layout call then copies the filled-row count into it and returns
+    after the stream caught up (read it as .num_valid)."""
 
-    def __init__(self, routing: Routing, device="cuda", workspace: torch.Tensor | None = None, stream=None):
+    def __init__(self, routing: Routing, device="cuda", workspace: torch.Tensor | None = None, stream=None,
+                 report_num_valid: bool = False):
         T, E, R = routing.T, routing.E, routing.R
         i32 = dict(dtype=torch.int32, device=device)
         self.num_tokens_per_expert = torch.empty(E, **i32)
@@ -228,10 +237,19 @@ class Layout:
         elif workspace.numel() * workspace.element_size() < need:
             raise ValueError("workspace too small: %d < %d" % (workspace.numel(), need))
         self.workspace = workspace
+        self.num_valid_host = torch.zeros(1, dtype=torch.int32).pin_memory() if report_num_valid else None
         self.desc = LayoutDesc(*(None if t is None else t.data_ptr() for t in (
             self.num_tokens_per_expert, self.expert_offsets, self.num_tokens_per_rank, self.is_token_in_rank,
             self.slot, self.token_offsets, self.token_slots, self.workspace)),
-            self.workspace.numel() * self.workspace.element_size())
+            self.workspace.numel() * self.workspace.element_size(),
+            None if self.num_valid_host is None else self.num_valid_host.data_ptr())
+
+    @property
+    def num_valid(self) -> int:
+        """Filled rows reported by the last layout call (needs report_num_valid)."""
+        if self.num_valid_host is None:
+            raise ValueError("this layout was made without report_num_valid")
+        return int(self.num_valid_host[0])
 
 
 class LayoutView:
@@ -241,6 +259,7 @@ class LayoutView:
     def __init__(self, parent: Layout, t0: int, k: int):
         self.parent = parent
         self.desc = LayoutDesc.from_buffer_copy(parent.desc)
+        self.desc.num_valid_host = None  # counts are the parent's; a view never reports them
         if parent.slot is not None:
             self.desc.slot = parent.desc.slot + t0 * k * 4
         self.desc.is_token_in_rank = parent.desc.is_token_in_rank + t0 * parent.num_tokens_per_rank.numel()

@@ -1,6 +1,7 @@
 // ep_api.cu -- the C ABI declared in include/ep.h: argument checks on the
 // host, then one launcher per operation.  Nothing here allocates device
-// memory; only ep_get_device_error synchronises.
+// memory; only ep_get_device_error, and a layout call given a
+// num_valid_host pointer, synchronise.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -114,7 +115,26 @@ ep::TcRows tc_rows(const ep_routing_desc_t* r, const ep_layout_t* l, ep_buffer_m
     return rows;
 }
 
+// ep_get_layout without the host report: argument checks and the launch.
+ep_status_t get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream);
+
 } // namespace
+
+namespace ep {
+
+ep_status_t report_num_valid(const ep_routing_desc_t* routing, const ep_layout_t* layout, cudaStream_t stream)
+{
+    if (layout->num_valid_host == nullptr)
+        return EP_OK;
+    const int32_t* total = routing->routing == EP_ROUTING_TOPK ? layout->expert_offsets + routing->num_experts
+                                                               : layout->token_offsets + routing->num_tokens;
+    cudaError_t e = cudaMemcpyAsync(layout->num_valid_host, total, sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(stream);
+    return from_cuda(e);
+}
+
+} // namespace ep
 
 extern "C" {
 
@@ -136,6 +156,18 @@ ep_status_t ep_workspace_init(void* workspace, size_t bytes, ep_stream_t stream)
 ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream)
 {
     CallRange range_("ep_get_layout");
+    const ep_status_t st = get_layout(routing, layout, stream);
+    if (st != EP_OK)
+        return st;
+    return ep::report_num_valid(routing, layout, reinterpret_cast<cudaStream_t>(stream));
+}
+
+} // extern "C"
+
+namespace {
+
+ep_status_t get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream)
+{
     ep_status_t st = check_routing(routing);
     if (st != EP_OK)
         return st;
@@ -189,8 +221,6 @@ ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* l
     return from_cuda(ep::launch_ec_layout(a, s));
 }
 
-namespace {
-
 // Host-side checks of a token-choice dispatch call (ep_dispatch and the
 // dispatch half of ep_dispatch_low_latency).
 ep_status_t check_dispatch_args(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
@@ -234,6 +264,8 @@ ep_status_t check_dispatch_args(const void* x, int32_t hidden, const ep_routing_
 }
 
 } // namespace
+
+extern "C" {
 
 ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing, const ep_layout_t* layout,
                         ep_buffer_mode_t mode, int32_t max_tokens_per_expert, int64_t num_recv_rows,
@@ -312,13 +344,16 @@ ep_status_t ep_dispatch_low_latency(const void* x, int32_t hidden, const ep_rout
                                layout->expert_offsets,
                                layout->num_tokens_per_rank,
                                ep::error_word(layout->workspace)};
-        return from_cuda(ep::launch_ll_dispatch(a, s));
+        st = from_cuda(ep::launch_ll_dispatch(a, s));
+    } else {
+        st = get_layout(routing, layout, stream);
+        if (st == EP_OK)
+            st = ep_dispatch(x, hidden, routing, layout, EP_LAYOUT_PADDED, max_tokens_per_expert, rows, out_dtype,
+                             topk_weights, recv_x, recv_scales, recv_src, recv_weights, stream);
     }
-    st = ep_get_layout(routing, layout, stream);
     if (st != EP_OK)
         return st;
-    return ep_dispatch(x, hidden, routing, layout, EP_LAYOUT_PADDED, max_tokens_per_expert, rows, out_dtype,
-                       topk_weights, recv_x, recv_scales, recv_src, recv_weights, stream);
+    return ep::report_num_valid(routing, layout, s);
 }
 
 ep_status_t ep_combine(const void* y, int32_t hidden, int64_t num_y_rows, const ep_routing_desc_t* routing,

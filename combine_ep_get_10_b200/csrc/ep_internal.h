@@ -20,6 +20,10 @@ inline uint32_t* error_word(void* workspace)
     return static_cast<uint32_t*>(workspace);
 }
 
+// When layout->num_valid_host is set: copy the routing's filled-row count
+// (expert_offsets[E] or token_offsets[T]) to it and synchronise the stream.
+ep_status_t report_num_valid(const ep_routing_desc_t* routing, const ep_layout_t* layout, cudaStream_t stream);
+
 // ------------------------------------------------------------------ layout
 struct TcLayoutLaunch {
     const int64_t* topk_idx;

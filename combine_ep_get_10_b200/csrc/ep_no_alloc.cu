@@ -2,15 +2,14 @@
 // callers that cannot allocate device memory.
 //
 // Some callers cannot call cudaMalloc (or any allocator) at the point where
-// they need a layout: a host that captures the MoE step into a CUDA graph
-// (cudaMalloc is not allowed while a stream is being captured), a plugin
-// inside an inference server or framework that only hands the plugin its
-// input and output tensors and owns every other byte of device memory, or a
-// latency-critical decode loop where an allocation could synchronise the
-// device.  ep_get_layout needs a caller-provided workspace (the expert-choice
-// layout keeps per-token counters and an unordered slot list there); this
-// variant takes its scratch from a fixed-size array in the library's own
-// device memory instead.
+// they need a layout: a plugin inside an inference server or framework that
+// only hands the plugin its input and output tensors and owns every other
+// byte of device memory, or a latency-critical decode loop where an
+// allocation could synchronise the device.  ep_get_layout needs a
+// caller-provided workspace (the expert-choice layout keeps per-token
+// counters and an unordered slot list there); this variant takes its
+// scratch from a fixed-size array in the library's own device memory
+// instead.
 //
 // The array is a file-scope __device__ object: every GPU that loads the
 // library holds kStaticWorkspaceBytes of it until the process exits.  Its
@@ -18,7 +17,9 @@
 // device current); host code must never pass the symbol itself to a kernel.
 // All calls share the one array, so calls whose kernels overlap on the GPU
 // (two streams, or two host threads) race on it and must be serialised by
-// the caller.
+// the caller.  Every call zeroes the array's 256-byte header first (the
+// error word and the grid barrier's arrival and generation words), so a call
+// whose barrier wait ran out leaves nothing behind for the next one.
 #include <cstdint>
 #include <mutex>
 
@@ -102,10 +103,13 @@ ep_status_t ep_get_layout_no_alloc(const ep_routing_desc_t* routing, const ep_la
     if (ws == nullptr)
         return EP_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // the error word starts every call at zero: in the caller's word when one
-    // is given, else in the array's header (where nobody reads it)
+    // the header (error word, grid-barrier words) starts every call at zero,
+    // and so does the caller's error word when one is given (the kernels
+    // report there instead of in the header, where nobody reads it)
+    if (cudaMemsetAsync(ws, 0, ep::kWorkspaceHeaderBytes, s) != cudaSuccess)
+        return EP_ERR_CUDA;
     uint32_t* err = device_error_flags != nullptr ? device_error_flags : ep::error_word(ws);
-    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), s) != cudaSuccess)
+    if (device_error_flags != nullptr && cudaMemsetAsync(err, 0, sizeof(uint32_t), s) != cudaSuccess)
         return EP_ERR_CUDA;
 
     if (topk) {
@@ -121,7 +125,9 @@ ep_status_t ep_get_layout_no_alloc(const ep_routing_desc_t* routing, const ep_la
                              layout->slot,
                              err,
                              ws};
-        return ep::launch_tc_layout(a, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+        if (ep::launch_tc_layout(a, s) != cudaSuccess)
+            return EP_ERR_CUDA;
+        return ep::report_num_valid(routing, layout, s);
     }
     ep::EcLayoutLaunch a{routing->token_indices,
                          T,
@@ -135,7 +141,9 @@ ep_status_t ep_get_layout_no_alloc(const ep_routing_desc_t* routing, const ep_la
                          layout->token_slots,
                          ws,
                          err};
-    return ep::launch_ec_layout(a, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    if (ep::launch_ec_layout(a, s) != cudaSuccess)
+        return EP_ERR_CUDA;
+    return ep::report_num_valid(routing, layout, s);
 }
 
 } // extern "C"

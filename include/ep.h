@@ -4,8 +4,9 @@
  * C ABI of libep_b200.so.  All tensors are plain device pointers, row-major
  * and densely packed; all memory belongs to the caller.  No entry point
  * allocates or frees device memory, and none synchronises the host except
- * ep_get_device_error().  Every call is asynchronous on `stream`
- * (a cudaStream_t; NULL = the legacy default stream).
+ * ep_get_device_error() and a layout call given a num_valid_host pointer.
+ * Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ * default stream).
  *
  * The operations follow these pages (title, section):
  *   [README] "DeepEP-Ascend" README (sgl-kernel-npu python/deep_ep),
@@ -41,7 +42,7 @@
 extern "C" {
 #endif
 
-#define EP_ABI_VERSION 1
+#define EP_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define EP_API __attribute__((visibility("default")))
@@ -146,7 +147,17 @@ typedef struct {
  *                         layout's per-token arrays.  Zero it once
  *                         (ep_workspace_init) before first use; calls leave
  *                         it reusable.  One workspace per stream: calls that
- *                         share one must not overlap on the GPU. */
+ *                         share one must not overlap on the GPU.
+ *   num_valid_host        optional HOST pointer to one int32 (pinned or
+ *                         pageable), NULL = not used.  When set, the layout
+ *                         call copies the number of rows the routing fills
+ *                         (TOPK: expert_offsets[E], the routed pairs; EC:
+ *                         token_offsets[T], the filled slots) into it and
+ *                         synchronises `stream` before returning, so the
+ *                         caller can size its receive buffer without a read
+ *                         of its own.  This is the only synchronisation a
+ *                         layout call ever makes; leave it NULL while the
+ *                         stream is being captured. */
 typedef struct {
     int32_t* num_tokens_per_expert;
     int32_t* expert_offsets;
@@ -157,6 +168,7 @@ typedef struct {
     int32_t* token_slots;
     void* workspace;
     size_t workspace_bytes;
+    int32_t* num_valid_host;
 } ep_layout_t;
 
 /* Bytes of workspace the layout of this routing needs (>= 256; the first
@@ -172,7 +184,10 @@ EP_API ep_status_t ep_workspace_init(void* workspace, size_t bytes, ep_stream_t 
  * is_token_in_rank and slot.  EXPERT_CHOICE ([EC] Solution 1) writes
  * num_tokens_per_expert, num_tokens_per_rank, is_token_in_rank,
  * token_offsets and token_slots.  Deterministic: the same routing gives the
- * same bytes on every call. */
+ * same bytes on every call.  With layout->num_valid_host set, the number of
+ * filled rows is also copied to the host and the call returns after the
+ * stream has caught up (the [README] dispatch returns the received-token
+ * count to the host in the same way). */
 EP_API ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream);
 
 /* Token-choice dispatch ([README] API Overview: dispatch; low_latency_dispatch
@@ -294,10 +309,10 @@ EP_API ep_status_t ep_combine_ranks(const void* y, int32_t hidden, int64_t num_y
  * have no counterpart: this is a deployment variant of the layout call.
  *
  * Who needs it: code that must not call cudaMalloc (or any allocator) when
- * it builds a layout -- a host capturing the MoE step into a CUDA graph
- * (allocation is not allowed during stream capture), a plugin inside an
- * inference server or framework that is handed only its input and output
- * tensors, or a decode loop where an allocation could synchronise the device.
+ * it builds a layout -- a plugin inside an inference server or framework that
+ * is handed only its input and output tensors while the host program owns
+ * every other byte of device memory, or a decode loop where an allocation
+ * could synchronise the device and stall the step.
  *
  * It computes exactly what ep_get_layout computes, writing the same outputs
  * in `layout`, but ignores layout->workspace / workspace_bytes: its scratch is
@@ -310,11 +325,15 @@ EP_API ep_status_t ep_combine_ranks(const void* y, int32_t hidden, int64_t num_y
  *   device_error_flags  optional device pointer to one uint32: zeroed at the
  *                       start of the call, then receives the EP_DEVERR_* bits
  *                       the layout kernels raise (NULL: not reported).
+ * layout->num_valid_host is honoured as by ep_get_layout.
  * The first call on a device looks up the array's device address (with that
  * device current), so make one call per device before any stream capture.
  * All calls share the array and it keeps the last call's contents: calls that
  * overlap on the GPU (other streams, other host threads) race on it and must
- * be serialised by the caller. */
+ * be serialised by the caller.  Every call first zeroes the array's 256-byte
+ * header (error word and grid-barrier words) on `stream`, so a call that
+ * follows one whose wait ran out (EP_DEVERR_TIMEOUT) starts clean: there is
+ * nothing for the caller to reset. */
 #define EP_STATIC_WORKSPACE_BYTES ((size_t)4 << 20)
 EP_API ep_status_t ep_get_layout_no_alloc(const ep_routing_desc_t* routing, const ep_layout_t* layout,
                                           uint32_t* device_error_flags, ep_stream_t stream);
@@ -322,7 +341,8 @@ EP_API ep_status_t ep_get_layout_no_alloc(const ep_routing_desc_t* routing, cons
 /* Synchronise `stream`, read the device error word of layout->workspace into
  * *flags (EP_DEVERR_* bits), clear it if `clear`, and return EP_OK when it is
  * zero, else the status of the lowest set bit (BAD_INDEX, OVERFLOW, TIMEOUT).
- * After EP_ERR_TIMEOUT re-run ep_workspace_init on the workspace. */
+ * After EP_ERR_TIMEOUT re-run ep_workspace_init on the workspace (the
+ * grid-barrier words may hold a partial count). */
 EP_API ep_status_t ep_get_device_error(const ep_layout_t* layout, uint32_t* flags, int clear, ep_stream_t stream);
 
 EP_API const char* ep_status_string(ep_status_t status);

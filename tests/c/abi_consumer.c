@@ -113,6 +113,12 @@ static int gpu_mode(void)
     l.workspace = d_ws;
     l.workspace_bytes = ws;
     CHECK(ep_get_layout(&r, &l, NULL) == EP_OK, "layout");
+    /* the same layout again, reporting the routed-pair count to the host */
+    int32_t num_valid = -1;
+    l.num_valid_host = &num_valid;
+    CHECK(ep_get_layout(&r, &l, NULL) == EP_OK, "layout with num_valid_host");
+    CHECK(num_valid == 7, "num_valid_host holds the routed pairs");
+    l.num_valid_host = NULL;
     CHECK(ep_dispatch(d_x, H, &r, &l, EP_LAYOUT_COMPACT, 0, T * K, EP_BF16, NULL, d_recv, NULL, NULL, NULL, NULL) ==
               EP_OK,
           "dispatch");

@@ -43,7 +43,10 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert B.ep_version() == 1
+    assert B.ep_version() == B.EP_ABI_VERSION == 2
+    # ep_layout_t: nine pointer-sized fields, then num_valid_host (version 2)
+    assert ctypes.sizeof(B.LayoutDesc) == 10 * 8
+    assert B.LayoutDesc.num_valid_host.offset == 9 * 8
     for s in range(8):
         assert B.ep_status_string(s)
     assert B.ep_status_string(99) == "unknown status"
@@ -171,6 +174,7 @@ def test_binding_constants_match_the_header():
     here = os.path.dirname(os.path.abspath(__file__))
     text = open(os.path.join(here, "..", "include", "ep.h")).read()
     values = {m.group(1): int(m.group(2), 0) for m in re.finditer(r"\b(EP_[A-Z0-9_]+) = (\d+)\b", text)}
+    values["EP_ABI_VERSION"] = int(re.search(r"#define EP_ABI_VERSION (\d+)", text).group(1))
     values.update({m.group(1): int(m.group(2), 16) for m in
                    re.finditer(r"#define (EP_DEVERR_[A-Z_]+) 0x([0-9a-fA-F]+)u", text)})
     assert len(values) >= 22, sorted(values)

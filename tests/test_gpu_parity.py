@@ -484,9 +484,9 @@ def test_long_sequence_in_rounds():
     assert len(rounds) == 4
     for t0, t1 in rounds:
         r = routing.tokens(t0, t1)
-        lay = B.Layout(r)
-        B.ep_get_layout(r, lay)
-        n = int(lay.expert_offsets[-1].item())
+        lay = B.Layout(r, report_num_valid=True)
+        B.ep_get_layout(r, lay)  # returns with the round's routed-pair count on the host
+        n = lay.num_valid
         assert n == int((idx[t0:t1] >= 0).sum()) <= P * K
         B.ep_dispatch(xd[t0:t1], r, lay, recv, num_recv_rows=n)
         B.ep_combine(recv, r, lay, wd[t0:t1], out[t0:t1], num_y_rows=n)
@@ -524,3 +524,41 @@ def test_combine_into_pinned_host_memory():
     torch.cuda.synchronize()
     assert B.ep_get_device_error(lay) == 0
     assert torch.equal(out_d.cpu().view(torch.int16), out_h.view(torch.int16))
+
+
+def test_num_valid_host_reports_the_filled_rows():
+    """layout->num_valid_host: the layout call copies the filled-row count to
+    the host and returns after the stream caught up; the value equals the
+    oracle's expert_offsets[E] (token choice) or token_offsets[T] (expert
+    choice), for the plain, the fused low-latency and the no-alloc layouts."""
+    for wl in (2, 5):
+        inp = inputs(wl, T=3000)
+        c = inp["cfg"]
+        idx = inp["topk_idx"]
+        ref = oracle.tc_layout(idx, c["E"], c["R"])
+        routing = B.Routing.topk(to_dev(idx), c["E"], c["R"])
+        lay = B.Layout(routing, report_num_valid=True)
+        lay.num_valid_host[0] = -5
+        B.ep_get_layout(routing, lay)
+        assert lay.num_valid == int(ref["expert_offsets"][-1])
+        lay.num_valid_host[0] = -5
+        B.ep_get_layout_no_alloc(routing, lay)
+        assert lay.num_valid == int(ref["expert_offsets"][-1])
+    inp = inputs(3)
+    c = inp["cfg"]
+    idx, mt = inp["topk_idx"], c["max_tokens"]
+    routing = B.Routing.topk(to_dev(idx), c["E"], c["R"])
+    lay = B.Layout(routing, report_num_valid=True)
+    q = torch.empty((c["E"] * mt, c["H"]), dtype=torch.uint8, device="cuda")
+    sc = torch.empty((c["E"] * mt, c["H"] // 128), dtype=torch.float32, device="cuda")
+    B.ep_dispatch_low_latency(to_dev(inp["x"], bf16=True), routing, lay, q, max_tokens_per_expert=mt,
+                              recv_scales=sc)
+    assert lay.num_valid == int(oracle.tc_layout(idx, c["E"], c["R"])["expert_offsets"][-1])
+    inp = inputs(4)
+    c = inp["cfg"]
+    ti = inp["token_indices"]
+    routing = B.Routing.expert_choice(to_dev(ti), c["T"], 1)
+    lay = B.Layout(routing, report_num_valid=True)
+    B.ep_get_layout(routing, lay)
+    assert lay.num_valid == int(oracle.ec_layout(ti, c["T"], 1)["token_offsets"][-1])
+    assert B.ep_get_device_error(lay) == 0

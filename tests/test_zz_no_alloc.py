@@ -1,6 +1,6 @@
 """ep_get_layout_no_alloc: the layout entry point for callers that cannot
-allocate device memory (graph capture, plugins handed only their tensors,
-latency-critical loops).  It must write exactly what ep_get_layout writes;
+allocate device memory (plugins handed only their tensors, latency-critical
+decode loops where an allocation could stall the step).  It must write exactly what ep_get_layout writes;
 here both are called through the C ABI on the same routing and compared
 (integer outputs: bit for bit), twice in a row so that a second call over the
 shared scratch array left by the first is covered too.
@@ -81,6 +81,16 @@ def test_no_alloc_matches_layout_expert_choice():
     rng = np.random.Generator(np.random.PCG64(4))
     ti = W.random_token_indices(rng, 40, 16, 8, p_neg=0.2, p_bad=0.05)
     _compare(B.Routing.expert_choice(_dev(ti), 40, 4))
+
+
+def test_no_alloc_matches_layout_expert_choice_past_the_cluster_limits():
+    # 20000 tokens (more than one thread-block cluster handles): the
+    # multi-kernel expert-choice layout, whose per-token counters and
+    # unordered slot list live in the scratch array (256 + 4 (2T + EC) bytes,
+    # about 226 KB here, inside the 4 MiB)
+    rng = np.random.Generator(np.random.PCG64(5))
+    ti = W.random_token_indices(rng, 20000, 64, 256, p_neg=0.1, p_bad=0.01)
+    _compare(B.Routing.expert_choice(_dev(ti), 20000, 8))
 
 
 def test_no_alloc_rejects_problems_beyond_the_fixed_scratch():
