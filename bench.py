@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--e2e-chunks", type=int, default=8, help="token chunks of the pipelined end-to-end step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the per-op timings of the decode, expert-choice and skewed workloads")
+    ap.add_argument("--other-reps", type=int, default=30)
     ap.add_argument("--print-digests", action="store_true", help="print kernel source digests and exit")
     ap.add_argument("--workloads", action="store_true",
                     help="time every op on all five workloads (one JSON line each) instead of the step")
@@ -433,6 +436,13 @@ def run_ours(args):
     if B.ep_get_device_error(lay) != 0:
         raise RuntimeError("device error flagged during the end-to-end steps")
 
+    # the other workloads' ops, timed in this process with clocks sampled
+    other, other_clocks = None, None
+    if rank == 0 and not args.no_other_workloads:
+        with ClockSampler(local, uuid) as clocks2:
+            other = time_other_workloads(dev, flush, args.other_reps)
+        other_clocks = clocks2.summary()
+
     if rank == 0:
         peak, peak_kind = measured_peak()
         mean = lambda a: float(sum(a) / len(a))  # noqa: E731
@@ -469,6 +479,11 @@ def run_ours(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "clocks": clocks.summary(),
         }
+        if other is not None:
+            line["other_workloads"] = {"per_op": other, "reps": args.other_reps,
+                                       "timing": "CUDA events around each op alone, L2 flushed (256 MiB memset) "
+                                                 "before each repetition, median; frac against the same peak",
+                                       "clocks": other_clocks}
         if world == 1 and not args.no_cpu_baseline:
             n_tok = 1024
             times, b = cpu_oracle_run(args.workload, seed, n_tok, reps_budget_s=10.0)
@@ -483,6 +498,96 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def time_other_workloads(dev, flush, reps):
+    """Per-op event timings of the decode (3), expert-choice (4) and skewed
+    (5) workloads, each op alone after an L2 flush, median of `reps`; returned
+    as {workload: {op: {"us", "gbs", "frac", "bytes"}}} for the bench line."""
+    import torch
+
+    from combine_ep_get_10_b200 import binding as B
+    from combine_ep_get_10_b200 import workloads as W
+
+    peak, _ = measured_peak()
+
+    def timeit(fn):
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize(dev)
+            if i >= 3:
+                ts.append(a.elapsed_time(b) * 1e3)
+        return statistics.median(ts)
+
+    def rec(us, nbytes):
+        return {"us": round(us, 2), "bytes": int(nbytes), "gbs": round(nbytes / us / 1e3, 1),
+                "frac": round(nbytes / us / 1e3 / peak, 3)}
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    res = {}
+    for wl in (3, 4, 5):
+        inp = W.make_inputs(wl)
+        cfg = inp["cfg"]
+        T, H, E, R = cfg["T"], cfg["H"], cfg["E"], cfg["R"]
+        x = bf(inp["x"])
+        ops = {}
+        if cfg["routing"] == "topk":
+            K = cfg["K"]
+            n_valid = int((inp["topk_idx"] >= 0).sum())
+            idx = torch.from_numpy(inp["topk_idx"]).to(dev)
+            w = torch.from_numpy(inp["topk_weights"]).to(dev)
+            rt = B.Routing.topk(idx, E, R)
+            lay = B.Layout(rt, device=dev)
+            ops["layout"] = rec(timeit(lambda: B.ep_get_layout(rt, lay)), T * K * 12 + T * R + E * 8 + R * 4)
+            mode, mt = cfg["mode"], cfg["max_tokens"]
+            rows = E * mt if mode == W.PADDED else T * K
+            meta = T * K * 12 + E * 4
+            y = torch.zeros((rows, H), dtype=torch.bfloat16, device=dev)
+            if cfg["dispatch_dtype"] == W.FP8_E4M3:
+                q = torch.empty((rows, H), dtype=torch.uint8, device=dev)
+                sc = torch.empty((rows, H // 128), dtype=torch.float32, device=dev)
+                ops["dispatch_fp8"] = rec(timeit(lambda: B.ep_dispatch(x, rt, lay, q, mode=mode, max_tokens_per_expert=mt,
+                                                                      recv_scales=sc)),
+                                          T * H * 2 + n_valid * (H + H // 128 * 4) + meta)
+                ops["low_latency_layout_dispatch_fp8"] = rec(
+                    timeit(lambda: B.ep_dispatch_low_latency(x, rt, lay, q, max_tokens_per_expert=mt, recv_scales=sc)),
+                    T * K * 12 + T * R + E * 8 + R * 4 + T * H * 2 + n_valid * (H + H // 128 * 4))
+                del q, sc
+            else:
+                ops["dispatch"] = rec(timeit(lambda: B.ep_dispatch(x, rt, lay, y, mode=mode, max_tokens_per_expert=mt)),
+                                      T * H * 2 + n_valid * H * 2 + meta)
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+            ops["combine"] = rec(timeit(lambda: B.ep_combine(y, rt, lay, w, out, mode=mode, max_tokens_per_expert=mt)),
+                                 n_valid * H * 2 + T * H * 2 + T * K * 16 + E * 4)
+        else:
+            C = cfg["C"]
+            ti_np = inp["token_indices"]
+            S = E * C
+            uniq = len(np.unique(ti_np[ti_np >= 0]))
+            ti = torch.from_numpy(ti_np).to(dev)
+            ew = torch.from_numpy(inp["expert_weights"]).to(dev)
+            rt = B.Routing.expert_choice(ti, T, R)
+            lay = B.Layout(rt, device=dev)
+            ops["ec_layout"] = rec(timeit(lambda: B.ep_get_layout(rt, lay)), S * 4 + (T + 1) * 4 + S * 4 + T * R + E * 4 + R * 4)
+            y = torch.empty((S, H), dtype=torch.bfloat16, device=dev)
+            ops["ec_dispatch"] = rec(timeit(lambda: B.ep_dispatch_expert_choice(x, rt, lay, y)), uniq * H * 2 + S * H * 2 + S * 4)
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+            ops["ec_combine"] = rec(timeit(lambda: B.ep_combine_expert_choice(y, rt, lay, ew, out)),
+                                    S * H * 2 + T * H * 2 + S * 8 + (T + 1) * 4)
+        if B.ep_get_device_error(lay) != 0:
+            raise RuntimeError("device error flagged on workload %d" % wl)
+        res[cfg["name"]] = ops
+        del x, y, out, lay
+        torch.cuda.empty_cache()
+    return res
 
 
 # quantised dispatch formats: (name, dtype code, code bytes per row, scale bytes per row)

@@ -34,6 +34,21 @@ __device__ __forceinline__ void flag_error(uint32_t* err, uint32_t bits)
         atomicOr(err, bits);
 }
 
+// ------------------------------------------- programmatic dependent launch
+// A layout kernel lets the next kernel of the stream start early (when that
+// one is launched with programmatic stream serialisation); the dispatch
+// kernels issue their input-row loads first and wait for the layout's
+// results here before reading them.  Without such a launch both are no-ops.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
 {
@@ -49,6 +64,14 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
                  : "memory");
+}
+
+// One arrival (no transaction bytes) on `bar`; release semantics at CTA
+// scope, so this thread's earlier shared-memory writes are visible to a
+// thread whose wait on the phase returns.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
@@ -126,6 +149,18 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p)
         : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
         : "l"(p));
     return r;
+}
+
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p)
+{
+    uint2 r;
+    asm("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_cs_v2(void* p, uint2 v)
+{
+    asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
 
 __device__ __forceinline__ void st_cs_v4(void* p, uint4 v)

@@ -34,6 +34,32 @@ namespace {
 
 constexpr int64_t kChunkTarget = EP_DISPATCH_CHUNK; // bytes per bulk-copy item
 
+// Dispatch kernels are launched with programmatic stream serialisation: when
+// the kernel before them is a layout (which lets its dependents start at
+// once), their CTAs start while it runs, load their source rows, and wait for
+// the layout's results (griddepcontrol.wait) before reading them.
+#ifndef EP_DISPATCH_PDL
+#define EP_DISPATCH_PDL 1
+#endif
+
+// <<<grid, block, smem, stream>>> with programmatic stream serialisation.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = EP_DISPATCH_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 struct RowMap {
     const int64_t* topk_idx;
     const int32_t* slot;
@@ -135,8 +161,10 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
     if (kExpertChoice) {
         const int t = __ldg(a.token_indices + r);
         if (t < 0 || t >= a.T) {
-            if (lane == 0 && c == 0 && t != -1)
+            if (lane == 0 && c == 0 && t != -1) {
+                pdl_wait(); // the error word is shared with the layout before
                 flag_error(a.err, EP_DEVERR_BAD_INDEX);
+            }
             return;
         }
         src_row = t;
@@ -150,6 +178,7 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
         mbar_arrive_expect_tx(&bar, bytes);
         bulk_load_g2s(buf, a.src + src_row * a.row_bytes + off, bytes, &bar);
     }
+    pdl_wait(); // the layout's results (slot, offsets, rank rows) are final from here on
     // destination rows of the first 32 pairs while the load is in flight
     int64_t dst_row = -1;
     if constexpr (kSrc == kSrcEc) {
@@ -301,15 +330,30 @@ __device__ __forceinline__ uint2 encode8(uint4 r, float mul)
 // issued by different threads.  Rows whose byte size is not a multiple of 16
 // are written with 8-byte stores instead.  Registers stay low, so many CTAs
 // (and their row loads) are resident per SM.
-//   shared memory: x row [2H] | codes [code_row] | scales [scale_row -> 16] | rows [K]
+// Up to kInPlaceIters vectors per thread (rows of up to 8192 channels) the
+// codes overwrite the staged row: every thread first takes its vectors into
+// registers, the CTA meets at a barrier, and the codes are written over the
+// bf16 row, so a token CTA needs 2H bytes of row buffer instead of 3H (2.5H
+// for FP4) and a third more tokens fit on an SM.
+//   shared memory: x row [2H] | codes [code_row] (not in place) | scales [scale_row -> 16] | rows [K]
 // Shared-memory bytes of one token CTA: x row | codes | scales | rows [K]
 // (| fused layout: expert -> k mask [E], histogram [E], per-token rank bits
 // [T], small arrays [4 x 32]).
+constexpr int kInPlaceIters = 8;
+#ifndef EP_QUANT_IN_PLACE
+#define EP_QUANT_IN_PLACE 0
+#endif
+
+__host__ __device__ inline bool quant_in_place(int fmt, int H)
+{
+    return EP_QUANT_IN_PLACE && fmt != kQBf16 && H / 8 <= kInPlaceIters * kQuantThreads;
+}
+
 __host__ __device__ inline size_t quant_smem_bytes(int fmt, int H, int K, int E, int T, bool fused)
 {
     const size_t nvec = static_cast<size_t>(H) / 8;
     const bool mx = fmt == kQMxE4m3 || fmt == kQMxE5m2 || fmt == kQMxE2m1;
-    const size_t code_row = fmt == kQBf16 ? 0 : nvec * (fmt == kQMxE2m1 ? 4 : 8);
+    const size_t code_row = fmt == kQBf16 || quant_in_place(fmt, H) ? 0 : nvec * (fmt == kQMxE2m1 ? 4 : 8);
     const size_t scale_row =
         fmt == kQBf16 ? 0 : (mx ? nvec / 4 : ((fmt == kQInt8Tok || fmt == kQFp8Tok) ? 4 : nvec / 16 * 4));
     size_t n = nvec * 16 + code_row + ((scale_row + 15) & ~static_cast<size_t>(15)) + sizeof(int64_t) * K;
@@ -446,9 +490,10 @@ __device__ __forceinline__ void fused_layout(const QuantArgs& a, int64_t t, int6
     }
 }
 
-template <int kFmt, bool kFused>
+template <int kFmt, bool kFused, bool kInPlace>
 __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs a)
 {
+    static_assert(!(kInPlace && kFmt == kQBf16), "the bf16 copy encodes nothing");
     constexpr bool kMx = kFmt == kQMxE4m3 || kFmt == kQMxE5m2 || kFmt == kQMxE2m1;
     constexpr bool kPerToken = kFmt == kQInt8Tok || kFmt == kQFp8Tok;
     constexpr bool kCopy = kFmt == kQBf16;
@@ -464,8 +509,8 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
     const int code_row = kCopy ? row_bytes : nvec * kCodeBytes;
     const int scale_row = kCopy ? 0 : (kMx ? nvec / 4 : (kPerToken ? 4 : nvec / 16 * 4));
     uint8_t* s_x = qsmem;
-    uint8_t* s_codes = kCopy ? s_x : qsmem + row_bytes;
-    uint8_t* s_scales = qsmem + row_bytes + (kCopy ? 0 : code_row);
+    uint8_t* s_codes = kCopy || kInPlace ? s_x : qsmem + row_bytes;
+    uint8_t* s_scales = qsmem + row_bytes + (kCopy || kInPlace ? 0 : code_row);
     int64_t* rows = reinterpret_cast<int64_t*>(s_scales + ((scale_row + 15) & ~15));
 
     if (tid == 0) {
@@ -475,6 +520,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
         bulk_load_g2s(s_x, reinterpret_cast<const uint8_t*>(a.x) + t * static_cast<int64_t>(row_bytes),
                       static_cast<uint32_t>(row_bytes), &bar);
     }
+    pdl_wait(); // the layout's results are final from here on
     uint32_t errbits = 0;
     if constexpr (kFused) {
         fused_layout(a, t, rows, reinterpret_cast<uint32_t*>(rows + a.map.K), errbits);
@@ -496,11 +542,29 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
     if (!mbar_wait_bounded(&bar, 0, a.err))
         return;
 
+    // in place: this thread's vectors in registers, then a barrier, so that
+    // no code is written over a vector another thread has yet to read
+    uint4 held[kInPlace ? kInPlaceIters : 1];
+    if constexpr (kInPlace) {
+#pragma unroll
+        for (int i = 0; i < kInPlaceIters; ++i) {
+            const int v = i * kQuantThreads + tid;
+            held[i] = v < nvec ? *reinterpret_cast<const uint4*>(s_x + v * 16) : make_uint4(0, 0, 0, 0);
+        }
+        __syncthreads();
+    }
+
     float tok_mul = 0.0f;
     if constexpr (kPerToken) {
         float amax = 0.0f;
-        for (int v = tid; v < nvec; v += kQuantThreads)
-            amax = fmaxf(amax, amax8(*reinterpret_cast<const uint4*>(s_x + v * 16)));
+        if constexpr (kInPlace) {
+#pragma unroll
+            for (int i = 0; i < kInPlaceIters; ++i)
+                amax = fmaxf(amax, amax8(held[i])); // zero vectors past the row leave the max alone
+        } else {
+            for (int v = tid; v < nvec; v += kQuantThreads)
+                amax = fmaxf(amax, amax8(*reinterpret_cast<const uint4*>(s_x + v * 16)));
+        }
 #pragma unroll
         for (int d = 16; d >= 1; d >>= 1)
             amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
@@ -521,11 +585,11 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
             *reinterpret_cast<float*>(s_scales) = scale;
     }
 
-    // uniform trip count: every lane takes part in the group shuffles
-    for (int base = 0; !kCopy && base < nvec; base += kQuantThreads) {
+    // one vector per thread and step, uniform trip count: every lane takes
+    // part in the group shuffles
+    auto encode_step = [&](int base, uint4 raw) {
         const int v = base + tid;
         const bool active = v < nvec; // a scale group is all-in or all-out
-        const uint4 raw = active ? *reinterpret_cast<const uint4*>(s_x + v * 16) : make_uint4(0, 0, 0, 0);
         float mul = tok_mul;
         if constexpr (!kPerToken) {
             float amax = amax8(raw);
@@ -559,6 +623,19 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
                 sts_v2(s_codes + v * 8, q);
             else
                 reinterpret_cast<uint32_t*>(s_codes)[v] = q.x;
+        }
+    };
+    if constexpr (kInPlace) {
+#pragma unroll
+        for (int i = 0; i < kInPlaceIters; ++i) {
+            if (i * kQuantThreads >= nvec)
+                break; // CTA-uniform
+            encode_step(i * kQuantThreads, held[i]);
+        }
+    } else if constexpr (!kCopy) {
+        for (int base = 0; base < nvec; base += kQuantThreads) {
+            const int v = base + tid;
+            encode_step(base, v < nvec ? *reinterpret_cast<const uint4*>(s_x + v * 16) : make_uint4(0, 0, 0, 0));
         }
     }
     fence_proxy_async_shared();
@@ -615,14 +692,15 @@ template <int kFmt, bool kFused>
 cudaError_t launch_quant(const QuantArgs& a, int32_t T, int32_t K, cudaStream_t stream)
 {
     const size_t smem = quant_smem_bytes(kFmt, a.H, K, a.map.E, kFused ? T : 0, kFused);
+    constexpr bool kCanInPlace = kFmt != kQBf16;
+    auto kernel = kCanInPlace && quant_in_place(kFmt, a.H) ? quant_dispatch_kernel<kFmt, kFused, kCanInPlace>
+                                                           : quant_dispatch_kernel<kFmt, kFused, false>;
     if (smem > 48 * 1024) {
-        cudaError_t st = cudaFuncSetAttribute(quant_dispatch_kernel<kFmt, kFused>,
-                                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        cudaError_t st = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (st != cudaSuccess)
             return st;
     }
-    quant_dispatch_kernel<kFmt, kFused><<<T, kQuantThreads, smem, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kernel, static_cast<unsigned>(T), kQuantThreads, smem, stream, a);
 }
 
 template <bool kFused>
@@ -658,8 +736,7 @@ cudaError_t launch_bulk(BulkArgs k, int64_t items, cudaStream_t stream)
     for (int64_t base = 0; base < items; base += kMaxGrid) {
         k.item_base = base;
         const unsigned n = static_cast<unsigned>(std::min(kMaxGrid, items - base));
-        bulk_dispatch_kernel<kSrc><<<n, 32, static_cast<size_t>(k.chunk_bytes), stream>>>(k);
-        cudaError_t st = cudaGetLastError();
+        cudaError_t st = launch_pdl(bulk_dispatch_kernel<kSrc>, n, 32, static_cast<size_t>(k.chunk_bytes), stream, k);
         if (st != cudaSuccess)
             return st;
     }

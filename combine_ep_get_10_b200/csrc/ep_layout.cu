@@ -125,6 +125,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& 
 
 __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(TcArgs a)
 {
+    pdl_launch_dependents(); // a dispatch launched after this may load its rows now
     cg::cluster_group cluster = cg::this_cluster();
     const int cs = static_cast<int>(cluster.num_blocks());
     const int b = static_cast<int>(cluster.block_rank());
@@ -402,6 +403,7 @@ __device__ __forceinline__ bool grid_sync(GridBar bar, uint32_t nblocks, uint32_
 __global__ void __launch_bounds__(kGridThreads) tc_layout_grid_kernel(TcArgs a, int32_t* tile_counts,
                                                                       int32_t* tile_ranks, GridBar bar)
 {
+    pdl_launch_dependents(); // a dispatch launched after this may load its rows now
     const int G = static_cast<int>(gridDim.x);
     const int b = static_cast<int>(blockIdx.x);
     extern __shared__ __align__(16) int32_t smem[];
@@ -783,6 +785,7 @@ size_t ec_cluster_smem_bytes(int64_t T, int64_t spc, int64_t E)
 
 __global__ void __launch_bounds__(kEcClusterThreads, 1) ec_layout_cluster_kernel(EcClusterArgs a, int32_t spc)
 {
+    pdl_launch_dependents(); // a dispatch launched after this may load its rows now
     cg::cluster_group cluster = cg::this_cluster();
     const int cs = static_cast<int>(cluster.num_blocks());
     const int b = static_cast<int>(cluster.block_rank());

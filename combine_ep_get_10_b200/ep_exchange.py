@@ -1,0 +1,192 @@
+"""Expert parallelism across GPUs: the exchange between the per-rank dispatch
+and the rank-level combine.
+
+The DeepEP-Ascend README ("Normal Mode (Prefill / Training)"; the strategy
+table's ``alltoall`` entry, a ``torch.distributed`` all-to-all-v) sends each
+token once to every rank that holds one of its experts and brings one
+partial row per (token, rank) back.  Here the W processes of a process group
+are those ranks: rank r owns experts [r*E/W, (r+1)*E/W), the logical ranks of
+the layout are the W processes, and the step is
+
+    ep_get_layout (R = W) -> ep_get_rank_layout -> ep_dispatch_ranks
+        send rows grouped by destination rank, each with its K top-k entries
+        seen by that rank (local expert id or -1, gate weight or 0)
+    counts exchange            rows each rank sends to each rank
+    row exchange               all-to-all-v of the rows and their entries
+        -> every rank holds the rows of all ranks' tokens for its experts,
+           source rank 0's rows first, each source's rows in token order
+    local experts              per received row: sum over its local entries
+                               (ascending k) of weight * expert(row), fp32
+                               fmaf chain, one bf16 row (the same layout ->
+                               dispatch -> combine path with R = 1)
+    reverse row exchange       the partial rows go back to their source ranks,
+                               landing in the send order
+    ep_combine_ranks           out[t] = sum over the token's ranks, ascending,
+                               fp32 additions from 0
+
+so a token's result is the two-level sum (per rank, then over ranks) that
+DeepEP's combine forms.  The transfers are ``torch.distributed``
+all-to-all-v calls (NCCL over NVLink between GPUs, gloo between CPU
+processes): the counts on the host size the receive buffers, which is the
+one host synchronisation of a step.  bf16 rows travel as their 16-bit
+patterns.  No transfer here uses TMA multicast or hands a peer's memory to a
+library kernel.
+
+The compute steps are the CUDA kernels of the C ABI (``CudaRowOps``); the
+exchange itself takes any object with the same three methods, so that the
+protocol can be exercised on CPU processes.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+import torch.distributed as dist
+
+
+# ------------------------------------------------------------------ protocol
+def exchange_counts(send_counts: torch.Tensor, group=None) -> torch.Tensor:
+    """send_counts[j] = rows this rank sends to rank j (int64 [W]); returns
+    recv_counts[i] = rows rank i sends to this rank."""
+    if send_counts.dtype != torch.int64 or send_counts.dim() != 1:
+        raise TypeError("send_counts must be an int64 vector of one entry per rank")
+    recv_counts = torch.empty_like(send_counts)
+    dist.all_to_all_single(recv_counts, send_counts, group=group)
+    return recv_counts
+
+
+def exchange_rows(send: torch.Tensor, send_splits: list[int], recv_splits: list[int], group=None) -> torch.Tensor:
+    """All-to-all-v of the rows of `send` (rows for rank 0 first, then rank 1,
+    ...; send_splits[j] rows for rank j).  Returns the received rows, rank 0's
+    first, recv_splits[i] rows from rank i.  bf16 rows travel as their bit
+    patterns, two values per int32 (every backend moves int32)."""
+    if sum(send_splits) != send.shape[0]:
+        raise ValueError("send splits cover %d rows, the buffer has %d" % (sum(send_splits), send.shape[0]))
+    send = send.contiguous()
+    bf16 = send.dtype == torch.bfloat16
+    if bf16 and send.shape[-1] % 2 != 0:
+        raise ValueError("bf16 rows travel in pairs: the last dimension must be even")
+    wire = send.view(torch.int32) if bf16 else send
+    recv = torch.empty((sum(recv_splits),) + tuple(wire.shape[1:]), dtype=wire.dtype, device=send.device)
+    dist.all_to_all_single(recv, wire, output_split_sizes=list(recv_splits),
+                           input_split_sizes=list(send_splits), group=group)
+    return recv.view(torch.bfloat16) if bf16 else recv
+
+
+@dataclass
+class SendRows:
+    """What a rank's per-rank dispatch produced: rows for rank j at
+    [offsets[j], offsets[j+1]) of x / topk_idx / topk_weights, and the handle
+    its rank-level combine needs."""
+    x: torch.Tensor             # bf16 [N_send, H]
+    topk_idx: torch.Tensor      # int64 [N_send, K]: local expert id on the destination rank, or -1
+    topk_weights: torch.Tensor  # fp32 [N_send, K]
+    counts: list[int]           # rows per destination rank
+    handle: object              # passed back to combine_ranks
+
+
+@dataclass
+class Received:
+    """The rows this rank's experts process, source rank 0's first."""
+    x: torch.Tensor
+    topk_idx: torch.Tensor
+    topk_weights: torch.Tensor
+    recv_counts: list[int]
+    send: SendRows
+
+
+class ExpertParallel:
+    """The exchange of one process group (W ranks; rank r owns experts
+    [r*E/W, (r+1)*E/W)).  ``ops`` runs the compute steps (CudaRowOps by
+    default)."""
+
+    def __init__(self, num_experts: int, group=None, ops=None):
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        if num_experts % self.world != 0:
+            raise ValueError("%d experts do not split over %d ranks" % (num_experts, self.world))
+        self.num_experts = num_experts
+        self.local_experts = num_experts // self.world
+        self.ops = ops if ops is not None else CudaRowOps()
+
+    def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor) -> Received:
+        send = self.ops.rank_rows(x, topk_idx, topk_weights, self.num_experts, self.world)
+        if len(send.counts) != self.world:
+            raise ValueError("rank_rows returned %d counts for %d ranks" % (len(send.counts), self.world))
+        send_counts = torch.tensor(send.counts, dtype=torch.int64, device=self._wire_device(x))
+        recv_counts = exchange_counts(send_counts, self.group).tolist()
+        rx = exchange_rows(send.x, send.counts, recv_counts, self.group)
+        ridx = exchange_rows(send.topk_idx, send.counts, recv_counts, self.group)
+        rw = exchange_rows(send.topk_weights, send.counts, recv_counts, self.group)
+        return Received(rx, ridx, rw, recv_counts, send)
+
+    def experts(self, recv: Received, expert_fn) -> torch.Tensor:
+        """One bf16 row per received row: the fmaf chain over its local
+        entries (ascending k) of weight * expert_fn output."""
+        return self.ops.local_experts(recv.x, recv.topk_idx, recv.topk_weights, self.local_experts, expert_fn)
+
+    def combine(self, y: torch.Tensor, recv: Received, out_dtype=torch.bfloat16) -> torch.Tensor:
+        """Send the partial rows back and reduce them per token (ascending
+        rank, fp32 additions)."""
+        if y.shape[0] != sum(recv.recv_counts):
+            raise ValueError("y has %d rows, %d were received" % (y.shape[0], sum(recv.recv_counts)))
+        back = exchange_rows(y, recv.recv_counts, recv.send.counts, self.group)
+        return self.ops.combine_ranks(back, recv.send.handle, out_dtype)
+
+    def _wire_device(self, x):
+        # NCCL moves device tensors; gloo host tensors
+        backend = dist.get_backend(self.group)
+        return x.device if backend == "nccl" else torch.device("cpu")
+
+
+# ------------------------------------------------------------ compute steps
+class CudaRowOps:
+    """The compute steps on the GPU, through the C ABI."""
+
+    def __init__(self, stream=None):
+        from . import binding as B
+
+        self.B = B
+        self.stream = stream
+
+    def rank_rows(self, x, topk_idx, topk_weights, num_experts, world) -> SendRows:
+        B = self.B
+        routing = B.Routing.topk(topk_idx, num_experts, world)
+        layout = B.Layout(routing, device=x.device)
+        B.ep_get_layout(routing, layout, stream=self.stream)
+        rl = B.RankLayout(routing, device=x.device)
+        B.ep_get_rank_layout(routing, layout, rl, stream=self.stream)
+        counts = layout.num_tokens_per_rank.tolist()  # sizes the send buffer
+        n = sum(counts)
+        H, K = x.shape[1], topk_idx.shape[1]
+        sx = torch.empty((n, H), dtype=torch.bfloat16, device=x.device)
+        sidx = torch.empty((n, K), dtype=torch.int64, device=x.device)
+        sw = torch.empty((n, K), dtype=torch.float32, device=x.device)
+        B.ep_dispatch_ranks(x, routing, layout, rl, sx, topk_weights=topk_weights, recv_topk_idx=sidx,
+                            recv_topk_weights=sw, stream=self.stream)
+        return SendRows(sx, sidx, sw, counts, (routing, layout, rl))
+
+    def local_experts(self, x, topk_idx, topk_weights, local_experts, expert_fn):
+        B = self.B
+        n, H = x.shape
+        y = torch.empty((n, H), dtype=torch.bfloat16, device=x.device)
+        if n == 0:
+            return y
+        routing = B.Routing.topk(topk_idx, local_experts, 1)
+        layout = B.Layout(routing, device=x.device, report_num_valid=True)
+        B.ep_get_layout(routing, layout, stream=self.stream)
+        rows = torch.empty((max(layout.num_valid, 1), H), dtype=torch.bfloat16, device=x.device)
+        B.ep_dispatch(x, routing, layout, rows, num_recv_rows=layout.num_valid, stream=self.stream)
+        out_rows = expert_fn(rows[:layout.num_valid], layout.expert_offsets)
+        B.ep_combine(out_rows, routing, layout, topk_weights, y, num_y_rows=layout.num_valid, stream=self.stream)
+        return y
+
+    def combine_ranks(self, back, handle, out_dtype):
+        B = self.B
+        routing, layout, rl = handle
+        out = torch.empty((routing.T, back.shape[1]), dtype=out_dtype, device=back.device)
+        B.ep_combine_ranks(back, routing, layout, rl, out, num_y_rows=back.shape[0], stream=self.stream)
+        if B.ep_get_device_error(layout) != 0:
+            raise B.EPError(B.EP_ERR_BAD_INDEX, "device error flagged in the exchange step")
+        return out
