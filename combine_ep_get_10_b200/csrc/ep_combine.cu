@@ -144,23 +144,13 @@ constexpr int kHeavy0Vec = EP_COMBINE_HEAVY0_VEC;
 constexpr int kHeavy0Group = EP_COMBINE_HEAVY0_GROUP;
 // 16-byte vectors of CSR bounds each thread loads per round of the heavy listing
 constexpr int kHeavyVecs = 8;
-
-// expert choice through the TMA engine (ec_stream_kernel): consumer warps
-// per CTA (a column segment is 16 bytes per consumer thread) and ring stages
-#ifndef EP_EC_STREAM
-#define EP_EC_STREAM 0
+// expert choice: the rows of unpicked tokens are written whole by TMA bulk
+// stores from a zeroed shared buffer while the heavy tokens are listed (1),
+// or by the light runs' vector stores (0)
+#ifndef EP_COMBINE_EC_ZERO_BULK
+#define EP_COMBINE_EC_ZERO_BULK 1
 #endif
-#ifndef EP_EC_STREAM_WARPS
-#define EP_EC_STREAM_WARPS 4
-#endif
-#ifndef EP_EC_STREAM_STAGES
-#define EP_EC_STREAM_STAGES 32
-#endif
-constexpr int kStreamWarps = EP_EC_STREAM_WARPS;
-constexpr int kStreamThreads = (kStreamWarps + 1) * 32; // + one producer warp
-constexpr int kStreamSeg = kStreamWarps * 32 * 16;      // bytes of a row per CTA
-constexpr int kStreamStages = EP_EC_STREAM_STAGES;
-static_assert(kStreamStages >= 32, "the producer's 32 lanes fill 32 distinct stages at once");
+constexpr int kZeroBytes = 4096; // zeroed shared memory behind the bulk stores
 
 enum CombineSrc : int {
     kSrcTopk = 0,  // entries: the token's K (expert, slot) pairs, gate weights
@@ -360,7 +350,7 @@ __device__ __forceinline__ void store_segment(const CombineArgs& a, int64_t t, c
 // CSR order, as in reduce_segment.  Tokens without entries store zeros.
 template <bool kOutF32, int kVecPerLane, int kGroup, int kLookup>
 __device__ __forceinline__ void reduce_run(const CombineArgs& a, int64_t t0, int cnt, int seg, bool skip_heavy,
-                                           int lane, uint32_t& errbits)
+                                           bool zeros_written, int lane, uint32_t& errbits)
 {
     constexpr int kSegVec = 32 * kVecPerLane;
     int v[kVecPerLane];
@@ -384,7 +374,7 @@ __device__ __forceinline__ void reduce_run(const CombineArgs& a, int64_t t0, int
     }
     const bool mine = lane < cnt && !(skip_heavy && my_n >= kHeavyDeg);
     const int my_cnt = mine ? max(my_n, 0) : 0;
-    uint32_t zeros = __ballot_sync(kFullMask, mine && my_cnt == 0);
+    uint32_t zeros = zeros_written ? 0u : __ballot_sync(kFullMask, mine && my_cnt == 0);
     while (zeros) { // warp-uniform
         const int j = __ffs(zeros) - 1;
         zeros &= zeros - 1u;
@@ -594,6 +584,7 @@ __device__ __forceinline__ void reduce_heavy(const CombineArgs& a, int64_t t, in
 template <int kSrc, bool kOutF32, int kVecPerLane, int kGroup>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 {
+    pdl_wait(); // every input is final once the kernel before has finished
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarpsPerCta;
@@ -612,8 +603,9 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 
 // Expert choice.  A few tokens are picked by up to all E experts and most by
 // none, so the work per token varies by 100x.  Every CTA first lists the
-// tokens with at least kHeavyDeg picks (the same tokens in every CTA): by
-// degree class, longest first (>= 4x, >= 2x, >= 1x kHeavyDeg).  The items are then: one per (heavy token, segment),
+// tokens with at least kHeavyDeg picks (the same list in every CTA, which
+// the items below rely on): by degree class, longest first (>= 4x, >= 2x,
+// >= 1x kHeavyDeg), in token order inside a class.  The items are then: one per (heavy token, segment),
 // followed by one per (run of kEcRun tokens, segment); a run item folds its
 // light tokens' entries as one list (reduce_run) and leaves the heavy tokens
 // to the heavy items.  Warps are numbered warp-major (warp w of every CTA
@@ -624,29 +616,42 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 template <bool kOutF32>
 __global__ void __launch_bounds__(kCombineThreads, kEcMinBlocks) ec_combine_kernel(CombineArgs a)
 {
+    pdl_wait(); // every input is final once the kernel before has finished
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     uint32_t errbits = 0;
 
-    __shared__ int s_list[kHeavyClasses][kMaxHeavy];
-    __shared__ int s_cnt[kHeavyClasses];
-    int n_cls[kHeavyClasses];
-#pragma unroll
-    for (int c = 0; c < kHeavyClasses; ++c)
-        n_cls[c] = 0;
+    __shared__ int s_heavy[kMaxHeavy];
+    __shared__ uint32_t s_flags[kHeavyClasses][kHeavyFirstMaxT / 32];
+    __shared__ int s_wsum[kWarpsPerCta];
+    __shared__ __align__(128) uint8_t s_zero[EP_COMBINE_EC_ZERO_BULK ? kZeroBytes : 16];
     int n_heavy = 0, n_long = 0;
     if (a.heavy_first) {
         // Every CTA reads the whole CSR bound array once, coalesced and all at
         // once (16-byte vectors, kHeavyVecs per thread, plus the bound after
-        // each vector) and appends each heavy token to its degree class's list
-        // with a shared-memory atomic.  The order inside a class varies from
-        // run to run; it decides only which warp computes a token, not how
-        // (every token's chain is fixed), so the output does not vary.
+        // each vector), flags the heavy tokens in one shared bit mask per
+        // degree class, then lists them class by class (count per 32-token
+        // word, CTA scan).
         const int tid = threadIdx.x;
-        if (tid < kHeavyClasses)
-            s_cnt[tid] = 0;
+        const int nwords = (a.T + 31) / 32;
+        for (int i = tid; i < nwords; i += kCombineThreads)
+#pragma unroll
+            for (int c = 0; c < kHeavyClasses; ++c)
+                s_flags[c][i] = 0u;
+        if (EP_COMBINE_EC_ZERO_BULK) {
+            for (int i = tid; i < kZeroBytes / 16; i += kCombineThreads)
+                reinterpret_cast<uint4*>(s_zero)[i] = make_uint4(0, 0, 0, 0);
+            fence_proxy_async_shared(); // the bulk stores below read it
+        }
         __syncthreads();
-        // 4 bounds per 16-byte vector (1 when the array is not 16-byte aligned)
+        // this CTA also writes the whole output rows of the unpicked tokens in
+        // [z0, z1), by bulk stores from the zeroed buffer
+        const int64_t z0 = static_cast<int64_t>(a.T) * blockIdx.x / gridDim.x;
+        const int64_t z1 = static_cast<int64_t>(a.T) * (blockIdx.x + 1) / gridDim.x;
+        const int64_t out_row = static_cast<int64_t>(a.H) * (kOutF32 ? 4 : 2);
+        bool issued = false;
+        // 4 bounds per 16-byte vector (1 when the array is not 16-byte aligned),
+        // kHeavyVecs vectors per thread per round, all loads of a round at once
         const int per = (reinterpret_cast<uintptr_t>(a.token_offsets) & 15u) == 0 ? 4 : 1;
         const int nv = (a.T + per - 1) / per; // vectors holding bounds 0 .. T-1
         for (int base = 0; base < nv; base += kHeavyVecs * kCombineThreads) {
@@ -683,28 +688,65 @@ __global__ void __launch_bounds__(kCombineThreads, kEcMinBlocks) ec_combine_kern
                     const int deg = (j + 1 < per ? o[j + 1] : o[4]) - o[j];
                     if (j < per && t < a.T && deg >= kHeavyDeg) {
                         const int c = kHeavyClasses == 1 ? 0 : deg >= 4 * kHeavyDeg ? 0 : deg >= 2 * kHeavyDeg ? 1 : 2;
-                        const int pos = atomicAdd(&s_cnt[c], 1);
-                        if (pos < kMaxHeavy)
-                            s_list[c][pos] = t;
+                        atomicOr(&s_flags[c][t / 32], 1u << (t % 32));
+                    }
+                    if (EP_COMBINE_EC_ZERO_BULK && j < per && t >= z0 && t < z1 && deg == 0) {
+                        uint8_t* row = static_cast<uint8_t*>(a.out) + t * out_row;
+                        for (int64_t b0 = 0; b0 < out_row; b0 += kZeroBytes)
+                            bulk_store_s2g(row + b0, s_zero,
+                                           static_cast<uint32_t>(min(static_cast<int64_t>(kZeroBytes), out_row - b0)));
+                        issued = true;
                     }
                 }
             }
         }
+        if (issued)
+            bulk_commit();
         __syncthreads();
-        bool fits = true;
-#pragma unroll
+        // words w0 .. w1 of this thread, scanned over the CTA, class by class
+        const int wpt = (nwords + kCombineThreads - 1) / kCombineThreads;
+        const int w0 = min(nwords, tid * wpt);
+        const int w1 = min(nwords, w0 + wpt);
+        int listed = 0;
+#pragma unroll 1
         for (int c = 0; c < kHeavyClasses; ++c) {
-            n_cls[c] = s_cnt[c];
-            fits &= n_cls[c] <= kMaxHeavy;
-            n_heavy += n_cls[c];
-        }
-        if (!fits) { // too many to list: every token goes through the runs
+            if (c == 1)
+                n_long = listed; // class 0: the longest lists
+            int cnt = 0;
+            for (int w = w0; w < w1; ++w)
+                cnt += __popc(s_flags[c][w]);
+            int inc = cnt;
 #pragma unroll
-            for (int c = 0; c < kHeavyClasses; ++c)
-                n_cls[c] = 0;
-            n_heavy = 0;
+            for (int d = 1; d < 32; d <<= 1) {
+                const int v = __shfl_up_sync(kFullMask, inc, d);
+                if (lane >= d)
+                    inc += v;
+            }
+            if (lane == 31)
+                s_wsum[warp] = inc;
+            __syncthreads();
+            int before = 0, n_c = 0;
+            for (int w = 0; w < kWarpsPerCta; ++w) {
+                before += w < warp ? s_wsum[w] : 0;
+                n_c += s_wsum[w];
+            }
+            if (listed + n_c <= kMaxHeavy) {
+                int pos = listed + before + inc - cnt;
+                for (int w = w0; w < w1; ++w) {
+                    uint32_t bits = s_flags[c][w];
+                    while (bits) {
+                        const int i = __ffs(bits) - 1;
+                        bits &= bits - 1u;
+                        s_heavy[pos++] = w * 32 + i;
+                    }
+                }
+            }
+            listed += n_c;
+            __syncthreads(); // s_wsum is reused by the next class
         }
-        n_long = kHeavyClasses == 1 ? 0 : n_cls[0];
+        n_heavy = listed <= kMaxHeavy ? listed : 0; // too many to list: every token goes through the runs
+        if (n_heavy == 0 || kHeavyClasses == 1)
+            n_long = 0;
     }
     const int nseg_h = (a.nvec + 32 * kHeavyVec - 1) / (32 * kHeavyVec);
     const int nseg_l = (a.nvec + 32 * kHeavy0Vec - 1) / (32 * kHeavy0Vec);
@@ -721,14 +763,7 @@ __global__ void __launch_bounds__(kCombineThreads, kEcMinBlocks) ec_combine_kern
         const bool is_long = it < long_items;
         const int64_t k = is_long ? it : it - long_items;
         const int ns = is_long ? nseg_l : nseg_h;
-        int64_t t;
-        if (is_long || kHeavyClasses == 1) {
-            t = s_list[0][k / ns];
-        } else { // the other classes' lists, one after the other
-            const int64_t j = k / ns;
-            const int c1 = 1 % kHeavyClasses, c2 = 2 % kHeavyClasses;
-            t = j < n_cls[c1] ? s_list[c1][j] : s_list[c2][j - n_cls[c1]];
-        }
+        const int64_t t = s_heavy[(is_long ? 0 : n_long) + k / ns];
         const int seg = static_cast<int>(k % ns);
         const int beg = __ldg(a.token_offsets + t);
         const int n = __ldg(a.token_offsets + t + 1) - beg;
@@ -751,7 +786,8 @@ __global__ void __launch_bounds__(kCombineThreads, kEcMinBlocks) ec_combine_kern
         const int64_t t0 = r * kEcRun;
         const int cnt = static_cast<int>(min(static_cast<int64_t>(kEcRun), a.T - t0));
 #if EP_COMBINE_EC_FLAT
-        reduce_run<kOutF32, kEcVec, kEcGroup, kEcLookup>(a, t0, cnt, seg, n_heavy > 0, lane, errbits);
+        reduce_run<kOutF32, kEcVec, kEcGroup, kEcLookup>(a, t0, cnt, seg, n_heavy > 0,
+                                                         EP_COMBINE_EC_ZERO_BULK && a.heavy_first, lane, errbits);
 #else
         // lane j holds the CSR bounds of the run's j-th token; one token at a time
         int my_beg = 0, my_n = 0;
@@ -771,222 +807,32 @@ __global__ void __launch_bounds__(kCombineThreads, kEcMinBlocks) ec_combine_kern
     const uint32_t any = __reduce_or_sync(kFullMask, errbits);
     if (lane == 0)
         flag_error(a.err, any);
+    if (EP_COMBINE_EC_ZERO_BULK)
+        bulk_wait_read_all(); // the zero rows' bulk stores have read s_zero
 }
 
-// Expert choice through the TMA engine.  The reads of the gather are rows of
-// y picked in no particular order, 2 KB of each per CTA; issued as 16-byte
-// loads per lane they need one outstanding request per 512 bytes and stall
-// on the SM's request tracking long before HBM is busy.  Here one producer
-// warp per CTA issues one bulk copy (cp.async.bulk) per (pick, segment) into
-// a ring of shared-memory stages, each completing on its own mbarrier, and
-// the consumer warps fold the stages in order:
-//   * the CTA owns one column segment (kStreamSeg bytes, 16 per consumer
-//     thread) of a contiguous range of tokens; the ranges of the CTAs of a
-//     segment split the cost off[t] + t (one unit per pick read, one per
-//     output row written) evenly, so a token with 128 picks and a run of 128
-//     unpicked tokens cost the same;
-//   * per token the consumers run the fmaf chain over its picks in CSR order
-//     (ascending slot) from zero, as the other combine kernels do, and store
-//     the segment of its output row; unpicked tokens store zeros;
-//   * the producer looks the picks up 32 at a time (slot, weight), waits for
-//     each stage to be released (empty barrier, one arrival per consumer
-//     warp) and issues the copy with its weight beside it.
-// Every wait is bounded; a wait that runs out flags EP_DEVERR_TIMEOUT and
-// the CTA stops (its producer drains the copies it issued before leaving).
-struct StreamSmem {
-    uint8_t ring[kStreamStages][kStreamSeg];
-    float w[kStreamStages];
-    int32_t ok[kStreamStages];
-    uint64_t full[kStreamStages];
-    uint64_t empty[kStreamStages];
-    int32_t range[2];
-    int32_t red[2][kStreamWarps + 1];
-    int32_t dead;
-};
+// Combine kernels are launched with programmatic stream serialisation: their
+// CTAs may be placed while the kernel before them (normally the dispatch)
+// retires its last CTAs, and wait in griddepcontrol.wait before any read, so
+// only the launch latency is hidden.
+#ifndef EP_COMBINE_PDL
+#define EP_COMBINE_PDL 1
+#endif
 
-template <bool kOutF32>
-__global__ void __launch_bounds__(kStreamThreads) ec_stream_kernel(CombineArgs a, int32_t per_seg)
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(void (*kernel)(KArgs...), unsigned grid, cudaStream_t stream, Args... args)
 {
-    extern __shared__ __align__(128) uint8_t stream_smem[];
-    StreamSmem& sm = *reinterpret_cast<StreamSmem*>(stream_smem);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool producer = warp == kStreamWarps;
-    const int nseg = a.nseg;
-    const int sigma = static_cast<int>(blockIdx.x) % nseg; // column segment
-    const int part = static_cast<int>(blockIdx.x) / nseg;  // token range among the CTAs of the segment
-    const int64_t row_bytes = static_cast<int64_t>(a.H) * 2;
-    const int64_t seg_off = static_cast<int64_t>(sigma) * kStreamSeg;
-    const uint32_t seg_bytes = static_cast<uint32_t>(min(static_cast<int64_t>(kStreamSeg), row_bytes - seg_off));
-    const int32_t* off = a.token_offsets;
-
-    if (tid == 0) {
-        for (int i = 0; i < kStreamStages; ++i) {
-            mbar_init(&sm.full[i], 1);
-            mbar_init(&sm.empty[i], kStreamWarps);
-        }
-        sm.dead = 0;
-        fence_mbar_init();
-    }
-    // token range: t_a = #{t : off[t] + t < C * part / P}, t_b likewise for
-    // part + 1 (the cost off[t] + t rises with t), counted by every thread
-    // over a strided share of the bounds
-    const int64_t C = static_cast<int64_t>(__ldg(off + a.T)) + a.T;
-    const int64_t target_a = C * part / per_seg;
-    const int64_t target_b = part + 1 == per_seg ? C : C * (part + 1) / per_seg;
-    int cnt_a = 0, cnt_b = 0;
-    for (int i0 = 0; i0 <= a.T; i0 += 8 * kStreamThreads) {
-        int64_t c[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * kStreamThreads + tid;
-            c[u] = i <= a.T ? static_cast<int64_t>(__ldg(off + i)) + i : C;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            cnt_a += c[u] < target_a ? 1 : 0;
-            cnt_b += c[u] < target_b ? 1 : 0;
-        }
-    }
-#pragma unroll
-    for (int d = 16; d >= 1; d >>= 1) {
-        cnt_a += __shfl_xor_sync(kFullMask, cnt_a, d);
-        cnt_b += __shfl_xor_sync(kFullMask, cnt_b, d);
-    }
-    if (lane == 0) {
-        sm.red[0][warp] = cnt_a;
-        sm.red[1][warp] = cnt_b;
-    }
-    __syncthreads();
-    int t_a = 0, t_b = 0;
-#pragma unroll
-    for (int w = 0; w <= kStreamWarps; ++w) {
-        t_a += sm.red[0][w];
-        t_b += sm.red[1][w];
-    }
-
-    if (producer) {
-        uint32_t ctr = 0; // records issued
-        volatile int32_t* dead = &sm.dead; // written by a warp whose wait ran out
-        for (int tb = t_a; tb < t_b && *dead == 0; tb += 32) {
-            const int t = tb + lane;
-            int beg = 0, n = 0;
-            if (t < t_b) {
-                beg = __ldg(off + t);
-                n = __ldg(off + t + 1) - beg;
-            }
-            int incl = n;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const int o = __shfl_up_sync(kFullMask, incl, d);
-                if (lane >= d)
-                    incl += o;
-            }
-            const int total = __shfl_sync(kFullMask, incl, 31);
-            const int start = incl - n;
-            for (int r0 = 0; r0 < total; r0 += 32) {
-                const int r = r0 + lane;
-                // owner of record r: the lanes whose picks end at or before r
-                int j = 0;
-#pragma unroll
-                for (int step = 16; step >= 1; step >>= 1) {
-                    const int end = __shfl_sync(kFullMask, incl, j + step - 1);
-                    if (end <= r)
-                        j += step;
-                }
-                const int jbeg = __shfl_sync(kFullMask, beg, j);
-                const int jstart = __shfl_sync(kFullMask, start, j);
-                if (r < total) {
-                    const int32_t sl = __ldg(a.token_slots + jbeg + (r - jstart));
-                    const bool ok = sl >= 0 && sl < a.num_y_rows;
-                    const float w = ok ? __ldg(a.expert_weights + sl) : 0.0f;
-                    if (!ok)
-                        flag_error(a.err, EP_DEVERR_OVERFLOW);
-                    const uint32_t c = ctr + static_cast<uint32_t>(r);
-                    const int st = static_cast<int>(c % kStreamStages);
-                    bool go = true;
-                    if (c >= kStreamStages)
-                        go = mbar_wait_bounded(&sm.empty[st], ((c / kStreamStages) - 1u) & 1u, a.err);
-                    if (!go) {
-                        *dead = 1;
-                    } else {
-                        sm.w[st] = w;
-                        sm.ok[st] = ok ? 1 : 0;
-                        if (ok) {
-                            mbar_arrive_expect_tx(&sm.full[st], seg_bytes);
-                            bulk_load_g2s(sm.ring[st], a.y + static_cast<int64_t>(sl) * row_bytes + seg_off, seg_bytes,
-                                          &sm.full[st]);
-                        } else {
-                            mbar_arrive(&sm.full[st]);
-                        }
-                    }
-                }
-                __syncwarp();
-            }
-            ctr += static_cast<uint32_t>(total);
-        }
-        // drain: every issued copy has landed before the CTA leaves (at once
-        // unless a consumer stopped early)
-        for (int st = lane; st < kStreamStages; st += 32) {
-            if (static_cast<uint32_t>(st) < ctr) {
-                const uint32_t last = (ctr - 1u - static_cast<uint32_t>(st)) / kStreamStages * kStreamStages + st;
-                mbar_wait_bounded(&sm.full[st], (last / kStreamStages) & 1u, a.err);
-            }
-        }
-        return;
-    }
-
-    // consumers: thread tid owns bytes [16 tid, 16 tid + 16) of the segment
-    const bool mine = static_cast<uint32_t>(tid) * 16u < seg_bytes;
-    const int64_t col = seg_off + static_cast<int64_t>(tid) * 16; // byte of the bf16 row
-    uint32_t ctr = 0;
-    for (int tb = t_a; tb < t_b; tb += 32) {
-        const int t = tb + lane;
-        int n = 0;
-        if (t < t_b)
-            n = __ldg(off + t + 1) - __ldg(off + t);
-        const int m = min(32, t_b - tb);
-        for (int jt = 0; jt < m; ++jt) {
-            const int nj = __shfl_sync(kFullMask, n, jt);
-            float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-            for (int e = 0; e < nj; ++e) {
-                const int st = static_cast<int>(ctr % kStreamStages);
-                if (!mbar_wait_bounded(&sm.full[st], (ctr / kStreamStages) & 1u, a.err)) {
-                    *reinterpret_cast<volatile int32_t*>(&sm.dead) = 1;
-                    return;
-                }
-                if (sm.ok[st] && mine) {
-                    const float w = sm.w[st];
-                    const uint4 d = *reinterpret_cast<const uint4*>(sm.ring[st] + tid * 16);
-                    acc[0] = fmaf(w, bf16_lo(d.x), acc[0]);
-                    acc[1] = fmaf(w, bf16_hi(d.x), acc[1]);
-                    acc[2] = fmaf(w, bf16_lo(d.y), acc[2]);
-                    acc[3] = fmaf(w, bf16_hi(d.y), acc[3]);
-                    acc[4] = fmaf(w, bf16_lo(d.z), acc[4]);
-                    acc[5] = fmaf(w, bf16_hi(d.z), acc[5]);
-                    acc[6] = fmaf(w, bf16_lo(d.w), acc[6]);
-                    acc[7] = fmaf(w, bf16_hi(d.w), acc[7]);
-                }
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&sm.empty[st]);
-                ++ctr;
-            }
-            if (mine) {
-                const int64_t tok = tb + jt;
-                if (kOutF32) {
-                    float* o = static_cast<float*>(a.out) + tok * a.H + col / 2;
-                    st_cs_v4(o, make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
-                                           __float_as_uint(acc[3])));
-                    st_cs_v4(o + 4, make_uint4(__float_as_uint(acc[4]), __float_as_uint(acc[5]),
-                                               __float_as_uint(acc[6]), __float_as_uint(acc[7])));
-                } else {
-                    st_cs_v4(static_cast<uint8_t*>(a.out) + tok * row_bytes + col,
-                             make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                                        pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7])));
-                }
-            }
-        }
-    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kCombineThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = EP_COMBINE_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 // Blocks of 256 threads of `kernel` resident on the whole device (SMs x
@@ -1031,11 +877,8 @@ cudaError_t launch_combine(CombineArgs k, bool out_f32, bool persistent, cudaStr
     for (int64_t b0 = 0; b0 < blocks; b0 += kMaxBlocks) {
         k.warp_base = b0 * kWarpsPerCta;
         const unsigned n = static_cast<unsigned>(blocks - b0 < kMaxBlocks ? blocks - b0 : kMaxBlocks);
-        if (out_f32)
-            combine_kernel<kSrc, true, kVec, kGrp><<<n, kCombineThreads, 0, stream>>>(k);
-        else
-            combine_kernel<kSrc, false, kVec, kGrp><<<n, kCombineThreads, 0, stream>>>(k);
-        cudaError_t st = cudaGetLastError();
+        cudaError_t st = out_f32 ? launch_after(combine_kernel<kSrc, true, kVec, kGrp>, n, stream, k)
+                                 : launch_after(combine_kernel<kSrc, false, kVec, kGrp>, n, stream, k);
         if (st != cudaSuccess)
             return st;
     }
@@ -1043,52 +886,8 @@ cudaError_t launch_combine(CombineArgs k, bool out_f32, bool persistent, cudaStr
 }
 
 // Expert choice: one resident wave of warps over the heavy and run items.
-std::atomic<int> stream_blocks_cache[2][64];
-
-// The TMA-fed expert-choice combine: resident CTAs rounded down to a
-// multiple of the row's column segments (at least one CTA per segment).
-cudaError_t launch_ec_stream(CombineArgs k, bool out_f32, cudaStream_t stream)
-{
-    const int64_t row_bytes = static_cast<int64_t>(k.H) * 2;
-    k.nseg = static_cast<int32_t>((row_bytes + kStreamSeg - 1) / kStreamSeg);
-    const size_t smem = sizeof(StreamSmem);
-    int dev = 0;
-    cudaError_t st = cudaGetDevice(&dev);
-    if (st != cudaSuccess)
-        return st;
-    std::atomic<int>& cache = stream_blocks_cache[out_f32 ? 1 : 0][dev >= 0 && dev < 64 ? dev : 0];
-    int resident = cache.load(std::memory_order_relaxed);
-    if (resident == 0) {
-        auto kernel = out_f32 ? ec_stream_kernel<true> : ec_stream_kernel<false>;
-        st = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        int sms = 0, per_sm = 0;
-        if (st == cudaSuccess)
-            st = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (st == cudaSuccess)
-            st = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStreamThreads, smem);
-        if (st != cudaSuccess)
-            return st;
-        resident = std::max(1, sms * per_sm);
-        if (dev >= 0 && dev < 64)
-            cache.store(resident, std::memory_order_relaxed);
-    }
-    const int64_t per_seg = std::max<int64_t>(1, resident / k.nseg);
-    const int64_t blocks = per_seg * k.nseg;
-    if (blocks >= (int64_t{1} << 31))
-        return cudaErrorInvalidValue;
-    if (out_f32)
-        ec_stream_kernel<true><<<static_cast<unsigned>(blocks), kStreamThreads, smem, stream>>>(
-            k, static_cast<int32_t>(per_seg));
-    else
-        ec_stream_kernel<false><<<static_cast<unsigned>(blocks), kStreamThreads, smem, stream>>>(
-            k, static_cast<int32_t>(per_seg));
-    return cudaGetLastError();
-}
-
 cudaError_t launch_ec(CombineArgs k, bool out_f32, cudaStream_t stream)
 {
-    if (EP_EC_STREAM)
-        return launch_ec_stream(k, out_f32, stream);
     k.nseg = (k.nvec + 32 * kEcVec - 1) / (32 * kEcVec);
     const int64_t runs = (static_cast<int64_t>(k.T) + kEcRun - 1) / kEcRun;
     const int64_t items = std::max<int64_t>(1, runs * k.nseg);
@@ -1098,11 +897,8 @@ cudaError_t launch_ec(CombineArgs k, bool out_f32, cudaStream_t stream)
     int64_t blocks = res > 0 ? res : (items + kWarpsPerCta - 1) / kWarpsPerCta;
     blocks = std::min<int64_t>(blocks, int64_t{1} << 30);
     k.warp_base = 0;
-    if (out_f32)
-        ec_combine_kernel<true><<<static_cast<unsigned>(blocks), kCombineThreads, 0, stream>>>(k);
-    else
-        ec_combine_kernel<false><<<static_cast<unsigned>(blocks), kCombineThreads, 0, stream>>>(k);
-    return cudaGetLastError();
+    return out_f32 ? launch_after(ec_combine_kernel<true>, static_cast<unsigned>(blocks), stream, k)
+                   : launch_after(ec_combine_kernel<false>, static_cast<unsigned>(blocks), stream, k);
 }
 
 } // namespace

@@ -330,30 +330,15 @@ __device__ __forceinline__ uint2 encode8(uint4 r, float mul)
 // issued by different threads.  Rows whose byte size is not a multiple of 16
 // are written with 8-byte stores instead.  Registers stay low, so many CTAs
 // (and their row loads) are resident per SM.
-// Up to kInPlaceIters vectors per thread (rows of up to 8192 channels) the
-// codes overwrite the staged row: every thread first takes its vectors into
-// registers, the CTA meets at a barrier, and the codes are written over the
-// bf16 row, so a token CTA needs 2H bytes of row buffer instead of 3H (2.5H
-// for FP4) and a third more tokens fit on an SM.
-//   shared memory: x row [2H] | codes [code_row] (not in place) | scales [scale_row -> 16] | rows [K]
+//   shared memory: x row [2H] | codes [code_row] | scales [scale_row -> 16] | rows [K]
 // Shared-memory bytes of one token CTA: x row | codes | scales | rows [K]
 // (| fused layout: expert -> k mask [E], histogram [E], per-token rank bits
 // [T], small arrays [4 x 32]).
-constexpr int kInPlaceIters = 8;
-#ifndef EP_QUANT_IN_PLACE
-#define EP_QUANT_IN_PLACE 0
-#endif
-
-__host__ __device__ inline bool quant_in_place(int fmt, int H)
-{
-    return EP_QUANT_IN_PLACE && fmt != kQBf16 && H / 8 <= kInPlaceIters * kQuantThreads;
-}
-
 __host__ __device__ inline size_t quant_smem_bytes(int fmt, int H, int K, int E, int T, bool fused)
 {
     const size_t nvec = static_cast<size_t>(H) / 8;
     const bool mx = fmt == kQMxE4m3 || fmt == kQMxE5m2 || fmt == kQMxE2m1;
-    const size_t code_row = fmt == kQBf16 || quant_in_place(fmt, H) ? 0 : nvec * (fmt == kQMxE2m1 ? 4 : 8);
+    const size_t code_row = fmt == kQBf16 ? 0 : nvec * (fmt == kQMxE2m1 ? 4 : 8);
     const size_t scale_row =
         fmt == kQBf16 ? 0 : (mx ? nvec / 4 : ((fmt == kQInt8Tok || fmt == kQFp8Tok) ? 4 : nvec / 16 * 4));
     size_t n = nvec * 16 + code_row + ((scale_row + 15) & ~static_cast<size_t>(15)) + sizeof(int64_t) * K;
@@ -490,10 +475,9 @@ __device__ __forceinline__ void fused_layout(const QuantArgs& a, int64_t t, int6
     }
 }
 
-template <int kFmt, bool kFused, bool kInPlace>
+template <int kFmt, bool kFused>
 __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs a)
 {
-    static_assert(!(kInPlace && kFmt == kQBf16), "the bf16 copy encodes nothing");
     constexpr bool kMx = kFmt == kQMxE4m3 || kFmt == kQMxE5m2 || kFmt == kQMxE2m1;
     constexpr bool kPerToken = kFmt == kQInt8Tok || kFmt == kQFp8Tok;
     constexpr bool kCopy = kFmt == kQBf16;
@@ -509,8 +493,8 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
     const int code_row = kCopy ? row_bytes : nvec * kCodeBytes;
     const int scale_row = kCopy ? 0 : (kMx ? nvec / 4 : (kPerToken ? 4 : nvec / 16 * 4));
     uint8_t* s_x = qsmem;
-    uint8_t* s_codes = kCopy || kInPlace ? s_x : qsmem + row_bytes;
-    uint8_t* s_scales = qsmem + row_bytes + (kCopy || kInPlace ? 0 : code_row);
+    uint8_t* s_codes = kCopy ? s_x : qsmem + row_bytes;
+    uint8_t* s_scales = qsmem + row_bytes + (kCopy ? 0 : code_row);
     int64_t* rows = reinterpret_cast<int64_t*>(s_scales + ((scale_row + 15) & ~15));
 
     if (tid == 0) {
@@ -542,29 +526,11 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
     if (!mbar_wait_bounded(&bar, 0, a.err))
         return;
 
-    // in place: this thread's vectors in registers, then a barrier, so that
-    // no code is written over a vector another thread has yet to read
-    uint4 held[kInPlace ? kInPlaceIters : 1];
-    if constexpr (kInPlace) {
-#pragma unroll
-        for (int i = 0; i < kInPlaceIters; ++i) {
-            const int v = i * kQuantThreads + tid;
-            held[i] = v < nvec ? *reinterpret_cast<const uint4*>(s_x + v * 16) : make_uint4(0, 0, 0, 0);
-        }
-        __syncthreads();
-    }
-
     float tok_mul = 0.0f;
     if constexpr (kPerToken) {
         float amax = 0.0f;
-        if constexpr (kInPlace) {
-#pragma unroll
-            for (int i = 0; i < kInPlaceIters; ++i)
-                amax = fmaxf(amax, amax8(held[i])); // zero vectors past the row leave the max alone
-        } else {
-            for (int v = tid; v < nvec; v += kQuantThreads)
-                amax = fmaxf(amax, amax8(*reinterpret_cast<const uint4*>(s_x + v * 16)));
-        }
+        for (int v = tid; v < nvec; v += kQuantThreads)
+            amax = fmaxf(amax, amax8(*reinterpret_cast<const uint4*>(s_x + v * 16)));
 #pragma unroll
         for (int d = 16; d >= 1; d >>= 1)
             amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
@@ -625,14 +591,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
                 reinterpret_cast<uint32_t*>(s_codes)[v] = q.x;
         }
     };
-    if constexpr (kInPlace) {
-#pragma unroll
-        for (int i = 0; i < kInPlaceIters; ++i) {
-            if (i * kQuantThreads >= nvec)
-                break; // CTA-uniform
-            encode_step(i * kQuantThreads, held[i]);
-        }
-    } else if constexpr (!kCopy) {
+    if constexpr (!kCopy) {
         for (int base = 0; base < nvec; base += kQuantThreads) {
             const int v = base + tid;
             encode_step(base, v < nvec ? *reinterpret_cast<const uint4*>(s_x + v * 16) : make_uint4(0, 0, 0, 0));
@@ -692,9 +651,7 @@ template <int kFmt, bool kFused>
 cudaError_t launch_quant(const QuantArgs& a, int32_t T, int32_t K, cudaStream_t stream)
 {
     const size_t smem = quant_smem_bytes(kFmt, a.H, K, a.map.E, kFused ? T : 0, kFused);
-    constexpr bool kCanInPlace = kFmt != kQBf16;
-    auto kernel = kCanInPlace && quant_in_place(kFmt, a.H) ? quant_dispatch_kernel<kFmt, kFused, kCanInPlace>
-                                                           : quant_dispatch_kernel<kFmt, kFused, false>;
+    auto kernel = quant_dispatch_kernel<kFmt, kFused>;
     if (smem > 48 * 1024) {
         cudaError_t st = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (st != cudaSuccess)

@@ -60,7 +60,7 @@ def test_token_choice_random_shapes(seed):
     ref_d = oracle.tc_dispatch(x, idx, E, ref_l)
     assert np.array_equal(host(recv)[:n], ref_d["recv"])
     for dt, tdt in ((W.FP32, torch.float32), (W.BF16, torch.bfloat16)):
-        out = torch.empty((T, H), dtype=tdt, device="cuda")
+        out = torch.full((T, H), float("nan"), dtype=tdt, device="cuda")
         B.ep_combine(recv, routing, lay, wd, out, num_y_rows=n)
         ref_c = oracle.tc_combine(ref_d["recv"], idx, E, ref_l, w, out_dtype=dt)
         assert_combine_close(host(out), ref_c, dt == W.BF16, "combine seed %d" % seed)
@@ -91,7 +91,7 @@ def test_token_choice_random_shapes(seed):
         rrecv = torch.empty((nr, H), dtype=torch.bfloat16, device="cuda")
         B.ep_dispatch_ranks(xd, routing, lay, rl, rrecv)
         assert np.array_equal(host(rrecv), oracle.rank_dispatch(x, idx, E, R, ref_rl)["recv"])
-        rout = torch.empty((T, H), dtype=torch.float32, device="cuda")
+        rout = torch.full((T, H), float("nan"), dtype=torch.float32, device="cuda")
         B.ep_combine_ranks(rrecv, routing, lay, rl, rout)
         assert_combine_close(host(rout), oracle.rank_combine(host(rrecv), ref_rl, out_dtype=W.FP32), False, "ranks")
     assert B.ep_get_device_error(lay) & ~B.EP_DEVERR_OVERFLOW == 0
@@ -119,7 +119,7 @@ def test_expert_choice_random_shapes(seed):
     B.ep_dispatch_expert_choice(to_dev(x, bf16=True), routing, lay, recv)
     ref_d = oracle.ec_dispatch(x, ti)
     assert np.array_equal(host(recv), ref_d)
-    out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    out = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
     B.ep_combine_expert_choice(recv, routing, lay, to_dev(ew), out)
     assert_combine_close(host(out), oracle.ec_combine(ref_d, ref_l, ew, T, out_dtype=W.BF16), True, "ec")
     assert B.ep_get_device_error(lay) == 0

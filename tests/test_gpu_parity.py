@@ -43,6 +43,12 @@ def rng(seed):
     return np.random.Generator(np.random.PCG64(seed))
 
 
+def nan_filled(shape, dtype):
+    """An output buffer holding NaN bit patterns, so that a row the kernel
+    fails to write (or writes for the wrong token) cannot match the oracle."""
+    return torch.full(shape, float("nan"), dtype=dtype, device="cuda")
+
+
 # ---------------------------------------------------------------- helpers
 def gpu_tc_layout(idx_np, E, R, stream=None):
     idx = to_dev(np.ascontiguousarray(idx_np, np.int64))
@@ -232,7 +238,7 @@ def _combine_both(y_np, routing, lay, w_np, T, H, mode=W.COMPACT, mt=0, num_rows
     wd = to_dev(w_np)
     outs = {}
     for dt in (W.FP32, W.BF16):
-        out = torch.empty((T, H), dtype=torch.float32 if dt == W.FP32 else torch.bfloat16, device="cuda")
+        out = nan_filled((T, H), torch.float32 if dt == W.FP32 else torch.bfloat16)
         B.ep_combine(yd, routing, lay, wd, out, mode=mode, max_tokens_per_expert=mt, num_y_rows=num_rows)
         outs[dt] = host(out)
     return outs
@@ -387,7 +393,7 @@ def test_ec_workload(R):
     assert np.array_equal(host(recv), ref_recv)
     wd = to_dev(ew)
     for dt, bf in ((W.FP32, False), (W.BF16, True)):
-        out = torch.empty((T, H), dtype=torch.float32 if dt == W.FP32 else torch.bfloat16, device="cuda")
+        out = nan_filled((T, H), torch.float32 if dt == W.FP32 else torch.bfloat16)
         B.ep_combine_expert_choice(to_dev(ref_recv, bf16=True), routing, lay, wd, out)
         ref = oracle.ec_combine(ref_recv, ref_l, ew, T, out_dtype=dt)
         got = host(out)
@@ -428,7 +434,7 @@ def test_ec_edges(case):
     assert np.array_equal(host(recv), ref_recv)
     y = W.to_bf16_bits(r.standard_normal((E * C, H)).astype(np.float32))
     for dt, bf in ((W.FP32, False), (W.BF16, True)):
-        out = torch.empty((T, H), dtype=torch.float32 if dt == W.FP32 else torch.bfloat16, device="cuda")
+        out = nan_filled((T, H), torch.float32 if dt == W.FP32 else torch.bfloat16)
         B.ep_combine_expert_choice(to_dev(y, bf16=True), routing, lay, to_dev(ew), out)
         ref = oracle.ec_combine(y, ref_l, ew, T, out_dtype=dt)
         assert_combine_close(host(out), ref, bf, "ec edges")
@@ -450,7 +456,7 @@ def test_ec_skewed_mixed(T, E, C, H):
     assert flags == 0
     y = W.to_bf16_bits(r.standard_normal((E * C, H)).astype(np.float32))
     for dt, bf in ((W.FP32, False), (W.BF16, True)):
-        out = torch.empty((T, H), dtype=torch.float32 if dt == W.FP32 else torch.bfloat16, device="cuda")
+        out = nan_filled((T, H), torch.float32 if dt == W.FP32 else torch.bfloat16)
         B.ep_combine_expert_choice(to_dev(y, bf16=True), routing, lay, to_dev(ew), out)
         ref = oracle.ec_combine(y, ref_l, ew, T, out_dtype=dt)
         assert_combine_close(host(out), ref, bf, "ec skewed")
@@ -479,7 +485,7 @@ def test_long_sequence_in_rounds():
     xd, idxd, wd = to_dev(x, bf16=True), to_dev(idx), to_dev(w)
     routing = B.Routing.topk(idxd, E, R)
     recv = torch.empty((P * K, H), dtype=torch.bfloat16, device="cuda")
-    out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    out = nan_filled((T, H), torch.bfloat16)
     rounds = B.token_rounds(T, P)
     assert len(rounds) == 4
     for t0, t1 in rounds:
