@@ -96,6 +96,7 @@ struct CombineArgs {
     uint32_t* err;
     int64_t warp_base; // first (token, segment) item of this launch
     int32_t heavy_first; // expert choice: list heavy tokens first (persistent launch)
+    int32_t wide;        // rows and y 32-byte aligned: pairs of vectors by one 32-byte load
 };
 
 // expert choice, heavy first (see combine_kernel)
@@ -219,11 +220,13 @@ __device__ __forceinline__ void reduce_segment(const CombineArgs& a, int64_t t, 
                                                uint32_t& errbits)
 {
     constexpr int kSegVec = 32 * kVecPerLane;
+    const bool wide = kVecPerLane % 2 == 0 && a.wide != 0;
     int v[kVecPerLane];
     bool vin[kVecPerLane];
 #pragma unroll
     for (int j = 0; j < kVecPerLane; ++j) {
-        v[j] = seg * kSegVec + j * 32 + lane;
+        // 32-byte loads: lane covers vectors 2 lane, 2 lane + 1 of each 64-vector run
+        v[j] = wide ? seg * kSegVec + (j >> 1) * 64 + 2 * lane + (j & 1) : seg * kSegVec + j * 32 + lane;
         vin[j] = v[j] < a.nvec;
     }
     float acc[kVecPerLane][8];
@@ -269,13 +272,23 @@ __device__ __forceinline__ void reduce_segment(const CombineArgs& a, int64_t t, 
                 }
                 uint4 d[kGroup][kVecPerLane];
 #pragma unroll
-                for (int g = 0; g < kGroup; ++g)
+                for (int g = 0; g < kGroup; ++g) {
+                    const bool on = rows[g] >= 0;
+                    const uint8_t* src = a.y + static_cast<int64_t>(on ? rows[g] : 0) * row_bytes;
+                    if (wide) {
 #pragma unroll
-                    for (int j = 0; j < kVecPerLane; ++j)
-                        d[g][j] = (rows[g] >= 0 && vin[j])
-                                      ? ld_nc_v4(a.y + static_cast<int64_t>(rows[g]) * row_bytes +
-                                                 static_cast<int64_t>(v[j]) * 16)
-                                      : make_uint4(0, 0, 0, 0);
+                        for (int j = 0; j < kVecPerLane; j += 2) {
+                            if (on && vin[j])
+                                ld_nc_v8(src + static_cast<int64_t>(v[j]) * 16, d[g][j], d[g][j + 1]);
+                            else
+                                d[g][j] = d[g][j + 1] = make_uint4(0, 0, 0, 0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < kVecPerLane; ++j)
+                            d[g][j] = (on && vin[j]) ? ld_nc_v4(src + static_cast<int64_t>(v[j]) * 16) : make_uint4(0, 0, 0, 0);
+                    }
+                }
 #pragma unroll
                 for (int g = 0; g < kGroup; ++g) {
                     if (rows[g] < 0)
@@ -353,11 +366,13 @@ __device__ __forceinline__ void reduce_run(const CombineArgs& a, int64_t t0, int
                                            bool zeros_written, int lane, uint32_t& errbits)
 {
     constexpr int kSegVec = 32 * kVecPerLane;
+    const bool wide = kVecPerLane % 2 == 0 && a.wide != 0;
     int v[kVecPerLane];
     bool vin[kVecPerLane];
 #pragma unroll
     for (int j = 0; j < kVecPerLane; ++j) {
-        v[j] = seg * kSegVec + j * 32 + lane;
+        // 32-byte loads: lane covers vectors 2 lane, 2 lane + 1 of each 64-vector run
+        v[j] = wide ? seg * kSegVec + (j >> 1) * 64 + 2 * lane + (j & 1) : seg * kSegVec + j * 32 + lane;
         vin[j] = v[j] < a.nvec;
     }
     float acc[kVecPerLane][8];
@@ -443,13 +458,23 @@ __device__ __forceinline__ void reduce_run(const CombineArgs& a, int64_t t0, int
                 }
                 uint4 d[kGroup][kVecPerLane];
 #pragma unroll
-                for (int g = 0; g < kGroup; ++g)
+                for (int g = 0; g < kGroup; ++g) {
+                    const bool on = rows[g] >= 0;
+                    const uint8_t* src = a.y + static_cast<int64_t>(on ? rows[g] : 0) * (static_cast<int64_t>(a.H) * 2);
+                    if (wide) {
 #pragma unroll
-                    for (int j = 0; j < kVecPerLane; ++j)
-                        d[g][j] = (rows[g] >= 0 && vin[j])
-                                      ? ld_nc_v4(a.y + static_cast<int64_t>(rows[g]) * a.H * 2 +
-                                                 static_cast<int64_t>(v[j]) * 16)
-                                      : make_uint4(0, 0, 0, 0);
+                        for (int j = 0; j < kVecPerLane; j += 2) {
+                            if (on && vin[j])
+                                ld_nc_v8(src + static_cast<int64_t>(v[j]) * 16, d[g][j], d[g][j + 1]);
+                            else
+                                d[g][j] = d[g][j + 1] = make_uint4(0, 0, 0, 0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < kVecPerLane; ++j)
+                            d[g][j] = (on && vin[j]) ? ld_nc_v4(src + static_cast<int64_t>(v[j]) * 16) : make_uint4(0, 0, 0, 0);
+                    }
+                }
 #pragma unroll
                 for (int g = 0; g < kGroup; ++g) {
                     if (g0 + g >= m)
@@ -497,11 +522,13 @@ __device__ __forceinline__ void reduce_heavy(const CombineArgs& a, int64_t t, in
 {
     constexpr int kSegVec = 32 * kVecPerLane;
     static_assert(32 % kGroup == 0, "a group never straddles two lookups");
+    const bool wide = kVecPerLane % 2 == 0 && a.wide != 0;
     int v[kVecPerLane];
     bool vin[kVecPerLane];
 #pragma unroll
     for (int j = 0; j < kVecPerLane; ++j) {
-        v[j] = seg * kSegVec + j * 32 + lane;
+        // 32-byte loads: lane covers vectors 2 lane, 2 lane + 1 of each 64-vector run
+        v[j] = wide ? seg * kSegVec + (j >> 1) * 64 + 2 * lane + (j & 1) : seg * kSegVec + j * 32 + lane;
         vin[j] = v[j] < a.nvec;
     }
     float acc[kVecPerLane][8];
@@ -543,13 +570,23 @@ __device__ __forceinline__ void reduce_heavy(const CombineArgs& a, int64_t t, in
             }
             uint4 d[kGroup][kVecPerLane];
 #pragma unroll
-            for (int g = 0; g < kGroup; ++g)
+            for (int g = 0; g < kGroup; ++g) {
+                const bool on = rows[g] >= 0;
+                const uint8_t* src = a.y + static_cast<int64_t>(on ? rows[g] : 0) * row_bytes;
+                if (wide) {
 #pragma unroll
-                for (int j = 0; j < kVecPerLane; ++j)
-                    d[g][j] = (rows[g] >= 0 && vin[j])
-                                  ? ld_nc_v4(a.y + static_cast<int64_t>(rows[g]) * row_bytes +
-                                             static_cast<int64_t>(v[j]) * 16)
-                                  : make_uint4(0, 0, 0, 0);
+                    for (int j = 0; j < kVecPerLane; j += 2) {
+                        if (on && vin[j])
+                            ld_nc_v8(src + static_cast<int64_t>(v[j]) * 16, d[g][j], d[g][j + 1]);
+                        else
+                            d[g][j] = d[g][j + 1] = make_uint4(0, 0, 0, 0);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < kVecPerLane; ++j)
+                        d[g][j] = (on && vin[j]) ? ld_nc_v4(src + static_cast<int64_t>(v[j]) * 16) : make_uint4(0, 0, 0, 0);
+                }
+            }
             if (g0 == 0) { // the next 32 entries' weights, and the slots of the 32 after them
                 r_nxt = valid(k0 + 32 + lane, s_nxt) ? s_nxt : -1;
                 w_nxt = r_nxt >= 0 ? __ldg(a.expert_weights + r_nxt) : 0.0f;
@@ -901,6 +938,19 @@ cudaError_t launch_ec(CombineArgs k, bool out_f32, cudaStream_t stream)
                    : launch_after(ec_combine_kernel<false>, static_cast<unsigned>(blocks), stream, k);
 }
 
+// Pairs of 16-byte vectors by one 32-byte load (sm_100's 256-bit loads) in
+// the token-choice and per-rank combines from this many tokens on: measured
+// faster at 16384 tokens (skewed workload 305 -> 293 us) and slower at 4096
+// (91 -> 99 us); the expert-choice combine measured no gain and keeps 16-byte
+// loads.  32-byte loads need y aligned to 32 and rows a multiple of 32 bytes.
+#ifndef EP_COMBINE_WIDE_MIN_TOKENS
+#define EP_COMBINE_WIDE_MIN_TOKENS 8192
+#endif
+int32_t wide_loads(const void* y, int32_t H, int32_t T)
+{
+    return T >= EP_COMBINE_WIDE_MIN_TOKENS && H % 16 == 0 && (reinterpret_cast<uintptr_t>(y) & 31u) == 0 ? 1 : 0;
+}
+
 } // namespace
 
 cudaError_t launch_tc_combine(const TcCombineLaunch& a, cudaStream_t stream)
@@ -921,6 +971,7 @@ cudaError_t launch_tc_combine(const TcCombineLaunch& a, cudaStream_t stream)
     k.topk_weights = a.topk_weights;
     k.out = a.out;
     k.err = a.err;
+    k.wide = wide_loads(a.y, a.H, a.T);
     return launch_combine<kSrcTopk, kTcVec, kTcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0, stream);
 }
 
@@ -938,6 +989,7 @@ cudaError_t launch_ec_combine(const EcCombineLaunch& a, cudaStream_t stream)
     k.out = a.out;
     k.err = a.err;
     k.heavy_first = EP_COMBINE_HEAVY_FIRST && a.T <= kHeavyFirstMaxT ? 1 : 0;
+    k.wide = 0;
     if (a.T == 0)
         return cudaSuccess;
     return launch_ec(k, a.out_dtype == EP_FP32, stream);
@@ -955,6 +1007,7 @@ cudaError_t launch_rank_combine(const RankCombineLaunch& a, cudaStream_t stream)
     k.rank_row = a.rank_row;
     k.out = a.out;
     k.err = a.err;
+    k.wide = wide_loads(a.y, a.H, a.T);
     return launch_combine<kSrcRanks, kTcVec, kTcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0, stream);
 }
 

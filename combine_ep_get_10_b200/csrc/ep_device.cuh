@@ -143,6 +143,14 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p)
     return r;
 }
 
+// 32 bytes (256-bit load, sm_100) into two 16-byte halves; p 32-byte aligned.
+__device__ __forceinline__ void ld_nc_v8(const void* p, uint4& lo, uint4& hi)
+{
+    asm("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+        : "l"(p));
+}
+
 __device__ __forceinline__ uint2 ld_nc_v2(const void* p)
 {
     uint2 r;
@@ -158,6 +166,12 @@ __device__ __forceinline__ void st_cs_v2(void* p, uint2 v)
 __device__ __forceinline__ void st_cs_v4(void* p, uint4 v)
 {
     asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v)
+{
+    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
 }
 

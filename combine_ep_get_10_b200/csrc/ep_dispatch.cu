@@ -34,6 +34,10 @@ namespace {
 
 constexpr int64_t kChunkTarget = EP_DISPATCH_CHUNK; // bytes per bulk-copy item
 
+#ifndef EP_QUANT_BULK_SCALES
+#define EP_QUANT_BULK_SCALES 0
+#endif
+
 // Dispatch kernels are launched with programmatic stream serialisation: when
 // the kernel before them is a layout (which lets its dependents start at
 // once), their CTAs start while it runs, load their source rows, and wait for
@@ -601,8 +605,12 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
     __syncthreads();
 
     const bool bulk_codes = (code_row & 15) == 0;
+    // A scale row is small (224 bytes at 7168 channels): one bulk copy each
+    // would double the copy engine's operations per token for 3% of the
+    // bytes, so scales leave by plain 16-byte stores from the threads (or by
+    // the copy engine, EP_QUANT_BULK_SCALES)
     const bool bulk_scales =
-        kCopy || ((scale_row & 15) == 0 && (reinterpret_cast<uintptr_t>(a.scales) & 15) == 0);
+        kCopy || (EP_QUANT_BULK_SCALES && (scale_row & 15) == 0 && (reinterpret_cast<uintptr_t>(a.scales) & 15) == 0);
     if (bulk_codes) {
         bool issued = false;
         for (int k = tid; k < a.map.K; k += kQuantThreads) {
@@ -627,7 +635,18 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
                 st_v2(dst + i * 8, *reinterpret_cast<const uint2*>(s_codes + i * 8));
         }
     }
-    if (!kCopy && !(bulk_codes && bulk_scales)) {
+    if (!kCopy && !(bulk_codes && bulk_scales) && (scale_row & 15) == 0 &&
+        (reinterpret_cast<uintptr_t>(a.scales) & 15) == 0) {
+        // every (destination, 16-byte vector) pair of the scale rows by one thread
+        const int vpr = scale_row / 16;
+        for (int i = tid; i < a.map.K * vpr; i += kQuantThreads) {
+            const int k = i / vpr;
+            const int64_t rk = rows[k];
+            if (rk >= 0)
+                st_v4(static_cast<uint8_t*>(a.scales) + rk * scale_row + (i - k * vpr) * 16,
+                      *reinterpret_cast<const uint4*>(s_scales + (i - k * vpr) * 16));
+        }
+    } else if (!kCopy && !(bulk_codes && bulk_scales)) {
         // scales by plain stores (per-token: 4 bytes; rows not 16-byte multiples)
         for (int k = 0; k < a.map.K; ++k) {
             const int64_t rk = rows[k];

@@ -568,3 +568,40 @@ def test_num_valid_host_reports_the_filled_rows():
     B.ep_get_layout(routing, lay)
     assert lay.num_valid == int(oracle.ec_layout(ti, c["T"], 1)["token_offsets"][-1])
     assert B.ep_get_device_error(lay) == 0
+
+
+
+@pytest.mark.parametrize("T,H", [(8192, 512), (9000, 264)])
+def test_tc_combine_large_batches_every_output(T, H):
+    """From 8192 tokens on, the token-choice and per-rank combines read pairs
+    of 16-byte vectors with one 32-byte load when the rows allow it (H = 512
+    here; H = 264 keeps 16-byte loads): every output element against the
+    oracle, fp32 and bf16, from NaN-filled buffers."""
+    r = rng(41)
+    E, R, K = 64, 8, 6
+    idx = W.random_topk(r, T, E, K, p_neg=0.1)
+    x = W.to_bf16_bits(r.standard_normal((T, H)).astype(np.float32))
+    w = r.random((T, K)).astype(np.float32)
+    ref_l = oracle.tc_layout(idx, E, R)
+    routing, lay, flags = gpu_tc_layout(idx, E, R)
+    assert flags == 0
+    n = int(ref_l["expert_offsets"][-1])
+    y = W.to_bf16_bits(r.standard_normal((n, H)).astype(np.float32))
+    yd = to_dev(y, bf16=True)
+    for dt, bf in ((W.FP32, False), (W.BF16, True)):
+        out = nan_filled((T, H), torch.float32 if dt == W.FP32 else torch.bfloat16)
+        B.ep_combine(yd, routing, lay, to_dev(w), out)
+        ref = oracle.tc_combine(y, idx, E, ref_l, w, out_dtype=dt)
+        assert_combine_close(host(out), ref, bf, "large-batch combine")
+        assert exact_fraction(host(out), ref) == 1.0
+    # per rank: the rank rows of the same routing, summed per token
+    ref_rl = oracle.rank_layout(ref_l["is_token_in_rank"])
+    rl = B.RankLayout(routing)
+    B.ep_get_rank_layout(routing, lay, rl)
+    nr = int(ref_rl["rank_offsets"][-1])
+    yr = W.to_bf16_bits(r.standard_normal((nr, H)).astype(np.float32))
+    rout = nan_filled((T, H), torch.float32)
+    B.ep_combine_ranks(to_dev(yr, bf16=True), routing, lay, rl, rout)
+    ref_r = oracle.rank_combine(yr, ref_rl, out_dtype=W.FP32)
+    assert np.array_equal(host(rout).view(np.uint32), ref_r.view(np.uint32))
+    assert B.ep_get_device_error(lay) == 0
