@@ -27,9 +27,9 @@ the layout are the W processes, and the step is
 so a token's result is the two-level sum (per rank, then over ranks) that
 DeepEP's combine forms.  The transfers are ``torch.distributed``
 all-to-all-v calls (NCCL over NVLink between GPUs, gloo between CPU
-processes): the counts on the host size the receive buffers, which is the
-one host synchronisation of a step.  bf16 rows travel as their 16-bit
-patterns.  No transfer here uses TMA multicast or hands a peer's memory to a
+processes; device tensors are staged through host memory for gloo): the
+counts on the host size the receive buffers, which is the one host
+synchronisation of a step.  bf16 rows travel as their 16-bit patterns.  No transfer here uses TMA multicast or hands a peer's memory to a
 library kernel.
 
 The compute steps are the CUDA kernels of the C ABI (``CudaRowOps``); the
@@ -45,14 +45,21 @@ import torch.distributed as dist
 
 
 # ------------------------------------------------------------------ protocol
+def _host_transport(t: torch.Tensor, group) -> bool:
+    """gloo moves host tensors only: device tensors are staged through host
+    memory (a process group of CPU processes sharing a GPU, or a test)."""
+    return t.is_cuda and dist.get_backend(group) == "gloo"
+
+
 def exchange_counts(send_counts: torch.Tensor, group=None) -> torch.Tensor:
     """send_counts[j] = rows this rank sends to rank j (int64 [W]); returns
     recv_counts[i] = rows rank i sends to this rank."""
     if send_counts.dtype != torch.int64 or send_counts.dim() != 1:
         raise TypeError("send_counts must be an int64 vector of one entry per rank")
-    recv_counts = torch.empty_like(send_counts)
-    dist.all_to_all_single(recv_counts, send_counts, group=group)
-    return recv_counts
+    wire = send_counts.cpu() if _host_transport(send_counts, group) else send_counts
+    recv_counts = torch.empty_like(wire)
+    dist.all_to_all_single(recv_counts, wire, group=group)
+    return recv_counts.to(send_counts.device)
 
 
 def exchange_rows(send: torch.Tensor, send_splits: list[int], recv_splits: list[int], group=None) -> torch.Tensor:
@@ -67,9 +74,14 @@ def exchange_rows(send: torch.Tensor, send_splits: list[int], recv_splits: list[
     if bf16 and send.shape[-1] % 2 != 0:
         raise ValueError("bf16 rows travel in pairs: the last dimension must be even")
     wire = send.view(torch.int32) if bf16 else send
-    recv = torch.empty((sum(recv_splits),) + tuple(wire.shape[1:]), dtype=wire.dtype, device=send.device)
+    staged = _host_transport(wire, group)
+    if staged:
+        wire = wire.cpu()
+    recv = torch.empty((sum(recv_splits),) + tuple(wire.shape[1:]), dtype=wire.dtype, device=wire.device)
     dist.all_to_all_single(recv, wire, output_split_sizes=list(recv_splits),
                            input_split_sizes=list(send_splits), group=group)
+    if staged:
+        recv = recv.to(send.device)
     return recv.view(torch.bfloat16) if bf16 else recv
 
 
@@ -114,7 +126,7 @@ class ExpertParallel:
         send = self.ops.rank_rows(x, topk_idx, topk_weights, self.num_experts, self.world)
         if len(send.counts) != self.world:
             raise ValueError("rank_rows returned %d counts for %d ranks" % (len(send.counts), self.world))
-        send_counts = torch.tensor(send.counts, dtype=torch.int64, device=self._wire_device(x))
+        send_counts = torch.tensor(send.counts, dtype=torch.int64, device=x.device)
         recv_counts = exchange_counts(send_counts, self.group).tolist()
         rx = exchange_rows(send.x, send.counts, recv_counts, self.group)
         ridx = exchange_rows(send.topk_idx, send.counts, recv_counts, self.group)
@@ -134,10 +146,6 @@ class ExpertParallel:
         back = exchange_rows(y, recv.recv_counts, recv.send.counts, self.group)
         return self.ops.combine_ranks(back, recv.send.handle, out_dtype)
 
-    def _wire_device(self, x):
-        # NCCL moves device tensors; gloo host tensors
-        backend = dist.get_backend(self.group)
-        return x.device if backend == "nccl" else torch.device("cpu")
 
 
 # ------------------------------------------------------------ compute steps

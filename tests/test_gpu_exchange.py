@@ -77,3 +77,78 @@ def test_exchange_on_one_rank_matches_the_oracle():
             yf[a:b] = oracle.f32_to_bf16((oracle.bf16_to_f32(yf[a:b]) * np.float32(e + 1)).astype(np.float32))
     ref = oracle.tc_combine(yf, idx, E, L, w, out_dtype=oracle.BF16)
     assert np.array_equal(host(out), ref)
+
+
+def _two_rank_worker(rank, world, port, q):
+    import os
+    import sys
+    from datetime import timedelta
+
+    import torch.distributed as dist
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    sys.path.insert(0, os.path.join(root, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        from combine_ep_get_10_b200.ep_exchange import ExpertParallel
+        from test_ep_exchange_cpu import E, _inputs
+
+        ep = ExpertParallel(E)  # the CUDA compute steps
+        x, idx, w = _inputs(rank, world)
+        recv = ep.dispatch(to_dev(x, bf16=True), to_dev(idx), to_dev(w))
+        first = rank * (E // world)
+
+        def experts(rows, offsets):
+            out = torch.empty_like(rows)
+            off = offsets.tolist()
+            for j in range(len(off) - 1):
+                if off[j + 1] > off[j]:
+                    out[off[j]:off[j + 1]] = (rows[off[j]:off[j + 1]].float() * (first + j + 1)).to(torch.bfloat16)
+            return out
+
+        y = ep.experts(recv, experts)
+        out = ep.combine(y, recv, torch.bfloat16)
+        torch.cuda.synchronize()
+        q.put((rank, "ok", host(out)))
+        dist.barrier()
+    except BaseException:
+        import traceback
+
+        q.put((rank, "error", traceback.format_exc()))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+def test_exchange_two_ranks_sharing_the_gpu():
+    """Two processes on the one GPU, each a rank of a gloo group (rows staged
+    through host memory): the CUDA compute steps of both ranks and the
+    protocol between them give each rank the single-process oracle's
+    two-level result bit for bit.  No kernel waits on the other process."""
+    import torch.multiprocessing as mp
+
+    from test_ep_exchange_cpu import _reference
+
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_two_rank_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    try:
+        for _ in range(world):
+            item = q.get(timeout=300)
+            assert item[1] == "ok", "rank %d failed:\n%s" % (item[0], item[2])
+            res[item[0]] = item[2]
+    finally:
+        for p in procs:
+            p.join(timeout=120 if len(res) == world else 5)
+            if p.exitcode is None:
+                p.kill()
+    ref = _reference(oracle, world)
+    for r in range(world):
+        assert np.array_equal(res[r], ref[r]["two_bf16"]), r
