@@ -147,7 +147,6 @@ class ExpertParallel:
         return self.ops.combine_ranks(back, recv.send.handle, out_dtype)
 
 
-
 # ------------------------------------------------------------ compute steps
 class CudaRowOps:
     """The compute steps on the GPU, through the C ABI."""

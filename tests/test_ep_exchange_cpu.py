@@ -2,7 +2,8 @@
 combine_ep_get_10_b200/ep_exchange.py on 2 and 4 gloo ranks on CPU.
 
 Each rank holds its own token batch (the prefill routing recipe at a small
-size: 256 experts, top-8, sigmoid router with bias), and rank r owns experts
+size: 256 experts, top-8, sigmoid router with bias; 48 + 20 r tokens on rank
+r, so the counts differ in both directions), and rank r owns experts
 [r*E/W, (r+1)*E/W).  The compute steps run in the CPU oracle (the CUDA
 kernels need a GPU); what is under test is the protocol: the counts exchange,
 the receive-buffer sizes, the all-to-all-v of rows and their top-k entries,
@@ -29,7 +30,12 @@ import torch
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-E, H, T = 256, 128, 48
+E, H = 256, 128
+
+
+def tokens_of(rank):
+    """Uneven batches: rank r holds 48 + 20 r tokens."""
+    return 48 + 20 * rank
 
 
 def _free_port():
@@ -46,6 +52,7 @@ def _inputs(rank, world):
     the layout allows), so that single-rank and multi-rank tokens both occur."""
     from combine_ep_get_10_b200 import workloads as W
 
+    T = tokens_of(rank)
     inp = W.make_inputs(2, seed=7000 + rank, T=T)
     x = np.ascontiguousarray(inp["x"][:, :H])
     idx = inp["topk_idx"].copy()
@@ -185,6 +192,7 @@ def _reference(oracle, world):
         flat = oracle.tc_combine(yf, idx, E, LF, w, out_dtype=oracle.FP32)
         flat_bf16 = oracle.tc_combine(yf, idx, E, LF, w, out_dtype=oracle.BF16)
         # |w * y| summed per token, for the tolerance of multi-rank tokens
+        T = tokens_of(i)
         mag = np.zeros((T, H), np.float64)
         for t in range(T):
             for k in range(idx.shape[1]):

@@ -123,16 +123,17 @@ def _two_rank_worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_exchange_two_ranks_sharing_the_gpu():
-    """Two processes on the one GPU, each a rank of a gloo group (rows staged
-    through host memory): the CUDA compute steps of both ranks and the
+@pytest.mark.parametrize("world", [2, 4])
+def test_exchange_ranks_sharing_the_gpu(world):
+    """2 or 4 processes on the one GPU, each a rank of a gloo group (rows
+    staged through host memory): the CUDA compute steps of every rank and the
     protocol between them give each rank the single-process oracle's
-    two-level result bit for bit.  No kernel waits on the other process."""
+    two-level result bit for bit.  No kernel waits on another process."""
     import torch.multiprocessing as mp
 
     from test_ep_exchange_cpu import _reference
 
-    world, port = 2, _free_port()
+    port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     procs = [ctx.Process(target=_two_rank_worker, args=(r, world, port, q)) for r in range(world)]
