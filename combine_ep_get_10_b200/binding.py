@@ -31,7 +31,7 @@ EP_DEVERR_BAD_INDEX, EP_DEVERR_OVERFLOW, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 EXPORTED = ("ep_workspace_bytes", "ep_workspace_init", "ep_get_layout", "ep_dispatch", "ep_combine",
             "ep_dispatch_expert_choice", "ep_combine_expert_choice", "ep_get_device_error", "ep_status_string",
             "ep_version", "ep_get_layout_no_alloc", "ep_get_rank_layout", "ep_dispatch_ranks", "ep_combine_ranks",
-            "ep_dispatch_low_latency")
+            "ep_dispatch_low_latency", "ep_layout_dispatch")
 
 
 class EPError(RuntimeError):
@@ -103,6 +103,8 @@ def lib():
         L.ep_combine_ranks.argtypes = [P, i32, i64, RP, LP, KP, P, st, P]
         L.ep_dispatch_low_latency.restype = st
         L.ep_dispatch_low_latency.argtypes = [P, i32, RP, LP, i32, st, P, P, P, P, P, P]
+        L.ep_layout_dispatch.restype = st
+        L.ep_layout_dispatch.argtypes = [P, i32, RP, LP, st, i32, i64, st, P, P, P, P, P, P]
         if L.ep_version() != EP_ABI_VERSION:
             raise ImportError("libep_b200.so has ABI version %d, the binding expects %d; rebuild it"
                               % (L.ep_version(), EP_ABI_VERSION))
@@ -300,6 +302,19 @@ def ep_dispatch(x: torch.Tensor, routing: Routing, layout: Layout, recv_x: torch
     _check(lib().ep_dispatch(_ptr(x), x.shape[1], ctypes.byref(routing.desc), ctypes.byref(layout.desc), int(mode),
                              int(max_tokens_per_expert), rows, out_dtype, _ptr(topk_weights), _ptr(recv_x),
                              _ptr(recv_scales), _ptr(recv_src), _ptr(recv_weights), _stream(stream)), "ep_dispatch")
+
+
+def ep_layout_dispatch(x: torch.Tensor, routing: Routing, layout: Layout, recv_x: torch.Tensor, *,
+                       mode=EP_LAYOUT_COMPACT, max_tokens_per_expert=0, num_recv_rows=None, topk_weights=None,
+                       recv_scales=None, recv_src=None, recv_weights=None, out_dtype=None, stream=None) -> None:
+    """ep_get_layout + ep_dispatch in one call (the dispatch's row loads
+    overlap the layout kernel); arguments as for ep_dispatch."""
+    out_dtype = _dtype_code(recv_x) if out_dtype is None else int(out_dtype)
+    rows = recv_x.shape[0] if num_recv_rows is None else int(num_recv_rows)
+    _check(lib().ep_layout_dispatch(_ptr(x), x.shape[1], ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                                    int(mode), int(max_tokens_per_expert), rows, out_dtype, _ptr(topk_weights),
+                                    _ptr(recv_x), _ptr(recv_scales), _ptr(recv_src), _ptr(recv_weights),
+                                    _stream(stream)), "ep_layout_dispatch")
 
 
 def ep_dispatch_low_latency(x: torch.Tensor, routing: Routing, layout: Layout, recv_x: torch.Tensor, *,

@@ -263,6 +263,31 @@ ep_status_t check_dispatch_args(const void* x, int32_t hidden, const ep_routing_
     return EP_OK;
 }
 
+// The dispatch launch of ep_dispatch (early_load 0: wait for the kernel
+// before, whatever it is, before reading anything) and of ep_layout_dispatch
+// (early_load 1: the kernel before is this library's layout, launched just
+// now on the same stream).  Arguments are checked by the caller.
+ep_status_t launch_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                            const ep_layout_t* layout, ep_buffer_mode_t mode, int32_t max_tokens_per_expert,
+                            int64_t num_recv_rows, ep_dtype_t out_dtype, const float* topk_weights, void* recv_x,
+                            void* recv_scales, int32_t* recv_src, float* recv_weights, ep_stream_t stream,
+                            bool early_load)
+{
+    ep::TcDispatchLaunch a{x,
+                           routing->num_tokens,
+                           hidden,
+                           tc_rows(routing, layout, mode, max_tokens_per_expert, num_recv_rows),
+                           static_cast<int32_t>(out_dtype),
+                           topk_weights,
+                           recv_x,
+                           recv_scales,
+                           recv_src,
+                           recv_weights,
+                           ep::error_word(layout->workspace),
+                           early_load ? 1 : 0};
+    return from_cuda(ep::launch_tc_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 } // namespace
 
 extern "C" {
@@ -277,19 +302,29 @@ ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* 
                                          out_dtype, topk_weights, recv_x, recv_scales, recv_src, recv_weights);
     if (st != EP_OK)
         return st;
-    const int32_t T = routing->num_tokens;
-    ep::TcDispatchLaunch a{x,
-                           T,
-                           hidden,
-                           tc_rows(routing, layout, mode, max_tokens_per_expert, num_recv_rows),
-                           static_cast<int32_t>(out_dtype),
-                           topk_weights,
-                           recv_x,
-                           recv_scales,
-                           recv_src,
-                           recv_weights,
-                           ep::error_word(layout->workspace)};
-    return from_cuda(ep::launch_tc_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+    return launch_dispatch(x, hidden, routing, layout, mode, max_tokens_per_expert, num_recv_rows, out_dtype,
+                           topk_weights, recv_x, recv_scales, recv_src, recv_weights, stream, false);
+}
+
+ep_status_t ep_layout_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                               const ep_layout_t* layout, ep_buffer_mode_t mode, int32_t max_tokens_per_expert,
+                               int64_t num_recv_rows, ep_dtype_t out_dtype, const float* topk_weights, void* recv_x,
+                               void* recv_scales, int32_t* recv_src, float* recv_weights, ep_stream_t stream)
+{
+    CallRange range_("ep_layout_dispatch");
+    // the dispatch's checks first: nothing is launched unless both calls can run
+    ep_status_t st = check_dispatch_args(x, hidden, routing, layout, mode, max_tokens_per_expert, num_recv_rows,
+                                         out_dtype, topk_weights, recv_x, recv_scales, recv_src, recv_weights);
+    if (st != EP_OK)
+        return st;
+    st = get_layout(routing, layout, stream);
+    if (st != EP_OK)
+        return st;
+    st = launch_dispatch(x, hidden, routing, layout, mode, max_tokens_per_expert, num_recv_rows, out_dtype,
+                         topk_weights, recv_x, recv_scales, recv_src, recv_weights, stream, true);
+    if (st != EP_OK)
+        return st;
+    return ep::report_num_valid(routing, layout, reinterpret_cast<cudaStream_t>(stream));
 }
 
 ep_status_t ep_dispatch_low_latency(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
@@ -348,8 +383,8 @@ ep_status_t ep_dispatch_low_latency(const void* x, int32_t hidden, const ep_rout
     } else {
         st = get_layout(routing, layout, stream);
         if (st == EP_OK)
-            st = ep_dispatch(x, hidden, routing, layout, EP_LAYOUT_PADDED, max_tokens_per_expert, rows, out_dtype,
-                             topk_weights, recv_x, recv_scales, recv_src, recv_weights, stream);
+            st = launch_dispatch(x, hidden, routing, layout, EP_LAYOUT_PADDED, max_tokens_per_expert, rows,
+                                 out_dtype, topk_weights, recv_x, recv_scales, recv_src, recv_weights, stream, true);
     }
     if (st != EP_OK)
         return st;

@@ -38,10 +38,15 @@ constexpr int64_t kChunkTarget = EP_DISPATCH_CHUNK; // bytes per bulk-copy item
 #define EP_QUANT_BULK_SCALES 0
 #endif
 
-// Dispatch kernels are launched with programmatic stream serialisation: when
-// the kernel before them is a layout (which lets its dependents start at
-// once), their CTAs start while it runs, load their source rows, and wait for
-// the layout's results (griddepcontrol.wait) before reading them.
+// Dispatch kernels are launched with programmatic stream serialisation.  By
+// default a dispatch waits for the kernel before it (griddepcontrol.wait)
+// before it reads anything: that kernel may have written x or the routing,
+// and its writes are only guaranteed visible after the wait.  When the
+// library itself has just launched the layout on the stream
+// (ep_layout_dispatch: the kernel before is that layout, which lets its
+// dependents start at once and writes neither x nor the routing), the
+// dispatch's CTAs start while the layout runs, load their source rows, and
+// wait only before reading the layout's results (early_load).
 #ifndef EP_DISPATCH_PDL
 #define EP_DISPATCH_PDL 1
 #endif
@@ -117,6 +122,7 @@ struct BulkArgs {
     float* recv_topk_weights;
     uint32_t* err;
     int64_t item_base; // first item of this launch
+    int32_t early_load; // load source rows before waiting for the kernel before (see launch_pdl)
 };
 
 enum BulkSrc : int {
@@ -161,14 +167,14 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
     const uint32_t bytes = static_cast<uint32_t>(min(a.chunk_bytes, a.row_bytes - off));
     uint32_t errbits = 0;
 
+    if (!a.early_load)
+        pdl_wait(); // the kernel before may have written x or the routing
     int64_t src_row;
     if (kExpertChoice) {
         const int t = __ldg(a.token_indices + r);
         if (t < 0 || t >= a.T) {
-            if (lane == 0 && c == 0 && t != -1) {
-                pdl_wait(); // the error word is shared with the layout before
+            if (lane == 0 && c == 0 && t != -1)
                 flag_error(a.err, EP_DEVERR_BAD_INDEX);
-            }
             return;
         }
         src_row = t;
@@ -182,7 +188,8 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
         mbar_arrive_expect_tx(&bar, bytes);
         bulk_load_g2s(buf, a.src + src_row * a.row_bytes + off, bytes, &bar);
     }
-    pdl_wait(); // the layout's results (slot, offsets, rank rows) are final from here on
+    if (a.early_load)
+        pdl_wait(); // the layout's results (slot, offsets) are final from here on
     // destination rows of the first 32 pairs while the load is in flight
     int64_t dst_row = -1;
     if constexpr (kSrc == kSrcEc) {
@@ -261,6 +268,7 @@ struct QuantArgs {
     int32_t* recv_src;
     float* recv_weights;
     uint32_t* err;
+    int32_t early_load; // load the row before waiting for the kernel before (see launch_pdl)
     // fused low-latency mode: the layout is computed in the same launch
     int32_t T, R;
     int32_t* slot;
@@ -501,6 +509,8 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
     uint8_t* s_scales = qsmem + row_bytes + (kCopy ? 0 : code_row);
     int64_t* rows = reinterpret_cast<int64_t*>(s_scales + ((scale_row + 15) & ~15));
 
+    if (!a.early_load)
+        pdl_wait(); // the kernel before may have written x or the routing
     if (tid == 0) {
         mbar_init(&bar, 1);
         fence_mbar_init();
@@ -508,7 +518,8 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
         bulk_load_g2s(s_x, reinterpret_cast<const uint8_t*>(a.x) + t * static_cast<int64_t>(row_bytes),
                       static_cast<uint32_t>(row_bytes), &bar);
     }
-    pdl_wait(); // the layout's results are final from here on
+    if (a.early_load)
+        pdl_wait(); // the layout's results are final from here on
     uint32_t errbits = 0;
     if constexpr (kFused) {
         fused_layout(a, t, rows, reinterpret_cast<uint32_t*>(rows + a.map.K), errbits);
@@ -768,6 +779,7 @@ cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream)
         k.recv_src = a.recv_src;
         k.recv_weights = a.recv_weights;
         k.err = a.err;
+        k.early_load = a.early_load;
         return launch_quant_fmt<false>(a.out_dtype, k, a.T, a.rows.K, stream);
     }
     BulkArgs k{};
@@ -782,6 +794,7 @@ cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream)
     k.recv_src = a.recv_src;
     k.recv_weights = a.recv_weights;
     k.err = a.err;
+    k.early_load = a.early_load;
     return launch_bulk<kSrcTopk>(k, static_cast<int64_t>(a.T) * k.nchunks, stream);
 }
 

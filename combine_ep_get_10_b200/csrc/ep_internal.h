@@ -83,6 +83,7 @@ struct TcDispatchLaunch {
     int32_t* recv_src;
     float* recv_weights;
     uint32_t* err;
+    int32_t early_load; // 1 only right after this library's own layout launch on the stream
 };
 cudaError_t launch_tc_dispatch(const TcDispatchLaunch& a, cudaStream_t stream);
 

@@ -213,6 +213,22 @@ EP_API ep_status_t ep_dispatch(const void* x, int32_t hidden, const ep_routing_d
                         ep_dtype_t out_dtype, const float* topk_weights, void* recv_x, void* recv_scales,
                         int32_t* recv_src, float* recv_weights, ep_stream_t stream);
 
+/* Layout and dispatch in one call ([README] API Overview: get_dispatch_layout
+ * followed by dispatch): exactly ep_get_layout(routing, layout) followed by
+ * ep_dispatch(x, hidden, routing, layout, mode, ...), with the same outputs,
+ * arguments and errors (nothing is launched unless both calls' arguments
+ * pass).  Being the library's own back-to-back launches, the dispatch's
+ * threads start while the layout kernel runs and load their source rows
+ * before waiting for it; ep_dispatch alone must first wait for whatever
+ * kernel precedes it on the stream, which may have written x.
+ * layout->workspace must have ep_workspace_bytes() bytes;
+ * layout->num_valid_host is honoured as by ep_get_layout. */
+EP_API ep_status_t ep_layout_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                      const ep_layout_t* layout, ep_buffer_mode_t mode, int32_t max_tokens_per_expert,
+                                      int64_t num_recv_rows, ep_dtype_t out_dtype, const float* topk_weights,
+                                      void* recv_x, void* recv_scales, int32_t* recv_src, float* recv_weights,
+                                      ep_stream_t stream);
+
 /* Low-latency dispatch ([README] API Overview: low_latency_dispatch, which
  * takes topk_idx and num_max_dispatch_tokens_per_rank and needs no separate
  * layout call): exactly ep_get_layout(routing, layout) followed by

@@ -168,6 +168,21 @@ def test_token_rounds_cover_the_batch_in_order():
         B.token_rounds(10, 0)
 
 
+def test_layout_dispatch_checks_both_calls_before_launching(L):
+    """ep_layout_dispatch rejects what either ep_dispatch or ep_get_layout
+    would reject, before anything is launched (no GPU here)."""
+    desc = _topk_desc()
+    good_ws = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x100000, 1 << 20)
+    call = lambda lay, hidden=256, x=0x2000: L.ep_layout_dispatch(  # noqa: E731
+        x, hidden, ctypes.byref(desc), ctypes.byref(lay), 0, 0, 32, 0, None, 0x4000, None, None, None, None)
+    assert call(good_ws, hidden=12) == 1  # hidden not a multiple of 8
+    assert call(good_ws, x=0x2008) == 1  # x not 16-byte aligned
+    small = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x100000, 256)
+    assert call(small) == 4  # the layout needs its whole workspace
+    no_counts = B.LayoutDesc(None, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x100000, 1 << 20)
+    assert call(no_counts) == 1
+
+
 def test_binding_constants_match_the_header():
     """Every enum value and device-error bit of include/ep.h has the same value
     in the binding (the binding marshals them as plain ints)."""

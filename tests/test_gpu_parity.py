@@ -605,3 +605,55 @@ def test_tc_combine_large_batches_every_output(T, H):
     ref_r = oracle.rank_combine(yr, ref_rl, out_dtype=W.FP32)
     assert np.array_equal(host(rout).view(np.uint32), ref_r.view(np.uint32))
     assert B.ep_get_device_error(lay) == 0
+
+
+def test_layout_dispatch_one_call_equals_the_two_calls():
+    """ep_layout_dispatch: the layout and the dispatch in one call (the
+    dispatch's row loads overlap the layout kernel) writes the same layout,
+    rows and quantised codes as ep_get_layout + ep_dispatch, against the
+    oracle, and reports the filled rows through num_valid_host."""
+    inp = inputs(2, T=2048)
+    c = inp["cfg"]
+    x, idx, w = inp["x"], inp["topk_idx"], inp["topk_weights"]
+    E, R, H = c["E"], c["R"], c["H"]
+    ref_l = oracle.tc_layout(idx, E, R)
+    n = int(ref_l["expert_offsets"][-1])
+    routing = B.Routing.topk(to_dev(idx), E, R)
+    lay = B.Layout(routing, report_num_valid=True)
+    recv = to_dev(np.full((n, H), 0x7FC1, np.uint16), bf16=True)
+    B.ep_layout_dispatch(to_dev(x, bf16=True), routing, lay, recv)
+    assert lay.num_valid == n
+    check_tc_layout(lay, ref_l)
+    assert np.array_equal(host(recv), oracle.tc_dispatch(x, idx, E, ref_l)["recv"])
+    q = torch.zeros((n, H), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros((n, H // 128), dtype=torch.float32, device="cuda")
+    B.ep_layout_dispatch(to_dev(x, bf16=True), routing, lay, q, recv_scales=sc, topk_weights=to_dev(w),
+                         recv_weights=(rw := torch.zeros(n, dtype=torch.float32, device="cuda")))
+    ref_q = oracle.tc_dispatch(x, idx, E, ref_l, out_dtype=W.FP8_E4M3, topk_weights=w, want_weights=True)
+    assert np.array_equal(host(q), ref_q["recv"])
+    assert np.array_equal(host(sc).view(np.uint32), ref_q["recv_scales"].view(np.uint32))
+    assert np.array_equal(host(rw), ref_q["recv_weights"])
+    assert B.ep_get_device_error(lay) == 0
+
+
+def test_dispatch_reads_x_written_by_the_kernel_just_before():
+    """ep_dispatch after a kernel that writes x on the same stream (the
+    layout computed earlier): the dispatch waits for that kernel before its
+    first read, so every dispatched row is the new x."""
+    inp = inputs(2, T=1024)
+    c = inp["cfg"]
+    idx = inp["topk_idx"]
+    E, R, H = c["E"], c["R"], c["H"]
+    ref_l = oracle.tc_layout(idx, E, R)
+    n = int(ref_l["expert_offsets"][-1])
+    routing, lay, flags = gpu_tc_layout(idx, E, R)
+    assert flags == 0
+    r = rng(5)
+    xd = torch.empty((1024, H), dtype=torch.bfloat16, device="cuda")
+    recv = torch.empty((n, H), dtype=torch.bfloat16, device="cuda")
+    for it in range(4):
+        x = W.to_bf16_bits(r.standard_normal((1024, H)).astype(np.float32))
+        src = to_dev(x, bf16=True)
+        xd.copy_(src)  # a kernel on the stream writing x right before the dispatch
+        B.ep_dispatch(xd, routing, lay, recv)
+        assert np.array_equal(host(recv), oracle.tc_dispatch(x, idx, E, ref_l)["recv"]), it
