@@ -59,7 +59,8 @@ def parse():
     ap.add_argument("--quant", action="store_true",
                     help="with --workloads: also time every quantised dispatch format on the token-choice workloads")
     ap.add_argument("--ranks", action="store_true",
-                    help="with --workloads: also time the per-rank (deduplicated) dispatch and combine")
+                    help="with --workloads: also time the per-rank (deduplicated) dispatch and combine, "
+                         "and the same over peer memory with the ranks emulated on this GPU")
     ap.add_argument("--rounds", type=int, default=0,
                     help="with --workloads: also time the whole batch in rounds of this many tokens "
                          "(per-round layout, dispatch and combine; receive buffer of one round)")
@@ -603,6 +604,41 @@ QUANT_FORMATS = [
 ]
 
 
+def time_peer_path(cfg, x, w, rt, lay, rl, n_rank, dev, timeit, emit):
+    """The per-rank path over peer memory, its R ranks emulated on this GPU:
+    this process is rank R/2 of R ranks that all hold this routing (so every
+    row of the counts matrix is this rank's num_tokens_per_rank), and each
+    rank's receive, entry, source and partial-row buffers are separate
+    allocations here.  The dispatch stores this rank's (token, rank) rows
+    into the R ranks' buffers at their offsets behind ranks 0 .. R/2-1, and
+    the combine reads them back from there: the same bytes as
+    dispatch_ranks / combine_ranks, over local HBM instead of NVLink."""
+    import torch
+
+    from combine_ep_get_10_b200 import binding as B
+
+    T, H, K, R = cfg["T"], cfg["H"], cfg["K"], cfg["R"]
+    me = R // 2
+    counts = lay.num_tokens_per_rank.to(torch.int32)
+    capacity = (me + 1) * int(counts.max().item())
+    bufs = dict(recv_x=[torch.empty((capacity, H), dtype=torch.bfloat16, device=dev) for _ in range(R)],
+                y=[torch.randn((capacity, H), device=dev).to(torch.bfloat16) for _ in range(R)],
+                idx=[torch.empty((capacity, K), dtype=torch.int64, device=dev) for _ in range(R)],
+                w=[torch.empty((capacity, K), dtype=torch.float32, device=dev) for _ in range(R)],
+                src=[torch.empty((capacity,), dtype=torch.int32, device=dev) for _ in range(R)],
+                counts=[counts.repeat(R, 1).contiguous() for _ in range(R)])
+    tab = {k: torch.tensor([t.data_ptr() for t in v], dtype=torch.int64, device=dev) for k, v in bufs.items()}
+    peers = B.Peers(me, capacity, tab["recv_x"], tab["y"], tab["counts"], recv_topk_idx=tab["idx"],
+                    recv_topk_weights=tab["w"], recv_src=tab["src"])
+    emit(cfg, "dispatch_peers_emulated",
+         timeit(lambda: B.ep_dispatch_peers(x, rt, lay, rl, peers, topk_weights=w)),
+         T * H * 2 + n_rank * H * 2 + n_rank * K * 12 + n_rank * 4 + T * R * 4 + T * K * 12, T)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    emit(cfg, "combine_peers_emulated", timeit(lambda: B.ep_combine_peers(rt, lay, rl, peers, out)),
+         n_rank * H * 2 + T * H * 2 + T * R * 4, T)
+    del bufs, tab, peers, out
+
+
 def run_workload_table(args):
     """Per-op timings on every workload (layout, dispatch, combine; expert
     choice for workload 4): one JSON line per (workload, op), L2 flushed
@@ -746,6 +782,7 @@ def run_workload_table(args):
                 print(json.dumps({"workload": cfg["name"], "rank_rows": n_rank, "expert_rows": n_valid,
                                   "rows_saved": round(1 - n_rank / max(n_valid, 1), 3)}), flush=True)
                 del rrecv, ridx, rwt, rout
+                time_peer_path(cfg, x, w, rt, lay, rl, n_rank, dev, timeit, emit)
             if args.quant:
                 del recv
                 for name, dt, code_b, scale_b in QUANT_FORMATS:

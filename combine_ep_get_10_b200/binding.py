@@ -16,7 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libep_b200.so")
 
 # ABI version and enums of include/ep.h
-EP_ABI_VERSION = 2  # the structures below follow this version of the header
+EP_ABI_VERSION = 3  # the structures below follow this version of the header
 EP_OK = 0
 EP_ERR_INVALID_ARG, EP_ERR_BAD_INDEX, EP_ERR_OVERFLOW, EP_ERR_WORKSPACE = 1, 2, 3, 4
 EP_ERR_CUDA, EP_ERR_UNSUPPORTED, EP_ERR_TIMEOUT = 5, 6, 7
@@ -31,7 +31,8 @@ EP_DEVERR_BAD_INDEX, EP_DEVERR_OVERFLOW, EP_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 EXPORTED = ("ep_workspace_bytes", "ep_workspace_init", "ep_get_layout", "ep_dispatch", "ep_combine",
             "ep_dispatch_expert_choice", "ep_combine_expert_choice", "ep_get_device_error", "ep_status_string",
             "ep_version", "ep_get_layout_no_alloc", "ep_get_rank_layout", "ep_dispatch_ranks", "ep_combine_ranks",
-            "ep_dispatch_low_latency", "ep_layout_dispatch")
+            "ep_dispatch_low_latency", "ep_layout_dispatch", "ep_peer_alloc", "ep_peer_free", "ep_peer_open",
+            "ep_peer_close", "ep_peer_publish_counts", "ep_dispatch_peers", "ep_combine_peers")
 
 
 class EPError(RuntimeError):
@@ -56,6 +57,13 @@ class LayoutDesc(ctypes.Structure):
 
 class RankLayoutDesc(ctypes.Structure):
     _fields_ = [("rank_offsets", ctypes.c_void_p), ("rank_row", ctypes.c_void_p)]
+
+
+class PeersDesc(ctypes.Structure):
+    _fields_ = [("num_ranks", ctypes.c_int32), ("rank", ctypes.c_int32), ("capacity", ctypes.c_int64),
+                ("recv_x", ctypes.c_void_p), ("recv_topk_idx", ctypes.c_void_p),
+                ("recv_topk_weights", ctypes.c_void_p), ("recv_src", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("rank_counts", ctypes.c_void_p)]
 
 
 _lib = None
@@ -105,6 +113,21 @@ def lib():
         L.ep_dispatch_low_latency.argtypes = [P, i32, RP, LP, i32, st, P, P, P, P, P, P]
         L.ep_layout_dispatch.restype = st
         L.ep_layout_dispatch.argtypes = [P, i32, RP, LP, st, i32, i64, st, P, P, P, P, P, P]
+        PP = ctypes.POINTER(PeersDesc)
+        L.ep_peer_alloc.restype = st
+        L.ep_peer_alloc.argtypes = [ctypes.c_size_t, ctypes.POINTER(P), P]
+        L.ep_peer_free.restype = st
+        L.ep_peer_free.argtypes = [P]
+        L.ep_peer_open.restype = st
+        L.ep_peer_open.argtypes = [P, ctypes.POINTER(P)]
+        L.ep_peer_close.restype = st
+        L.ep_peer_close.argtypes = [P]
+        L.ep_peer_publish_counts.restype = st
+        L.ep_peer_publish_counts.argtypes = [RP, LP, PP, P]
+        L.ep_dispatch_peers.restype = st
+        L.ep_dispatch_peers.argtypes = [P, i32, RP, LP, KP, P, PP, P]
+        L.ep_combine_peers.restype = st
+        L.ep_combine_peers.argtypes = [i32, RP, LP, KP, PP, P, st, P]
         if L.ep_version() != EP_ABI_VERSION:
             raise ImportError("libep_b200.so has ABI version %d, the binding expects %d; rebuild it"
                               % (L.ep_version(), EP_ABI_VERSION))
@@ -400,6 +423,94 @@ def ep_combine_ranks(y: torch.Tensor, routing: Routing, layout: Layout, rank_lay
     _check(lib().ep_combine_ranks(_ptr(y), y.shape[1], rows, ctypes.byref(routing.desc), ctypes.byref(layout.desc),
                                   ctypes.byref(rank_layout.desc), _ptr(out), _dtype_code(out), _stream(stream)),
            "ep_combine_ranks")
+
+
+# ------------------------------------------------------ per rank over peer memory
+EP_IPC_HANDLE_BYTES = 64
+
+
+def ep_peer_alloc(nbytes: int) -> tuple[int, bytes]:
+    """Device memory other processes can map: (address, IPC handle)."""
+    ptr = ctypes.c_void_p()
+    handle = ctypes.create_string_buffer(EP_IPC_HANDLE_BYTES)
+    _check(lib().ep_peer_alloc(int(nbytes), ctypes.byref(ptr), handle), "ep_peer_alloc")
+    return int(ptr.value), handle.raw
+
+
+def ep_peer_free(ptr: int) -> None:
+    _check(lib().ep_peer_free(ctypes.c_void_p(ptr)), "ep_peer_free")
+
+
+def ep_peer_open(handle: bytes) -> int:
+    """Map another process's ep_peer_alloc buffer; returns its address here."""
+    if len(handle) != EP_IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle has %d bytes, got %d" % (EP_IPC_HANDLE_BYTES, len(handle)))
+    ptr = ctypes.c_void_p()
+    _check(lib().ep_peer_open(ctypes.create_string_buffer(handle, EP_IPC_HANDLE_BYTES), ctypes.byref(ptr)),
+           "ep_peer_open")
+    return int(ptr.value)
+
+
+def ep_peer_close(ptr: int) -> None:
+    _check(lib().ep_peer_close(ctypes.c_void_p(ptr)), "ep_peer_close")
+
+
+class _CudaArray:
+    """A device address, shape and element type in the CUDA array interface,
+    for torch.as_tensor to view without a copy."""
+
+    def __init__(self, ptr: int, shape: tuple, typestr: str):
+        self.__cuda_array_interface__ = {"data": (int(ptr), False), "shape": tuple(shape), "typestr": typestr,
+                                         "strides": None, "version": 3}
+
+
+_TYPESTR = {torch.bfloat16: "<i2", torch.int16: "<i2", torch.int32: "<i4", torch.int64: "<i8",
+            torch.float32: "<f4", torch.uint8: "|u1"}
+
+
+def device_view(ptr: int, shape: tuple, dtype: torch.dtype, device) -> torch.Tensor:
+    """A tensor over device memory the library handed out (no copy; the
+    memory must outlive the tensor)."""
+    t = torch.as_tensor(_CudaArray(ptr, shape, _TYPESTR[dtype]), device=device)
+    return t.view(torch.bfloat16) if dtype == torch.bfloat16 else t
+
+
+class Peers:
+    """The descriptor of ep_peers_t over device tables of R addresses each
+    (int64 tensors on this rank's GPU)."""
+
+    def __init__(self, rank: int, capacity: int, recv_x, y, rank_counts, recv_topk_idx=None,
+                 recv_topk_weights=None, recv_src=None):
+        tables = dict(recv_x=recv_x, y=y, rank_counts=rank_counts, recv_topk_idx=recv_topk_idx,
+                      recv_topk_weights=recv_topk_weights, recv_src=recv_src)
+        for name, t in tables.items():
+            if t is not None and (t.dtype != torch.int64 or t.dim() != 1 or t.shape[0] != recv_x.shape[0]):
+                raise ValueError("peer table %s must be an int64 vector of one address per rank" % name)
+        self.tables = tables  # keeps the tables alive
+        self.desc = PeersDesc(recv_x.shape[0], rank, capacity, *(None if tables[n] is None else tables[n].data_ptr()
+                                                                for n in ("recv_x", "recv_topk_idx",
+                                                                          "recv_topk_weights", "recv_src", "y",
+                                                                          "rank_counts")))
+
+
+def ep_peer_publish_counts(routing: Routing, layout: Layout, peers: Peers, stream=None) -> None:
+    _check(lib().ep_peer_publish_counts(ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                                        ctypes.byref(peers.desc), _stream(stream)), "ep_peer_publish_counts")
+
+
+def ep_dispatch_peers(x: torch.Tensor, routing: Routing, layout: Layout, rank_layout: RankLayout, peers: Peers, *,
+                      topk_weights=None, stream=None) -> None:
+    _check(lib().ep_dispatch_peers(_ptr(x), x.shape[1], ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                                   ctypes.byref(rank_layout.desc), _ptr(topk_weights), ctypes.byref(peers.desc),
+                                   _stream(stream)), "ep_dispatch_peers")
+
+
+def ep_combine_peers(routing: Routing, layout: Layout, rank_layout: RankLayout, peers: Peers, out: torch.Tensor, *,
+                     stream=None) -> None:
+    """out dtype follows `out` (bfloat16 or float32)."""
+    _check(lib().ep_combine_peers(out.shape[1], ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                                  ctypes.byref(rank_layout.desc), ctypes.byref(peers.desc), _ptr(out),
+                                  _dtype_code(out), _stream(stream)), "ep_combine_peers")
 
 
 def ep_get_layout_no_alloc(routing: Routing, layout: Layout, device_error_flags: torch.Tensor | None = None,

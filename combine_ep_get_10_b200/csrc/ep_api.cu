@@ -1,8 +1,10 @@
 // ep_api.cu -- the C ABI declared in include/ep.h: argument checks on the
 // host, then one launcher per operation.  Nothing here allocates device
-// memory; only ep_get_device_error, and a layout call given a
-// num_valid_host pointer, synchronise.
+// memory except ep_peer_alloc (buffers other processes map); only
+// ep_get_device_error, and a layout call given a num_valid_host pointer,
+// synchronise.
 #include <cstdint>
+#include <cstring>
 #include <cuda_runtime.h>
 
 #include <nvtx3/nvToolsExt.h>
@@ -507,6 +509,40 @@ ep_status_t check_rank_call(const ep_routing_desc_t* routing, const ep_layout_t*
     return EP_OK;
 }
 
+// Peer tables: one process per rank of the routing; the required tables
+// (recv_x, y, rank_counts) present, every table 8-byte aligned.
+ep_status_t check_peers(const ep_routing_desc_t* routing, const ep_peers_t* p)
+{
+    if (p == nullptr || p->num_ranks != routing->num_ranks || p->rank < 0 || p->rank >= p->num_ranks ||
+        p->capacity < 0)
+        return EP_ERR_INVALID_ARG;
+    const void* required[] = {p->recv_x, p->y, p->rank_counts};
+    for (const void* t : required)
+        if (t == nullptr || !aligned(t, 8))
+            return EP_ERR_INVALID_ARG;
+    const void* optional[] = {p->recv_topk_idx, p->recv_topk_weights, p->recv_src};
+    for (const void* t : optional)
+        if (t != nullptr && !aligned(t, 8))
+            return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+ep::PeerTables peer_tables(const ep_peers_t* p, const ep_rank_layout_t* rank_layout)
+{
+    auto table = [](const void* t) { return static_cast<const unsigned long long*>(t); };
+    ep::PeerTables k{};
+    k.recv_x = table(p->recv_x);
+    k.recv_topk_idx = table(p->recv_topk_idx);
+    k.recv_topk_weights = table(p->recv_topk_weights);
+    k.recv_src = table(p->recv_src);
+    k.y = table(p->y);
+    k.rank_counts = table(p->rank_counts);
+    k.rank_offsets = rank_layout->rank_offsets;
+    k.me = p->rank;
+    k.capacity = p->capacity;
+    return k;
+}
+
 } // namespace
 
 ep_status_t ep_get_rank_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout,
@@ -547,7 +583,7 @@ ep_status_t ep_dispatch_ranks(const void* x, int32_t hidden, const ep_routing_de
     if (recv_topk_idx != nullptr && !aligned(recv_topk_idx, 8))
         return EP_ERR_INVALID_ARG;
     if (recv_topk_weights != nullptr &&
-        (topk_weights == nullptr || !aligned(topk_weights, 4) || !aligned(recv_topk_weights, 4)))
+        ((T > 0 && topk_weights == nullptr) || !aligned(topk_weights, 4) || !aligned(recv_topk_weights, 4)))
         return EP_ERR_INVALID_ARG;
     if (recv_src != nullptr && !aligned(recv_src, 4))
         return EP_ERR_INVALID_ARG;
@@ -595,6 +631,146 @@ ep_status_t ep_combine_ranks(const void* y, int32_t hidden, int64_t num_y_rows, 
                             out,
                             static_cast<int32_t>(out_dtype),
                             ep::error_word(layout->workspace)};
+    return from_cuda(ep::launch_rank_combine(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_peer_alloc(size_t bytes, void** ptr, void* handle)
+{
+    CallRange range_("ep_peer_alloc");
+    if (bytes == 0 || ptr == nullptr || handle == nullptr)
+        return EP_ERR_INVALID_ARG;
+    static_assert(sizeof(cudaIpcMemHandle_t) == EP_IPC_HANDLE_BYTES, "IPC handle size");
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return EP_ERR_CUDA;
+    }
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, p) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(p);
+        return EP_ERR_CUDA;
+    }
+    std::memcpy(handle, &h, sizeof(h));
+    *ptr = p;
+    return EP_OK;
+}
+
+ep_status_t ep_peer_free(void* ptr)
+{
+    CallRange range_("ep_peer_free");
+    if (ptr == nullptr)
+        return EP_ERR_INVALID_ARG;
+    return from_cuda(cudaFree(ptr));
+}
+
+ep_status_t ep_peer_open(const void* handle, void** ptr)
+{
+    CallRange range_("ep_peer_open");
+    if (handle == nullptr || ptr == nullptr)
+        return EP_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof(h));
+    void* p = nullptr;
+    if (cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+        cudaGetLastError();
+        return EP_ERR_CUDA;
+    }
+    *ptr = p;
+    return EP_OK;
+}
+
+ep_status_t ep_peer_close(void* ptr)
+{
+    CallRange range_("ep_peer_close");
+    if (ptr == nullptr)
+        return EP_ERR_INVALID_ARG;
+    return from_cuda(cudaIpcCloseMemHandle(ptr));
+}
+
+ep_status_t ep_peer_publish_counts(const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                                   const ep_peers_t* peers, ep_stream_t stream)
+{
+    CallRange range_("ep_peer_publish_counts");
+    ep_status_t st = check_routing(routing);
+    if (st != EP_OK)
+        return st;
+    st = check_peers(routing, peers);
+    if (st != EP_OK)
+        return st;
+    if (layout == nullptr || layout->num_tokens_per_rank == nullptr || !aligned(layout->num_tokens_per_rank, 4))
+        return EP_ERR_INVALID_ARG;
+    ep::PublishCountsLaunch a{layout->num_tokens_per_rank, static_cast<const unsigned long long*>(
+                                                               static_cast<const void*>(peers->rank_counts)),
+                              peers->num_ranks, peers->rank};
+    return from_cuda(ep::launch_publish_counts(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_dispatch_peers(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                              const ep_layout_t* layout, const ep_rank_layout_t* rank_layout,
+                              const float* topk_weights, const ep_peers_t* peers, ep_stream_t stream)
+{
+    CallRange range_("ep_dispatch_peers");
+    ep_status_t st = check_rank_call(routing, layout, rank_layout);
+    if (st != EP_OK)
+        return st;
+    st = check_peers(routing, peers);
+    if (st != EP_OK)
+        return st;
+    if (routing->routing != EP_ROUTING_TOPK || hidden < 1 || hidden % 8 != 0)
+        return EP_ERR_INVALID_ARG;
+    const int32_t T = routing->num_tokens;
+    if (T > 0 && (x == nullptr || !aligned(x, 16)))
+        return EP_ERR_INVALID_ARG;
+    if (peers->recv_topk_weights != nullptr && ((T > 0 && topk_weights == nullptr) || !aligned(topk_weights, 4)))
+        return EP_ERR_INVALID_ARG;
+    ep::RankDispatchLaunch a{x,
+                             T,
+                             hidden,
+                             routing->num_topk,
+                             routing->num_experts,
+                             routing->num_ranks,
+                             routing->topk_idx,
+                             topk_weights,
+                             rank_layout->rank_row,
+                             peers->capacity,
+                             nullptr,
+                             nullptr,
+                             nullptr,
+                             nullptr,
+                             ep::error_word(layout->workspace),
+                             peer_tables(peers, rank_layout)};
+    return from_cuda(ep::launch_rank_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_combine_peers(int32_t hidden, const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                             const ep_rank_layout_t* rank_layout, const ep_peers_t* peers, void* out,
+                             ep_dtype_t out_dtype, ep_stream_t stream)
+{
+    CallRange range_("ep_combine_peers");
+    ep_status_t st = check_rank_call(routing, layout, rank_layout);
+    if (st != EP_OK)
+        return st;
+    st = check_peers(routing, peers);
+    if (st != EP_OK)
+        return st;
+    if (hidden < 1 || hidden % 8 != 0 || (out_dtype != EP_BF16 && out_dtype != EP_FP32))
+        return EP_ERR_INVALID_ARG;
+    const int32_t T = routing->num_tokens;
+    if (T > 0 && (out == nullptr || !aligned(out, 16)))
+        return EP_ERR_INVALID_ARG;
+    if (T == 0)
+        return EP_OK;
+    ep::RankCombineLaunch a{nullptr,
+                            T,
+                            hidden,
+                            routing->num_ranks,
+                            peers->capacity,
+                            rank_layout->rank_row,
+                            out,
+                            static_cast<int32_t>(out_dtype),
+                            ep::error_word(layout->workspace),
+                            peer_tables(peers, rank_layout)};
     return from_cuda(ep::launch_rank_combine(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -97,6 +97,7 @@ struct CombineArgs {
     int64_t warp_base; // first (token, segment) item of this launch
     int32_t heavy_first; // expert choice: list heavy tokens first (persistent launch)
     int32_t wide;        // rows and y 32-byte aligned: pairs of vectors by one 32-byte load
+    PeerTables peers;    // per rank over peer memory: the ranks' y buffers
 };
 
 // expert choice, heavy first (see combine_kernel)
@@ -156,7 +157,8 @@ constexpr int kZeroBytes = 4096; // zeroed shared memory behind the bulk stores
 enum CombineSrc : int {
     kSrcTopk = 0,  // entries: the token's K (expert, slot) pairs, gate weights
     kSrcEc = 1,    // entries: the token's CSR slots, expert weights
-    kSrcRanks = 2  // entries: the token's R rank rows, weight 1 (fmaf(1, y, acc) == acc + y)
+    kSrcRanks = 2, // entries: the token's R rank rows, weight 1 (fmaf(1, y, acc) == acc + y)
+    kSrcPeers = 3  // entries: the token's rows in the R ranks' y buffers, weight 1; row = its address
 };
 
 template <int kSrc>
@@ -165,7 +167,22 @@ __device__ __forceinline__ void entry(const CombineArgs& a, int64_t t, int64_t b
 {
     row = -1;
     w = 0.0f;
-    if constexpr (kSrc == kSrcRanks) {
+    if constexpr (kSrc == kSrcPeers) {
+        // rank j's rows: those of ranks 0 .. me-1 first, then this rank's in send order
+        const int64_t r = __ldg(a.rank_row + t * a.K + j);
+        if (r < 0)
+            return;
+        const int32_t* counts = reinterpret_cast<const int32_t*>(__ldg(a.peers.rank_counts + a.peers.me));
+        int64_t local = r - __ldg(a.peers.rank_offsets + j);
+        for (int i = 0; i < a.peers.me; ++i)
+            local += __ldg(counts + i * a.K + j);
+        if (local < 0 || local >= a.num_y_rows) {
+            errbits |= EP_DEVERR_OVERFLOW;
+            return;
+        }
+        row = static_cast<int64_t>(__ldg(a.peers.y + j)) + local * (static_cast<int64_t>(a.H) * 2);
+        w = 1.0f;
+    } else if constexpr (kSrc == kSrcRanks) {
         const int64_t r = __ldg(a.rank_row + t * a.K + j);
         if (r < 0)
             return;
@@ -274,7 +291,9 @@ __device__ __forceinline__ void reduce_segment(const CombineArgs& a, int64_t t, 
 #pragma unroll
                 for (int g = 0; g < kGroup; ++g) {
                     const bool on = rows[g] >= 0;
-                    const uint8_t* src = a.y + static_cast<int64_t>(on ? rows[g] : 0) * row_bytes;
+                    const uint8_t* src = kSrc == kSrcPeers
+                                             ? reinterpret_cast<const uint8_t*>(static_cast<uintptr_t>(rows[g]))
+                                             : a.y + static_cast<int64_t>(on ? rows[g] : 0) * row_bytes;
                     if (wide) {
 #pragma unroll
                         for (int j = 0; j < kVecPerLane; j += 2) {
@@ -1007,6 +1026,14 @@ cudaError_t launch_rank_combine(const RankCombineLaunch& a, cudaStream_t stream)
     k.rank_row = a.rank_row;
     k.out = a.out;
     k.err = a.err;
+    if (a.peers.y != nullptr) {
+        // the ranks' buffers: 16-byte loads (their alignment to 32 is not known here)
+        k.peers = a.peers;
+        k.num_y_rows = a.peers.capacity;
+        k.wide = 0;
+        return launch_combine<kSrcPeers, kTcVec, kTcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0,
+                                                            stream);
+    }
     k.wide = wide_loads(a.y, a.H, a.T);
     return launch_combine<kSrcRanks, kTcVec, kTcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0, stream);
 }

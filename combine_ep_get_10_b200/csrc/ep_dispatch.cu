@@ -123,13 +123,38 @@ struct BulkArgs {
     uint32_t* err;
     int64_t item_base; // first item of this launch
     int32_t early_load; // load source rows before waiting for the kernel before (see launch_pdl)
+    PeerTables peers;   // per rank over peer memory
 };
 
 enum BulkSrc : int {
     kSrcTopk = 0,  // item row = token t; destinations = its K routed pairs
     kSrcEc = 1,    // item row = slot s; source token_indices[s]; destination row s
-    kSrcRanks = 2  // item row = token t; destinations = its ranks' rows
+    kSrcRanks = 2, // item row = token t; destinations = its ranks' rows
+    kSrcPeers = 3  // item row = token t; destinations = its rows in the ranks' buffers
 };
+
+template <typename T>
+__device__ __forceinline__ T* table_at(const unsigned long long* table, int r)
+{
+    return reinterpret_cast<T*>(__ldg(table + r));
+}
+
+// Row of token t (rank_row[t, j] = row in this rank's send order) in rank
+// j's receive buffer: base(me, j) + rank_row - rank_offsets[j], base from
+// this rank's copy of every rank's counts; -1 with EP_DEVERR_OVERFLOW when
+// it falls outside the buffer.
+__device__ __forceinline__ int64_t peer_row(const PeerTables& p, int R, int j, int64_t row, uint32_t& errbits)
+{
+    const int32_t* counts = table_at<const int32_t>(p.rank_counts, p.me);
+    int64_t local = row - __ldg(p.rank_offsets + j);
+    for (int i = 0; i < p.me; ++i)
+        local += __ldg(counts + i * R + j);
+    if (local < 0 || local >= p.capacity) {
+        errbits |= EP_DEVERR_OVERFLOW;
+        return -1;
+    }
+    return local;
+}
 
 // Top-k entries of token t as rank r sees them (per-rank dispatch): local
 // expert id and weight for the experts of rank r, -1 and 0 for the others.
@@ -149,6 +174,31 @@ __device__ __forceinline__ void write_rank_topk(const BulkArgs& a, int64_t t, in
             a.recv_topk_idx[row * K + k] = local ? e - static_cast<int64_t>(r) * per_rank : -1;
         if (a.recv_topk_weights != nullptr)
             a.recv_topk_weights[row * K + k] = local ? __ldg(a.topk_weights + t * K + k) : 0.0f;
+    }
+}
+
+// The token's K entries as each of its ranks sees them, written into the
+// ranks' buffers: lane j holds the token's row in rank j's buffer (or -1).
+__device__ __forceinline__ void write_peer_topk(const BulkArgs& a, int64_t t, int lane, int64_t my_row)
+{
+    const int K = a.map.K;
+    const int per_rank = a.map.E / a.R;
+    const int n = a.R * K;
+    for (int j0 = 0; j0 < n; j0 += 32) { // warp-uniform trip count: every lane takes the shuffle
+        const int j = j0 + lane;
+        const int r = min(j / K, a.R - 1);
+        const int64_t row = __shfl_sync(kFullMask, my_row, r);
+        if (j >= n || row < 0)
+            continue;
+        const int k = j - r * K;
+        const int64_t e = __ldg(a.map.topk_idx + t * K + k);
+        const bool local = e >= 0 && e < a.map.E && e / per_rank == r;
+        if (a.peers.recv_topk_idx != nullptr)
+            table_at<int64_t>(a.peers.recv_topk_idx, r)[row * K + k] =
+                local ? e - static_cast<int64_t>(r) * per_rank : -1;
+        if (a.peers.recv_topk_weights != nullptr)
+            table_at<float>(a.peers.recv_topk_weights, r)[row * K + k] =
+                local ? __ldg(a.topk_weights + t * K + k) : 0.0f;
     }
 }
 
@@ -192,8 +242,17 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
         pdl_wait(); // the layout's results (slot, offsets) are final from here on
     // destination rows of the first 32 pairs while the load is in flight
     int64_t dst_row = -1;
+    uint8_t* dst = a.dst;
     if constexpr (kSrc == kSrcEc) {
         dst_row = lane == 0 ? r : -1;
+    } else if constexpr (kSrc == kSrcPeers) {
+        if (lane < a.R) {
+            const int64_t row = __ldg(a.rank_row + r * a.R + lane);
+            if (row >= 0) {
+                dst_row = peer_row(a.peers, a.R, lane, row, errbits);
+                dst = table_at<uint8_t>(a.peers.recv_x, lane);
+            }
+        }
     } else if constexpr (kSrc == kSrcRanks) {
         if (lane < a.R) {
             dst_row = __ldg(a.rank_row + r * a.R + lane);
@@ -209,7 +268,7 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
     const bool ok = mbar_wait_bounded(&bar, 0, a.err);
     if (ok) {
         if (dst_row >= 0)
-            bulk_store_s2g(a.dst + dst_row * a.row_bytes + off, buf, bytes);
+            bulk_store_s2g(dst + dst_row * a.row_bytes + off, buf, bytes);
         if constexpr (kSrc == kSrcTopk) {
             for (int k = lane + 32; k < a.map.K; k += 32) {
                 const int64_t rk = a.map.row(r, k, errbits);
@@ -226,6 +285,14 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
                 a.recv_src[dst_row] = static_cast<int32_t>(r);
             if (a.recv_topk_idx != nullptr || a.recv_topk_weights != nullptr)
                 write_rank_topk(a, r, lane);
+        }
+    }
+    if constexpr (kSrc == kSrcPeers) {
+        if (c == 0) {
+            if (dst_row >= 0 && a.peers.recv_src != nullptr)
+                table_at<int32_t>(a.peers.recv_src, lane)[dst_row] = static_cast<int32_t>(r);
+            if (a.peers.recv_topk_idx != nullptr || a.peers.recv_topk_weights != nullptr)
+                write_peer_topk(a, r, lane, dst_row);
         }
     }
     if (kSrc == kSrcTopk && c == 0 && (a.recv_src != nullptr || a.recv_weights != nullptr)) {
@@ -837,6 +904,10 @@ cudaError_t launch_rank_dispatch(const RankDispatchLaunch& a, cudaStream_t strea
     k.recv_topk_weights = a.recv_topk_weights;
     k.T = a.T;
     k.err = a.err;
+    if (a.peers.recv_x != nullptr) {
+        k.peers = a.peers;
+        return launch_bulk<kSrcPeers>(k, static_cast<int64_t>(a.T) * k.nchunks, stream);
+    }
     return launch_bulk<kSrcRanks>(k, static_cast<int64_t>(a.T) * k.nchunks, stream);
 }
 

@@ -118,6 +118,30 @@ struct EcDispatchLaunch {
 };
 cudaError_t launch_ec_dispatch(const EcDispatchLaunch& a, cudaStream_t stream);
 
+// Per rank over peer memory: device tables of R addresses (rank r's buffer
+// as this process reaches it) and this rank's place among the ranks.  A
+// source's row for rank j lands at base(me, j) + rank_row[t, j] -
+// rank_offsets[j] of rank j's buffer, base(me, j) = sum over i < me of
+// rank_counts[i, j] (this rank's own copy of the counts).
+struct PeerTables {
+    const unsigned long long* recv_x;            // nullptr: not the peer path
+    const unsigned long long* recv_topk_idx;     // or nullptr
+    const unsigned long long* recv_topk_weights; // or nullptr
+    const unsigned long long* recv_src;          // or nullptr
+    const unsigned long long* y;
+    const unsigned long long* rank_counts;
+    const int32_t* rank_offsets; // this rank's rank layout
+    int32_t me;
+    int64_t capacity; // rows of every rank's recv_x and y
+};
+
+struct PublishCountsLaunch {
+    const int32_t* num_tokens_per_rank; // [R]
+    const unsigned long long* rank_counts; // table of R [R, R] matrices
+    int32_t R, me;
+};
+cudaError_t launch_publish_counts(const PublishCountsLaunch& a, cudaStream_t stream);
+
 struct RankDispatchLaunch {
     const void* x;
     int32_t T, H, K, E, R;
@@ -130,6 +154,7 @@ struct RankDispatchLaunch {
     float* recv_topk_weights;
     int32_t* recv_src;
     uint32_t* err;
+    PeerTables peers; // peers.recv_x != nullptr: rows go to the ranks' buffers
 };
 cudaError_t launch_rank_dispatch(const RankDispatchLaunch& a, cudaStream_t stream);
 
@@ -166,6 +191,7 @@ struct RankCombineLaunch {
     void* out;
     int32_t out_dtype;
     uint32_t* err;
+    PeerTables peers; // peers.y != nullptr: rows read from the ranks' buffers
 };
 cudaError_t launch_rank_combine(const RankCombineLaunch& a, cudaStream_t stream);
 

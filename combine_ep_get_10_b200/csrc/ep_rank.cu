@@ -13,6 +13,11 @@
 // ranks its own tokens: a ballot per rank gives each lane its rank inside
 // the warp and one warp per rank scans the 32 warps' counts.  The rank
 // offsets come from the layout's num_tokens_per_rank (one warp scan).
+//
+// The per-rank path over peer memory also starts here: every rank publishes
+// its num_tokens_per_rank as one row of every rank's [R, R] counts matrix,
+// from which each rank's dispatch and combine find where its rows sit in
+// the other ranks' buffers.
 #include <algorithm>
 
 #include "ep_device.cuh"
@@ -134,7 +139,26 @@ __global__ void __launch_bounds__(kRankThreads) rank_layout_kernel(RankLayoutLau
     }
 }
 
+// Row `me` of every rank's [R, R] counts matrix <- this rank's
+// num_tokens_per_rank: thread (j, c) stores entry c into rank j's matrix.
+__global__ void __launch_bounds__(1024) publish_counts_kernel(PublishCountsLaunch a)
+{
+    const int i = threadIdx.x;
+    if (i >= a.R * a.R)
+        return;
+    const int j = i / a.R;
+    const int c = i - j * a.R;
+    int32_t* m = reinterpret_cast<int32_t*>(__ldg(a.rank_counts + j));
+    m[a.me * a.R + c] = __ldg(a.num_tokens_per_rank + c);
+}
+
 } // namespace
+
+cudaError_t launch_publish_counts(const PublishCountsLaunch& a, cudaStream_t stream)
+{
+    publish_counts_kernel<<<1, 1024, 0, stream>>>(a);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_rank_layout(const RankLayoutLaunch& a, cudaStream_t stream)
 {

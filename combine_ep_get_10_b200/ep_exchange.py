@@ -174,10 +174,10 @@ class CudaRowOps:
                             recv_topk_weights=sw, stream=self.stream)
         return SendRows(sx, sidx, sw, counts, (routing, layout, rl))
 
-    def local_experts(self, x, topk_idx, topk_weights, local_experts, expert_fn):
+    def local_experts(self, x, topk_idx, topk_weights, local_experts, expert_fn, out=None):
         B = self.B
         n, H = x.shape
-        y = torch.empty((n, H), dtype=torch.bfloat16, device=x.device)
+        y = torch.empty((n, H), dtype=torch.bfloat16, device=x.device) if out is None else out
         if n == 0:
             return y
         routing = B.Routing.topk(topk_idx, local_experts, 1)
@@ -197,3 +197,161 @@ class CudaRowOps:
         if B.ep_get_device_error(layout) != 0:
             raise B.EPError(B.EP_ERR_BAD_INDEX, "device error flagged in the exchange step")
         return out
+
+
+# ------------------------------------------------------ over peer memory
+def _align(n: int, a: int = 256) -> int:
+    return (n + a - 1) // a * a
+
+
+@dataclass
+class PeerReceived:
+    """The rows this rank's experts process (views of its receive buffers),
+    source rank 0's first, and what its combine needs."""
+    x: torch.Tensor
+    topk_idx: torch.Tensor
+    topk_weights: torch.Tensor
+    src: torch.Tensor
+    recv_counts: list[int]
+    handle: object
+
+
+class PeerExpertParallel:
+    """The same exchange with the all-to-all fused into the kernels over
+    peer memory (ep_dispatch_peers / ep_combine_peers): the dispatch stores
+    each (token, rank) row straight into that rank's receive buffer and the
+    combine reads the partial rows straight from the ranks' buffers.
+
+    Every rank allocates one block of device memory that the other processes
+    map (ep_peer_alloc; the handles travel by all_gather_object): receive
+    rows, their top-k entries and source tokens, the partial rows and the
+    [W, W] counts matrix, each at the same offset in every rank's block.
+    ``capacity`` bounds the rows a rank can receive.  Between the phases of a
+    step every rank synchronises its stream and passes a process-group
+    barrier (``barrier``), so no kernel ever waits for another rank:
+
+        layout -> rank layout -> publish counts | dispatch | experts | combine
+
+    A step's results equal ExpertParallel's (all-to-all-v) bit for bit."""
+
+    def __init__(self, num_experts: int, hidden: int, num_topk: int, capacity: int, group=None, device=None,
+                 barrier=None):
+        from . import binding as B
+
+        self.B = B
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        if num_experts % self.world != 0:
+            raise ValueError("%d experts do not split over %d ranks" % (num_experts, self.world))
+        if hidden % 8 != 0:
+            raise ValueError("rows travel in 16-byte vectors: hidden must be a multiple of 8")
+        self.num_experts, self.hidden, self.num_topk = num_experts, hidden, num_topk
+        self.local_experts = num_experts // self.world
+        self.capacity = int(capacity)
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self._barrier_fn = barrier
+        W, C, H, K = self.world, self.capacity, hidden, num_topk
+        sizes = dict(recv_x=C * H * 2, y=C * H * 2, recv_topk_idx=C * K * 8, recv_topk_weights=C * K * 4,
+                     recv_src=C * 4, rank_counts=W * W * 4)
+        self.offsets, total = {}, 0
+        for name, n in sizes.items():
+            self.offsets[name] = total
+            total += _align(max(n, 1))
+        self._own, handle = B.ep_peer_alloc(total)
+        handles = [None] * W
+        dist.all_gather_object(handles, handle, group=group)
+        self._opened = []
+        bases = []
+        try:
+            for r in range(W):
+                if r == self.rank:
+                    bases.append(self._own)
+                else:
+                    ptr = B.ep_peer_open(handles[r])
+                    self._opened.append(ptr)
+                    bases.append(ptr)
+        except Exception:
+            self._release()
+            raise
+        tables = {name: torch.tensor([b + off for b in bases], dtype=torch.int64, device=self.device)
+                  for name, off in self.offsets.items()}
+        self.peers = B.Peers(self.rank, C, tables["recv_x"], tables["y"], tables["rank_counts"],
+                             recv_topk_idx=tables["recv_topk_idx"], recv_topk_weights=tables["recv_topk_weights"],
+                             recv_src=tables["recv_src"])
+        own = lambda name, shape, dtype: B.device_view(self._own + self.offsets[name], shape, dtype, self.device)
+        self.recv_x = own("recv_x", (C, H), torch.bfloat16)
+        self.y = own("y", (C, H), torch.bfloat16)
+        self.recv_topk_idx = own("recv_topk_idx", (C, K), torch.int64)
+        self.recv_topk_weights = own("recv_topk_weights", (C, K), torch.float32)
+        self.recv_src = own("recv_src", (C,), torch.int32)
+        self.rank_counts = own("rank_counts", (W, W), torch.int32)
+        self.ops = CudaRowOps()
+        self._barrier()  # every rank has mapped every block before any store
+
+    def _barrier(self):
+        torch.cuda.current_stream(self.device).synchronize()
+        if self._barrier_fn is not None:
+            self._barrier_fn()
+        else:
+            dist.barrier(group=self.group)
+
+    def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor) -> PeerReceived:
+        B = self.B
+        if x.shape[1] != self.hidden or topk_idx.shape[1] != self.num_topk:
+            raise ValueError("x is [T, %d] and topk_idx [T, %d] for this exchange" % (self.hidden, self.num_topk))
+        routing = B.Routing.topk(topk_idx, self.num_experts, self.world)
+        layout = B.Layout(routing, device=x.device)
+        B.ep_get_layout(routing, layout)
+        rl = B.RankLayout(routing, device=x.device)
+        B.ep_get_rank_layout(routing, layout, rl)
+        B.ep_peer_publish_counts(routing, layout, self.peers)
+        self._barrier()
+        B.ep_dispatch_peers(x, routing, layout, rl, self.peers, topk_weights=topk_weights)
+        self._barrier()
+        counts = self.rank_counts.cpu()
+        recv_counts = counts[:, self.rank].tolist()
+        n = sum(recv_counts)
+        if n > self.capacity:
+            raise B.EPError(B.EP_ERR_OVERFLOW, "rank %d receives %d rows, the buffers hold %d"
+                            % (self.rank, n, self.capacity))
+        return PeerReceived(self.recv_x[:n], self.recv_topk_idx[:n], self.recv_topk_weights[:n], self.recv_src[:n],
+                            recv_counts, (routing, layout, rl))
+
+    def experts(self, recv: PeerReceived, expert_fn) -> torch.Tensor:
+        """The partial rows, written into this rank's y buffer."""
+        n = recv.x.shape[0]
+        return self.ops.local_experts(recv.x, recv.topk_idx, recv.topk_weights, self.local_experts, expert_fn,
+                                      out=self.y[:n])
+
+    def combine(self, y: torch.Tensor, recv: PeerReceived, out_dtype=torch.bfloat16) -> torch.Tensor:
+        B = self.B
+        n = recv.x.shape[0]
+        if y.shape != (n, self.hidden):
+            raise ValueError("y is %s, %d rows were received" % (tuple(y.shape), n))
+        if y.data_ptr() != self.y.data_ptr():
+            self.y[:n].copy_(y)
+        routing, layout, rl = recv.handle
+        self._barrier()
+        out = torch.empty((routing.T, self.hidden), dtype=out_dtype, device=self.device)
+        B.ep_combine_peers(routing, layout, rl, self.peers, out)
+        if B.ep_get_device_error(layout) != 0:
+            raise B.EPError(B.EP_ERR_OVERFLOW, "device error flagged in the peer exchange")
+        return out
+
+    def _release(self):
+        for ptr in self._opened:
+            self.B.ep_peer_close(ptr)
+        self._opened = []
+
+    def close(self):
+        """Unmap the peers' blocks and free this rank's (collective)."""
+        if self._own is None:
+            return
+        self._barrier()  # no rank still reads or writes another's block
+        self._release()
+        self._barrier()  # every mapping of this block is gone
+        for name in ("recv_x", "y", "recv_topk_idx", "recv_topk_weights", "recv_src", "rank_counts"):
+            setattr(self, name, None)
+        self.B.ep_peer_free(self._own)
+        self._own = None

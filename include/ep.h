@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define EP_ABI_VERSION 2
+#define EP_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define EP_API __attribute__((visibility("default")))
@@ -303,7 +303,7 @@ EP_API ep_status_t ep_get_rank_layout(const ep_routing_desc_t* routing, const ep
  *   recv_topk_idx     optional int64 [rows, K]: e - r*E/R for an expert e of
  *                     rank r, else -1
  *   recv_topk_weights optional fp32 [rows, K]: topk_weights[t, k] for those
- *                     entries, else 0 (needs topk_weights)
+ *                     entries, else 0 (needs topk_weights when T > 0)
  *   recv_src          optional int32 [rows]: source token
  * x bf16 [T, H], recv_x bf16 [num_recv_rows, H], both 16-byte aligned,
  * H % 8 == 0.  Rows >= num_recv_rows are skipped with EP_DEVERR_OVERFLOW. */
@@ -319,6 +319,116 @@ EP_API ep_status_t ep_dispatch_ranks(const void* x, int32_t hidden, const ep_rou
  * with no rank gets +0.  y bf16 [num_y_rows, H]; out [T, H]. */
 EP_API ep_status_t ep_combine_ranks(const void* y, int32_t hidden, int64_t num_y_rows, const ep_routing_desc_t* routing,
                                     const ep_layout_t* layout, const ep_rank_layout_t* rank_layout, void* out,
+                                    ep_dtype_t out_dtype, ep_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Per-rank path over peer memory: one process per GPU, the routing's R
+ * logical ranks are the R processes of a group, and the all-to-all of the
+ * per-rank path is fused into its kernels.  [README] "Normal Mode (Prefill /
+ * Training)" (intranode transfer) and the strategy table's all-to-all: each
+ * token goes once to every rank that holds one of its experts, and one
+ * partial row per (token, rank) comes back and is reduced on the token's
+ * rank.  Here the dispatch kernel stores each (token, rank) row straight
+ * into that rank's receive buffer, and the combine kernel reads the partial
+ * rows straight from the ranks' buffers: no staging buffer and no separate
+ * transfer.
+ *
+ * Every rank r holds, in device memory that the other processes map
+ * (ep_peer_alloc / ep_peer_open):
+ *   recv_x             bf16  [capacity, H]  rows it receives
+ *   recv_topk_idx      int64 [capacity, K]  their top-k entries as rank r
+ *                                           sees them (local expert id or -1)
+ *   recv_topk_weights  fp32  [capacity, K]  gate weight or 0
+ *   recv_src           int32 [capacity]     source token on the source rank
+ *   y                  bf16  [capacity, H]  partial rows it sends back, in
+ *                                           the order of recv_x
+ *   rank_counts        int32 [R, R]         row i = rank i's
+ *                                           num_tokens_per_rank
+ * Rank j's rows are those of source rank 0 first, each source's rows in
+ * ascending token order; source i's block starts at row
+ *   base(i, j) = sum over i' < i of rank_counts[i', j]
+ * and token t of source i lands at base(i, j) + rank_row[t, j] -
+ * rank_offsets[j] (its rank layout).  This is the order an all-to-all-v of
+ * the ep_dispatch_ranks rows delivers, and the results equal that path's bit
+ * for bit.
+ *
+ * ep_peers_t holds, per rank r, the address under which THIS process reaches
+ * rank r's buffer (its own allocation for r == rank, a mapping made by
+ * ep_peer_open otherwise), as device arrays of R addresses; each process
+ * builds its own tables, since mappings differ between processes.
+ *
+ * These calls only move data: none of their kernels waits for another rank.
+ * The caller separates the ranks' phases with a barrier that every rank
+ * passes only after its own kernels of the phase before have completed (for
+ * example: synchronise the stream, then a process-group barrier):
+ *   1. ep_get_layout (R ranks) -> ep_get_rank_layout -> ep_peer_publish_counts
+ *   2. barrier
+ *   3. ep_dispatch_peers
+ *   4. barrier; rank j's received rows: sum over i of its rank_counts[i, j]
+ *   5. local experts: rank j writes its partial rows to y[0 .. received)
+ *   6. barrier
+ *   7. ep_combine_peers
+ * and step 2 of the next round orders its writes after every rank's step 7.
+ * Rows that would land at or past `capacity` are skipped with
+ * EP_DEVERR_OVERFLOW in the calling rank's workspace error word.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    int32_t num_ranks;                /* R: the routing's num_ranks */
+    int32_t rank;                     /* this process's rank, 0 <= rank < R */
+    int64_t capacity;                 /* rows of every rank's recv_x and y */
+    void* const* recv_x;              /* device array of R addresses */
+    int64_t* const* recv_topk_idx;    /* device array of R addresses, or NULL */
+    float* const* recv_topk_weights;  /* device array of R addresses, or NULL */
+    int32_t* const* recv_src;         /* device array of R addresses, or NULL */
+    const void* const* y;             /* device array of R addresses */
+    int32_t* const* rank_counts;      /* device array of R addresses */
+} ep_peers_t;
+
+/* Bytes of an IPC handle (cudaIpcMemHandle_t) as ep_peer_alloc writes it. */
+#define EP_IPC_HANDLE_BYTES 64
+
+/* Device memory that other processes can map: `bytes` (>= 1) allocated with
+ * cudaMalloc on the current device (256-byte aligned) into *ptr, and its IPC
+ * handle written to handle[0 .. EP_IPC_HANDLE_BYTES).  Release with
+ * ep_peer_free after every process that opened it has closed it. */
+EP_API ep_status_t ep_peer_alloc(size_t bytes, void** ptr, void* handle);
+EP_API ep_status_t ep_peer_free(void* ptr);
+
+/* Map another process's ep_peer_alloc buffer (its handle, received by any
+ * host channel) into this process: *ptr is its address here (over NVLink
+ * when it lives on another GPU; peer access is enabled on first use).  A
+ * process cannot open its own handles: use the pointer it allocated.  Unmap
+ * with ep_peer_close. */
+EP_API ep_status_t ep_peer_open(const void* handle, void** ptr);
+EP_API ep_status_t ep_peer_close(void* ptr);
+
+/* Step 1: store layout->num_tokens_per_rank (written by ep_get_layout for
+ * `routing`, R = peers->num_ranks) as row `rank` of every rank's
+ * rank_counts. */
+EP_API ep_status_t ep_peer_publish_counts(const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                                          const ep_peers_t* peers, ep_stream_t stream);
+
+/* Step 3 (TOPK routing): for every token t and rank j with rank_row[t, j]
+ * >= 0, row base(rank, j) + rank_row[t, j] - rank_offsets[j] of rank j's
+ * recv_x gets x[t] (one read of x[t], one store per rank), and its
+ * recv_topk_idx / recv_topk_weights / recv_src entries (when the tables are
+ * given) the token's K entries as rank j sees them and t.  base() is read
+ * from this rank's own rank_counts, which must hold every rank's row (step
+ * 2).  x bf16 [T, H], 16-byte aligned, H % 8 == 0; topk_weights fp32 [T, K]
+ * (needed with recv_topk_weights when T > 0).  Every recv_x must be
+ * 16-byte aligned. */
+EP_API ep_status_t ep_dispatch_peers(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                     const ep_layout_t* layout, const ep_rank_layout_t* rank_layout,
+                                     const float* topk_weights, const ep_peers_t* peers, ep_stream_t stream);
+
+/* Step 7: out[t] = sum over the token's ranks j in ascending order of row
+ * base(rank, j) + rank_row[t, j] - rank_offsets[j] of rank j's y, fp32
+ * additions from 0, written as fp32 or rounded once (RNE) to bf16; a token
+ * with no rank gets +0 -- ep_combine_ranks with the rows read in place.
+ * out [T, H] (out_dtype BF16 or FP32), 16-byte aligned; every y must be
+ * 16-byte aligned. */
+EP_API ep_status_t ep_combine_peers(int32_t hidden, const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                                    const ep_rank_layout_t* rank_layout, const ep_peers_t* peers, void* out,
                                     ep_dtype_t out_dtype, ep_stream_t stream);
 
 /* ep_get_layout for callers that cannot allocate device memory.  The pages

@@ -43,10 +43,13 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert B.ep_version() == B.EP_ABI_VERSION == 2
+    assert B.ep_version() == B.EP_ABI_VERSION == 3
     # ep_layout_t: nine pointer-sized fields, then num_valid_host (version 2)
     assert ctypes.sizeof(B.LayoutDesc) == 10 * 8
     assert B.LayoutDesc.num_valid_host.offset == 9 * 8
+    # ep_peers_t (version 3): two int32, the int64 capacity, six tables
+    assert ctypes.sizeof(B.PeersDesc) == 8 + 8 + 6 * 8
+    assert B.PeersDesc.capacity.offset == 8 and B.PeersDesc.rank_counts.offset == 8 + 8 + 5 * 8
     for s in range(8):
         assert B.ep_status_string(s)
     assert B.ep_status_string(99) == "unknown status"
@@ -197,3 +200,54 @@ def test_binding_constants_match_the_header():
         assert getattr(B, name) == v, name
     for v, name in B.STATUS_NAMES.items():
         assert values[name] == v
+
+
+def test_peer_calls_reject_bad_args(L):
+    """The peer-memory calls check routing, layout, rank layout and tables on
+    the host before anything is launched or allocated (no GPU here)."""
+    d = _topk_desc(R=2)
+    lay = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x100000, 256)
+    rl = B.RankLayoutDesc(0x7000, 0x7100)
+
+    def peers(**kw):
+        f = dict(num_ranks=2, rank=0, capacity=64, recv_x=0x8000, recv_topk_idx=None, recv_topk_weights=None,
+                 recv_src=None, y=0x8100, rank_counts=0x8200)
+        f.update(kw)
+        return B.PeersDesc(*(f[n] for n, _ in B.PeersDesc._fields_))
+
+    def disp(p, x=0x2000, hidden=256, w=None, routing=d):
+        return L.ep_dispatch_peers(x, hidden, ctypes.byref(routing), ctypes.byref(lay), ctypes.byref(rl), w,
+                                   ctypes.byref(p), None)
+
+    def comb(p, hidden=256, out=0x5000, dt=B.EP_BF16):
+        return L.ep_combine_peers(hidden, ctypes.byref(d), ctypes.byref(lay), ctypes.byref(rl), ctypes.byref(p),
+                                  out, dt, None)
+
+    def publish(p, layout=lay):
+        return L.ep_peer_publish_counts(ctypes.byref(d), ctypes.byref(layout), ctypes.byref(p), None)
+
+    bad = [peers(num_ranks=4), peers(rank=2), peers(rank=-1), peers(capacity=-1), peers(recv_x=None),
+           peers(y=None), peers(rank_counts=None), peers(recv_x=0x8004), peers(recv_src=0x8304)]
+    for p in bad:
+        assert disp(p) == 1 and comb(p) == 1 and publish(p) == 1
+    assert L.ep_dispatch_peers(0x2000, 256, ctypes.byref(d), ctypes.byref(lay), ctypes.byref(rl), None, None,
+                               None) == 1  # no tables
+    assert disp(peers(), hidden=12) == 1
+    assert disp(peers(), x=0x2008) == 1
+    assert disp(peers(recv_topk_weights=0x8400)) == 1  # weights asked for, topk_weights missing
+    assert disp(peers(), routing=_ec_desc()) == 1  # token-choice routing only
+    assert comb(peers(), dt=B.EP_FP8_E4M3) == 1
+    assert comb(peers(), out=0x5008) == 1
+    no_rank_row = B.RankLayoutDesc(0x7000, None)
+    assert L.ep_combine_peers(256, ctypes.byref(d), ctypes.byref(lay), ctypes.byref(no_rank_row),
+                              ctypes.byref(peers()), 0x5000, 0, None) == 1
+    no_counts = B.LayoutDesc(0x1000, 0x1000, None, 0x1000, 0x1000, None, None, 0x100000, 256)
+    assert publish(peers(), layout=no_counts) == 1
+    ptr = ctypes.c_void_p()
+    handle = ctypes.create_string_buffer(B.EP_IPC_HANDLE_BYTES)
+    assert L.ep_peer_alloc(0, ctypes.byref(ptr), handle) == 1
+    assert L.ep_peer_alloc(256, None, handle) == 1
+    assert L.ep_peer_alloc(256, ctypes.byref(ptr), None) == 1
+    assert L.ep_peer_open(None, ctypes.byref(ptr)) == 1
+    assert L.ep_peer_open(handle, None) == 1
+    assert L.ep_peer_close(None) == 1 and L.ep_peer_free(None) == 1
