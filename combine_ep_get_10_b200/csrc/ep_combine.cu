@@ -116,7 +116,7 @@ constexpr int kHeavyClasses = EP_COMBINE_HEAVY_SORT ? 3 : 1;
 #ifndef EP_COMBINE_HEAVY_LOOKUP
 #define EP_COMBINE_HEAVY_LOOKUP 1
 #endif
-constexpr int kHeavyLookup = EP_COMBINE_HEAVY_LOOKUP;
+[[maybe_unused]] constexpr int kHeavyLookup = EP_COMBINE_HEAVY_LOOKUP; // used without EP_COMBINE_HEAVY_PIPE
 // light runs: one list over the run's tokens (1) or one token at a time (0)
 #ifndef EP_COMBINE_EC_FLAT
 #define EP_COMBINE_EC_FLAT 1

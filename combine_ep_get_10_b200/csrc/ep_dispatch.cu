@@ -718,7 +718,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_dispatch_kernel(QuantArgs
         // every (destination, 16-byte vector) pair of the scale rows by one thread
         const int vpr = scale_row / 16;
         for (int i = tid; i < a.map.K * vpr; i += kQuantThreads) {
-            const int k = i / vpr;
+            const int k = i / max(vpr, 1); // vpr >= 1 here (a per-token scale row makes the loop empty)
             const int64_t rk = rows[k];
             if (rk >= 0)
                 st_v4(static_cast<uint8_t*>(a.scales) + rk * scale_row + (i - k * vpr) * 16,

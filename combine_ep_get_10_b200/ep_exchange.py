@@ -222,23 +222,23 @@ class PeerExpertParallel:
     each (token, rank) row straight into that rank's receive buffer and the
     combine reads the partial rows straight from the ranks' buffers.
 
-    Every rank allocates one block of device memory that the other processes
-    map (ep_peer_alloc; the handles travel by all_gather_object): receive
-    rows, their top-k entries and source tokens, the partial rows and the
-    [W, W] counts matrix, each at the same offset in every rank's block.
-    ``capacity`` bounds the rows a rank can receive.  Between the phases of a
-    step every rank synchronises its stream and passes a process-group
-    barrier (``barrier``), so no kernel ever waits for another rank:
+    Every rank allocates one block of memory that the other processes map
+    (the handles travel by all_gather_object): receive rows, their top-k
+    entries and source tokens, the partial rows and the [W, W] counts
+    matrix, each at the same offset in every rank's block.  ``capacity``
+    bounds the rows a rank can receive.  Between the phases of a step every
+    rank completes its own work and passes a process-group barrier
+    (``barrier``), so no kernel ever waits for another rank:
 
         layout -> rank layout -> publish counts | dispatch | experts | combine
 
-    A step's results equal ExpertParallel's (all-to-all-v) bit for bit."""
+    A step's results equal ExpertParallel's (all-to-all-v) bit for bit.
+    ``ops`` holds the memory and the compute steps (CudaPeerOps by default)."""
+
+    BUFFERS = ("recv_x", "y", "recv_topk_idx", "recv_topk_weights", "recv_src", "rank_counts")
 
     def __init__(self, num_experts: int, hidden: int, num_topk: int, capacity: int, group=None, device=None,
-                 barrier=None):
-        from . import binding as B
-
-        self.B = B
+                 barrier=None, ops=None):
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -249,16 +249,19 @@ class PeerExpertParallel:
         self.num_experts, self.hidden, self.num_topk = num_experts, hidden, num_topk
         self.local_experts = num_experts // self.world
         self.capacity = int(capacity)
-        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.ops = ops if ops is not None else CudaPeerOps(device)
         self._barrier_fn = barrier
         W, C, H, K = self.world, self.capacity, hidden, num_topk
-        sizes = dict(recv_x=C * H * 2, y=C * H * 2, recv_topk_idx=C * K * 8, recv_topk_weights=C * K * 4,
-                     recv_src=C * 4, rank_counts=W * W * 4)
+        shapes = dict(recv_x=((C, H), torch.bfloat16), y=((C, H), torch.bfloat16),
+                      recv_topk_idx=((C, K), torch.int64), recv_topk_weights=((C, K), torch.float32),
+                      recv_src=((C,), torch.int32), rank_counts=((W, W), torch.int32))
         self.offsets, total = {}, 0
-        for name, n in sizes.items():
+        for name in self.BUFFERS:
+            shape, dtype = shapes[name]
             self.offsets[name] = total
+            n = torch.Size(shape).numel() * torch.empty((), dtype=dtype).element_size()
             total += _align(max(n, 1))
-        self._own, handle = B.ep_peer_alloc(total)
+        self._own, handle = self.ops.alloc(total)
         handles = [None] * W
         dist.all_gather_object(handles, handle, group=group)
         self._opened = []
@@ -268,55 +271,40 @@ class PeerExpertParallel:
                 if r == self.rank:
                     bases.append(self._own)
                 else:
-                    ptr = B.ep_peer_open(handles[r])
-                    self._opened.append(ptr)
-                    bases.append(ptr)
+                    base = self.ops.open(handles[r])
+                    self._opened.append(base)
+                    bases.append(base)
         except Exception:
             self._release()
             raise
-        tables = {name: torch.tensor([b + off for b in bases], dtype=torch.int64, device=self.device)
-                  for name, off in self.offsets.items()}
-        self.peers = B.Peers(self.rank, C, tables["recv_x"], tables["y"], tables["rank_counts"],
-                             recv_topk_idx=tables["recv_topk_idx"], recv_topk_weights=tables["recv_topk_weights"],
-                             recv_src=tables["recv_src"])
-        own = lambda name, shape, dtype: B.device_view(self._own + self.offsets[name], shape, dtype, self.device)
-        self.recv_x = own("recv_x", (C, H), torch.bfloat16)
-        self.y = own("y", (C, H), torch.bfloat16)
-        self.recv_topk_idx = own("recv_topk_idx", (C, K), torch.int64)
-        self.recv_topk_weights = own("recv_topk_weights", (C, K), torch.float32)
-        self.recv_src = own("recv_src", (C,), torch.int32)
-        self.rank_counts = own("rank_counts", (W, W), torch.int32)
-        self.ops = CudaRowOps()
+        self.peers = self.ops.peers(self.rank, C, {name: [b + off for b in bases]
+                                                   for name, off in self.offsets.items()})
+        for name in self.BUFFERS:
+            shape, dtype = shapes[name]
+            setattr(self, name, self.ops.view(self._own + self.offsets[name], shape, dtype))
         self._barrier()  # every rank has mapped every block before any store
 
     def _barrier(self):
-        torch.cuda.current_stream(self.device).synchronize()
+        self.ops.sync()
         if self._barrier_fn is not None:
             self._barrier_fn()
         else:
             dist.barrier(group=self.group)
 
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor) -> PeerReceived:
-        B = self.B
         if x.shape[1] != self.hidden or topk_idx.shape[1] != self.num_topk:
             raise ValueError("x is [T, %d] and topk_idx [T, %d] for this exchange" % (self.hidden, self.num_topk))
-        routing = B.Routing.topk(topk_idx, self.num_experts, self.world)
-        layout = B.Layout(routing, device=x.device)
-        B.ep_get_layout(routing, layout)
-        rl = B.RankLayout(routing, device=x.device)
-        B.ep_get_rank_layout(routing, layout, rl)
-        B.ep_peer_publish_counts(routing, layout, self.peers)
+        handle = self.ops.layout(topk_idx, self.num_experts, self.world)
+        self.ops.publish(handle, self.peers)
         self._barrier()
-        B.ep_dispatch_peers(x, routing, layout, rl, self.peers, topk_weights=topk_weights)
+        self.ops.dispatch(x, topk_weights, handle, self.peers)
         self._barrier()
-        counts = self.rank_counts.cpu()
-        recv_counts = counts[:, self.rank].tolist()
+        recv_counts = [int(c) for c in self.rank_counts[:, self.rank].tolist()]
         n = sum(recv_counts)
         if n > self.capacity:
-            raise B.EPError(B.EP_ERR_OVERFLOW, "rank %d receives %d rows, the buffers hold %d"
-                            % (self.rank, n, self.capacity))
+            raise OverflowError("rank %d receives %d rows, the buffers hold %d" % (self.rank, n, self.capacity))
         return PeerReceived(self.recv_x[:n], self.recv_topk_idx[:n], self.recv_topk_weights[:n], self.recv_src[:n],
-                            recv_counts, (routing, layout, rl))
+                            recv_counts, handle)
 
     def experts(self, recv: PeerReceived, expert_fn) -> torch.Tensor:
         """The partial rows, written into this rank's y buffer."""
@@ -325,23 +313,17 @@ class PeerExpertParallel:
                                       out=self.y[:n])
 
     def combine(self, y: torch.Tensor, recv: PeerReceived, out_dtype=torch.bfloat16) -> torch.Tensor:
-        B = self.B
         n = recv.x.shape[0]
-        if y.shape != (n, self.hidden):
+        if tuple(y.shape) != (n, self.hidden):
             raise ValueError("y is %s, %d rows were received" % (tuple(y.shape), n))
         if y.data_ptr() != self.y.data_ptr():
             self.y[:n].copy_(y)
-        routing, layout, rl = recv.handle
         self._barrier()
-        out = torch.empty((routing.T, self.hidden), dtype=out_dtype, device=self.device)
-        B.ep_combine_peers(routing, layout, rl, self.peers, out)
-        if B.ep_get_device_error(layout) != 0:
-            raise B.EPError(B.EP_ERR_OVERFLOW, "device error flagged in the peer exchange")
-        return out
+        return self.ops.combine(recv.handle, self.peers, self.hidden, out_dtype)
 
     def _release(self):
-        for ptr in self._opened:
-            self.B.ep_peer_close(ptr)
+        for base in self._opened:
+            self.ops.close(base)
         self._opened = []
 
     def close(self):
@@ -351,7 +333,74 @@ class PeerExpertParallel:
         self._barrier()  # no rank still reads or writes another's block
         self._release()
         self._barrier()  # every mapping of this block is gone
-        for name in ("recv_x", "y", "recv_topk_idx", "recv_topk_weights", "recv_src", "rank_counts"):
+        for name in self.BUFFERS:
             setattr(self, name, None)
-        self.B.ep_peer_free(self._own)
+        self.ops.free(self._own)
         self._own = None
+
+
+class CudaPeerOps:
+    """The peer path's memory (ep_peer_alloc / open / close / free, device
+    tables) and compute steps (layout, counts publish, dispatch, local
+    experts, combine) on the GPU, through the C ABI."""
+
+    def __init__(self, device=None):
+        from . import binding as B
+
+        self.B = B
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.rows = CudaRowOps()
+
+    # memory
+    def alloc(self, nbytes: int):
+        return self.B.ep_peer_alloc(nbytes)
+
+    def open(self, handle: bytes) -> int:
+        return self.B.ep_peer_open(handle)
+
+    def close(self, base: int) -> None:
+        self.B.ep_peer_close(base)
+
+    def free(self, base: int) -> None:
+        self.B.ep_peer_free(base)
+
+    def view(self, addr: int, shape, dtype):
+        return self.B.device_view(addr, shape, dtype, self.device)
+
+    def peers(self, rank: int, capacity: int, tables: dict):
+        t = {name: torch.tensor(addrs, dtype=torch.int64, device=self.device) for name, addrs in tables.items()}
+        return self.B.Peers(rank, capacity, t["recv_x"], t["y"], t["rank_counts"], recv_topk_idx=t["recv_topk_idx"],
+                            recv_topk_weights=t["recv_topk_weights"], recv_src=t["recv_src"])
+
+    def sync(self) -> None:
+        torch.cuda.current_stream(self.device).synchronize()
+
+    # compute steps
+    def layout(self, topk_idx, num_experts, world):
+        B = self.B
+        routing = B.Routing.topk(topk_idx, num_experts, world)
+        layout = B.Layout(routing, device=topk_idx.device)
+        B.ep_get_layout(routing, layout)
+        rl = B.RankLayout(routing, device=topk_idx.device)
+        B.ep_get_rank_layout(routing, layout, rl)
+        return routing, layout, rl
+
+    def publish(self, handle, peers) -> None:
+        routing, layout, _ = handle
+        self.B.ep_peer_publish_counts(routing, layout, peers)
+
+    def dispatch(self, x, topk_weights, handle, peers) -> None:
+        routing, layout, rl = handle
+        self.B.ep_dispatch_peers(x, routing, layout, rl, peers, topk_weights=topk_weights)
+
+    def local_experts(self, x, topk_idx, topk_weights, local_experts, expert_fn, out):
+        return self.rows.local_experts(x, topk_idx, topk_weights, local_experts, expert_fn, out=out)
+
+    def combine(self, handle, peers, hidden, out_dtype):
+        B = self.B
+        routing, layout, rl = handle
+        out = torch.empty((routing.T, hidden), dtype=out_dtype, device=self.device)
+        B.ep_combine_peers(routing, layout, rl, peers, out)
+        if B.ep_get_device_error(layout) != 0:
+            raise B.EPError(B.EP_ERR_OVERFLOW, "device error flagged in the peer exchange")
+        return out
