@@ -292,6 +292,8 @@ class PeerExpertParallel:
             dist.barrier(group=self.group)
 
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor) -> PeerReceived:
+        """The rows every rank sends here land in this rank's buffers; the
+        returned tensors are views of them, valid until the next dispatch."""
         if x.shape[1] != self.hidden or topk_idx.shape[1] != self.num_topk:
             raise ValueError("x is [T, %d] and topk_idx [T, %d] for this exchange" % (self.hidden, self.num_topk))
         handle = self.ops.layout(topk_idx, self.num_experts, self.world)
