@@ -505,8 +505,10 @@ def run_ours(args):
 
 def time_other_workloads(dev, flush, reps):
     """Per-op event timings of the decode (3), expert-choice (4) and skewed
-    (5) workloads, each op alone after an L2 flush, median of `reps`; returned
-    as {workload: {op: {"us", "gbs", "frac", "bytes"}}} for the bench line."""
+    (5) workloads, and of the prefill workload's quantised, per-rank and
+    peer-path rows, each op alone after an L2 flush, median of `reps`;
+    returned as {workload: {op: {"us", "gbs", "frac", "bytes"}}} for the
+    bench line."""
     import torch
 
     from combine_ep_get_10_b200 import binding as B
@@ -590,7 +592,59 @@ def time_other_workloads(dev, flush, reps):
         res[cfg["name"]] = ops
         del x, y, out, lay
         torch.cuda.empty_cache()
+    res["prefill-topk-4096x7168-top8 (quantised, per-rank and peer-path rows)"] = time_prefill_rows(
+        dev, timeit, rec, bf)
+    torch.cuda.empty_cache()
     return res
+
+
+def time_prefill_rows(dev, timeit, rec, bf):
+    """The prefill workload's other rows: every quantised dispatch format
+    (compact), the per-rank (deduplicated) dispatch and combine, and the
+    same over peer memory with the ranks emulated on this GPU."""
+    import torch
+
+    from combine_ep_get_10_b200 import binding as B
+    from combine_ep_get_10_b200 import workloads as W
+
+    inp = W.make_inputs(2)
+    cfg = inp["cfg"]
+    T, H, E, R, K = cfg["T"], cfg["H"], cfg["E"], cfg["R"], cfg["K"]
+    x = bf(inp["x"])
+    n_valid = int((inp["topk_idx"] >= 0).sum())
+    idx = torch.from_numpy(inp["topk_idx"]).to(dev)
+    w = torch.from_numpy(inp["topk_weights"]).to(dev)
+    rt = B.Routing.topk(idx, E, R)
+    lay = B.Layout(rt, device=dev)
+    B.ep_get_layout(rt, lay)
+    ops = {}
+    meta = T * K * 12 + E * 4
+    for name, dt, code_b, scale_b in QUANT_FORMATS:
+        cb, sb = code_b(H), scale_b(H)
+        q = torch.empty((n_valid, cb), dtype=torch.uint8, device=dev)
+        sc = torch.empty((n_valid, sb), dtype=torch.uint8, device=dev)
+        ops["dispatch_" + name] = rec(timeit(lambda: B.ep_dispatch(x, rt, lay, q, recv_scales=sc, out_dtype=dt)),
+                                      T * H * 2 + n_valid * (cb + sb) + meta)
+        del q, sc
+    rl = B.RankLayout(rt, device=dev)
+    ops["rank_layout"] = rec(timeit(lambda: B.ep_get_rank_layout(rt, lay, rl)),
+                             T * R + R * 4 + (R + 1) * 4 + T * R * 4)
+    n_rank = int(rl.rank_offsets[-1].item())
+    rrecv = torch.empty((n_rank, H), dtype=torch.bfloat16, device=dev)
+    ridx = torch.empty((n_rank, K), dtype=torch.int64, device=dev)
+    rwt = torch.empty((n_rank, K), dtype=torch.float32, device=dev)
+    ops["dispatch_ranks"] = rec(timeit(lambda: B.ep_dispatch_ranks(x, rt, lay, rl, rrecv, topk_weights=w,
+                                                                   recv_topk_idx=ridx, recv_topk_weights=rwt)),
+                                T * H * 2 + n_rank * H * 2 + n_rank * K * 12 + T * R * 4 + T * K * 12)
+    rout = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    ops["combine_ranks"] = rec(timeit(lambda: B.ep_combine_ranks(rrecv, rt, lay, rl, rout)),
+                               n_rank * H * 2 + T * H * 2 + T * R * 4)
+    del rrecv, ridx, rwt, rout
+    time_peer_path(cfg, x, w, rt, lay, rl, n_rank, dev, timeit,
+                   lambda cfg_, op, us, nbytes, tokens: ops.__setitem__(op, rec(us, nbytes)))
+    if B.ep_get_device_error(lay) != 0:
+        raise RuntimeError("device error flagged on the prefill rows")
+    return ops
 
 
 # quantised dispatch formats: (name, dtype code, code bytes per row, scale bytes per row)

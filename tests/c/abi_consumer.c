@@ -7,7 +7,9 @@
  *                          workspace sizing and argument rejection
  *   abi_consumer gpu    -- one small token-choice layout -> dispatch ->
  *                          combine on device memory from the CUDA runtime,
- *                          checked on the host against hand-computed values
+ *                          then the per-rank path over peer memory with two
+ *                          ranks in this process, checked on the host
+ *                          against hand-computed values
  *
  * Exit status 0 on success; each failed check prints a line and exits 1.
  */
@@ -62,6 +64,102 @@ static float bf16_to_f32(uint16_t b)
     float f;
     memcpy(&f, &u, 4);
     return f;
+}
+
+static void* peer_buffer(size_t bytes)
+{
+    void* p = NULL;
+    unsigned char handle[EP_IPC_HANDLE_BYTES];
+    CHECK(ep_peer_alloc(bytes, &p, handle) == EP_OK && p != NULL, "peer alloc");
+    CHECK(cudaMemset(p, 0xFF, bytes) == 0, "peer buffer fill");
+    return p;
+}
+
+static void* device_table(void* const* host, int n)
+{
+    void* d = NULL;
+    CHECK(cudaMalloc(&d, n * sizeof(void*)) == 0 && cudaMemcpy(d, host, n * sizeof(void*), H2D) == 0, "table");
+    return d;
+}
+
+/* The peer path with its two ranks in this process: both ranks hold the
+ * routing of gpu_mode (tokens 0..3 go to ranks {0,1}, {0}, {0,1}, {1}), so
+ * every rank receives 3 rows from each source, source 0's first.  The
+ * partial rows are the received rows themselves, so out[t] = (number of
+ * ranks of t) * (t + 1): 2, 2, 6, 4. */
+static void peer_mode(const void* d_x, const ep_routing_desc_t* r, const ep_layout_t* l, int T, int H, int K)
+{
+    enum { R = 2, CAP = 6 };
+    int32_t *d_roff, *d_rrow;
+    CHECK(cudaMalloc((void**)&d_roff, (R + 1) * 4) == 0 && cudaMalloc((void**)&d_rrow, T * R * 4) == 0, "cudaMalloc");
+    ep_rank_layout_t rl = {d_roff, d_rrow};
+    CHECK(ep_get_rank_layout(r, l, &rl, NULL) == EP_OK, "rank layout");
+    void *rx[R], *y[R], *ridx[R], *rsrc[R], *cnt[R];
+    for (int j = 0; j < R; ++j) {
+        rx[j] = peer_buffer(CAP * H * 2);
+        y[j] = peer_buffer(CAP * H * 2);
+        ridx[j] = peer_buffer(CAP * K * 8);
+        rsrc[j] = peer_buffer(CAP * 4);
+        cnt[j] = peer_buffer(R * R * 4);
+    }
+    ep_peers_t p[R];
+    for (int me = 0; me < R; ++me) {
+        memset(&p[me], 0, sizeof p[me]);
+        p[me].num_ranks = R;
+        p[me].rank = me;
+        p[me].capacity = CAP;
+        p[me].recv_x = (void* const*)device_table(rx, R);
+        p[me].recv_topk_idx = (int64_t* const*)device_table(ridx, R);
+        p[me].recv_src = (int32_t* const*)device_table(rsrc, R);
+        p[me].y = (const void* const*)device_table(y, R);
+        p[me].rank_counts = (int32_t* const*)device_table(cnt, R);
+    }
+    for (int me = 0; me < R; ++me)
+        CHECK(ep_peer_publish_counts(r, l, &p[me], NULL) == EP_OK, "publish counts");
+    for (int me = 0; me < R; ++me)
+        CHECK(ep_dispatch_peers(d_x, H, r, l, &rl, NULL, &p[me], NULL) == EP_OK, "dispatch peers");
+    const float want_row[R][CAP] = {{1, 2, 3, 1, 2, 3}, {1, 3, 4, 1, 3, 4}};
+    const int32_t want_src[R][CAP] = {{0, 1, 2, 0, 1, 2}, {0, 2, 3, 0, 2, 3}};
+    for (int j = 0; j < R; ++j) {
+        uint16_t rows[CAP * 8];
+        int32_t src[CAP], counts[R * R];
+        int64_t entries[2];
+        CHECK(cudaMemcpy(rows, rx[j], sizeof rows, D2H) == 0 && cudaMemcpy(src, rsrc[j], sizeof src, D2H) == 0 &&
+                  cudaMemcpy(counts, cnt[j], sizeof counts, D2H) == 0 &&
+                  cudaMemcpy(entries, ridx[j], sizeof entries, D2H) == 0,
+              "copy peer buffers");
+        for (int i = 0; i < R * R; ++i)
+            CHECK(counts[i] == 3, "every rank holds every rank's counts");
+        for (int row = 0; row < CAP; ++row) {
+            CHECK(bf16_to_f32(rows[row * H]) == want_row[j][row], "received row");
+            CHECK(src[row] == want_src[j][row], "received source token");
+        }
+        /* token 0 (experts 0 and 3): rank 0 sees (0, -1), rank 1 sees (-1, 1) */
+        CHECK(entries[0] == (j == 0 ? 0 : -1) && entries[1] == (j == 0 ? -1 : 1), "received top-k entries");
+        CHECK(cudaMemcpy(y[j], rx[j], CAP * H * 2, cudaMemcpyDeviceToDevice) == 0, "partial rows");
+    }
+    const float want_out[4] = {2.0f, 2.0f, 6.0f, 4.0f};
+    float* d_out;
+    CHECK(cudaMalloc((void**)&d_out, T * H * 4) == 0, "cudaMalloc");
+    for (int me = 0; me < R; ++me) {
+        float out[4 * 8];
+        CHECK(ep_combine_peers(H, r, l, &rl, &p[me], d_out, EP_FP32, NULL) == EP_OK, "combine peers");
+        CHECK(cudaMemcpy(out, d_out, sizeof out, D2H) == 0, "copy out");
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < H; ++h)
+                CHECK(out[t * H + h] == want_out[t], "peer combined value");
+    }
+    uint32_t flags = 1;
+    CHECK(ep_get_device_error(l, &flags, 1, NULL) == EP_OK && flags == 0, "device error word after the peer path");
+    for (int me = 0; me < R; ++me) {
+        cudaFree((void*)p[me].recv_x), cudaFree((void*)p[me].recv_topk_idx), cudaFree((void*)p[me].recv_src);
+        cudaFree((void*)p[me].y), cudaFree((void*)p[me].rank_counts);
+    }
+    for (int j = 0; j < R; ++j)
+        CHECK(ep_peer_free(rx[j]) == EP_OK && ep_peer_free(y[j]) == EP_OK && ep_peer_free(ridx[j]) == EP_OK &&
+                  ep_peer_free(rsrc[j]) == EP_OK && ep_peer_free(cnt[j]) == EP_OK,
+              "peer free");
+    cudaFree(d_out), cudaFree(d_roff), cudaFree(d_rrow);
 }
 
 static int gpu_mode(void)
@@ -148,6 +246,7 @@ static int gpu_mode(void)
     for (int t = 0; t < T; ++t)
         for (int h = 0; h < H; ++h)
             CHECK(out[t * H + h] == want_out[t], "combined value");
+    peer_mode(d_x, &r, &l, T, H, K);
     cudaDeviceSynchronize();
     cudaFree(d_idx), cudaFree(d_w), cudaFree(d_x), cudaFree(d_recv), cudaFree(d_out), cudaFree(d_ws);
     cudaFree(d_cnt), cudaFree(d_off), cudaFree(d_rcnt), cudaFree(d_slot), cudaFree(d_inr);

@@ -297,6 +297,33 @@ def test_peer_calls_check_their_tables():
         B.ep_dispatch_peers(to_dev(x, bf16=True), routing, layout, rl, L.peers[0])
 
 
+def test_peer_exchange_on_one_rank_nccl_matches_the_oracle():
+    """PeerExpertParallel on a one-rank NCCL group (the barrier between the
+    phases is NCCL's): its own block only, every token's experts local."""
+    import torch.distributed as dist
+
+    from combine_ep_get_10_b200.ep_exchange import PeerExpertParallel
+
+    E, H = 256, 1024
+    inputs = [rank_inputs(0, 1, 512, H, E)]
+    x, idx, w = inputs[0]
+    dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % _free_port(), rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        ep = PeerExpertParallel(E, H, idx.shape[1], capacity=len(x))
+        recv = ep.dispatch(to_dev(x, bf16=True), to_dev(idx), to_dev(w))
+        y = ep.experts(recv, expert_fn_for(0))
+        ob = ep.combine(y, recv, torch.bfloat16)
+        got = (host(recv.x).copy(), host(recv.src).copy(), recv.recv_counts, host(ob).copy())
+        ep.close()
+    finally:
+        dist.destroy_process_group()
+    ref = two_level_reference(inputs, E, 1)[0]
+    assert got[2] == ref["counts"]
+    assert np.array_equal(got[0], ref["x"]) and np.array_equal(got[1], ref["src"])
+    assert np.array_equal(got[3], ref["out_bf16"])
+
+
 def _ipc_worker(rank, world, port, q):
     import os
     import sys
