@@ -232,3 +232,70 @@ def test_peer_exchange_protocol_matches_the_single_process_oracle(world, oracle_
         assert ((rsrc >= 0) & (rsrc < 48 + 20 * (world - 1))).all()
         assert np.array_equal(out_bf16, ref[r]["two_bf16"])
         assert np.array_equal(out_f32.view(np.uint32), ref[r]["two_f32"].view(np.uint32))
+
+
+def _leaving_worker(rank, world, port, directory, kind, q):
+    """Rank 1 leaves between steps (after the exchange is set up, before the
+    step's first collective); rank 0 then runs a step."""
+    import sys
+    import time
+    from datetime import timedelta
+
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=5))
+    import oracle
+    from combine_ep_get_10_b200.ep_exchange import ExpertParallel, PeerExpertParallel
+    from test_ep_exchange_cpu import E, H, OracleRowOps, _bits_to_t, _inputs, tokens_of
+
+    oracle.build()
+    x, idx, w = _inputs(rank, world)
+    if kind == "peer":
+        ep = PeerExpertParallel(E, H, idx.shape[1], sum(tokens_of(i) for i in range(world)),
+                                ops=FilePeerOps(oracle, directory))
+    else:
+        ep = ExpertParallel(E, ops=OracleRowOps(oracle, rank, E // world))
+        dist.barrier()
+    if rank == 1:
+        q.put((rank, "left", 0.0))
+        q.close()
+        q.join_thread()
+        os._exit(0)  # no destroy_process_group: the rank is simply gone
+    t0 = time.time()
+    try:
+        ep.dispatch(_bits_to_t(x), torch.from_numpy(idx), torch.from_numpy(w))
+        q.put((rank, "no error", time.time() - t0))
+    except Exception as e:  # the collective fails: the peer is gone or the timeout ran out
+        q.put((rank, "raised " + type(e).__name__, time.time() - t0))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+@pytest.mark.parametrize("kind", ["peer", "alltoall"])
+def test_a_rank_that_leaves_fails_the_next_step_instead_of_hanging(kind, tmp_path):
+    """Failure detection on the host: with a short process-group timeout,
+    the remaining rank's next collective of the step (the barrier after the
+    counts publish, or the counts all-to-all) raises instead of waiting."""
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_leaving_worker, args=(r, 2, port, str(tmp_path), kind, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = {}
+    try:
+        for _ in range(2):
+            rank, what, secs = q.get(timeout=120)
+            res[rank] = (what, secs)
+    finally:
+        for p in procs:
+            p.join(timeout=30)
+            if p.exitcode is None:
+                p.kill()
+    assert res[1][0] == "left"
+    assert res[0][0].startswith("raised"), res[0]
+    assert res[0][1] < 60.0, res[0]
