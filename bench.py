@@ -439,8 +439,10 @@ def run_ours(args):
         raise RuntimeError("device error flagged during the end-to-end steps")
 
     # the other workloads' ops, timed in this process with clocks sampled
+    # (one GPU only: under torchrun the other ranks would wait at the final
+    # barrier meanwhile)
     other, other_clocks = None, None
-    if rank == 0 and not args.no_other_workloads:
+    if world == 1 and not args.no_other_workloads:
         with ClockSampler(local, uuid) as clocks2:
             other = time_other_workloads(dev, flush, args.other_reps)
         other_clocks = clocks2.summary()
