@@ -277,6 +277,54 @@ def test_peer_dispatch_beyond_capacity_is_flagged_and_stays_in_bounds():
         assert (host(L.idx[r][60:]) == -7).all() and (host(L.src[r][60:]) == -9).all(), r
 
 
+def test_peer_path_at_the_bench_configuration():
+    """Full size, as bench.py times the peer path: the prefill workload
+    (4096 x 7168, top-8 of 256, 8 ranks), this process as rank 4 of 8 ranks
+    that all hold its routing.  Every rank's block of received rows, entries
+    and source tokens equals the oracle's per-rank dispatch rows for that
+    rank, at rows 4 * count .. 5 * count of its buffer (rows around it
+    untouched); with each rank's received rows as its partial rows, the
+    combine equals the oracle's rank combine of the same rows, bit for bit
+    on all outputs."""
+    inp = W.make_inputs(2)
+    cfg = inp["cfg"]
+    T, H, E, R, K = cfg["T"], cfg["H"], cfg["E"], cfg["R"], cfg["K"]
+    x_np, idx_np, w_np = inp["x"], inp["topk_idx"], inp["topk_weights"]
+    L = oracle.tc_layout(idx_np, E, R)
+    RL = oracle.rank_layout(L["is_token_in_rank"])
+    D = oracle.rank_dispatch(x_np, idx_np, E, R, RL, topk_weights=w_np, want_src=True)
+    want_out = oracle.rank_combine(D["recv"], RL, out_dtype=oracle.BF16)
+
+    x, w = to_dev(x_np, bf16=True), to_dev(w_np)
+    rt = B.Routing.topk(to_dev(idx_np), E, R)
+    lay = B.Layout(rt)
+    B.ep_get_layout(rt, lay)
+    rl = B.RankLayout(rt)
+    B.ep_get_rank_layout(rt, lay, rl)
+    counts = host(lay.num_tokens_per_rank).astype(np.int64)
+    me = R // 2
+    capacity = int((me + 1) * counts.max())
+    Lr = LocalRanks(R, capacity, H, K)
+    for j in range(R):
+        Lr.counts[j].copy_(lay.num_tokens_per_rank.repeat(R, 1))
+    B.ep_dispatch_peers(x, rt, lay, rl, Lr.peers[me], topk_weights=w)
+    torch.cuda.synchronize()
+    offs = RL["rank_offsets"]
+    for j in range(R):
+        a, n = me * int(counts[j]), int(counts[j])
+        blk = slice(int(offs[j]), int(offs[j + 1]))
+        assert np.array_equal(host(Lr.recv_x[j][a:a + n]), D["recv"][blk]), j
+        assert np.array_equal(host(Lr.idx[j][a:a + n]), D["recv_topk_idx"][blk]), j
+        assert np.array_equal(host(Lr.w[j][a:a + n]).view(np.uint32), D["recv_topk_weights"][blk].view(np.uint32)), j
+        assert np.array_equal(host(Lr.src[j][a:a + n]), D["recv_src"][blk]), j
+        assert torch.isnan(Lr.recv_x[j][a - 1].float()).all() and (host(Lr.src[j][a + n:]) == -9).all(), j
+        Lr.y[j][a:a + n].copy_(Lr.recv_x[j][a:a + n])
+    out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    B.ep_combine_peers(rt, lay, rl, Lr.peers[me], out)
+    assert np.array_equal(host(out), want_out)
+    assert B.ep_get_device_error(lay) == 0
+
+
 def test_peer_calls_check_their_tables():
     E, world = 64, 2
     x, idx, w = rank_inputs(0, world, 16, 64, E, K=4)
