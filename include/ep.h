@@ -59,7 +59,7 @@ typedef enum {
     EP_ERR_OVERFLOW = 3,    /* device: destination row beyond the buffer */
     EP_ERR_WORKSPACE = 4,   /* workspace missing, misaligned or too small */
     EP_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
-    EP_ERR_UNSUPPORTED = 6, /* valid request this build does not handle */
+    EP_ERR_UNSUPPORTED = 6, /* valid request the library does not handle */
     EP_ERR_TIMEOUT = 7      /* device: a bounded wait gave up */
 } ep_status_t;
 
