@@ -123,3 +123,31 @@ def test_expert_choice_random_shapes(seed):
     B.ep_combine_expert_choice(recv, routing, lay, to_dev(ew), out)
     assert_combine_close(host(out), oracle.ec_combine(ref_d, ref_l, ew, T, out_dtype=W.BF16), True, "ec")
     assert B.ep_get_device_error(lay) == 0
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_peer_path_random_shapes(seed):
+    """The per-rank path over peer memory with its ranks emulated on the one
+    GPU (tests/test_gpu_peers.py): random rank counts (1..32), uneven token
+    batches per rank (some empty), -1 and duplicate ids, hidden sizes from 8
+    to 8800 (rows of two bulk chunks past 16 KB), capacity with or without
+    slack; received rows, entries, source tokens and both output precisions
+    bit for bit against the oracle's two-level composition."""
+    from test_gpu_peers import check_step, run_local
+
+    r = np.random.Generator(np.random.PCG64(5000 + seed))
+    world = int(r.choice([1, 2, 3, 4, 8, 16, 32]))
+    E = world * int(r.integers(1, 9))
+    K = int(r.integers(1, min(E, 10) + 1))
+    H = 8 * int(r.integers(1030, 1126) if seed % 4 == 3 else r.integers(1, 1101))  # every 4th: two chunks
+    inputs = []
+    for _ in range(world):
+        T = int(r.choice([0, 1, 5, 33, 100, 257]))
+        idx = W.random_topk(r, T, E, K, p_neg=float(r.choice([0.0, 0.2])), allow_dup=bool(r.random() < 0.3),
+                            p_bad=0.0)
+        x = W.to_bf16_bits((r.standard_normal((T, H)) * 10.0 ** r.uniform(-2, 2)).astype(np.float32))
+        w = r.standard_normal((T, K)).astype(np.float32)
+        inputs.append((np.ascontiguousarray(x), np.ascontiguousarray(idx, np.int64), np.ascontiguousarray(w)))
+    capacity = sum(len(x) for x, _, _ in inputs) + int(r.choice([0, 3]))
+    L, state = run_local(inputs, E, world, capacity)
+    check_step(L, state, inputs, E, world)
