@@ -1,7 +1,8 @@
 """Seeded random shapes through every entry point, against the CPU oracle:
 token counts, expert / rank / top-k counts, hidden sizes (ragged against the
 kernels' tiles), -1 and duplicate ids, padded overflow, every quantised
-format, the per-rank path and expert choice.  Deterministic (fixed seeds)."""
+format, the per-rank path, the per-rank path over peer memory and expert
+choice.  Deterministic (fixed seeds)."""
 import numpy as np
 import pytest
 import torch
