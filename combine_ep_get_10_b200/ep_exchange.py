@@ -29,8 +29,8 @@ DeepEP's combine forms.  The transfers are ``torch.distributed``
 all-to-all-v calls (NCCL over NVLink between GPUs, gloo between CPU
 processes; device tensors are staged through host memory for gloo): the
 counts on the host size the receive buffers, which is the one host
-synchronisation of a step.  bf16 rows travel as their 16-bit patterns.  No transfer here uses TMA multicast or hands a peer's memory to a
-library kernel.
+synchronisation of a step.  bf16 rows travel as their 16-bit patterns.  No
+transfer here hands a peer's memory to a library kernel.
 
 The compute steps are the CUDA kernels of the C ABI (``CudaRowOps``); the
 exchange itself takes any object with the same three methods, so that the
