@@ -262,11 +262,11 @@ class PeerExpertParallel:
             n = torch.Size(shape).numel() * torch.empty((), dtype=dtype).element_size()
             total += _align(max(n, 1))
         self._own, handle = self.ops.alloc(total)
-        handles = [None] * W
-        dist.all_gather_object(handles, handle, group=group)
         self._opened = []
         bases = []
         try:
+            handles = [None] * W
+            dist.all_gather_object(handles, handle, group=group)
             for r in range(W):
                 if r == self.rank:
                     bases.append(self._own)
@@ -274,8 +274,10 @@ class PeerExpertParallel:
                     base = self.ops.open(handles[r])
                     self._opened.append(base)
                     bases.append(base)
-        except Exception:
+        except Exception:  # no step has run: unmap what was mapped, free this rank's block
             self._release()
+            self.ops.free(self._own)
+            self._own = None
             raise
         self.peers = self.ops.peers(self.rank, C, {name: [b + off for b in bases]
                                                    for name, off in self.offsets.items()})
