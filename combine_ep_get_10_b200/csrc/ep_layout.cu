@@ -41,6 +41,12 @@ namespace {
 #define EP_LAYOUT_MAX_CLUSTER 16
 #endif
 // from this many (token, k) pairs on, the grid-wide kernel is used
+// one-CTA layouts launched without the cluster attribute: every launch is an
+// implicit cluster of one CTA, and the plain launch measured ~1 us faster
+// (decode and tiny batches: 14.3 -> 13.2 us, 12.3 -> 11.3 us event-timed)
+#ifndef EP_LAYOUT_SINGLE_PLAIN
+#define EP_LAYOUT_SINGLE_PLAIN 1
+#endif
 #ifndef EP_LAYOUT_GRID_MIN_PAIRS
 #define EP_LAYOUT_GRID_MIN_PAIRS 8192
 #endif
@@ -1212,7 +1218,7 @@ cudaError_t launch_tc_layout(const TcLayoutLaunch& a, cudaStream_t stream)
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = (EP_LAYOUT_SINGLE_PLAIN && cs == 1) ? 0 : 1;
     return cudaLaunchKernelEx(&cfg, tc_layout_cluster_kernel, k);
 }
 
