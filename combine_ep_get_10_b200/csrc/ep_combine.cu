@@ -130,6 +130,14 @@ constexpr int kEcLookup = EP_COMBINE_EC_LOOKUP;
 #define EP_COMBINE_EC_MINB 2
 #endif
 constexpr int kEcMinBlocks = EP_COMBINE_EC_MINB;
+// per-rank combines: when a token's rank rows are spread over more groups
+// than they fill, they are packed to the front (ascending rank kept) so that
+// their loads go out in fewer rounds.  Measured on the skewed 16384-token
+// batch (2.7 ranks per token): 153.6 -> 148.5 us; unchanged at 4096 tokens
+// (5.3 ranks per token; packing every token measured 2 us slower there)
+#ifndef EP_COMBINE_RANKS_COMPACT
+#define EP_COMBINE_RANKS_COMPACT 1
+#endif
 // heavy items: lookups pipelined (reduce_heavy) or not (reduce_segment)
 #ifndef EP_COMBINE_HEAVY_PIPE
 #define EP_COMBINE_HEAVY_PIPE 1
@@ -270,12 +278,32 @@ __device__ __forceinline__ void reduce_segment(const CombineArgs& a, int64_t t, 
                 my_row[i] = static_cast<RowT>(r);
             }
         }
+        int m_valid = 32;
+#if EP_COMBINE_RANKS_COMPACT
+        if constexpr ((kSrc == kSrcRanks || kSrc == kSrcPeers) && kLookup == 1) {
+            // the token's ranks first, in ascending order: its loads then fill
+            // the first group instead of spreading over all of them
+            const uint32_t valid = __ballot_sync(kFullMask, my_row[0] >= 0);
+            const int cnt = __popc(valid);
+            static_assert(kGroup == 4, "group occupancy by nibbles");
+            // groups (aligned nibbles) holding at least one of the token's ranks
+            const int touched = __popc((valid | (valid >> 1) | (valid >> 2) | (valid >> 3)) & 0x11111111u);
+            if ((cnt + kGroup - 1) / kGroup < touched) { // packing saves a round of loads
+                m_valid = cnt;
+                const int src = lane < cnt ? static_cast<int>(__fns(valid, 0, lane + 1)) : lane;
+                const RowT r = __shfl_sync(kFullMask, my_row[0], src);
+                const float wv = __shfl_sync(kFullMask, my_w[0], src);
+                my_row[0] = lane < cnt ? r : -1;
+                my_w[0] = lane < cnt ? wv : 0.0f;
+            }
+        }
+#endif
 #pragma unroll
         for (int i = 0; i < kLookup; ++i) {
             const int kb = k0 + 32 * i;
             if (kb >= n)
                 break; // warp-uniform
-            const int m = min(32, n - kb);
+            const int m = min(m_valid, n - kb);
             for (int g0 = 0; g0 < m; g0 += kGroup) {
                 RowT rows[kGroup];
                 float ws[kGroup];
