@@ -586,6 +586,9 @@ def time_other_workloads(dev, flush, reps):
             ops["ec_layout"] = rec(timeit(lambda: B.ep_get_layout(rt, lay)), S * 4 + (T + 1) * 4 + S * 4 + T * R + E * 4 + R * 4)
             y = torch.empty((S, H), dtype=torch.bfloat16, device=dev)
             ops["ec_dispatch"] = rec(timeit(lambda: B.ep_dispatch_expert_choice(x, rt, lay, y)), uniq * H * 2 + S * H * 2 + S * 4)
+            ops["ec_layout_dispatch"] = rec(timeit(lambda: B.ep_layout_dispatch_expert_choice(x, rt, lay, y)),
+                                            S * 4 + (T + 1) * 4 + S * 4 + T * R + E * 4 + R * 4
+                                            + uniq * H * 2 + S * H * 2 + S * 4)
             out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
             ops["ec_combine"] = rec(timeit(lambda: B.ep_combine_expert_choice(y, rt, lay, ew, out)),
                                     S * H * 2 + T * H * 2 + S * 8 + (T + 1) * 4)
@@ -864,6 +867,8 @@ def run_workload_table(args):
             recv = torch.empty((S, H), dtype=torch.bfloat16, device=dev)
             emit(cfg, "ec_dispatch", timeit(lambda: B.ep_dispatch_expert_choice(x, rt, lay, recv)),
                  uniq * H * 2 + S * H * 2 + S * 4, T)
+            emit(cfg, "ec_layout_dispatch (one call)", timeit(lambda: B.ep_layout_dispatch_expert_choice(x, rt, lay, recv)),
+                 S * 4 + (T + 1) * 4 + S * 4 + T * R + E * 4 + R * 4 + uniq * H * 2 + S * H * 2 + S * 4, T)
             out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
             emit(cfg, "ec_combine", timeit(lambda: B.ep_combine_expert_choice(recv, rt, lay, ew, out)),
                  S * H * 2 + T * H * 2 + S * 8 + (T + 1) * 4, T)

@@ -32,7 +32,8 @@ EXPORTED = ("ep_workspace_bytes", "ep_workspace_init", "ep_get_layout", "ep_disp
             "ep_dispatch_expert_choice", "ep_combine_expert_choice", "ep_get_device_error", "ep_status_string",
             "ep_version", "ep_get_layout_no_alloc", "ep_get_rank_layout", "ep_dispatch_ranks", "ep_combine_ranks",
             "ep_dispatch_low_latency", "ep_layout_dispatch", "ep_peer_alloc", "ep_peer_free", "ep_peer_open",
-            "ep_peer_close", "ep_peer_publish_counts", "ep_dispatch_peers", "ep_combine_peers")
+            "ep_peer_close", "ep_peer_publish_counts", "ep_dispatch_peers", "ep_combine_peers",
+            "ep_layout_dispatch_expert_choice")
 
 
 class EPError(RuntimeError):
@@ -92,6 +93,8 @@ def lib():
         L.ep_combine.argtypes = [P, i32, i64, RP, LP, st, i32, P, P, st, P]
         L.ep_dispatch_expert_choice.restype = st
         L.ep_dispatch_expert_choice.argtypes = [P, i32, RP, LP, P, P]
+        L.ep_layout_dispatch_expert_choice.restype = st
+        L.ep_layout_dispatch_expert_choice.argtypes = [P, i32, RP, LP, P, P]
         L.ep_combine_expert_choice.restype = st
         L.ep_combine_expert_choice.argtypes = [P, i32, RP, LP, P, P, st, P]
         L.ep_get_device_error.restype = st
@@ -366,6 +369,16 @@ def ep_dispatch_expert_choice(x: torch.Tensor, routing: Routing, layout: Layout,
     _check(lib().ep_dispatch_expert_choice(_ptr(x), x.shape[1], ctypes.byref(routing.desc),
                                            ctypes.byref(layout.desc), _ptr(recv_x), _stream(stream)),
            "ep_dispatch_expert_choice")
+
+
+def ep_layout_dispatch_expert_choice(x: torch.Tensor, routing: Routing, layout: Layout, recv_x: torch.Tensor,
+                                     stream=None) -> Layout:
+    """ep_get_layout + ep_dispatch_expert_choice in one call; the copy runs
+    under the layout kernel."""
+    _check(lib().ep_layout_dispatch_expert_choice(_ptr(x), x.shape[1], ctypes.byref(routing.desc),
+                                                  ctypes.byref(layout.desc), _ptr(recv_x), _stream(stream)),
+           "ep_layout_dispatch_expert_choice")
+    return layout
 
 
 def ep_combine_expert_choice(y: torch.Tensor, routing: Routing, layout: Layout, expert_weights: torch.Tensor,

@@ -427,10 +427,11 @@ ep_status_t ep_combine(const void* y, int32_t hidden, int64_t num_y_rows, const 
     return from_cuda(ep::launch_tc_combine(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-ep_status_t ep_dispatch_expert_choice(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
-                                      const ep_layout_t* layout, void* recv_x, ep_stream_t stream)
+namespace {
+
+ep_status_t check_ec_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                              const ep_layout_t* layout, const void* recv_x)
 {
-    CallRange range_("ep_dispatch_expert_choice");
     ep_status_t st = check_routing(routing);
     if (st != EP_OK)
         return st;
@@ -443,6 +444,12 @@ ep_status_t ep_dispatch_expert_choice(const void* x, int32_t hidden, const ep_ro
         return EP_ERR_INVALID_ARG;
     if ((routing->num_tokens > 0 && (x == nullptr || !aligned(x, 16))) || recv_x == nullptr || !aligned(recv_x, 16))
         return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+ep_status_t launch_ec_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                               const ep_layout_t* layout, void* recv_x, ep_stream_t stream, bool early_load)
+{
     ep::EcDispatchLaunch a{x,
                            routing->num_tokens,
                            hidden,
@@ -450,8 +457,38 @@ ep_status_t ep_dispatch_expert_choice(const void* x, int32_t hidden, const ep_ro
                            routing->capacity,
                            routing->token_indices,
                            recv_x,
-                           ep::error_word(layout->workspace)};
+                           ep::error_word(layout->workspace),
+                           early_load ? 1 : 0};
     return from_cuda(ep::launch_ec_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+} // namespace
+
+ep_status_t ep_dispatch_expert_choice(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                      const ep_layout_t* layout, void* recv_x, ep_stream_t stream)
+{
+    CallRange range_("ep_dispatch_expert_choice");
+    const ep_status_t st = check_ec_dispatch(x, hidden, routing, layout, recv_x);
+    if (st != EP_OK)
+        return st;
+    return launch_ec_dispatch(x, hidden, routing, layout, recv_x, stream, false);
+}
+
+ep_status_t ep_layout_dispatch_expert_choice(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                             const ep_layout_t* layout, void* recv_x, ep_stream_t stream)
+{
+    CallRange range_("ep_layout_dispatch_expert_choice");
+    // the dispatch's checks first: nothing is launched unless both calls can run
+    ep_status_t st = check_ec_dispatch(x, hidden, routing, layout, recv_x);
+    if (st != EP_OK)
+        return st;
+    st = get_layout(routing, layout, stream);
+    if (st != EP_OK)
+        return st;
+    st = launch_ec_dispatch(x, hidden, routing, layout, recv_x, stream, true);
+    if (st != EP_OK)
+        return st;
+    return ep::report_num_valid(routing, layout, reinterpret_cast<cudaStream_t>(stream));
 }
 
 ep_status_t ep_combine_expert_choice(const void* y, int32_t hidden, const ep_routing_desc_t* routing,

@@ -46,7 +46,12 @@ constexpr int64_t kChunkTarget = EP_DISPATCH_CHUNK; // bytes per bulk-copy item
 // (ep_layout_dispatch: the kernel before is that layout, which lets its
 // dependents start at once and writes neither x nor the routing), the
 // dispatch's CTAs start while the layout runs, load their source rows, and
-// wait only before reading the layout's results (early_load).
+// wait only before reading the layout's results (early_load).  The
+// expert-choice copy reads no layout result at all
+// (ep_layout_dispatch_expert_choice): its CTAs run under the whole layout
+// and only the grid's last CTA waits, before it ends, so that the grid never
+// completes before the layout does (a kernel launched after it in the same
+// way then sees the layout's CSR) while the other CTAs leave at once.
 #ifndef EP_DISPATCH_PDL
 #define EP_DISPATCH_PDL 1
 #endif
@@ -225,6 +230,8 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
         if (t < 0 || t >= a.T) {
             if (lane == 0 && c == 0 && t != -1)
                 flag_error(a.err, EP_DEVERR_BAD_INDEX);
+            if (a.early_load && blockIdx.x == gridDim.x - 1)
+                pdl_wait(); // this grid ends only after the layout before it
             return;
         }
         src_row = t;
@@ -238,8 +245,10 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
         mbar_arrive_expect_tx(&bar, bytes);
         bulk_load_g2s(buf, a.src + src_row * a.row_bytes + off, bytes, &bar);
     }
-    if (a.early_load)
-        pdl_wait(); // the layout's results (slot, offsets) are final from here on
+    // the layout's results (slot, offsets) are final from here on; the
+    // expert-choice copy reads none of them and waits only before it ends
+    if (a.early_load && !kExpertChoice)
+        pdl_wait();
     // destination rows of the first 32 pairs while the load is in flight
     int64_t dst_row = -1;
     uint8_t* dst = a.dst;
@@ -312,6 +321,10 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
         if (lane == 0)
             flag_error(a.err, any);
     }
+    // this grid ends only after the layout before it (for the kernels after
+    // it): its last CTA waits; the others leave at once and free their slots
+    if (kExpertChoice && a.early_load && blockIdx.x == gridDim.x - 1)
+        pdl_wait();
 }
 
 // Quantised payload formats (values of ep_dtype_t handled by the kernel).
@@ -878,6 +891,7 @@ cudaError_t launch_ec_dispatch(const EcDispatchLaunch& a, cudaStream_t stream)
     k.token_indices = a.token_indices;
     k.T = a.T;
     k.err = a.err;
+    k.early_load = a.early_load;
     return launch_bulk<kSrcEc>(k, S * k.nchunks, stream);
 }
 

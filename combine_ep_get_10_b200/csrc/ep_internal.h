@@ -115,6 +115,7 @@ struct EcDispatchLaunch {
     const int32_t* token_indices;
     void* recv_x;
     uint32_t* err;
+    int32_t early_load; // the layout kernel was launched just before by the library (see launch_pdl)
 };
 cudaError_t launch_ec_dispatch(const EcDispatchLaunch& a, cudaStream_t stream);
 

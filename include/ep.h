@@ -265,6 +265,17 @@ EP_API ep_status_t ep_combine(const void* y, int32_t hidden, int64_t num_y_rows,
 EP_API ep_status_t ep_dispatch_expert_choice(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
                                       const ep_layout_t* layout, void* recv_x, ep_stream_t stream);
 
+/* ep_get_layout followed by ep_dispatch_expert_choice, in one call (same
+ * arguments, results and checks; nothing is launched unless both calls can
+ * run).  The copy reads no result of the layout, so it runs while the layout
+ * kernel runs instead of after it; it still ends only after the layout has,
+ * so work that the caller queues next on `stream` sees both.  The separate
+ * calls cannot overlap this way: a dispatch alone must first wait for
+ * whatever kernel precedes it, which may have written x or token_indices.
+ * layout->num_valid_host is honoured as by ep_get_layout. */
+EP_API ep_status_t ep_layout_dispatch_expert_choice(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                                    const ep_layout_t* layout, void* recv_x, ep_stream_t stream);
+
 /* Expert-choice combine ([EC] Solution 1, the combine of the new API pair):
  *   out[t] = sum over the token's slots s in token_slots[token_offsets[t] ..
  *   token_offsets[t+1]) (ascending s) of expert_weights[s] * y[s], as an fmaf

@@ -251,3 +251,22 @@ def test_peer_calls_reject_bad_args(L):
     assert L.ep_peer_open(None, ctypes.byref(ptr)) == 1
     assert L.ep_peer_open(handle, None) == 1
     assert L.ep_peer_close(None) == 1 and L.ep_peer_free(None) == 1
+
+
+def test_layout_dispatch_expert_choice_checks_both_calls_before_launching(L):
+    """ep_layout_dispatch_expert_choice rejects what either
+    ep_dispatch_expert_choice or ep_get_layout would reject, before anything
+    is launched (no GPU here)."""
+    ec = _ec_desc()
+    ws = L.ep_workspace_bytes(ctypes.byref(ec))
+    good = B.LayoutDesc(0x1000, None, 0x1000, 0x1000, None, 0x1000, 0x1000, 0x100000, ws)
+    call = lambda lay, routing=ec, hidden=256, x=0x2000, recv=0x4000: L.ep_layout_dispatch_expert_choice(  # noqa: E731
+        x, hidden, ctypes.byref(routing), ctypes.byref(lay), recv, None)
+    assert call(good, routing=_topk_desc()) == 1  # token-choice routing
+    assert call(good, hidden=12) == 1
+    assert call(good, x=0x2008) == 1
+    assert call(good, recv=None) == 1
+    small = B.LayoutDesc(0x1000, None, 0x1000, 0x1000, None, 0x1000, 0x1000, 0x100000, 256)
+    assert call(small) == 4  # the layout needs its whole workspace
+    no_csr = B.LayoutDesc(0x1000, None, 0x1000, 0x1000, None, None, 0x1000, 0x100000, ws)
+    assert call(no_csr) == 1

@@ -464,6 +464,53 @@ def test_ec_skewed_mixed(T, E, C, H):
     assert B.ep_get_device_error(lay) == 0
 
 
+EC_ONE_CALL = [None, EC_EDGE[1], EC_EDGE[2], EC_EDGE[5], EC_EDGE[7]]  # None: the expert-choice workload, R = 8
+
+
+@pytest.mark.parametrize("case", EC_ONE_CALL, ids=["workload"] + [str(c[:4]) for c in EC_ONE_CALL[1:]])
+def test_ec_layout_dispatch_one_call_equals_the_two_calls(case):
+    """ep_layout_dispatch_expert_choice: the layout and the copy in one call
+    (the copy runs under the layout kernel and ends after it) writes the same
+    CSR, counts, rows and error bits as the two calls, against the oracle,
+    with the rows of empty or bad slots untouched and num_valid_host
+    reported; a combine queued right after it on the same stream, with no
+    synchronisation in between, reads the finished CSR (bit for bit)."""
+    if case is None:
+        inp = inputs(4)
+        c = inp["cfg"]
+        T, E, C, H, R = c["T"], c["E"], c["C"], c["H"], 8
+        ti, ew, x = inp["token_indices"], inp["expert_weights"], inp["x"]
+        r = rng(44)
+    else:
+        T, E, C, R, H, p_neg, p_bad, seed = case
+        r = rng(seed)
+        ti = W.random_token_indices(r, T, E, C, p_neg=p_neg, p_bad=p_bad)
+        x = W.to_bf16_bits(r.standard_normal((T, H)).astype(np.float32))
+        ew = r.standard_normal((E, C)).astype(np.float32)
+    ref_l = oracle.ec_layout(ti, T, R)
+    sentinel = np.full((E * C, H), 0x7FC1, np.uint16)
+    ref_recv = oracle.ec_dispatch(x, ti, recv=sentinel.copy())
+    tid, xd = to_dev(np.ascontiguousarray(ti, np.int32)), to_dev(x, bf16=True)
+    routing = B.Routing.expert_choice(tid, T, R)
+    lay = B.Layout(routing, report_num_valid=True)
+    recv = to_dev(sentinel, bf16=True)
+    B.ep_layout_dispatch_expert_choice(xd, routing, lay, recv)
+    assert lay.num_valid == int(ref_l["token_offsets"][-1])
+    check_ec_layout(lay, ref_l)
+    assert np.array_equal(host(recv), ref_recv)
+    flags = B.ep_get_device_error(lay)
+    assert bool(flags & B.EP_DEVERR_BAD_INDEX) == (ref_l["bad_index_count"] > 0)
+    # again without the host report, the combine queued straight behind it
+    lay2 = B.Layout(routing)
+    recv2 = to_dev(sentinel, bf16=True)
+    out = nan_filled((T, H), torch.float32)
+    B.ep_layout_dispatch_expert_choice(xd, routing, lay2, recv2)
+    B.ep_combine_expert_choice(recv2, routing, lay2, to_dev(ew), out)
+    ref = oracle.ec_combine(ref_recv, ref_l, ew, T, out_dtype=W.FP32)
+    assert exact_fraction(host(out), ref) == 1.0
+    assert np.array_equal(host(recv2), ref_recv)
+
+
 def test_device_error_word_clears():
     idx = np.array([[0, 9], [1, -1]], np.int64)  # 9 is out of range for E = 4
     _, lay, flags = gpu_tc_layout(idx, 4, 2)
