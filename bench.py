@@ -641,6 +641,11 @@ def time_prefill_rows(dev, timeit, rec, bf):
     ops["dispatch_ranks"] = rec(timeit(lambda: B.ep_dispatch_ranks(x, rt, lay, rl, rrecv, topk_weights=w,
                                                                    recv_topk_idx=ridx, recv_topk_weights=rwt)),
                                 T * H * 2 + n_rank * H * 2 + n_rank * K * 12 + T * R * 4 + T * K * 12)
+    ops["layout_dispatch_ranks"] = rec(
+        timeit(lambda: B.ep_layout_dispatch_ranks(x, rt, lay, rl, rrecv, topk_weights=w, recv_topk_idx=ridx,
+                                                  recv_topk_weights=rwt)),
+        T * K * 12 + T * R + E * 8 + R * 4 + T * R + R * 4 + (R + 1) * 4 + T * R * 4
+        + T * H * 2 + n_rank * H * 2 + n_rank * K * 12 + T * R * 4 + T * K * 12)
     rout = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     ops["combine_ranks"] = rec(timeit(lambda: B.ep_combine_ranks(rrecv, rt, lay, rl, rout)),
                                n_rank * H * 2 + T * H * 2 + T * R * 4)
@@ -835,6 +840,11 @@ def run_workload_table(args):
                      timeit(lambda: B.ep_dispatch_ranks(x, rt, lay, rl, rrecv, topk_weights=w, recv_topk_idx=ridx,
                                                         recv_topk_weights=rwt)),
                      T * H * 2 + n_rank * H * 2 + n_rank * K * 12 + T * R * 4 + T * K * 12, T)
+                emit(cfg, "layout_dispatch_ranks (one call: layout, rank layout, dispatch)",
+                     timeit(lambda: B.ep_layout_dispatch_ranks(x, rt, lay, rl, rrecv, topk_weights=w,
+                                                               recv_topk_idx=ridx, recv_topk_weights=rwt)),
+                     T * K * 12 + T * R + E * 8 + R * 4 + T * R + R * 4 + (R + 1) * 4 + T * R * 4
+                     + T * H * 2 + n_rank * H * 2 + n_rank * K * 12 + T * R * 4 + T * K * 12, T)
                 rout = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
                 emit(cfg, "combine_ranks", timeit(lambda: B.ep_combine_ranks(rrecv, rt, lay, rl, rout)),
                      n_rank * H * 2 + T * H * 2 + T * R * 4, T)

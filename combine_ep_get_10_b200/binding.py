@@ -33,7 +33,7 @@ EXPORTED = ("ep_workspace_bytes", "ep_workspace_init", "ep_get_layout", "ep_disp
             "ep_version", "ep_get_layout_no_alloc", "ep_get_rank_layout", "ep_dispatch_ranks", "ep_combine_ranks",
             "ep_dispatch_low_latency", "ep_layout_dispatch", "ep_peer_alloc", "ep_peer_free", "ep_peer_open",
             "ep_peer_close", "ep_peer_publish_counts", "ep_dispatch_peers", "ep_combine_peers",
-            "ep_layout_dispatch_expert_choice")
+            "ep_layout_dispatch_expert_choice", "ep_layout_dispatch_ranks")
 
 
 class EPError(RuntimeError):
@@ -110,6 +110,8 @@ def lib():
         L.ep_get_rank_layout.argtypes = [RP, LP, KP, P]
         L.ep_dispatch_ranks.restype = st
         L.ep_dispatch_ranks.argtypes = [P, i32, RP, LP, KP, i64, P, P, P, P, P, P]
+        L.ep_layout_dispatch_ranks.restype = st
+        L.ep_layout_dispatch_ranks.argtypes = [P, i32, RP, LP, KP, i64, P, P, P, P, P, P]
         L.ep_combine_ranks.restype = st
         L.ep_combine_ranks.argtypes = [P, i32, i64, RP, LP, KP, P, st, P]
         L.ep_dispatch_low_latency.restype = st
@@ -427,6 +429,18 @@ def ep_dispatch_ranks(x: torch.Tensor, routing: Routing, layout: Layout, rank_la
                                    ctypes.byref(rank_layout.desc), rows, _ptr(topk_weights), _ptr(recv_x),
                                    _ptr(recv_topk_idx), _ptr(recv_topk_weights), _ptr(recv_src), _stream(stream)),
            "ep_dispatch_ranks")
+
+
+def ep_layout_dispatch_ranks(x: torch.Tensor, routing: Routing, layout: Layout, rank_layout: RankLayout,
+                             recv_x: torch.Tensor, *, num_recv_rows=None, topk_weights=None, recv_topk_idx=None,
+                             recv_topk_weights=None, recv_src=None, stream=None) -> None:
+    """ep_get_layout + ep_get_rank_layout + ep_dispatch_ranks in one call;
+    the rows are loaded while the rank layout runs."""
+    rows = recv_x.shape[0] if num_recv_rows is None else int(num_recv_rows)
+    _check(lib().ep_layout_dispatch_ranks(_ptr(x), x.shape[1], ctypes.byref(routing.desc), ctypes.byref(layout.desc),
+                                          ctypes.byref(rank_layout.desc), rows, _ptr(topk_weights), _ptr(recv_x),
+                                          _ptr(recv_topk_idx), _ptr(recv_topk_weights), _ptr(recv_src),
+                                          _stream(stream)), "ep_layout_dispatch_ranks")
 
 
 def ep_combine_ranks(y: torch.Tensor, routing: Routing, layout: Layout, rank_layout: RankLayout, out: torch.Tensor,

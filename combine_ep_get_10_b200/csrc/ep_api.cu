@@ -118,7 +118,12 @@ ep::TcRows tc_rows(const ep_routing_desc_t* r, const ep_layout_t* l, ep_buffer_m
 }
 
 // ep_get_layout without the host report: argument checks and the launch.
-ep_status_t get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream);
+// trigger: the caller launches its own dispatch next, which may start while
+// the layout runs (it reads the layout's results only after waiting for it,
+// and through L2); without it the kernel launched next starts after the
+// layout has finished.
+ep_status_t get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream,
+                       bool trigger = false);
 
 } // namespace
 
@@ -168,7 +173,8 @@ ep_status_t ep_get_layout(const ep_routing_desc_t* routing, const ep_layout_t* l
 
 namespace {
 
-ep_status_t get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream)
+ep_status_t get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout, ep_stream_t stream,
+                       bool trigger)
 {
     ep_status_t st = check_routing(routing);
     if (st != EP_OK)
@@ -202,7 +208,8 @@ ep_status_t get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layo
                              layout->is_token_in_rank,
                              layout->slot,
                              err,
-                             layout->workspace};
+                             layout->workspace,
+                             trigger ? 1 : 0};
         return from_cuda(ep::launch_tc_layout(a, s));
     }
     if (layout->token_offsets == nullptr || layout->token_slots == nullptr || !aligned(layout->token_offsets, 4) ||
@@ -219,7 +226,8 @@ ep_status_t get_layout(const ep_routing_desc_t* routing, const ep_layout_t* layo
                          layout->token_offsets,
                          layout->token_slots,
                          layout->workspace,
-                         err};
+                         err,
+                         trigger ? 1 : 0};
     return from_cuda(ep::launch_ec_layout(a, s));
 }
 
@@ -319,7 +327,7 @@ ep_status_t ep_layout_dispatch(const void* x, int32_t hidden, const ep_routing_d
                                          out_dtype, topk_weights, recv_x, recv_scales, recv_src, recv_weights);
     if (st != EP_OK)
         return st;
-    st = get_layout(routing, layout, stream);
+    st = get_layout(routing, layout, stream, true);
     if (st != EP_OK)
         return st;
     st = launch_dispatch(x, hidden, routing, layout, mode, max_tokens_per_expert, num_recv_rows, out_dtype,
@@ -383,7 +391,7 @@ ep_status_t ep_dispatch_low_latency(const void* x, int32_t hidden, const ep_rout
                                ep::error_word(layout->workspace)};
         st = from_cuda(ep::launch_ll_dispatch(a, s));
     } else {
-        st = get_layout(routing, layout, stream);
+        st = get_layout(routing, layout, stream, true);
         if (st == EP_OK)
             st = launch_dispatch(x, hidden, routing, layout, EP_LAYOUT_PADDED, max_tokens_per_expert, rows,
                                  out_dtype, topk_weights, recv_x, recv_scales, recv_src, recv_weights, stream, true);
@@ -482,7 +490,7 @@ ep_status_t ep_layout_dispatch_expert_choice(const void* x, int32_t hidden, cons
     ep_status_t st = check_ec_dispatch(x, hidden, routing, layout, recv_x);
     if (st != EP_OK)
         return st;
-    st = get_layout(routing, layout, stream);
+    st = get_layout(routing, layout, stream, true);
     if (st != EP_OK)
         return st;
     st = launch_ec_dispatch(x, hidden, routing, layout, recv_x, stream, true);
@@ -601,12 +609,103 @@ ep_status_t ep_get_rank_layout(const ep_routing_desc_t* routing, const ep_layout
     return from_cuda(ep::launch_rank_layout(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+
+ep_status_t check_rank_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                const ep_layout_t* layout, const ep_rank_layout_t* rank_layout, int64_t num_recv_rows,
+                                const float* topk_weights, const void* recv_x, const int64_t* recv_topk_idx,
+                                const float* recv_topk_weights, const int32_t* recv_src);
+
+ep_status_t launch_rank_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                 const ep_layout_t* layout, const ep_rank_layout_t* rank_layout,
+                                 int64_t num_recv_rows, const float* topk_weights, void* recv_x,
+                                 int64_t* recv_topk_idx, float* recv_topk_weights, int32_t* recv_src,
+                                 ep_stream_t stream, bool early_load)
+{
+    ep::RankDispatchLaunch a{x,
+                             routing->num_tokens,
+                             hidden,
+                             routing->num_topk,
+                             routing->num_experts,
+                             routing->num_ranks,
+                             routing->topk_idx,
+                             topk_weights,
+                             rank_layout->rank_row,
+                             num_recv_rows,
+                             recv_x,
+                             recv_topk_idx,
+                             recv_topk_weights,
+                             recv_src,
+                             ep::error_word(layout->workspace),
+                             ep::PeerTables{},
+                             early_load ? 1 : 0};
+    return from_cuda(ep::launch_rank_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t launch_rank_layout(const ep_routing_desc_t* routing, const ep_layout_t* layout,
+                               const ep_rank_layout_t* rank_layout, ep_stream_t stream)
+{
+    ep::RankLayoutLaunch a{layout->is_token_in_rank,
+                           layout->num_tokens_per_rank,
+                           routing->num_tokens,
+                           routing->num_ranks,
+                           rank_layout->rank_offsets,
+                           rank_layout->rank_row,
+                           1}; // the per-rank dispatch of the same call follows
+    return from_cuda(ep::launch_rank_layout(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+} // namespace
+
+ep_status_t ep_layout_dispatch_ranks(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                     const ep_layout_t* layout, const ep_rank_layout_t* rank_layout,
+                                     int64_t num_recv_rows, const float* topk_weights, void* recv_x,
+                                     int64_t* recv_topk_idx, float* recv_topk_weights, int32_t* recv_src,
+                                     ep_stream_t stream)
+{
+    CallRange range_("ep_layout_dispatch_ranks");
+    // every call's checks first: nothing is launched unless all three can run
+    ep_status_t st = check_rank_dispatch(x, hidden, routing, layout, rank_layout, num_recv_rows, topk_weights,
+                                         recv_x, recv_topk_idx, recv_topk_weights, recv_src);
+    if (st != EP_OK)
+        return st;
+    st = check_workspace(routing, layout, true);
+    if (st != EP_OK)
+        return st;
+    if (layout->num_tokens_per_rank == nullptr || !aligned(layout->num_tokens_per_rank, 4) ||
+        (routing->num_tokens > 0 && layout->is_token_in_rank == nullptr))
+        return EP_ERR_INVALID_ARG;
+    st = get_layout(routing, layout, stream);
+    if (st != EP_OK)
+        return st;
+    st = launch_rank_layout(routing, layout, rank_layout, stream);
+    if (st != EP_OK)
+        return st;
+    return launch_rank_dispatch(x, hidden, routing, layout, rank_layout, num_recv_rows, topk_weights, recv_x,
+                                recv_topk_idx, recv_topk_weights, recv_src, stream, true);
+}
+
 ep_status_t ep_dispatch_ranks(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
                               const ep_layout_t* layout, const ep_rank_layout_t* rank_layout, int64_t num_recv_rows,
                               const float* topk_weights, void* recv_x, int64_t* recv_topk_idx,
                               float* recv_topk_weights, int32_t* recv_src, ep_stream_t stream)
 {
     CallRange range_("ep_dispatch_ranks");
+    const ep_status_t st = check_rank_dispatch(x, hidden, routing, layout, rank_layout, num_recv_rows, topk_weights,
+                                               recv_x, recv_topk_idx, recv_topk_weights, recv_src);
+    if (st != EP_OK)
+        return st;
+    return launch_rank_dispatch(x, hidden, routing, layout, rank_layout, num_recv_rows, topk_weights, recv_x,
+                                recv_topk_idx, recv_topk_weights, recv_src, stream, false);
+}
+
+namespace {
+
+ep_status_t check_rank_dispatch(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                const ep_layout_t* layout, const ep_rank_layout_t* rank_layout, int64_t num_recv_rows,
+                                const float* topk_weights, const void* recv_x, const int64_t* recv_topk_idx,
+                                const float* recv_topk_weights, const int32_t* recv_src)
+{
     ep_status_t st = check_rank_call(routing, layout, rank_layout);
     if (st != EP_OK)
         return st;
@@ -624,23 +723,10 @@ ep_status_t ep_dispatch_ranks(const void* x, int32_t hidden, const ep_routing_de
         return EP_ERR_INVALID_ARG;
     if (recv_src != nullptr && !aligned(recv_src, 4))
         return EP_ERR_INVALID_ARG;
-    ep::RankDispatchLaunch a{x,
-                             T,
-                             hidden,
-                             routing->num_topk,
-                             routing->num_experts,
-                             routing->num_ranks,
-                             routing->topk_idx,
-                             topk_weights,
-                             rank_layout->rank_row,
-                             num_recv_rows,
-                             recv_x,
-                             recv_topk_idx,
-                             recv_topk_weights,
-                             recv_src,
-                             ep::error_word(layout->workspace)};
-    return from_cuda(ep::launch_rank_dispatch(a, reinterpret_cast<cudaStream_t>(stream)));
+    return EP_OK;
 }
+
+} // namespace
 
 ep_status_t ep_combine_ranks(const void* y, int32_t hidden, int64_t num_y_rows, const ep_routing_desc_t* routing,
                              const ep_layout_t* layout, const ep_rank_layout_t* rank_layout, void* out,

@@ -134,6 +134,22 @@ __device__ __forceinline__ void bulk_wait_read_all()
 }
 
 // ------------------------------------------------------------ plain memory
+// Loads of the layout's results (slots, offsets, rank rows, counts) in the
+// dispatch kernels.  A dispatch runs as a programmatic dependent of the
+// kernel before it, and inside the library's one-call entry points that
+// kernel is the layout, which lets the dispatch start at once: the
+// dispatch's CTAs are then resident while the layout still writes these
+// arrays.  After griddepcontrol.wait they are read through L2 (.cg), never
+// through the read-only (.nc) path, which was measured returning stale
+// values in exactly that situation.  (The combine kernels keep the
+// read-only path: no kernel that lets its dependents start early is ever
+// launched directly before a combine.)
+template <typename T>
+__device__ __forceinline__ T ld_meta(const T* p)
+{
+    return __ldcg(p);
+}
+
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p)
 {
     uint4 r;

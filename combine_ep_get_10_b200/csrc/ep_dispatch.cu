@@ -85,7 +85,7 @@ struct RowMap {
     __device__ __forceinline__ int64_t row(int64_t t, int k, uint32_t& errbits) const
     {
         const int64_t e = __ldg(topk_idx + t * K + k);
-        const int32_t s = __ldg(slot + t * K + k);
+        const int32_t s = ld_meta(slot + t * K + k);
         if (e < 0 || e >= E || s < 0) {
             if (e < -1 || e >= E)
                 errbits |= EP_DEVERR_BAD_INDEX;
@@ -99,7 +99,7 @@ struct RowMap {
             }
             r = e * max_tokens + s;
         } else {
-            r = static_cast<int64_t>(__ldg(offsets + e)) + s;
+            r = static_cast<int64_t>(ld_meta(offsets + e)) + s;
         }
         if (r >= num_rows) {
             errbits |= EP_DEVERR_OVERFLOW;
@@ -151,9 +151,9 @@ __device__ __forceinline__ T* table_at(const unsigned long long* table, int r)
 __device__ __forceinline__ int64_t peer_row(const PeerTables& p, int R, int j, int64_t row, uint32_t& errbits)
 {
     const int32_t* counts = table_at<const int32_t>(p.rank_counts, p.me);
-    int64_t local = row - __ldg(p.rank_offsets + j);
+    int64_t local = row - ld_meta(p.rank_offsets + j);
     for (int i = 0; i < p.me; ++i)
-        local += __ldg(counts + i * R + j);
+        local += ld_meta(counts + i * R + j);
     if (local < 0 || local >= p.capacity) {
         errbits |= EP_DEVERR_OVERFLOW;
         return -1;
@@ -170,7 +170,7 @@ __device__ __forceinline__ void write_rank_topk(const BulkArgs& a, int64_t t, in
     for (int j = lane; j < a.R * K; j += 32) {
         const int r = j / K;
         const int k = j - r * K;
-        const int64_t row = __ldg(a.rank_row + t * a.R + r);
+        const int64_t row = ld_meta(a.rank_row + t * a.R + r);
         if (row < 0 || row >= a.map.num_rows)
             continue;
         const int64_t e = __ldg(a.map.topk_idx + t * K + k);
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
         dst_row = lane == 0 ? r : -1;
     } else if constexpr (kSrc == kSrcPeers) {
         if (lane < a.R) {
-            const int64_t row = __ldg(a.rank_row + r * a.R + lane);
+            const int64_t row = ld_meta(a.rank_row + r * a.R + lane);
             if (row >= 0) {
                 dst_row = peer_row(a.peers, a.R, lane, row, errbits);
                 dst = table_at<uint8_t>(a.peers.recv_x, lane);
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(32) bulk_dispatch_kernel(BulkArgs a)
         }
     } else if constexpr (kSrc == kSrcRanks) {
         if (lane < a.R) {
-            dst_row = __ldg(a.rank_row + r * a.R + lane);
+            dst_row = ld_meta(a.rank_row + r * a.R + lane);
             if (dst_row >= a.map.num_rows) {
                 errbits |= EP_DEVERR_OVERFLOW;
                 dst_row = -1;
@@ -918,6 +918,7 @@ cudaError_t launch_rank_dispatch(const RankDispatchLaunch& a, cudaStream_t strea
     k.recv_topk_weights = a.recv_topk_weights;
     k.T = a.T;
     k.err = a.err;
+    k.early_load = a.early_load;
     if (a.peers.recv_x != nullptr) {
         k.peers = a.peers;
         return launch_bulk<kSrcPeers>(k, static_cast<int64_t>(a.T) * k.nchunks, stream);

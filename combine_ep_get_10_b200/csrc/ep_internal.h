@@ -35,6 +35,9 @@ struct TcLayoutLaunch {
     int32_t* slot;
     uint32_t* err;
     void* workspace; // header + per-CTA totals of the grid-wide kernel
+    // let the kernel launched next start at once (a dispatch of the same call
+    // that reads the layout's results through L2 only after griddepcontrol.wait)
+    int32_t trigger_dependents;
 };
 size_t tc_layout_workspace_bytes(int64_t E);
 cudaError_t launch_tc_layout(const TcLayoutLaunch& a, cudaStream_t stream);
@@ -49,6 +52,7 @@ struct EcLayoutLaunch {
     int32_t* token_slots;
     void* workspace; // header, then tmask[T], fill[T], scratch[E*C]
     uint32_t* err;
+    int32_t trigger_dependents; // as for TcLayoutLaunch
 };
 size_t ec_layout_workspace_bytes(int64_t T, int64_t E, int64_t C);
 cudaError_t launch_ec_layout(const EcLayoutLaunch& a, cudaStream_t stream);
@@ -59,6 +63,7 @@ struct RankLayoutLaunch {
     int32_t T, R;
     int32_t* rank_offsets;
     int32_t* rank_row;
+    int32_t trigger_dependents; // as for TcLayoutLaunch
 };
 cudaError_t launch_rank_layout(const RankLayoutLaunch& a, cudaStream_t stream);
 
@@ -155,7 +160,8 @@ struct RankDispatchLaunch {
     float* recv_topk_weights;
     int32_t* recv_src;
     uint32_t* err;
-    PeerTables peers; // peers.recv_x != nullptr: rows go to the ranks' buffers
+    PeerTables peers;   // peers.recv_x != nullptr: rows go to the ranks' buffers
+    int32_t early_load; // the rank layout was launched just before by the library (see launch_pdl)
 };
 cudaError_t launch_rank_dispatch(const RankDispatchLaunch& a, cudaStream_t stream);
 

@@ -70,6 +70,7 @@ struct TcArgs {
     int32_t* slot;
     uint32_t* err;
     int32_t in_rank_words; // 1: write is_token_in_rank as 32-bit words
+    int32_t trigger;       // let the dispatch launched next start at once
 };
 
 __device__ __forceinline__ void write_rank_row(const TcArgs& a, int64_t t, uint32_t mask)
@@ -131,7 +132,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& 
 
 __global__ void __launch_bounds__(kLayoutThreads, 1) tc_layout_cluster_kernel(TcArgs a)
 {
-    pdl_launch_dependents(); // a dispatch launched after this may load its rows now
+    if (a.trigger)
+        pdl_launch_dependents(); // the dispatch of the same call may load its rows now
     cg::cluster_group cluster = cg::this_cluster();
     const int cs = static_cast<int>(cluster.num_blocks());
     const int b = static_cast<int>(cluster.block_rank());
@@ -409,7 +411,8 @@ __device__ __forceinline__ bool grid_sync(GridBar bar, uint32_t nblocks, uint32_
 __global__ void __launch_bounds__(kGridThreads) tc_layout_grid_kernel(TcArgs a, int32_t* tile_counts,
                                                                       int32_t* tile_ranks, GridBar bar)
 {
-    pdl_launch_dependents(); // a dispatch launched after this may load its rows now
+    if (a.trigger)
+        pdl_launch_dependents(); // the dispatch of the same call may load its rows now
     const int G = static_cast<int>(gridDim.x);
     const int b = static_cast<int>(blockIdx.x);
     extern __shared__ __align__(16) int32_t smem[];
@@ -776,6 +779,7 @@ struct EcClusterArgs {
     int32_t* token_offsets;
     int32_t* token_slots;
     uint32_t* err;
+    int32_t trigger; // let the dispatch launched next start at once
 };
 
 // per-token arrays are padded to a multiple of 4 tokens for 16-byte DSMEM access
@@ -791,7 +795,8 @@ size_t ec_cluster_smem_bytes(int64_t T, int64_t spc, int64_t E)
 
 __global__ void __launch_bounds__(kEcClusterThreads, 1) ec_layout_cluster_kernel(EcClusterArgs a, int32_t spc)
 {
-    pdl_launch_dependents(); // a dispatch launched after this may load its rows now
+    if (a.trigger)
+        pdl_launch_dependents(); // the dispatch of the same call may load its rows now
     cg::cluster_group cluster = cg::this_cluster();
     const int cs = static_cast<int>(cluster.num_blocks());
     const int b = static_cast<int>(cluster.block_rank());
@@ -1192,6 +1197,7 @@ cudaError_t launch_tc_layout(const TcLayoutLaunch& a, cudaStream_t stream)
     k.slot = a.slot;
     k.err = a.err;
     k.in_rank_words = (a.R % 4 == 0 && (reinterpret_cast<uintptr_t>(a.in_rank) & 3u) == 0) ? 1 : 0;
+    k.trigger = a.trigger_dependents;
 
     if (static_cast<int64_t>(a.T) * a.K >= EP_LAYOUT_GRID_MIN_PAIRS && a.workspace != nullptr)
         return launch_tc_layout_grid(k, a.workspace, stream);
@@ -1262,7 +1268,7 @@ cudaError_t launch_ec_layout_cluster(const EcLayoutLaunch& a, cudaStream_t strea
             ec_smem_attr_dev[dev] = 1;
     }
     EcClusterArgs k{a.token_indices, a.T, a.E, a.C, a.R, a.E / a.R, a.counts, a.rank_counts, a.in_rank,
-                    a.token_offsets, a.token_slots, a.err};
+                    a.token_offsets, a.token_slots, a.err, a.trigger_dependents};
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     cfg.gridDim = dim3(cs);

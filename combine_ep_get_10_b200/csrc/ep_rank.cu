@@ -51,7 +51,8 @@ __device__ __forceinline__ uint32_t token_mask(const uint8_t* in_rank, int64_t t
 
 __global__ void __launch_bounds__(kRankThreads) rank_layout_kernel(RankLayoutLaunch a)
 {
-    pdl_launch_dependents(); // a per-rank dispatch launched after this may load its rows now
+    if (a.trigger_dependents)
+        pdl_launch_dependents(); // the per-rank dispatch of the same call may load its rows now
     __shared__ int32_t s_base[32];             // first row of each rank in this tile
     __shared__ int32_t s_wpre[kRankWarps][33]; // per warp, per rank: counts, then rows before the warp
     const int tid = threadIdx.x;

@@ -324,6 +324,18 @@ EP_API ep_status_t ep_dispatch_ranks(const void* x, int32_t hidden, const ep_rou
                                      int64_t* recv_topk_idx, float* recv_topk_weights, int32_t* recv_src,
                                      ep_stream_t stream);
 
+/* ep_get_layout, ep_get_rank_layout and ep_dispatch_ranks in one call (the
+ * same arguments, results and checks; nothing is launched unless all three
+ * can run).  The dispatch's CTAs load their source rows while the rank
+ * layout kernel runs and wait for it only before they read rank_row; the
+ * separate calls cannot overlap this way, since a dispatch alone must first
+ * wait for whatever kernel precedes it (it may have written x). */
+EP_API ep_status_t ep_layout_dispatch_ranks(const void* x, int32_t hidden, const ep_routing_desc_t* routing,
+                                            const ep_layout_t* layout, const ep_rank_layout_t* rank_layout,
+                                            int64_t num_recv_rows, const float* topk_weights, void* recv_x,
+                                            int64_t* recv_topk_idx, float* recv_topk_weights, int32_t* recv_src,
+                                            ep_stream_t stream);
+
 /* Rank-level combine: out[t] = sum over the token's ranks r in ascending
  * order of y[rank_row[t, r]], fp32 additions from 0 (the ranks have applied
  * the gate weights), written as fp32 or rounded once (RNE) to bf16; a token

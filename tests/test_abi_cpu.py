@@ -270,3 +270,23 @@ def test_layout_dispatch_expert_choice_checks_both_calls_before_launching(L):
     assert call(small) == 4  # the layout needs its whole workspace
     no_csr = B.LayoutDesc(0x1000, None, 0x1000, 0x1000, None, None, 0x1000, 0x100000, ws)
     assert call(no_csr) == 1
+
+
+def test_layout_dispatch_ranks_checks_every_call_before_launching(L):
+    """ep_layout_dispatch_ranks rejects what ep_get_layout, ep_get_rank_layout
+    or ep_dispatch_ranks would reject, before anything is launched."""
+    d = _topk_desc()
+    ws = L.ep_workspace_bytes(ctypes.byref(d))
+    good = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x100000, ws)
+    rl = B.RankLayoutDesc(0x7000, 0x7100)
+    call = lambda lay, hidden=256, x=0x2000, rank_layout=rl, routing=d: L.ep_layout_dispatch_ranks(  # noqa: E731
+        x, hidden, ctypes.byref(routing), ctypes.byref(lay), ctypes.byref(rank_layout), 32, None, 0x4000, None, None,
+        None, None)
+    assert call(good, hidden=12) == 1
+    assert call(good, x=0x2008) == 1
+    assert call(good, routing=_ec_desc()) == 1
+    assert call(good, rank_layout=B.RankLayoutDesc(None, 0x7100)) == 1
+    small = B.LayoutDesc(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x100000, 256)
+    assert call(small) == 4  # the layout needs its whole workspace
+    no_in_rank = B.LayoutDesc(0x1000, 0x1000, 0x1000, None, 0x1000, None, None, 0x100000, ws)
+    assert call(no_in_rank) == 1

@@ -169,3 +169,40 @@ def test_rank_dispatch_overflow_is_flagged():
     out = torch.empty((T, H), dtype=torch.float32, device="cuda")
     B.ep_combine_ranks(recv, routing, lay, rl, out, num_y_rows=cut)
     assert B.ep_get_device_error(lay) & B.EP_DEVERR_OVERFLOW
+
+
+@pytest.mark.parametrize("wl", [2, 5])
+def test_layout_dispatch_ranks_one_call_equals_the_three_calls(wl):
+    """ep_layout_dispatch_ranks: the layout, the rank layout and the per-rank
+    dispatch in one call (the rows are loaded while the rank layout runs)
+    writes the same layouts, rows, entries and sources as the three calls,
+    bit for bit, on the full prefill and skewed workloads."""
+    inp = W.make_inputs(wl)
+    c = inp["cfg"]
+    x, idx, w = inp["x"], inp["topk_idx"], inp["topk_weights"]
+    T, H, E, R, K = c["T"], c["H"], c["E"], c["R"], c["K"]
+    xd, wd = to_dev(x, bf16=True), to_dev(w)
+    routing, lay, rl = _layouts(idx, E, R)
+    rows = int(host(rl.rank_offsets)[-1])
+    outs = []
+    for one_call in (False, True):
+        recv = torch.full((rows, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ridx = torch.full((rows, K), -7, dtype=torch.int64, device="cuda")
+        rw = torch.full((rows, K), float("nan"), dtype=torch.float32, device="cuda")
+        src = torch.full((rows,), -9, dtype=torch.int32, device="cuda")
+        if one_call:
+            lay = B.Layout(routing)
+            rl = B.RankLayout(routing)
+            B.ep_layout_dispatch_ranks(xd, routing, lay, rl, recv, topk_weights=wd, recv_topk_idx=ridx,
+                                       recv_topk_weights=rw, recv_src=src)
+        else:
+            B.ep_dispatch_ranks(xd, routing, lay, rl, recv, topk_weights=wd, recv_topk_idx=ridx, recv_topk_weights=rw,
+                                recv_src=src)
+        assert B.ep_get_device_error(lay) == 0
+        outs.append((host(rl.rank_offsets), host(rl.rank_row), host(lay.slot), host(recv), host(ridx),
+                     host(rw).view(np.uint32), host(src)))
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)
+    ref_rl = oracle.rank_layout(oracle.tc_layout(idx, E, R)["is_token_in_rank"])
+    _check_rank_layout(rl, ref_rl)
+    assert np.array_equal(outs[1][3], x[outs[1][6]])  # every received row is its source token's row
