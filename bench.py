@@ -802,6 +802,14 @@ def run_workload_table(args):
                 emit(cfg, "dispatch", timeit(lambda: B.ep_dispatch(x, rt, lay, recv, mode=mode,
                                                                    max_tokens_per_expert=mt)),
                      T * H * 2 + n_valid * H * 2 + meta, T)
+                lb = T * K * 12 + T * R + E * 8 + R * 4
+                emit(cfg, "layout + dispatch (two calls)",
+                     timeit(lambda: (B.ep_get_layout(rt, lay),
+                                     B.ep_dispatch(x, rt, lay, recv, mode=mode, max_tokens_per_expert=mt))),
+                     lb + T * H * 2 + n_valid * H * 2 + meta, T)
+                emit(cfg, "layout + dispatch (one call, ep_layout_dispatch)",
+                     timeit(lambda: B.ep_layout_dispatch(x, rt, lay, recv, mode=mode, max_tokens_per_expert=mt)),
+                     lb + T * H * 2 + n_valid * H * 2 + meta, T)
                 y = recv
             out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
             emit(cfg, "combine", timeit(lambda: B.ep_combine(y, rt, lay, w, out, mode=mode,
@@ -840,6 +848,12 @@ def run_workload_table(args):
                      timeit(lambda: B.ep_dispatch_ranks(x, rt, lay, rl, rrecv, topk_weights=w, recv_topk_idx=ridx,
                                                         recv_topk_weights=rwt)),
                      T * H * 2 + n_rank * H * 2 + n_rank * K * 12 + T * R * 4 + T * K * 12, T)
+                emit(cfg, "layout + rank layout + dispatch_ranks (three calls)",
+                     timeit(lambda: (B.ep_get_layout(rt, lay), B.ep_get_rank_layout(rt, lay, rl),
+                                     B.ep_dispatch_ranks(x, rt, lay, rl, rrecv, topk_weights=w, recv_topk_idx=ridx,
+                                                         recv_topk_weights=rwt))),
+                     T * K * 12 + T * R + E * 8 + R * 4 + T * R + R * 4 + (R + 1) * 4 + T * R * 4
+                     + T * H * 2 + n_rank * H * 2 + n_rank * K * 12 + T * R * 4 + T * K * 12, T)
                 emit(cfg, "layout_dispatch_ranks (one call: layout, rank layout, dispatch)",
                      timeit(lambda: B.ep_layout_dispatch_ranks(x, rt, lay, rl, rrecv, topk_weights=w,
                                                                recv_topk_idx=ridx, recv_topk_weights=rwt)),
@@ -877,6 +891,9 @@ def run_workload_table(args):
             recv = torch.empty((S, H), dtype=torch.bfloat16, device=dev)
             emit(cfg, "ec_dispatch", timeit(lambda: B.ep_dispatch_expert_choice(x, rt, lay, recv)),
                  uniq * H * 2 + S * H * 2 + S * 4, T)
+            emit(cfg, "ec_layout + ec_dispatch (two calls)",
+                 timeit(lambda: (B.ep_get_layout(rt, lay), B.ep_dispatch_expert_choice(x, rt, lay, recv))),
+                 S * 4 + (T + 1) * 4 + S * 4 + T * R + E * 4 + R * 4 + uniq * H * 2 + S * H * 2 + S * 4, T)
             emit(cfg, "ec_layout_dispatch (one call)", timeit(lambda: B.ep_layout_dispatch_expert_choice(x, rt, lay, recv)),
                  S * 4 + (T + 1) * 4 + S * 4 + T * R + E * 4 + R * 4 + uniq * H * 2 + S * H * 2 + S * 4, T)
             out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
