@@ -683,6 +683,34 @@ def test_layout_dispatch_one_call_equals_the_two_calls():
     assert B.ep_get_device_error(lay) == 0
 
 
+@pytest.mark.parametrize("wl", [2, 5])
+def test_layout_dispatch_full_size_equals_the_two_calls(wl):
+    """ep_layout_dispatch at full size (the dispatch's CTAs start under the
+    layout and read its slots and offsets after waiting for it), three times
+    with layout outputs pre-filled with zeros: every received row equals the
+    row the separate ep_get_layout + ep_dispatch calls write."""
+    inp = inputs(wl)
+    c = inp["cfg"]
+    E, R, H = c["E"], c["R"], c["H"]
+    xd = to_dev(inp["x"], bf16=True)
+    routing = B.Routing.topk(to_dev(inp["topk_idx"]), E, R)
+    lay0 = B.Layout(routing)
+    B.ep_get_layout(routing, lay0)
+    n = int(host(lay0.expert_offsets)[-1])
+    ref = torch.full((n, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    B.ep_dispatch(xd, routing, lay0, ref, num_recv_rows=n)
+    want = ref.view(torch.int16)
+    for _ in range(3):
+        lay = B.Layout(routing)
+        lay.slot.fill_(0)
+        lay.expert_offsets.fill_(0)
+        out = torch.full((n, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        B.ep_layout_dispatch(xd, routing, lay, out, num_recv_rows=n)
+        assert B.ep_get_device_error(lay) == 0
+        assert int((out.view(torch.int16) != want).any(dim=1).sum().item()) == 0
+        del out
+
+
 def test_dispatch_reads_x_written_by_the_kernel_just_before():
     """ep_dispatch after a kernel that writes x on the same stream (the
     layout computed earlier): the dispatch waits for that kernel before its
