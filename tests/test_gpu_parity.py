@@ -711,6 +711,41 @@ def test_layout_dispatch_full_size_equals_the_two_calls(wl):
         del out
 
 
+def test_combine_queued_right_behind_a_layout_reads_the_finished_layout():
+    """A combine (and a rank combine) queued directly behind ep_get_layout
+    (and ep_get_rank_layout), with no synchronisation in between: the plain
+    layout calls do not let the next kernel start early, so the combine's
+    read-only loads of slots, offsets and rank rows see the finished
+    layout; outputs bit for bit against the oracle."""
+    inp = inputs(2, T=2048)
+    c = inp["cfg"]
+    idx, w = inp["topk_idx"], inp["topk_weights"]
+    E, R, H, T = c["E"], c["R"], c["H"], 2048
+    ref_l = oracle.tc_layout(idx, E, R)
+    n = int(ref_l["expert_offsets"][-1])
+    r = rng(77)
+    y = W.to_bf16_bits(r.standard_normal((n, H)).astype(np.float32))
+    yd, wd = to_dev(y, bf16=True), to_dev(w)
+    routing = B.Routing.topk(to_dev(idx), E, R)
+    lay = B.Layout(routing)
+    lay.slot.fill_(0)
+    lay.expert_offsets.fill_(0)
+    out = nan_filled((T, H), torch.float32)
+    B.ep_get_layout(routing, lay)
+    B.ep_combine(yd, routing, lay, wd, out, num_y_rows=n)
+    assert exact_fraction(host(out), oracle.tc_combine(y, idx, E, ref_l, w, out_dtype=W.FP32)) == 1.0
+    ref_rl = oracle.rank_layout(ref_l["is_token_in_rank"])
+    m = int(ref_rl["rank_offsets"][-1])
+    yr = W.to_bf16_bits(r.standard_normal((m, H)).astype(np.float32))
+    rl = B.RankLayout(routing)
+    rl.rank_row.fill_(0)
+    out_r = nan_filled((T, H), torch.float32)
+    B.ep_get_rank_layout(routing, lay, rl)
+    B.ep_combine_ranks(to_dev(yr, bf16=True), routing, lay, rl, out_r)
+    assert exact_fraction(host(out_r), oracle.rank_combine(yr, ref_rl, out_dtype=W.FP32)) == 1.0
+    assert B.ep_get_device_error(lay) == 0
+
+
 def test_dispatch_reads_x_written_by_the_kernel_just_before():
     """ep_dispatch after a kernel that writes x on the same stream (the
     layout computed earlier): the dispatch waits for that kernel before its
