@@ -681,8 +681,11 @@ ep_status_t ep_layout_dispatch_ranks(const void* x, int32_t hidden, const ep_rou
     st = launch_rank_layout(routing, layout, rank_layout, stream);
     if (st != EP_OK)
         return st;
-    return launch_rank_dispatch(x, hidden, routing, layout, rank_layout, num_recv_rows, topk_weights, recv_x,
-                                recv_topk_idx, recv_topk_weights, recv_src, stream, true);
+    st = launch_rank_dispatch(x, hidden, routing, layout, rank_layout, num_recv_rows, topk_weights, recv_x,
+                              recv_topk_idx, recv_topk_weights, recv_src, stream, true);
+    if (st != EP_OK)
+        return st;
+    return ep::report_num_valid(routing, layout, reinterpret_cast<cudaStream_t>(stream));
 }
 
 ep_status_t ep_dispatch_ranks(const void* x, int32_t hidden, const ep_routing_desc_t* routing,

@@ -191,10 +191,11 @@ def test_layout_dispatch_ranks_one_call_equals_the_three_calls(wl):
         rw = torch.full((rows, K), float("nan"), dtype=torch.float32, device="cuda")
         src = torch.full((rows,), -9, dtype=torch.int32, device="cuda")
         if one_call:
-            lay = B.Layout(routing)
+            lay = B.Layout(routing, report_num_valid=True)
             rl = B.RankLayout(routing)
             B.ep_layout_dispatch_ranks(xd, routing, lay, rl, recv, topk_weights=wd, recv_topk_idx=ridx,
                                        recv_topk_weights=rw, recv_src=src)
+            assert lay.num_valid == int((idx >= 0).sum())  # num_valid_host, as ep_get_layout reports it
         else:
             B.ep_dispatch_ranks(xd, routing, lay, rl, recv, topk_weights=wd, recv_topk_idx=ridx, recv_topk_weights=rw,
                                 recv_src=src)
