@@ -130,6 +130,12 @@ constexpr int kEcLookup = EP_COMBINE_EC_LOOKUP;
 #define EP_COMBINE_EC_MINB 2
 #endif
 constexpr int kEcMinBlocks = EP_COMBINE_EC_MINB;
+// expert choice: each group's weights (looked up from its slots, one more
+// round trip) are taken from their lanes after the group's row loads are
+// issued, not before (fp32 out 61.4 -> 60.4 us; bf16 unchanged)
+#ifndef EP_COMBINE_EC_LATE_W
+#define EP_COMBINE_EC_LATE_W 1
+#endif
 // per-rank combines: when a token's rank rows are spread over more groups
 // than they fill, they are packed to the front (ascending rank kept) so that
 // their loads go out in fewer rounds.  Measured on the skewed 16384-token
@@ -499,7 +505,8 @@ __device__ __forceinline__ void reduce_run(const CombineArgs& a, int64_t t0, int
                 for (int g = 0; g < kGroup; ++g) {
                     const int src = (g0 + g) & 31;
                     rows[g] = __shfl_sync(kFullMask, my_row[i], src);
-                    ws[g] = __shfl_sync(kFullMask, my_w[i], src);
+                    if (!EP_COMBINE_EC_LATE_W)
+                        ws[g] = __shfl_sync(kFullMask, my_w[i], src);
                     if (g0 + g >= m)
                         rows[g] = -1;
                 }
@@ -521,6 +528,11 @@ __device__ __forceinline__ void reduce_run(const CombineArgs& a, int64_t t0, int
                         for (int j = 0; j < kVecPerLane; ++j)
                             d[g][j] = (on && vin[j]) ? ld_nc_v4(src + static_cast<int64_t>(v[j]) * 16) : make_uint4(0, 0, 0, 0);
                     }
+                }
+                if (EP_COMBINE_EC_LATE_W) { // the weights' lookups finish under the row loads
+#pragma unroll
+                    for (int g = 0; g < kGroup; ++g)
+                        ws[g] = __shfl_sync(kFullMask, my_w[i], (g0 + g) & 31);
                 }
 #pragma unroll
                 for (int g = 0; g < kGroup; ++g) {
@@ -611,7 +623,8 @@ __device__ __forceinline__ void reduce_heavy(const CombineArgs& a, int64_t t, in
 #pragma unroll
             for (int g = 0; g < kGroup; ++g) {
                 rows[g] = __shfl_sync(kFullMask, r_cur, g0 + g);
-                ws[g] = __shfl_sync(kFullMask, w_cur, g0 + g);
+                if (!EP_COMBINE_EC_LATE_W)
+                    ws[g] = __shfl_sync(kFullMask, w_cur, g0 + g);
                 if (g0 + g >= m)
                     rows[g] = -1;
             }
@@ -638,6 +651,11 @@ __device__ __forceinline__ void reduce_heavy(const CombineArgs& a, int64_t t, in
                 r_nxt = valid(k0 + 32 + lane, s_nxt) ? s_nxt : -1;
                 w_nxt = r_nxt >= 0 ? __ldg(a.expert_weights + r_nxt) : 0.0f;
                 s_after = slot_at(k0 + 64 + lane);
+            }
+            if (EP_COMBINE_EC_LATE_W) { // the weights' lookups finish under the row loads
+#pragma unroll
+                for (int g = 0; g < kGroup; ++g)
+                    ws[g] = __shfl_sync(kFullMask, w_cur, g0 + g);
             }
 #pragma unroll
             for (int g = 0; g < kGroup; ++g) {
