@@ -34,7 +34,7 @@ def _gpu():
 
 
 def test_grid_barrier_wait_runs_out_and_is_reported():
-    inp = W.make_inputs(2, T=2048)  # 16384 (token, k) pairs: the grid-wide layout
+    inp = W.make_inputs(2, T=4608)  # 36864 (token, k) pairs: the grid-wide layout
     idx = inp["topk_idx"]
     routing = B.Routing.topk(to_dev(idx), 256, 8)
     lay = B.Layout(routing)

@@ -67,7 +67,9 @@ def _compare(routing):
 
 
 def test_no_alloc_matches_layout_token_choice():
-    inp = W.make_inputs(2)
+    inp = W.make_inputs(2)  # 32768 pairs: the 16-CTA cluster layout
+    _compare(B.Routing.topk(_dev(inp["topk_idx"]), 256, 8))
+    inp = W.make_inputs(5)  # 131072 pairs: the grid-wide layout (its barrier words in the scratch array)
     _compare(B.Routing.topk(_dev(inp["topk_idx"]), 256, 8))
     rng = np.random.Generator(np.random.PCG64(3))
     idx = W.random_topk(rng, 300, 24, 5, p_neg=0.2, allow_dup=True, p_bad=0.05)
