@@ -2,11 +2,13 @@
  * ep.h -- MoE token layout, dispatch and combine on one B200 (sm_100a).
  *
  * C ABI of libep_b200.so.  All tensors are plain device pointers, row-major
- * and densely packed; all memory belongs to the caller.  No entry point
- * allocates or frees device memory, and none synchronises the host except
- * ep_get_device_error() and a layout call given a num_valid_host pointer.
- * Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
- * default stream).
+ * and densely packed; all memory belongs to the caller.  Only ep_peer_alloc /
+ * ep_peer_free (device memory other processes map) and ep_peer_open /
+ * ep_peer_close (those mappings) allocate, free or map device memory, and no
+ * entry point synchronises the host except ep_get_device_error() and a
+ * layout call (or a one-call layout + dispatch) given a num_valid_host
+ * pointer.  Every other call is asynchronous on `stream` (a cudaStream_t;
+ * NULL = the legacy default stream).
  *
  * The operations follow these pages (title, section):
  *   [README] "DeepEP-Ascend" README (sgl-kernel-npu python/deep_ep),
