@@ -35,6 +35,16 @@ transfer here hands a peer's memory to a library kernel.
 The compute steps are the CUDA kernels of the C ABI (``CudaRowOps``); the
 exchange itself takes any object with the same three methods, so that the
 protocol can be exercised on CPU processes.
+
+``PeerExpertParallel`` runs the same step with the transfers fused into the
+kernels over peer memory instead of a library all-to-all between them: the
+dispatch (ep_dispatch_peers) stores each (token, rank) row straight into
+that rank's receive buffer, mapped into this process through CUDA IPC, and
+the combine (ep_combine_peers) reads the partial rows straight from the
+ranks' buffers.  No kernel waits for another rank: the phases are separated
+by a stream synchronisation and a process-group barrier.  Its memory and
+compute steps likewise come from an object (``CudaPeerOps``) that a test can
+replace.
 """
 from __future__ import annotations
 
