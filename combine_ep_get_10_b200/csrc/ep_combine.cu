@@ -710,11 +710,12 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 // >= 1x kHeavyDeg), in token order inside a class.  The items are then: one per (heavy token, segment),
 // followed by one per (run of kEcRun tokens, segment); a run item folds its
 // light tokens' entries as one list (reduce_run) and leaves the heavy tokens
-// to the heavy items.  Warps are numbered warp-major (warp w of every CTA
-// before warp w + 1): heavy items go to the first warps, so they spread over
-// all SMs, and light items to the last warps first, so that when there are
-// more items than warps the extra light work lands on the warps holding the
-// shortest heavy lists.
+// to the heavy items.  The items, in that order (roughly longest first), are
+// dealt to the CTAs one round of gridDim items at a time in a serpentine (CTA
+// c takes item c of an even round and item gridDim - 1 - c of an odd one), so
+// every CTA holds a like mix of long and short work; a CTA's warps take its
+// rounds in order from a shared-memory ticket, so a warp that finishes early
+// takes the next item instead of the tail waiting on fixed shares.
 template <bool kOutF32>
 __global__ void __launch_bounds__(kCombineThreads, kEcMinBlocks) ec_combine_kernel(CombineArgs a)
 {
@@ -726,7 +727,11 @@ __global__ void __launch_bounds__(kCombineThreads, kEcMinBlocks) ec_combine_kern
     __shared__ int s_heavy[kMaxHeavy];
     __shared__ uint32_t s_flags[kHeavyClasses][kHeavyFirstMaxT / 32];
     __shared__ int s_wsum[kWarpsPerCta];
+    __shared__ int s_ticket; // this CTA's next round of items
     __shared__ __align__(128) uint8_t s_zero[EP_COMBINE_EC_ZERO_BULK ? kZeroBytes : 16];
+    if (threadIdx.x == 0)
+        s_ticket = 0;
+    __syncthreads();
     int n_heavy = 0, n_long = 0;
     if (a.heavy_first) {
         // Every CTA reads the whole CSR bound array once, coalesced and all at
@@ -856,35 +861,43 @@ __global__ void __launch_bounds__(kCombineThreads, kEcMinBlocks) ec_combine_kern
     const int64_t heavy_items = long_items + static_cast<int64_t>(n_heavy - n_long) * nseg_h;
     const int64_t runs = (static_cast<int64_t>(a.T) + kEcRun - 1) / kEcRun;
     const int64_t items = heavy_items + runs * a.nseg;
-    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerCta;
-    const int64_t g = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x; // warp-major
-    // heavy items from the first warps, light items from the last warps
-    // backwards, so a warp with a long list gets light work only when there
-    // are more items than warps
-    for (int64_t it = g; it < heavy_items; it += nwarps) {
-        const bool is_long = it < long_items;
-        const int64_t k = is_long ? it : it - long_items;
-        const int ns = is_long ? nseg_l : nseg_h;
-        const int64_t t = s_heavy[(is_long ? 0 : n_long) + k / ns];
-        const int seg = static_cast<int>(k % ns);
-        const int beg = __ldg(a.token_offsets + t);
-        const int n = __ldg(a.token_offsets + t + 1) - beg;
+    // this CTA's round k holds item k * G + c (k even) or k * G + G - 1 - c (k odd)
+    const int64_t G = gridDim.x;
+    auto take = [&]() -> int {
+        int k = 0;
+        if (lane == 0)
+            k = atomicAdd(&s_ticket, 1);
+        return __shfl_sync(kFullMask, k, 0);
+    };
+    for (int k = take();; k = take()) {
+        const int64_t it = static_cast<int64_t>(k) * G + ((k & 1) ? G - 1 - blockIdx.x : blockIdx.x);
+        if (it >= items)
+            break; // every later round of this CTA lies past the end too
+        if (it < heavy_items) {
+            const bool is_long = it < long_items;
+            const int64_t h = is_long ? it : it - long_items;
+            const int ns = is_long ? nseg_l : nseg_h;
+            const int64_t t = s_heavy[(is_long ? 0 : n_long) + h / ns];
+            const int seg = static_cast<int>(h % ns);
+            const int beg = __ldg(a.token_offsets + t);
+            const int n = __ldg(a.token_offsets + t + 1) - beg;
 #if EP_COMBINE_HEAVY_PIPE
-        if (is_long)
-            reduce_heavy<kOutF32, kHeavy0Vec, kHeavy0Group>(a, t, seg, beg, n, lane, errbits);
-        else
-            reduce_heavy<kOutF32, kHeavyVec, kHeavyGroup>(a, t, seg, beg, n, lane, errbits);
+            if (is_long)
+                reduce_heavy<kOutF32, kHeavy0Vec, kHeavy0Group>(a, t, seg, beg, n, lane, errbits);
+            else
+                reduce_heavy<kOutF32, kHeavyVec, kHeavyGroup>(a, t, seg, beg, n, lane, errbits);
 #else
-        if (is_long)
-            reduce_segment<kSrcEc, kOutF32, kHeavy0Vec, kHeavy0Group, kHeavyLookup>(a, t, seg, beg, n, lane, errbits);
-        else
-            reduce_segment<kSrcEc, kOutF32, kHeavyVec, kHeavyGroup, kHeavyLookup>(a, t, seg, beg, n, lane, errbits);
+            if (is_long)
+                reduce_segment<kSrcEc, kOutF32, kHeavy0Vec, kHeavy0Group, kHeavyLookup>(a, t, seg, beg, n, lane,
+                                                                                       errbits);
+            else
+                reduce_segment<kSrcEc, kOutF32, kHeavyVec, kHeavyGroup, kHeavyLookup>(a, t, seg, beg, n, lane, errbits);
 #endif
-    }
-    const int64_t light_items = items - heavy_items;
-    for (int64_t it = nwarps - 1 - g; it < light_items; it += nwarps) {
-        const int64_t r = it / a.nseg;
-        const int seg = static_cast<int>(it - r * a.nseg);
+            continue;
+        }
+        const int64_t l = it - heavy_items; // a light item
+        const int64_t r = l / a.nseg;
+        const int seg = static_cast<int>(l - r * a.nseg);
         const int64_t t0 = r * kEcRun;
         const int cnt = static_cast<int>(min(static_cast<int64_t>(kEcRun), a.T - t0));
 #if EP_COMBINE_EC_FLAT
