@@ -144,6 +144,15 @@ constexpr int kEcMinBlocks = EP_COMBINE_EC_MINB;
 #ifndef EP_COMBINE_RANKS_COMPACT
 #define EP_COMBINE_RANKS_COMPACT 1
 #endif
+// per-rank and peer combines: 16-byte vectors per lane and rows per load round
+#ifndef EP_COMBINE_RANKS_VEC
+#define EP_COMBINE_RANKS_VEC EP_COMBINE_VEC
+#endif
+#ifndef EP_COMBINE_RANKS_GROUP
+#define EP_COMBINE_RANKS_GROUP EP_COMBINE_GROUP
+#endif
+constexpr int kRanksVec = EP_COMBINE_RANKS_VEC;
+constexpr int kRanksGroup = EP_COMBINE_RANKS_GROUP;
 // heavy items: lookups pipelined (reduce_heavy) or not (reduce_segment)
 #ifndef EP_COMBINE_HEAVY_PIPE
 #define EP_COMBINE_HEAVY_PIPE 1
@@ -286,12 +295,12 @@ __device__ __forceinline__ void reduce_segment(const CombineArgs& a, int64_t t, 
         }
         int m_valid = 32;
 #if EP_COMBINE_RANKS_COMPACT
-        if constexpr ((kSrc == kSrcRanks || kSrc == kSrcPeers) && kLookup == 1) {
+        if constexpr ((kSrc == kSrcRanks || kSrc == kSrcPeers) && kLookup == 1 && kGroup == 4) {
             // the token's ranks first, in ascending order: its loads then fill
-            // the first group instead of spreading over all of them
+            // the first group instead of spreading over all of them (group
+            // occupancy counted by nibbles)
             const uint32_t valid = __ballot_sync(kFullMask, my_row[0] >= 0);
             const int cnt = __popc(valid);
-            static_assert(kGroup == 4, "group occupancy by nibbles");
             // groups (aligned nibbles) holding at least one of the token's ranks
             const int touched = __popc((valid | (valid >> 1) | (valid >> 2) | (valid >> 3)) & 0x11111111u);
             if ((cnt + kGroup - 1) / kGroup < touched) { // packing saves a round of loads
@@ -1090,11 +1099,12 @@ cudaError_t launch_rank_combine(const RankCombineLaunch& a, cudaStream_t stream)
         k.peers = a.peers;
         k.num_y_rows = a.peers.capacity;
         k.wide = 0;
-        return launch_combine<kSrcPeers, kTcVec, kTcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0,
-                                                            stream);
+        return launch_combine<kSrcPeers, kRanksVec, kRanksGroup>(k, a.out_dtype == EP_FP32,
+                                                                  EP_COMBINE_PERSIST_TC != 0, stream);
     }
     k.wide = wide_loads(a.y, a.H, a.T);
-    return launch_combine<kSrcRanks, kTcVec, kTcGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0, stream);
+    return launch_combine<kSrcRanks, kRanksVec, kRanksGroup>(k, a.out_dtype == EP_FP32, EP_COMBINE_PERSIST_TC != 0,
+                                                              stream);
 }
 
 } // namespace ep
