@@ -517,6 +517,7 @@ def time_other_workloads(dev, flush, reps):
     from combine_ep_get_10_b200 import workloads as W
 
     peak, _ = measured_peak()
+    spread = {}  # min, p90 and mean of the last timeit, for the record that reports it
 
     def timeit(fn):
         ts = []
@@ -530,11 +531,13 @@ def time_other_workloads(dev, flush, reps):
             torch.cuda.synchronize(dev)
             if i >= 3:
                 ts.append(a.elapsed_time(b) * 1e3)
+        ts.sort()
+        spread.update(us_min=ts[0], us_p90=ts[min(len(ts) - 1, (9 * len(ts)) // 10)], us_mean=sum(ts) / len(ts))
         return statistics.median(ts)
 
     def rec(us, nbytes):
-        return {"us": round(us, 2), "bytes": int(nbytes), "gbs": round(nbytes / us / 1e3, 1),
-                "frac": round(nbytes / us / 1e3 / peak, 3)}
+        return {"us": round(us, 2), **{k: round(v, 2) for k, v in spread.items()}, "bytes": int(nbytes),
+                "gbs": round(nbytes / us / 1e3, 1), "frac": round(nbytes / us / 1e3 / peak, 3)}
 
     def bf(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -717,6 +720,7 @@ def run_workload_table(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     peak, peak_kind = measured_peak()
     reps = max(10, min(args.steps, 200))
+    spread = {}  # min, p90 and mean of the last timeit, for the line that reports it
 
     def timeit(fn):
         ts = []
@@ -731,10 +735,12 @@ def run_workload_table(args):
             if i >= 3:
                 ts.append(a.elapsed_time(b) * 1e3)
         ts.sort()
+        spread.update(us_min=ts[0], us_p90=ts[min(len(ts) - 1, (9 * len(ts)) // 10)], us_mean=sum(ts) / len(ts))
         return ts[len(ts) // 2]
 
     def emit(cfg, op, us, nbytes, tokens):
-        print(json.dumps({"workload": cfg["name"], "op": op, "us": round(us, 2), "bytes": int(nbytes),
+        print(json.dumps({"workload": cfg["name"], "op": op, "us": round(us, 2),
+                          **{k: round(v, 2) for k, v in spread.items()}, "bytes": int(nbytes),
                           "gbs": round(nbytes / us / 1e3, 1), "frac_of_peak": round(nbytes / us / 1e3 / peak, 3),
                           "peak_gbs": peak, "peak_source": peak_kind, "tokens_per_s": round(tokens / us * 1e6),
                           "reps": reps, "l2": "flushed"}), flush=True)
