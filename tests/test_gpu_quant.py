@@ -112,6 +112,42 @@ def test_quant_dispatch_prefill_compact(dt):
 
 
 @pytest.mark.parametrize("dt", QUANT, ids=lambda d: NAMES[d])
+def test_quant_dispatch_full_prefill_sampled(dt):
+    """The full prefill workload (4096 tokens, hidden 7168, 256 experts,
+    top-8, compact) in the call the benchmark times: for a seeded sample of
+    tokens, every destination row the oracle's layout names holds the
+    oracle's codes and scales of that token, bit for bit (a token's codes
+    depend on its own row only, so the oracle encodes the sample alone)."""
+    inp = W.make_inputs(2)
+    c = inp["cfg"]
+    T, H, E, R = c["T"], c["H"], c["E"], c["R"]
+    x, idx = inp["x"], inp["topk_idx"]
+    ref_l = oracle.tc_layout(idx, E, R)
+    rows = int(ref_l["expert_offsets"][-1])
+    idx_d = to_dev(np.ascontiguousarray(idx, np.int64))
+    routing = B.Routing.topk(idx_d, E, R)
+    lay = B.Layout(routing)
+    B.ep_get_layout(routing, lay)
+    codes, scales = _buffers(dt, rows, H)
+    B.ep_dispatch(to_dev(x, bf16=True), routing, lay, codes, recv_scales=scales, out_dtype=dt)
+    assert B.ep_get_device_error(lay) == 0
+    sample = np.sort(_rng(2024).choice(T, size=48, replace=False))
+    one = np.zeros((len(sample), 1), np.int64)  # every sampled token to one expert, in sample order
+    ref = oracle.tc_dispatch(x[sample], one, 1, oracle.tc_layout(one, 1, 1), out_dtype=dt)
+    rc, rs = _host_bytes(ref, dt, len(sample), H)
+    want_rows, want_i = [], []
+    for i, t in enumerate(sample):
+        for k in range(idx.shape[1]):
+            e = int(idx[t, k])
+            if e >= 0:
+                want_rows.append(int(ref_l["expert_offsets"][e]) + int(ref_l["slot"][t, k]))
+                want_i.append(i)
+    sel = torch.tensor(want_rows, dtype=torch.int64, device="cuda")
+    gc, gs = host(codes[sel]), host(scales[sel])
+    assert np.array_equal(gc, rc[want_i]) and np.array_equal(gs, rs[want_i])
+
+
+@pytest.mark.parametrize("dt", QUANT, ids=lambda d: NAMES[d])
 @pytest.mark.parametrize("H", [128, 4224, 32768])
 def test_quant_dispatch_ragged_hidden_and_magnitudes(dt, H):
     """Row widths that leave threads idle (4224 = 528 vectors) or fill the
