@@ -363,7 +363,10 @@ constexpr int kFusedMaxPairs = 8192;
 constexpr int kFusedMaxK = 32;
 constexpr int kFusedMaxE = 1024;
 
-constexpr int kQuantThreads = 128; // threads per token CTA
+#ifndef EP_QUANT_THREADS
+#define EP_QUANT_THREADS 256
+#endif
+constexpr int kQuantThreads = EP_QUANT_THREADS; // threads per token CTA
 
 __device__ __forceinline__ float amax8(uint4 r)
 {
