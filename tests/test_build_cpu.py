@@ -11,6 +11,7 @@ import re
 import shutil
 import subprocess
 import sys
+import tempfile
 
 import pytest
 
@@ -27,14 +28,10 @@ def _report(source):
     if shutil.which("nvcc") is None and not os.path.exists("/usr/local/cuda/bin/nvcc"):
         pytest.skip("nvcc not available")
     flags = [f for f in BUILD.NVCC_FLAGS if f != "--shared"]
-    out = os.path.join(ROOT, "_build_report_%d.o" % os.getpid())
-    try:
+    with tempfile.TemporaryDirectory() as tmp:
         r = subprocess.run([BUILD.nvcc()] + BUILD.ARCH_FLAGS + flags +
-                           ["-I", BUILD.INCLUDE, "-I", CSRC, "-c", "-o", out, os.path.join(CSRC, source),
-                            "-Xptxas", "-v"], capture_output=True, text=True, timeout=600)
-    finally:
-        if os.path.exists(out):
-            os.remove(out)
+                           ["-I", BUILD.INCLUDE, "-I", CSRC, "-c", "-o", os.path.join(tmp, "k.o"),
+                            os.path.join(CSRC, source), "-Xptxas", "-v"], capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     kernels, name = {}, None
     spill = 0
